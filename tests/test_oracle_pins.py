@@ -1,0 +1,305 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Every check here compares the oracle with something other than itself: the
+worked example printed on the pages (tests/golden/running_example.json), a
+special case with a textbook closed form, an invariant the pages state, or a
+different algorithm of the oracle computing the same mathematical object.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import msr as omsr
+from retention_inputs import gamma_schedule
+
+
+def ex(golden):
+    Q = np.array(golden["Q"], float)[None, :, None, :]
+    K = np.array(golden["K"], float)[None, :, None, :]
+    V = np.array(golden["V"], float)[None, :, None, :]
+    return Q, K, V, np.array([golden["gamma"]])
+
+
+# ------------------------------------------------ the page's running example
+
+def test_recurrent_running_example_outputs(golden):
+    Q, K, V, g = ex(golden)
+    out, S4 = oracle.retention_recurrent(Q, K, V, g)
+    np.testing.assert_allclose(out[0, :, 0, :], golden["O"], atol=1e-12)
+    np.testing.assert_allclose(S4[0, 0], golden["S"][3], atol=1e-12)
+
+
+def test_recurrent_running_example_states_and_norms(golden):
+    Q, K, V, g = ex(golden)
+    for n in range(1, 5):
+        _, Sn = oracle.retention_recurrent(Q[:, :n], K[:, :n], V[:, :n], g)
+        np.testing.assert_allclose(Sn[0, 0], golden["S"][n - 1], atol=1e-12)
+        assert round(float(np.linalg.norm(Sn[0, 0])), 2) == pytest.approx(golden["state_norms_2dp"][n - 1])
+
+
+def test_parallel_running_example(golden):
+    Q, K, V, g = ex(golden)
+    out = oracle.retention_parallel(Q, K, V, g)
+    np.testing.assert_allclose(out[0, :, 0, :], golden["O"], atol=1e-12)
+    # the page's intermediates: (Q K^T (.) D) V with its printed Q K^T (.) D
+    np.testing.assert_allclose(np.array(golden["QKt_D"]) @ np.array(golden["V"]), golden["O"], atol=1e-12)
+    # D from the oracle's gamma power helper
+    D = np.array([[oracle.gamma_pow(0.9, n - m) if n >= m else 0.0 for m in range(4)] for n in range(4)])
+    np.testing.assert_allclose(D, golden["D"], atol=1e-12)
+
+
+def test_chunkwise_running_example(golden):
+    Q, K, V, g = ex(golden)
+    c = golden["chunk2"]
+    out, R2 = oracle.retention_chunkwise(Q, K, V, g, chunk=2)
+    np.testing.assert_allclose(out[0, :, 0, :], golden["O"], atol=1e-12)
+    np.testing.assert_allclose(R2[0, 0], c["R_2"], atol=1e-12)
+    # R_1: the state after the first chunk
+    out1, R1 = oracle.retention_chunkwise(Q[:, :2], K[:, :2], V[:, :2], g, chunk=2)
+    np.testing.assert_allclose(R1[0, 0], c["R_1"], atol=1e-12)
+    np.testing.assert_allclose(out1[0, :, 0, :], c["inner_1"], atol=1e-12)
+    # Inner_2: chunk 2 on its own (zero incoming state) is the inner term only
+    inner2, _ = oracle.retention_chunkwise(Q[:, 2:], K[:, 2:], V[:, 2:], g, chunk=2)
+    np.testing.assert_allclose(inner2[0, :, 0, :], c["inner_2"], atol=1e-12)
+    # Cross_2 = output of chunk 2 minus Inner_2, equal to (Q_[2] R_1) (.) xi
+    np.testing.assert_allclose(out[0, 2:, 0, :] - inner2[0, :, 0, :], c["cross_2"], atol=1e-12)
+    np.testing.assert_allclose(np.array(c["Q2_R1"]) * np.array(c["xi"])[:, None], c["cross_2"], atol=1e-12)
+    # zeta and xi from the gamma power helper, 0-based rows, B = 2
+    assert [oracle.gamma_pow(0.9, 2 - 1 - j) for j in range(2)] == pytest.approx(c["zeta"], abs=1e-15)
+    assert [oracle.gamma_pow(0.9, j + 1) for j in range(2)] == pytest.approx(c["xi"], abs=1e-15)
+
+
+def test_linear_attention_special_case(golden):
+    """gamma = 1 with phi(x) = elu(x) + 1 keys is the linear-attention state
+    of the page's section 1.1 (exact integers)."""
+    Q, K, V, _ = ex(golden)
+    phiK = np.where(K > 0, K, np.expm1(np.minimum(K, 0))) + 1.0
+    la = golden["linear_attention"]
+    for n in range(1, 5):
+        _, Sn = oracle.retention_recurrent(Q[:, :n], phiK[:, :n], V[:, :n], np.array([1.0]))
+        np.testing.assert_array_equal(Sn[0, 0], la["S"][n - 1])
+        assert round(float(np.linalg.norm(Sn[0, 0])), 2) == pytest.approx(la["norms_2dp"][n - 1])
+
+
+def test_decay_table(golden):
+    t = golden["decay_table"]
+    for e, val in t["powers"].items():
+        got = oracle.gamma_pow(t["gamma"], int(e))
+        # printed to 3 significant figures (2 for 0.0052): round to match
+        sig = 2 if val == 0.0052 else 3
+        assert float(f"{got:.{sig - 1}e}") == pytest.approx(val, rel=1e-12)
+    assert oracle.gamma_pow(0.0, 0) == 1.0 and oracle.gamma_pow(0.0, 3) == 0.0
+    assert oracle.gamma_pow(1.0, 10 ** 6) == 1.0
+
+
+def test_rotation_table(golden):
+    """A query at n = 4 against keys at m = 1..4 with theta = pi/4: the rotated
+    dot product gives cos((n-m) theta) for q = k = e_0 and sin((n-m) theta)
+    for q = e_0, k = e_1."""
+    t = golden["rotation_table"]
+    # d = 4 and theta_base = (4/pi)^2 make the pair p = 1 turn by pi/4 per step
+    base = (4.0 / math.pi) ** 2
+    assert base ** (-2 * 1 / 4) == pytest.approx(t["theta"], rel=1e-15)
+    N = 5
+    e0 = np.zeros((1, N, 1, 4)); e0[..., 2] = 1.0
+    e1 = np.zeros((1, N, 1, 4)); e1[..., 3] = 1.0
+    r0 = oracle.xpos_rotate(e0, 0, base)
+    r1 = oracle.xpos_rotate(e1, 0, base)
+    n = t["n"]
+    cos = [float(r0[0, n, 0] @ r0[0, m, 0]) for m in t["m"]]
+    sin = [float(r0[0, n, 0] @ r1[0, m, 0]) for m in t["m"]]
+    np.testing.assert_allclose(cos, t["cos"], atol=1e-3)
+    np.testing.assert_allclose(sin, t["sin"], atol=1e-3)
+
+
+def test_gamma_schedule(golden):
+    t = golden["gamma_schedule"]
+    np.testing.assert_array_equal(gamma_schedule(8), t["gamma"])
+    win = np.log(0.01) / np.log(np.array(t["gamma"]))
+    # the first four are printed from the exact formula; the rest are within 0.2%
+    np.testing.assert_allclose(np.round(win[:4]), t["window"][:4], atol=1.0)
+    np.testing.assert_allclose(win, t["window"], rtol=2e-3)
+
+
+# --------------------------------------------- forms agree, special cases
+
+def rand_qkv(rng, B, N, H, dk, dv):
+    return (rng.standard_normal((B, N, H, dk)), rng.standard_normal((B, N, H, dk)),
+            rng.standard_normal((B, N, H, dv)))
+
+
+@pytest.mark.parametrize("N", [1, 2, 5, 17, 33])
+def test_three_forms_agree(N):
+    rng = np.random.default_rng(100 + N)
+    B, H, dk, dv = 2, 3, 4, 6
+    q, k, v = rand_qkv(rng, B, N, H, dk, dv)
+    g = np.array([0.5, 0.9, 0.999])
+    rec, S = oracle.retention_recurrent(q, k, v, g)
+    par = oracle.retention_parallel(q, k, v, g)
+    scale = np.abs(rec).max() + 1.0
+    np.testing.assert_allclose(par, rec, atol=1e-12 * scale, rtol=0)
+    for c in sorted({1, 2, 3, 4, 8, N, N + 3}):
+        chk, R = oracle.retention_chunkwise(q, k, v, g, chunk=c)
+        np.testing.assert_allclose(chk, rec, atol=1e-12 * scale, rtol=0)
+        np.testing.assert_allclose(R, S, atol=1e-12 * (np.abs(S).max() + 1), rtol=0)
+
+
+def test_gamma_zero_closed_form():
+    """gamma = 0 (0^0 = 1): o_n = (q_n . k_n) v_n; gamma = 1e-30 is within
+    rounding of it."""
+    rng = np.random.default_rng(7)
+    q, k, v = rand_qkv(rng, 1, 9, 2, 5, 3)
+    expect = np.einsum("bnhd,bnhd->bnh", q, k)[..., None] * v
+    for g in (0.0, 1e-30):
+        gam = np.array([g, g])
+        rec, S = oracle.retention_recurrent(q, k, v, gam)
+        np.testing.assert_allclose(rec, expect, atol=1e-12)
+        np.testing.assert_allclose(oracle.retention_parallel(q, k, v, gam), expect, atol=1e-12)
+        np.testing.assert_allclose(oracle.retention_chunkwise(q, k, v, gam, 4)[0], expect, atol=1e-12)
+        np.testing.assert_allclose(S[0, :, :, :], np.einsum("hd,he->hde", k[0, -1], v[0, -1]), atol=1e-12)
+
+
+def test_gamma_one_is_causal_linear_attention():
+    """gamma = 1: un-normalised causal linear attention, tril(Q K^T) V."""
+    rng = np.random.default_rng(8)
+    q, k, v = rand_qkv(rng, 1, 12, 1, 4, 5)
+    expect = np.tril(q[0, :, 0] @ k[0, :, 0].T) @ v[0, :, 0]
+    rec, _ = oracle.retention_recurrent(q, k, v, np.array([1.0]))
+    np.testing.assert_allclose(rec[0, :, 0], expect, atol=1e-12)
+
+
+def test_relative_position_invariance():
+    """A common position offset on Q and K leaves retention unchanged
+    (the score depends only on n - m)."""
+    rng = np.random.default_rng(9)
+    q, k, v = rand_qkv(rng, 1, 11, 2, 8, 3)
+    g = np.array([0.9, 0.97])
+    outs = []
+    for off in (0, 5, 1000):
+        outs.append(oracle.retention_recurrent(oracle.xpos_rotate(q, off), oracle.xpos_rotate(k, off), v, g)[0])
+    np.testing.assert_allclose(outs[1], outs[0], atol=1e-9)
+    np.testing.assert_allclose(outs[2], outs[0], atol=1e-9)
+    # and the rotation does change the result against no rotation
+    plain = oracle.retention_recurrent(q, k, v, g)[0]
+    assert np.abs(plain - outs[0]).max() > 1e-3
+
+
+def test_rotation_preserves_pair_norms_and_position_zero():
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal((2, 7, 3, 8))
+    y = oracle.xpos_rotate(x, 3)
+    np.testing.assert_allclose(np.hypot(y[..., 0::2], y[..., 1::2]), np.hypot(x[..., 0::2], x[..., 1::2]), atol=1e-12)
+    z = oracle.xpos_rotate(x, 0)
+    np.testing.assert_array_equal(z[:, 0], x[:, 0])   # angle 0 at position 0
+    # pair 0 turns by exactly one radian per position
+    np.testing.assert_allclose(z[0, 1, 0, 0], x[0, 1, 0, 0] * math.cos(1) - x[0, 1, 0, 1] * math.sin(1), atol=1e-14)
+
+
+def test_bounded_state():
+    rng = np.random.default_rng(11)
+    N = 400
+    q, k, v = rand_qkv(rng, 1, N, 2, 3, 3)
+    k = np.clip(k, -1, 1); v = np.clip(v, -1, 1)
+    g = np.array([0.9, 0.99])
+    c = 1.0
+    for n in (1, 10, 100, 400):
+        _, S = oracle.retention_recurrent(q[:, :n], k[:, :n], v[:, :n], g)
+        for h in range(2):
+            bound = c * (1 - g[h] ** n) / (1 - g[h])
+            assert np.abs(S[0, h]).max() <= bound + 1e-12
+
+
+def test_decode_continues_the_recurrence():
+    """prefill then decode steps == the recurrence over the concatenation."""
+    rng = np.random.default_rng(12)
+    B, N, H, dk, dv, T = 2, 9, 2, 4, 5, 4
+    q, k, v = rand_qkv(rng, B, N + T, H, dk, dv)
+    g = np.array([0.8, 0.95])
+    full, Sfull = oracle.retention_recurrent(q, k, v, g)
+    _, S = oracle.retention_recurrent(q[:, :N], k[:, :N], v[:, :N], g)
+    for t in range(T):
+        o, S = oracle.decode_step(q[:, N + t], k[:, N + t], v[:, N + t], g, S)
+        np.testing.assert_allclose(o, full[:, N + t], atol=1e-12)
+    np.testing.assert_allclose(S, Sfull, atol=1e-12)
+    # and init_state of the recurrent form agrees with it
+    out2, S2 = oracle.retention_recurrent(q[:, N:], k[:, N:], v[:, N:], g,
+                                          init_state=oracle.retention_recurrent(q[:, :N], k[:, :N], v[:, :N], g)[1])
+    np.testing.assert_allclose(out2, full[:, N:], atol=1e-12)
+
+
+def test_threads_do_not_change_results():
+    rng = np.random.default_rng(13)
+    q, k, v = rand_qkv(rng, 2, 20, 3, 4, 4)
+    g = np.array([0.5, 0.9, 0.99])
+    a = oracle.retention_recurrent(q, k, v, g, nthreads=1)[0]
+    b = oracle.retention_recurrent(q, k, v, g, nthreads=4)[0]
+    np.testing.assert_array_equal(a, b)
+
+
+# ------------------------------------------------------- MSR layer pieces
+
+def test_swish_closed_form():
+    x = np.array([-30.0, -2.0, -0.5, 0.0, 0.5, 2.0, 30.0])
+    s = omsr.swish(x)
+    assert s[3] == 0.0
+    np.testing.assert_allclose(s[-1], 30.0, rtol=1e-12)
+    np.testing.assert_allclose(s[0], 0.0, atol=1e-11)
+    # swish(-x) = swish(x) - x  (since sigma(-x) = 1 - sigma(x))
+    np.testing.assert_allclose(omsr.swish(-x), s - x, atol=1e-12)
+    np.testing.assert_allclose(omsr.swish(np.array([1.0])), [1.0 / (1.0 + math.exp(-1.0))], rtol=1e-15)
+
+
+def test_group_norm_invariants():
+    rng = np.random.default_rng(14)
+    y = rng.standard_normal((2, 5, 3, 16)) * np.array([0.1, 1.0, 30.0])[None, None, :, None] + 2.0
+    z = omsr.group_norm_heads(y, 1e-5)
+    np.testing.assert_allclose(z.mean(-1), 0.0, atol=1e-12)
+    var = (z ** 2).mean(-1)
+    expect = (y.var(-1)) / (y.var(-1) + 1e-5)
+    np.testing.assert_allclose(var, expect, rtol=1e-12)
+    # scale invariance (exact when eps = 0), per head
+    z0 = omsr.group_norm_heads(y, 0.0)
+    z1 = omsr.group_norm_heads(y * np.array([3.0, 0.5, 7.0])[None, None, :, None], 0.0)
+    np.testing.assert_allclose(z1, z0, atol=1e-12)
+
+
+def test_project_brute_force():
+    rng = np.random.default_rng(15)
+    x = rng.standard_normal((2, 3, 4)); w = rng.standard_normal((4, 5))
+    got = omsr.project(x, w)
+    for a in range(2):
+        for b in range(3):
+            for j in range(5):
+                assert got[a, b, j] == pytest.approx(sum(x[a, b, i] * w[i, j] for i in range(4)), abs=1e-12)
+
+
+def _tiny_msr(rng, B=1, N=10, dm=8, H=2, dk=4, dv=6):
+    x = rng.standard_normal((B, N, dm))
+    W = dict(wq=rng.standard_normal((dm, H * dk)), wk=rng.standard_normal((dm, H * dk)),
+             wv=rng.standard_normal((dm, H * dv)), wg=rng.standard_normal((dm, H * dv)),
+             wo=rng.standard_normal((H * dv, dm)))
+    return x, W, np.array([0.9, 0.99])
+
+
+def test_msr_layer_invariants():
+    rng = np.random.default_rng(16)
+    x, W, g = _tiny_msr(rng)
+    H, dv = 2, 6
+    out = omsr.msr_forward(x, **W, gammas=g, H=H, k_scale=0.5, eps=0.0)
+    # scaling one head's value projection does not change the output: the
+    # normalisation is per head (a layer-wide norm would change it)
+    W2 = dict(W); W2["wv"] = W["wv"].copy(); W2["wv"][:, :dv] *= 5.0
+    np.testing.assert_allclose(omsr.msr_forward(x, **W2, gammas=g, H=H, k_scale=0.5, eps=0.0), out, atol=1e-9)
+    # causality: a change at token t leaves earlier outputs unchanged
+    x2 = x.copy(); x2[:, 6] += 1.0
+    out2 = omsr.msr_forward(x2, **W, gammas=g, H=H, k_scale=0.5, eps=0.0)
+    np.testing.assert_allclose(out2[:, :6], out[:, :6], atol=1e-12)
+    assert np.abs(out2[:, 6:] - out[:, 6:]).max() > 1e-6
+    # the sampled-heads form agrees with the full layer's gated heads
+    _, z, y, ret = omsr.msr_forward(x, **W, gammas=g, H=H, k_scale=0.5, eps=0.0, return_parts=True)
+    z1 = omsr.msr_forward(x, **W, gammas=g, H=H, k_scale=0.5, eps=0.0, heads=[1])
+    np.testing.assert_allclose(z1[:, :, 0], z[:, :, 1], atol=1e-12)
+    # output = Z W_O
+    np.testing.assert_allclose(out, z.reshape(1, 10, H * dv) @ W["wo"], atol=1e-12)
