@@ -1,0 +1,156 @@
+/*
+ * retention.h -- C ABI of the B200 (sm_100a) multi-scale retention library.
+ *
+ * The library computes retention, the sequence mixer of the Retentive Network:
+ *     o_n = sum_{m <= n} gamma_h^(n-m) (q_n . k_m) v_m        (per head h)
+ * defined by the recurrence S_n = gamma S_{n-1} + k_n v_n^T, o_n = q_n^T S_n
+ * ("Hybrid Architectures: RetNet and the Three Computation Paradigms",
+ * sections 2.1-2.2; RetNet paper summary, Eq. 6).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.  Row-major, last index fastest:
+ *     q, k          [B, N, H, dk]      (decode: [B, H, dk])
+ *     v, out        [B, N, H, dv]      (decode: [B, H, dv])
+ *     state         [B, H, dk, dv]     always fp32
+ * Positions are 0-based: token n sits at position pos_offset + n.
+ *
+ * Dtypes.  RET_BF16 inputs are multiplied in the tensor cores with fp32
+ * accumulation; RET_F32 inputs run on the CUDA cores in fp32 (no TF32).
+ * Every carried state is fp32.
+ *
+ * gammas.  A HOST pointer to H doubles, each in [0, 1].  The library turns
+ * them into per-head constants on the host in fp64 and passes those by value
+ * to the kernels, so the array may be freed as soon as the call returns.
+ *
+ * Ownership.  The caller allocates every device buffer.  The library keeps
+ * no pointer after a call returns and allocates nothing, except where an
+ * entry point says so.
+ *
+ * Asynchrony.  Every call enqueues its kernels on `stream` and returns
+ * without synchronising.  Results are valid once the stream has completed.
+ * Calls are thread-safe; the error string is per thread.
+ *
+ * Errors.  Every argument is checked before anything is launched; a failed
+ * check returns RET_ERR_INVALID_ARG (bad pointer, size, alignment or value)
+ * or RET_ERR_UNSUPPORTED (a valid combination no kernel implements) and
+ * launches nothing.  A failed launch returns RET_ERR_CUDA.  Kernels that wait
+ * on an mbarrier give up after a bounded number of polls, set a device-side
+ * error word and return; ret_check_device_error() reads it (RET_ERR_TIMEOUT).
+ * No entry point aborts, traps or prints.  ret_last_error_string() describes
+ * the last failure of the calling thread.
+ */
+#ifndef RETENTION_B200_H_
+#define RETENTION_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RET_OK = 0,
+    RET_ERR_INVALID_ARG = 1,
+    RET_ERR_UNSUPPORTED = 2,
+    RET_ERR_CUDA = 3,
+    RET_ERR_TIMEOUT = 4
+} ret_status;
+
+typedef enum { RET_F32 = 0, RET_BF16 = 1 } ret_dtype;
+
+/*
+ * xPos / rotary rotation of x [B, N, H, d], in place.
+ * "Hybrid Architectures ...", sections 6.6 and 6.8: pair (2p, 2p+1) of the
+ * vector at position n = pos_offset + t is turned by the angle n * theta_p,
+ *     [x0', x1'] = [x0 cos - x1 sin, x0 sin + x1 cos],
+ *     theta_p = theta_base^(-2p/d).
+ * Queries and keys are both turned this way; their dot product then depends
+ * only on the position difference (section 6.7).
+ * x: device, dtype dt, 4-byte aligned.  d even, all sizes >= 1, theta_base > 0.
+ */
+ret_status ret_xpos_rotate(void* x, ret_dtype dt, int B, int N, int H, int d,
+                           int64_t pos_offset, double theta_base, cudaStream_t stream);
+
+/*
+ * Chunkwise recurrent retention forward.
+ * "Hybrid Architectures ...", section 7.2, and the RetNet paper summary,
+ * Eq. 7: per chunk [i] of `chunk` tokens,
+ *     out_[i] = (Q_[i] K_[i]^T (.) D) V_[i] + (Q_[i] R_{i-1}) (.) xi,
+ *     R_i     = gamma^chunk R_{i-1} + K_[i]^T (V_[i] (.) zeta),
+ * xi_j = gamma^(j+1), zeta_j = gamma^(chunk-1-j) (0-based row j), R_0 = 0.
+ * A last chunk of L < chunk tokens uses L in place of chunk.
+ * q, k, v: device, dtype in_dt, 16-byte aligned, layouts above.
+ * out: device [B, N, H, dv], dtype out_dt, 16-byte aligned; must not overlap
+ *      q, k or v.
+ * final_state: device fp32 [B, H, dk, dv] receiving R after the last token,
+ *      or NULL.
+ * xpos != 0 applies the rotation of ret_xpos_rotate (positions pos_offset + n,
+ *      base theta_base) to q and k as they are loaded; the inputs are not
+ *      modified.
+ * Supported: in_dt RET_F32 (CUDA cores) for chunk * (2 dk + dv_tile + chunk)
+ * and dk * dv_tile small enough for shared memory; in_dt RET_BF16 through the
+ * tensor-core kernel for dk in {64, 128, 256}, dv a multiple of 64,
+ * chunk in {64, 128} and every gamma_h with gamma_h^chunk >= 2^-60, else
+ * through the CUDA-core kernel when it fits.  Other shapes: RET_ERR_UNSUPPORTED.
+ */
+ret_status ret_forward_chunkwise(const void* q, const void* k, const void* v,
+                                 const double* gammas, int B, int N, int H, int dk, int dv,
+                                 int chunk, void* out, float* final_state, cudaStream_t stream,
+                                 ret_dtype in_dt, ret_dtype out_dt, int xpos,
+                                 int64_t pos_offset, double theta_base);
+
+/*
+ * One recurrent decode step, state updated in place.
+ * "Hybrid Architectures ...", sections 2.1 and 5.2; RetNet paper summary,
+ * recurrent representation and inference protocol:
+ *     S <- gamma_h S + k v^T,   out = q^T S   (read-out after the update).
+ * q, k: device [B, H, dk], v: device [B, H, dv], dtype in_dt.
+ * state: device fp32 [B, H, dk, dv], read and written in place, 16-byte
+ *        aligned, dv a multiple of 4.
+ * out: device [B, H, dv], dtype out_dt.
+ */
+ret_status ret_decode_step(const void* q, const void* k, const void* v, const double* gammas,
+                           float* state, void* out, cudaStream_t stream, int B, int H, int dk,
+                           int dv, ret_dtype in_dt, ret_dtype out_dt);
+
+/*
+ * Parallel form, O(N^2), for cross-checking the chunkwise path on the GPU.
+ * "Hybrid Architectures ...", sections 4.2-4.3; RetNet paper summary, Eq. 5:
+ *     out = (Q K^T (.) D) V,  D_nm = gamma^(n-m) for n >= m, else 0.
+ * Arguments as ret_forward_chunkwise (no chunk, no state).  fp32 arithmetic
+ * on the CUDA cores.  dk <= 256.
+ */
+ret_status ret_forward_parallel(const void* q, const void* k, const void* v,
+                                const double* gammas, int B, int N, int H, int dk, int dv,
+                                void* out, cudaStream_t stream, ret_dtype in_dt, ret_dtype out_dt,
+                                int xpos, int64_t pos_offset, double theta_base);
+
+/*
+ * Recurrent form over a whole sequence, token by token, for cross-checking
+ * the chunkwise path on the GPU ("Hybrid Architectures ...", section 2.1).
+ * Arguments as ret_forward_chunkwise (no chunk).  The state lives in
+ * registers in fp32.  dk <= 256.
+ */
+ret_status ret_forward_recurrent(const void* q, const void* k, const void* v,
+                                 const double* gammas, int B, int N, int H, int dk, int dv,
+                                 void* out, float* final_state, cudaStream_t stream,
+                                 ret_dtype in_dt, ret_dtype out_dt, int xpos,
+                                 int64_t pos_offset, double theta_base);
+
+/*
+ * Synchronises `stream`, then reports (and clears) the device-side error word
+ * that kernels set when a bounded wait gives up.  RET_OK if none was set.
+ */
+ret_status ret_check_device_error(cudaStream_t stream);
+
+/* Description of the calling thread's last failure ("" if none). */
+const char* ret_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RETENTION_B200_H_ */

@@ -1,0 +1,192 @@
+"""Multi-scale retention on B200: Python binding of the C ABI in
+``include/retention.h``.
+
+The functions below carry the C entry points' names and do argument
+marshalling only (torch tensors -> device pointers, sizes, dtypes, the
+current CUDA stream); every step of the computation runs in the CUDA library
+``libretention.so`` built from ``csrc/``.  There is no fallback: importing
+this package fails if the library is missing, and every call raises
+``RetentionError`` when the library returns an error status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "RetentionError", "lib", "ret_xpos_rotate", "ret_forward_chunkwise", "ret_decode_step",
+    "ret_forward_parallel", "ret_forward_recurrent", "ret_check_device_error", "ret_last_error_string",
+    "RET_OK", "RET_ERR_INVALID_ARG", "RET_ERR_UNSUPPORTED", "RET_ERR_CUDA", "RET_ERR_TIMEOUT",
+    "RET_F32", "RET_BF16",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libretention.so")
+
+RET_OK, RET_ERR_INVALID_ARG, RET_ERR_UNSUPPORTED, RET_ERR_CUDA, RET_ERR_TIMEOUT = 0, 1, 2, 3, 4
+RET_F32, RET_BF16 = 0, 1
+_STATUS = {0: "RET_OK", 1: "RET_ERR_INVALID_ARG", 2: "RET_ERR_UNSUPPORTED", 3: "RET_ERR_CUDA",
+           4: "RET_ERR_TIMEOUT"}
+
+
+class RetentionError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def _load_library():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m linear_recurrent_sequence_chunkwise_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, d, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_int64
+    dp = ctypes.POINTER(ctypes.c_double)
+    L.ret_xpos_rotate.argtypes = [vp, i, i, i, i, i, i64, d, vp]
+    L.ret_forward_chunkwise.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d]
+    L.ret_decode_step.argtypes = [vp, vp, vp, dp, vp, vp, vp, i, i, i, i, i, i]
+    L.ret_forward_parallel.argtypes = [vp, vp, vp, dp, i, i, i, i, i, vp, vp, i, i, i, i64, d]
+    L.ret_forward_recurrent.argtypes = [vp, vp, vp, dp, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d]
+    L.ret_check_device_error.argtypes = [vp]
+    L.ret_last_error_string.restype = ctypes.c_char_p
+    L.ret_last_error_string.argtypes = []
+    for name in ("ret_xpos_rotate", "ret_forward_chunkwise", "ret_decode_step", "ret_forward_parallel",
+                 "ret_forward_recurrent", "ret_check_device_error"):
+        getattr(L, name).restype = ctypes.c_int
+    return L
+
+
+lib = _load_library()
+
+
+def ret_last_error_string() -> str:
+    return lib.ret_last_error_string().decode(errors="replace")
+
+
+def _check(status: int):
+    if status != RET_OK:
+        raise RetentionError(status, ret_last_error_string())
+
+
+def _dt(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return RET_F32
+    if t == torch.bfloat16:
+        return RET_BF16
+    raise TypeError(f"unsupported dtype {t}; expected float32 or bfloat16")
+
+
+def _ptr(t: Optional[torch.Tensor], name: str):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _gammas(gammas: Sequence[float], H: int):
+    g = [float(x) for x in gammas]
+    if len(g) != H:
+        raise ValueError(f"gammas has {len(g)} entries, expected H={H}")
+    return (ctypes.c_double * H)(*g)
+
+
+def ret_xpos_rotate(x: torch.Tensor, pos_offset: int = 0, theta_base: float = 10000.0, stream=None) -> torch.Tensor:
+    """Rotate x [B, N, H, d] in place (xPos / rotary, consecutive pairs)."""
+    B, N, H, d = x.shape
+    _check(lib.ret_xpos_rotate(_ptr(x, "x"), _dt(x.dtype), B, N, H, d, int(pos_offset), float(theta_base),
+                               _stream(stream)))
+    return x
+
+
+def _seq_shapes(q, k, v):
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise ValueError("expected q, k [B, N, H, dk] and v [B, N, H, dv]")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k and v must share a dtype")
+    B, N, H, dk = q.shape
+    return B, N, H, dk, v.shape[3]
+
+
+def ret_forward_chunkwise(q, k, v, gammas, chunk: int, out=None, final_state=None, out_dtype=None,
+                          xpos: bool = False, pos_offset: int = 0, theta_base: float = 10000.0,
+                          want_final_state: bool = False, stream=None):
+    """Chunkwise retention forward.  Returns ``out`` [B, N, H, dv], or
+    ``(out, final_state)`` when a final state is requested (passed in or
+    ``want_final_state``)."""
+    B, N, H, dk, dv = _seq_shapes(q, k, v)
+    if out is None:
+        out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
+    if final_state is None and want_final_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    if final_state is not None and final_state.dtype != torch.float32:
+        raise TypeError("final_state must be float32")
+    _check(lib.ret_forward_chunkwise(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N, H, dk,
+                                     dv, int(chunk), _ptr(out, "out"), _ptr(final_state, "final_state"),
+                                     _stream(stream), _dt(q.dtype), _dt(out.dtype), int(bool(xpos)),
+                                     int(pos_offset), float(theta_base)))
+    return (out, final_state) if final_state is not None else out
+
+
+def ret_forward_parallel(q, k, v, gammas, out=None, out_dtype=None, xpos: bool = False, pos_offset: int = 0,
+                         theta_base: float = 10000.0, stream=None):
+    """Parallel form (Q K^T (.) D) V, for cross-checks.  Returns ``out``."""
+    B, N, H, dk, dv = _seq_shapes(q, k, v)
+    if out is None:
+        out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
+    _check(lib.ret_forward_parallel(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N, H, dk,
+                                    dv, _ptr(out, "out"), _stream(stream), _dt(q.dtype), _dt(out.dtype),
+                                    int(bool(xpos)), int(pos_offset), float(theta_base)))
+    return out
+
+
+def ret_forward_recurrent(q, k, v, gammas, out=None, final_state=None, out_dtype=None, xpos: bool = False,
+                          pos_offset: int = 0, theta_base: float = 10000.0, want_final_state: bool = False,
+                          stream=None):
+    """Recurrent form token by token, for cross-checks."""
+    B, N, H, dk, dv = _seq_shapes(q, k, v)
+    if out is None:
+        out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
+    if final_state is None and want_final_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check(lib.ret_forward_recurrent(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N, H, dk,
+                                     dv, _ptr(out, "out"), _ptr(final_state, "final_state"), _stream(stream),
+                                     _dt(q.dtype), _dt(out.dtype), int(bool(xpos)), int(pos_offset),
+                                     float(theta_base)))
+    return (out, final_state) if final_state is not None else out
+
+
+def ret_decode_step(q, k, v, gammas, state, out=None, out_dtype=None, stream=None):
+    """One decode step: state [B, H, dk, dv] fp32 updated in place; returns
+    out [B, H, dv]."""
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("expected q, k [B, H, dk] and v [B, H, dv]")
+    B, H, dk = q.shape
+    dv = v.shape[2]
+    if state.shape != (B, H, dk, dv) or state.dtype != torch.float32:
+        raise ValueError("state must be float32 [B, H, dk, dv]")
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=out_dtype or torch.float32, device=q.device)
+    _check(lib.ret_decode_step(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H),
+                               _ptr(state, "state"), _ptr(out, "out"), _stream(stream), B, H, dk, dv,
+                               _dt(q.dtype), _dt(out.dtype)))
+    return out
+
+
+def ret_check_device_error(stream=None):
+    """Synchronise the stream and raise if a kernel gave up a bounded wait."""
+    _check(lib.ret_check_device_error(_stream(stream)))

@@ -1,0 +1,39 @@
+// kernels.h -- internal launch functions behind the C ABI.  Each returns
+// RET_OK after enqueueing, RET_ERR_UNSUPPORTED if the shape does not fit the
+// kernel (nothing launched), or RET_ERR_CUDA if the launch failed.  Argument
+// validation has already happened in ret_api.cu.
+#pragma once
+
+#include "common.cuh"
+
+namespace ret {
+
+struct RetArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    void* out;
+    float* final_state;  // may be null
+    int B, N, H, dk, dv, chunk;
+    ret_dtype in_dt, out_dt;
+    int xpos;
+    long long pos_offset;
+    double theta_base;
+    HeadConsts hc;
+    double gamma[kMaxHeads];
+};
+
+ret_status launch_xpos_rotate(void* x, ret_dtype dt, int B, int N, int H, int d, long long pos_offset,
+                              double theta_base, cudaStream_t s);
+ret_status launch_chunkwise_simt(const RetArgs& a, cudaStream_t s);
+ret_status launch_chunkwise_tc(const RetArgs& a, cudaStream_t s);
+ret_status launch_parallel_simt(const RetArgs& a, cudaStream_t s);
+ret_status launch_recurrent_simt(const RetArgs& a, cudaStream_t s);
+ret_status launch_decode(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
+                         void* out, int B, int H, int dk, int dv, ret_dtype in_dt, ret_dtype out_dt,
+                         cudaStream_t s);
+
+// Does the tensor-core chunkwise kernel take this problem?
+bool chunkwise_tc_supported(const RetArgs& a);
+
+}  // namespace ret

@@ -1,0 +1,182 @@
+// ret_api.cu -- the C ABI: argument validation, per-head constants and
+// dispatch to the kernels.  Nothing here allocates device memory.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "kernels.h"
+
+namespace ret {
+
+static thread_local char t_err[512] = "";
+
+ret_status fail(ret_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_err, sizeof(t_err), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+ret_status check_launch(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return RET_OK;
+}
+
+bool make_head_consts(const double* gammas, int H, HeadConsts* hc) {
+    if (H < 1 || H > kMaxHeads) return false;
+    for (int h = 0; h < H; h++) hc->log2g[h] = log2(gammas[h]);  // -inf for gamma = 0
+    for (int h = H; h < kMaxHeads; h++) hc->log2g[h] = 0.0;
+    return true;
+}
+
+static bool is_dtype(ret_dtype d) { return d == RET_F32 || d == RET_BF16; }
+static size_t esize(ret_dtype d) { return d == RET_F32 ? 4 : 2; }
+
+static bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    const char* pa = (const char*)a;
+    const char* pb = (const char*)b;
+    return pa < pb + nb && pb < pa + na;
+}
+
+static ret_status check_gammas(const double* gammas, int H, const char* who) {
+    if (!gammas) return fail(RET_ERR_INVALID_ARG, "%s: gammas is NULL", who);
+    if (H < 1 || H > kMaxHeads) return fail(RET_ERR_INVALID_ARG, "%s: H=%d outside [1, %d]", who, H, kMaxHeads);
+    for (int h = 0; h < H; h++)
+        if (!(gammas[h] >= 0.0 && gammas[h] <= 1.0))
+            return fail(RET_ERR_INVALID_ARG, "%s: gammas[%d]=%g outside [0, 1]", who, h, gammas[h]);
+    return RET_OK;
+}
+
+// Shared validation of the sequence-level entry points.
+static ret_status make_args(RetArgs* a, const char* who, const void* q, const void* k, const void* v,
+                            const double* gammas, int B, int N, int H, int dk, int dv, int chunk, void* out,
+                            float* final_state, ret_dtype in_dt, ret_dtype out_dt, int xpos, int64_t pos_offset,
+                            double theta_base) {
+    if (!q || !k || !v || !out) return fail(RET_ERR_INVALID_ARG, "%s: NULL q, k, v or out", who);
+    if (B < 1 || N < 1 || H < 1 || dk < 1 || dv < 1 || chunk < 1)
+        return fail(RET_ERR_INVALID_ARG, "%s: sizes must be >= 1 (B=%d N=%d H=%d dk=%d dv=%d chunk=%d)", who, B,
+                    N, H, dk, dv, chunk);
+    if (!is_dtype(in_dt) || !is_dtype(out_dt)) return fail(RET_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    ret_status st = check_gammas(gammas, H, who);
+    if (st != RET_OK) return st;
+    if (xpos && (dk % 2 != 0)) return fail(RET_ERR_INVALID_ARG, "%s: xpos needs an even dk (got %d)", who, dk);
+    if (xpos && !(theta_base > 0.0 && isfinite(theta_base)))
+        return fail(RET_ERR_INVALID_ARG, "%s: theta_base must be finite and > 0", who);
+    const size_t ntok = (size_t)B * N * H;
+    if (ntok * (size_t)(dk > dv ? dk : dv) > ((size_t)1 << 40))
+        return fail(RET_ERR_INVALID_ARG, "%s: problem too large", who);
+    for (const void* p : {q, k, v, (const void*)out})
+        if (!aligned(p, 16)) return fail(RET_ERR_INVALID_ARG, "%s: device pointers must be 16-byte aligned", who);
+    if (final_state && !aligned(final_state, 16))
+        return fail(RET_ERR_INVALID_ARG, "%s: final_state must be 16-byte aligned", who);
+    const size_t bq = ntok * dk * esize(in_dt), bv = ntok * dv * esize(in_dt), bo = ntok * dv * esize(out_dt);
+    if (overlaps(out, bo, q, bq) || overlaps(out, bo, k, bq) || overlaps(out, bo, v, bv))
+        return fail(RET_ERR_INVALID_ARG, "%s: out overlaps q, k or v", who);
+    if (final_state) {
+        const size_t bs = (size_t)B * H * dk * dv * 4;
+        if (overlaps(final_state, bs, out, bo) || overlaps(final_state, bs, q, bq) ||
+            overlaps(final_state, bs, k, bq) || overlaps(final_state, bs, v, bv))
+            return fail(RET_ERR_INVALID_ARG, "%s: final_state overlaps another buffer", who);
+    }
+    a->q = q; a->k = k; a->v = v; a->out = out; a->final_state = final_state;
+    a->B = B; a->N = N; a->H = H; a->dk = dk; a->dv = dv; a->chunk = chunk;
+    a->in_dt = in_dt; a->out_dt = out_dt;
+    a->xpos = xpos ? 1 : 0; a->pos_offset = pos_offset; a->theta_base = xpos ? theta_base : 10000.0;
+    make_head_consts(gammas, H, &a->hc);
+    for (int h = 0; h < kMaxHeads; h++) a->gamma[h] = h < H ? gammas[h] : 0.0;
+    return RET_OK;
+}
+
+}  // namespace ret
+
+using namespace ret;
+
+extern "C" {
+
+const char* ret_last_error_string(void) { return t_err; }
+
+ret_status ret_xpos_rotate(void* x, ret_dtype dt, int B, int N, int H, int d, int64_t pos_offset, double theta_base,
+                           cudaStream_t stream) {
+    t_err[0] = 0;
+    if (!x) return fail(RET_ERR_INVALID_ARG, "ret_xpos_rotate: x is NULL");
+    if (!is_dtype(dt)) return fail(RET_ERR_INVALID_ARG, "ret_xpos_rotate: unknown dtype");
+    if (B < 1 || N < 1 || H < 1 || d < 2 || d % 2)
+        return fail(RET_ERR_INVALID_ARG, "ret_xpos_rotate: sizes must be >= 1 and d even >= 2");
+    if (!(theta_base > 0.0 && isfinite(theta_base)))
+        return fail(RET_ERR_INVALID_ARG, "ret_xpos_rotate: theta_base must be finite and > 0");
+    if (!aligned(x, 4)) return fail(RET_ERR_INVALID_ARG, "ret_xpos_rotate: x must be 4-byte aligned");
+    return launch_xpos_rotate(x, dt, B, N, H, d, pos_offset, theta_base, stream);
+}
+
+ret_status ret_forward_chunkwise(const void* q, const void* k, const void* v, const double* gammas, int B, int N,
+                                 int H, int dk, int dv, int chunk, void* out, float* final_state,
+                                 cudaStream_t stream, ret_dtype in_dt, ret_dtype out_dt, int xpos,
+                                 int64_t pos_offset, double theta_base) {
+    t_err[0] = 0;
+    RetArgs a;
+    ret_status st = make_args(&a, "ret_forward_chunkwise", q, k, v, gammas, B, N, H, dk, dv, chunk, out,
+                              final_state, in_dt, out_dt, xpos, pos_offset, theta_base);
+    if (st != RET_OK) return st;
+    if (in_dt == RET_BF16 && chunkwise_tc_supported(a)) return launch_chunkwise_tc(a, stream);
+    return launch_chunkwise_simt(a, stream);
+}
+
+ret_status ret_forward_parallel(const void* q, const void* k, const void* v, const double* gammas, int B, int N,
+                                int H, int dk, int dv, void* out, cudaStream_t stream, ret_dtype in_dt,
+                                ret_dtype out_dt, int xpos, int64_t pos_offset, double theta_base) {
+    t_err[0] = 0;
+    RetArgs a;
+    ret_status st = make_args(&a, "ret_forward_parallel", q, k, v, gammas, B, N, H, dk, dv, 1, out, nullptr,
+                              in_dt, out_dt, xpos, pos_offset, theta_base);
+    if (st != RET_OK) return st;
+    return launch_parallel_simt(a, stream);
+}
+
+ret_status ret_forward_recurrent(const void* q, const void* k, const void* v, const double* gammas, int B, int N,
+                                 int H, int dk, int dv, void* out, float* final_state, cudaStream_t stream,
+                                 ret_dtype in_dt, ret_dtype out_dt, int xpos, int64_t pos_offset,
+                                 double theta_base) {
+    t_err[0] = 0;
+    RetArgs a;
+    ret_status st = make_args(&a, "ret_forward_recurrent", q, k, v, gammas, B, N, H, dk, dv, 1, out,
+                              final_state, in_dt, out_dt, xpos, pos_offset, theta_base);
+    if (st != RET_OK) return st;
+    return launch_recurrent_simt(a, stream);
+}
+
+ret_status ret_decode_step(const void* q, const void* k, const void* v, const double* gammas, float* state,
+                           void* out, cudaStream_t stream, int B, int H, int dk, int dv, ret_dtype in_dt,
+                           ret_dtype out_dt) {
+    t_err[0] = 0;
+    const char* who = "ret_decode_step";
+    if (!q || !k || !v || !state || !out) return fail(RET_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
+    if (B < 1 || H < 1 || dk < 1 || dv < 1)
+        return fail(RET_ERR_INVALID_ARG, "%s: sizes must be >= 1 (B=%d H=%d dk=%d dv=%d)", who, B, H, dk, dv);
+    if (!is_dtype(in_dt) || !is_dtype(out_dt)) return fail(RET_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    ret_status st = check_gammas(gammas, H, who);
+    if (st != RET_OK) return st;
+    if (dv % 4 != 0) return fail(RET_ERR_INVALID_ARG, "%s: dv must be a multiple of 4 (got %d)", who, dv);
+    if (!aligned(state, 16)) return fail(RET_ERR_INVALID_ARG, "%s: state must be 16-byte aligned", who);
+    for (const void* p : {q, k, v, (const void*)out})
+        if (!aligned(p, 4)) return fail(RET_ERR_INVALID_ARG, "%s: q, k, v, out must be 4-byte aligned", who);
+    const size_t bs = (size_t)B * H * dk * dv * 4, bo = (size_t)B * H * dv * esize(out_dt);
+    if (overlaps(out, bo, state, bs)) return fail(RET_ERR_INVALID_ARG, "%s: out overlaps state", who);
+    HeadConsts hc;
+    make_head_consts(gammas, H, &hc);
+    return launch_decode(q, k, v, hc, state, out, B, H, dk, dv, in_dt, out_dt, stream);
+}
+
+ret_status ret_check_device_error(cudaStream_t stream) {
+    t_err[0] = 0;
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "ret_check_device_error: %s", cudaGetErrorString(e));
+    int flag = 0;
+    e = read_clear_error_chunk_tc(&flag);
+    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "ret_check_device_error: %s", cudaGetErrorString(e));
+    if (flag) return fail(RET_ERR_TIMEOUT, "a kernel gave up a bounded wait (device error word %d)", flag);
+    return RET_OK;
+}
+
+}  // extern "C"

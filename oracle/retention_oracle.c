@@ -118,13 +118,11 @@ void orc_retention_recurrent(const double *q, const double *k, const double *v,
             for (int i = 0; i < dk; i++)
                 for (int j = 0; j < dv; j++)
                     S[(size_t)i * dv + j] = gamma * S[(size_t)i * dv + j] + kn[i] * vn[j];
-            /* o_n = q_n^T S_n */
+            /* o_n = q_n^T S_n  (for each j the sum runs over i = 0..dk-1 in order) */
             double *on = out + IDX4(b, n, h, 0, N, H, dv);
-            for (int j = 0; j < dv; j++) {
-                double acc = 0.0;
-                for (int i = 0; i < dk; i++) acc += qn[i] * S[(size_t)i * dv + j];
-                on[j] = acc;
-            }
+            for (int j = 0; j < dv; j++) on[j] = 0.0;
+            for (int i = 0; i < dk; i++)
+                for (int j = 0; j < dv; j++) on[j] += qn[i] * S[(size_t)i * dv + j];
         }
         if (final_state) memcpy(final_state + (size_t)bh * dk * dv, S, (size_t)dk * dv * sizeof(double));
         free(S);
@@ -247,10 +245,9 @@ void orc_decode_step(const double *q, const double *k, const double *v,
         for (int i = 0; i < dk; i++)
             for (int j = 0; j < dv; j++)
                 S[(size_t)i * dv + j] = gamma * S[(size_t)i * dv + j] + kb[i] * vb[j];
-        for (int j = 0; j < dv; j++) {
-            double acc = 0.0;
-            for (int i = 0; i < dk; i++) acc += qb[i] * S[(size_t)i * dv + j];
-            out[(size_t)bh * dv + j] = acc;
-        }
+        double *ob = out + (size_t)bh * dv;
+        for (int j = 0; j < dv; j++) ob[j] = 0.0;
+        for (int i = 0; i < dk; i++)
+            for (int j = 0; j < dv; j++) ob[j] += qb[i] * S[(size_t)i * dv + j];
     }
 }

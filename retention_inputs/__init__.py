@@ -42,21 +42,39 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
 
 
-@dataclass
 class Tensor:
-    """One synthetic tensor: the stored form and its exact fp64 value."""
-    dtype: str                 # "bf16" or "f32"
-    stored: np.ndarray         # uint16 bits (bf16) or float32
-    f64: np.ndarray            # the stored values widened exactly
+    """One synthetic tensor: its stored form (uint16 bf16 bits or float32)
+    and, on demand, the stored values widened exactly to float64."""
+
+    def __init__(self, dtype: str, stored: np.ndarray):
+        self.dtype = dtype
+        self.stored = stored
+        self._f64 = None
+
+    @property
+    def shape(self):
+        return self.stored.shape
+
+    def f64_at(self, index) -> np.ndarray:
+        """Widened values of ``stored[index]`` (no full-size copy)."""
+        part = self.stored[index]
+        if self.dtype == "bf16":
+            return bf16_bits_to_f32(part).astype(np.float64)
+        return np.asarray(part, dtype=np.float64)
+
+    @property
+    def f64(self) -> np.ndarray:
+        if self._f64 is None:
+            self._f64 = self.f64_at(...)
+        return self._f64
 
 
 def make_tensor(seed: int, stream: int, shape, dtype: str, scale: float = 1.0) -> Tensor:
     x = normal_f32(seed, stream, shape, scale)
     if dtype == "bf16":
-        bits = f32_to_bf16_bits(x)
-        return Tensor("bf16", bits, bf16_bits_to_f32(bits).astype(np.float64))
+        return Tensor("bf16", f32_to_bf16_bits(x))
     if dtype == "f32":
-        return Tensor("f32", x, x.astype(np.float64))
+        return Tensor("f32", x)
     raise ValueError(dtype)
 
 

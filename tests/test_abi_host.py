@@ -1,0 +1,120 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+that include/*.h declares, and rejects bad arguments before launching
+anything.  No GPU work happens here."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+import torch
+
+import linear_recurrent_sequence_chunkwise_b200 as R
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_entry_points():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s+(ret_[a-z_0-9]+)\s*\(", text, flags=re.M))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_entry_points()
+    for must in ("ret_xpos_rotate", "ret_forward_chunkwise", "ret_decode_step", "ret_forward_parallel",
+                 "ret_forward_recurrent", "ret_check_device_error", "ret_last_error_string"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(R.LIB_PATH)
+    missing = [n for n in declared_entry_points() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_library_exports_nothing_undeclared():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", R.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l and l.split()[-1].startswith("ret_")}
+    assert exported == set(declared_entry_points())
+
+
+# Fake, never-dereferenced device addresses.  Every call below fails argument
+# validation before any launch; the cases are skipped on a machine with a GPU
+# so that a validation bug can never turn into a launch on a bogus address.
+needs_no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="fake pointers: host-only checks")
+P = ctypes.c_void_p(0x10000)
+P2 = ctypes.c_void_p(0x20000)
+P3 = ctypes.c_void_p(0x30000)
+P4 = ctypes.c_void_p(0x90000000)
+G2 = (ctypes.c_double * 2)(0.9, 0.99)
+S0 = ctypes.c_void_p(0)
+
+
+def chunk_call(q=P, k=P2, v=P3, g=G2, B=1, N=8, H=2, dk=16, dv=16, chunk=4, out=P4, fs=None, in_dt=1, out_dt=1,
+               xpos=0, theta=10000.0):
+    return R.lib.ret_forward_chunkwise(q, k, v, g, B, N, H, dk, dv, chunk, out, fs, S0, in_dt, out_dt, xpos, 0,
+                                       theta)
+
+
+@needs_no_gpu
+@pytest.mark.parametrize("kw", [
+    dict(q=None), dict(k=None), dict(v=None), dict(out=None), dict(g=None),
+    dict(B=0), dict(N=0), dict(H=0), dict(dk=0), dict(dv=-1), dict(chunk=0),
+    dict(in_dt=7), dict(out_dt=-1),
+    dict(g=(ctypes.c_double * 2)(0.9, 1.5)), dict(g=(ctypes.c_double * 2)(-0.1, 0.5)),
+    dict(g=(ctypes.c_double * 2)(float("nan"), 0.5)),
+    dict(xpos=1, dk=15), dict(xpos=1, theta=0.0), dict(xpos=1, theta=float("inf")),
+    dict(q=ctypes.c_void_p(0x10004)), dict(out=ctypes.c_void_p(0x90000002)),
+    dict(out=ctypes.c_void_p(0x10000)),            # out aliases q
+    dict(fs=ctypes.c_void_p(0x90000008)),          # misaligned state
+    dict(H=200, g=(ctypes.c_double * 200)(*([0.9] * 200))),
+])
+def test_chunkwise_rejects_bad_arguments(kw):
+    st = chunk_call(**kw)
+    assert st == R.RET_ERR_INVALID_ARG, (kw, st, R.ret_last_error_string())
+    assert R.ret_last_error_string()
+
+
+@needs_no_gpu
+@pytest.mark.parametrize("fn", ["ret_forward_parallel", "ret_forward_recurrent"])
+def test_cross_check_paths_reject_bad_arguments(fn):
+    f = getattr(R.lib, fn)
+    if fn == "ret_forward_parallel":
+        st = f(P, P2, P3, G2, 1, 8, 2, 16, 16, None, S0, 1, 1, 0, 0, 1e4)
+    else:
+        st = f(P, P2, P3, G2, 1, 8, 2, 16, 16, None, None, S0, 1, 1, 0, 0, 1e4)
+    assert st == R.RET_ERR_INVALID_ARG
+
+
+@needs_no_gpu
+@pytest.mark.parametrize("args", [
+    (None, P2, P3, G2, P4, P, 1, 2, 16, 16),
+    (P, P2, P3, G2, ctypes.c_void_p(0x90000004), P, 1, 2, 16, 16),   # misaligned state
+    (P, P2, P3, G2, P4, P, 1, 2, 16, 18),                            # dv % 4
+    (P, P2, P3, (ctypes.c_double * 2)(0.9, 2.0), P4, P, 1, 2, 16, 16),
+    (P, P2, P3, G2, P4, P4, 1, 2, 16, 16),                           # out aliases state
+    (P, P2, P3, G2, P4, P, 0, 2, 16, 16),
+])
+def test_decode_rejects_bad_arguments(args):
+    q, k, v, g, state, out, B, H, dk, dv = args
+    st = R.lib.ret_decode_step(q, k, v, g, state, out, S0, B, H, dk, dv, 1, 0)
+    assert st == R.RET_ERR_INVALID_ARG, R.ret_last_error_string()
+
+
+@needs_no_gpu
+def test_rotate_rejects_bad_arguments():
+    assert R.lib.ret_xpos_rotate(None, 1, 1, 4, 2, 8, 0, 1e4, S0) == R.RET_ERR_INVALID_ARG
+    assert R.lib.ret_xpos_rotate(P, 1, 1, 4, 2, 7, 0, 1e4, S0) == R.RET_ERR_INVALID_ARG
+    assert R.lib.ret_xpos_rotate(P, 1, 1, 4, 2, 8, 0, -1.0, S0) == R.RET_ERR_INVALID_ARG
+    assert R.lib.ret_xpos_rotate(P, 9, 1, 4, 2, 8, 0, 1e4, S0) == R.RET_ERR_INVALID_ARG
+
+
+def test_binding_requires_cuda_tensors():
+    q = torch.zeros(1, 4, 1, 8)
+    with pytest.raises(ValueError):
+        R.ret_forward_chunkwise(q, q, q, [0.9], chunk=4, out=torch.zeros(1, 4, 1, 8))

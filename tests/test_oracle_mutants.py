@@ -17,8 +17,8 @@ MUTANTS = {
     "no_decay_in_recurrence": ("S[(size_t)i * dv + j] = gamma * S[(size_t)i * dv + j] + kn[i] * vn[j];",
                                "S[(size_t)i * dv + j] = S[(size_t)i * dv + j] + kn[i] * vn[j];"),
     "transposed_outer_product": ("+ kn[i] * vn[j];", "+ kn[j % dk] * vn[i % dv];"),
-    "readout_wrong_index": ("for (int i = 0; i < dk; i++) acc += qn[i] * S[(size_t)i * dv + j];\n                on[j] = acc;",
-                            "for (int i = 0; i < dk; i++) acc += qn[i] * S[(size_t)j % dk * dv + i % dv];\n                on[j] = acc;"),
+    "readout_wrong_index": ("for (int j = 0; j < dv; j++) on[j] += qn[i] * S[(size_t)i * dv + j];",
+                            "for (int j = 0; j < dv; j++) on[j] += qn[j % dk] * S[(size_t)(i % dv) * dv + (j + i) % dv];"),
     "rotation_sign": ("row[2 * p] = x0 * c - x1 * s;", "row[2 * p] = x0 * c + x1 * s;"),
     "rotation_frequency": ("-2.0 * p / (double)d", "-1.0 * p / (double)d"),
     "parallel_decay_off_by_one": ("orc_gamma_pow(gamma, n - m)", "orc_gamma_pow(gamma, n - m + 1)"),
