@@ -27,7 +27,7 @@ __global__ void __launch_bounds__(256) k_decode_step(const Tin* __restrict__ q, 
     extern __shared__ float smf[];
     float* qs = smf;            // [dk]
     float* ks = smf + dk;       // [dk]
-    float4* red = reinterpret_cast<float4*>(smf + 2 * dk);  // [8][32]
+    float4* red = reinterpret_cast<float4*>(smf + ((2 * dk + 3) & ~3));  // [8][32], 16-byte aligned
     const int bh = blockIdx.y, h = bh % H;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int j = blockIdx.x * kDecCols + lane * 4;
@@ -92,7 +92,7 @@ ret_status launch_decode(const void* q, const void* k, const void* v, const Head
                          void* out, int B, int H, int dk, int dv, ret_dtype in_dt, ret_dtype out_dt,
                          cudaStream_t s) {
     dim3 grid((dv + kDecCols - 1) / kDecCols, B * H);
-    const size_t smem = (size_t)2 * dk * sizeof(float) + kDecWarps * 32 * sizeof(float4);
+    const size_t smem = (size_t)((2 * dk + 3) & ~3) * sizeof(float) + kDecWarps * 32 * sizeof(float4);
     if (smem > 48 * 1024) return fail(RET_ERR_UNSUPPORTED, "ret_decode_step: dk too large");
 #define RET_LAUNCH_DEC(TI, TO)                                                                               \
     k_decode_step<TI, TO><<<grid, 256, smem, s>>>((const TI*)q, (const TI*)k, (const TI*)v, hc, H, dk, dv, \
