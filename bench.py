@@ -1,0 +1,409 @@
+#!/usr/bin/env python
+"""Throughput of the chunkwise retention forward on B200 (one JSON line).
+
+Step: one chunkwise retention forward (xPos rotation fused, fp32 inter-chunk
+state, final state written) over the long-sequence workload
+B=1, N=8192, H=16, d_k=256, d_v=512, chunk 128, bf16 in / bf16 out, through
+the C ABI (ret_forward_chunkwise).  value = tokens/s of the whole job
+(B*N per step per rank, summed over ranks; weak scaling, one replica per
+GPU, no collective on the data path).  The decode step (64 sequences x 16
+heads of 256x512 fp32 state) is timed in the same run and reported under
+"decode" in state GB/s.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the fp64 CPU oracle (the correctness reference) on
+bounded samples of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(workload="retention_bf16_1x8192x16x256x512", B=1, N=8192, H=16, dk=256, dv=512, chunk=128)
+DECODE = dict(workload="decode_bf16_64x16x256x512", B=64, H=16, dk=256, dv=512, prefill=1024, chunk=128)
+METRIC = "chunkwise retention fwd tokens/s"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def gammas(H):
+    return [1.0 - 2.0 ** (-5 - h) for h in range(H)]
+
+
+def flops_per_token_head(chunk, dk, dv):
+    """Algorithmic FLOPs of the chunkwise form per (token, head), full-chunk
+    count: Q K^T (2 C dk) + P V (2 C dv) + cross read-out (2 dk dv) + state
+    update (2 dk dv)."""
+    return 2 * chunk * dk + 2 * chunk * dv + 4 * dk * dv
+
+
+def algo_bytes(w, out_bytes=2):
+    """Read q, k, v once, write out once, write the final fp32 state once."""
+    tok = w["B"] * w["N"] * w["H"]
+    return tok * (2 * w["dk"] * 2 + w["dv"] * 2 + w["dv"] * out_bytes) + w["B"] * w["H"] * w["dk"] * w["dv"] * 4
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def load_traffic(kernel):
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f).get(kernel)
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        loaded = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ ours ---
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import linear_recurrent_sequence_chunkwise_b200 as R
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = dict(WORKLOAD)
+    B, N, H, dk, dv, C = w["B"], w["N"], w["H"], w["dk"], w["dv"], w["chunk"]
+    g = gammas(H)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0x5EED0003 + rank)
+    sc = dk ** -0.5
+    q = (torch.randn((B, N, H, dk), generator=gen, device=dev) * sc).to(torch.bfloat16)
+    k = (torch.randn((B, N, H, dk), generator=gen, device=dev) * sc).to(torch.bfloat16)
+    v = torch.randn((B, N, H, dv), generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty((B, N, H, dv), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        R.ret_forward_chunkwise(q, k, v, g, C, out=out, final_state=fs, xpos=True, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    R.ret_check_device_error()
+    torch.cuda.synchronize()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    R.ret_check_device_error()
+    times = [a.elapsed_time(b) for a, b in evs]  # ms, one launch each
+    total_ms = sum(times)
+    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * B * N / (ms_per_step / 1e3)
+
+    peaks = load_peaks()
+    flops = flops_per_token_head(C, dk, dv) * B * N * H
+    nbytes = algo_bytes(w, out_bytes=2)
+    t_s = statistics.mean(times) / 1e3
+    tflops = flops / t_s / 1e12
+    gbs = nbytes / t_s / 1e9
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    traffic = load_traffic("k_chunkwise_tc")
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    else:
+        roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(tflops / peaks["bf16_tflops"], 4)}
+    roof["traffic"] = traffic["bytes_per_launch"] if traffic else None
+    roof["peak_source"] = peaks["source"]
+    roof["kernel"] = "k_chunkwise_tc"
+    roof["algo_flops"] = flops
+    roof["algo_bytes"] = nbytes
+    roof["tensor_tflops"] = round(tflops, 1)
+    roof["tensor_frac"] = round(tflops / peaks["bf16_tflops"], 4)
+    roof["hbm_gbs"] = round(gbs, 1)
+    roof["hbm_frac"] = round(gbs / peaks["hbm_gbs"], 4)
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1); q, k scaled by d_k^-0.5)",
+        "config": {"workload": w["workload"], "B": B, "N": N, "H": H, "dk": dk, "dv": dv, "chunk": C, "xpos": True,
+                   "out_dtype": "bf16", "final_state": True, "global_batch": B * world, "seq_len": N,
+                   "parallelism": f"replicas x{world}", "l2": "flushed before every timed step (256 MiB write)"},
+        "roofline": roof, "clocks": clk.summary(), "gpu_launches": args.steps,
+    }
+    if not args.no_e2e:
+        result["e2e"] = e2e_ours(R, torch, dev, stream, w, g, args, world, barrier, dist)
+    if not args.no_decode:
+        result["decode"] = bench_decode(R, torch, dev, stream, args, peaks, world, barrier, dist, rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e_ours(R, torch, dev, stream, w, g, args, world, barrier, dist):
+    """Same metric through the C ABI from pinned host buffers: every step
+    copies q, k, v host->device, runs the forward, copies out device->host."""
+    B, N, H, dk, dv, C = w["B"], w["N"], w["H"], w["dk"], w["dv"], w["chunk"]
+    hq = torch.empty((B, N, H, dk), dtype=torch.bfloat16, pin_memory=True).normal_().mul_(dk ** -0.5)
+    hk = torch.empty((B, N, H, dk), dtype=torch.bfloat16, pin_memory=True).normal_().mul_(dk ** -0.5)
+    hv = torch.empty((B, N, H, dv), dtype=torch.bfloat16, pin_memory=True).normal_()
+    ho = torch.empty((B, N, H, dv), dtype=torch.bfloat16, pin_memory=True)
+    dq, dk_, dv_ = (torch.empty_like(x, device=dev) for x in (hq, hk, hv))
+    do = torch.empty((B, N, H, dv), dtype=torch.bfloat16, device=dev)
+    steps = max(3, min(args.steps, 10))
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk_.copy_(hk, non_blocking=True)
+        dv_.copy_(hv, non_blocking=True)
+        R.ret_forward_chunkwise(dq, dk_, dv_, g, C, out=do, xpos=True, stream=stream)
+        ho.copy_(do, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item()) / steps
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+    return {"value": round(world * B * N / (ms / 1e3), 1), "unit": UNIT, "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho.numel() * ho.element_size(), "steps": steps}
+
+
+def bench_decode(R, torch, dev, stream, args, peaks, world, barrier, dist, rank):
+    """Decode step on 64 sequences x 16 heads of 256x512 fp32 state, the state
+    initialised by a chunkwise prefill of a 1024-token prompt."""
+    d = DECODE
+    B, H, dk, dv = d["B"], d["H"], d["dk"], d["dv"]
+    g = gammas(H)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0x5EED0004 + rank)
+    P = d["prefill"]
+    pq = torch.randn((B, P, H, dk), generator=gen, device=dev).to(torch.bfloat16)
+    pk = torch.randn((B, P, H, dk), generator=gen, device=dev).to(torch.bfloat16)
+    pv = torch.randn((B, P, H, dv), generator=gen, device=dev).to(torch.bfloat16)
+    po = torch.empty((B, P, H, dv), dtype=torch.bfloat16, device=dev)
+    state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    R.ret_forward_chunkwise(pq, pk, pv, g, d["chunk"], out=po, final_state=state, stream=stream)
+    del pq, pk, pv, po
+    pool = 16
+    sq = torch.randn((pool, B, H, dk), generator=gen, device=dev).to(torch.bfloat16)
+    sk = torch.randn((pool, B, H, dk), generator=gen, device=dev).to(torch.bfloat16)
+    sv = torch.randn((pool, B, H, dv), generator=gen, device=dev).to(torch.bfloat16)
+    so = torch.empty((B, H, dv), dtype=torch.float32, device=dev)
+    steps = max(args.steps, 20)
+    for i in range(max(args.warmup, 3)):
+        R.ret_decode_step(sq[i % pool], sk[i % pool], sv[i % pool], g, state, out=so, stream=stream)
+    torch.cuda.synchronize()
+    barrier()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        evs[i][0].record(stream)
+        R.ret_decode_step(sq[i % pool], sk[i % pool], sv[i % pool], g, state, out=so, stream=stream)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    R.ret_check_device_error()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    nbytes = 2 * B * H * dk * dv * 4 + B * H * (2 * dk * 2 + dv * 2 + dv * 4)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": d["workload"], "metric": "decode-step state HBM GB/s", "value": round(gbs * world, 1),
+            "unit": "GB/s", "ms_per_step": round(ms, 4), "steps": steps, "bytes_per_step": nbytes,
+            "tokens_per_s": round(world * B / (ms / 1e3), 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "kernel": "k_decode_step",
+                         "traffic": (load_traffic("k_decode_step") or {}).get("bytes_per_launch")},
+            "l2": "state (537 MB) larger than L2"}
+
+
+# ---------------------------------------------------------- the oracle ---
+
+def oracle_sample(w, heads, n_tok):
+    """One bounded oracle run: ``heads`` heads of the workload over the first
+    ``n_tok`` tokens (rotation + recurrent definition, fp64, all host cores).
+    Returns (seconds, tokens of the full workload this sample stands for)."""
+    import numpy as np
+
+    import oracle
+    rng = np.random.default_rng(1)
+    B, dk, dv = w["B"], w["dk"], w["dv"]
+    q = rng.standard_normal((B, n_tok, heads, dk)) / 16
+    k = rng.standard_normal((B, n_tok, heads, dk)) / 16
+    v = rng.standard_normal((B, n_tok, heads, dv))
+    g = np.array(gammas(w["H"])[:heads])
+    t0 = time.perf_counter()
+    oracle.retention_recurrent(oracle.xpos_rotate(q), oracle.xpos_rotate(k), v, g)
+    dt = time.perf_counter() - t0
+    return dt, B * n_tok * heads / w["H"]
+
+
+def cpu_baseline(w, budget_s=20.0):
+    import oracle
+    cores = oracle.max_threads()
+    heads = min(w["H"], cores)
+    dt, tok = oracle_sample(w, heads, 256)           # calibrate
+    n = int(min(w["N"], max(256, 256 * budget_s / max(dt, 1e-3))))
+    dt, tok = oracle_sample(w, heads, n)
+    return {"value": round(tok / dt, 2), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{heads} of {w['H']} heads x first {n} of {w['N']} tokens, fp64 recurrent definition "
+                      f"with xPos, {dt:.1f} s; value scaled to tokens of the full workload"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    w = dict(WORKLOAD)
+    cores = oracle.max_threads()
+    heads = min(w["H"], cores)
+    n_tok = 512
+    for _ in range(args.warmup):
+        oracle_sample(w, heads, n_tok)
+    times, tok = [], 0
+    for _ in range(args.steps):
+        dt, tok = oracle_sample(w, heads, n_tok)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = tok / (ms / 1e3)
+    sample = (f"{heads} of {w['H']} heads x first {n_tok} of {w['N']} tokens per step, fp64 recurrent "
+              f"definition with xPos; value scaled to tokens of the full workload")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))",
+        "config": {"workload": w["workload"], "B": w["B"], "N": w["N"], "H": w["H"], "dk": w["dk"], "dv": w["dv"],
+                   "chunk": w["chunk"], "xpos": True, "global_batch": w["B"], "seq_len": w["N"],
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -90,11 +90,13 @@ ret_status ret_xpos_rotate(void* x, ret_dtype dt, int B, int N, int H, int d,
  * xpos != 0 applies the rotation of ret_xpos_rotate (positions pos_offset + n,
  *      base theta_base) to q and k as they are loaded; the inputs are not
  *      modified.
- * Supported: in_dt RET_F32 (CUDA cores) for chunk * (2 dk + dv_tile + chunk)
- * and dk * dv_tile small enough for shared memory; in_dt RET_BF16 through the
- * tensor-core kernel for dk in {64, 128, 256}, dv a multiple of 64,
- * chunk in {64, 128} and every gamma_h with gamma_h^chunk >= 2^-60, else
- * through the CUDA-core kernel when it fits.  Other shapes: RET_ERR_UNSUPPORTED.
+ * Kernels: in_dt RET_BF16 with dk in {128, 256}, dv a multiple of 64,
+ * chunk = 128 and every gamma_h^128 >= 2^-60 runs on the tensor cores
+ * (tcgen05/TMEM/TMA).  Otherwise the fp32 CUDA-core chunkwise kernel runs
+ * when its per-block working set (about 4 * chunk * (2 dk + chunk + 64)
+ * + 256 dk bytes) fits in shared memory, and else the token-by-token
+ * recurrent kernel (dk <= 256), which computes the same function.  Larger dk
+ * on neither path: RET_ERR_UNSUPPORTED.
  */
 ret_status ret_forward_chunkwise(const void* q, const void* k, const void* v,
                                  const double* gammas, int B, int N, int H, int dk, int dv,

@@ -120,7 +120,11 @@ ret_status ret_forward_chunkwise(const void* q, const void* k, const void* v, co
                               final_state, in_dt, out_dt, xpos, pos_offset, theta_base);
     if (st != RET_OK) return st;
     if (in_dt == RET_BF16 && chunkwise_tc_supported(a)) return launch_chunkwise_tc(a, stream);
-    return launch_chunkwise_simt(a, stream);
+    st = launch_chunkwise_simt(a, stream);
+    if (st != RET_ERR_UNSUPPORTED) return st;
+    // Same function, token by token: the shape fits neither chunkwise kernel.
+    t_err[0] = 0;
+    return launch_recurrent_simt(a, stream);
 }
 
 ret_status ret_forward_parallel(const void* q, const void* k, const void* v, const double* gammas, int B, int N,
