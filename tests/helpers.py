@@ -50,3 +50,31 @@ def err_out(got, ref):
 def err_state(got, ref):
     """[B, H, dk, dv] states: slices are (b, h)."""
     return max_rel_l2(got, ref, (0, 1))
+
+
+U_BF16 = 2.0 ** -8   # unit roundoff of bf16 (8 significant bits)
+
+
+def bf16_bound_check(got_out, got_state, q_rot, k_rot, v, gammas, ref_out, ref_state, out_is_bf16):
+    """Element-wise rounding bound for small shapes, where a per-slice relative
+    L2 of a handful of values is ill-conditioned (e.g. one token: the output is
+    the scalar q.k times v, and q.k may cancel).
+
+    The tensor-core path rounds to bf16 the rotated q, the zeta-scaled k, the
+    masked scores P and the bf16 copy of the state used for the read-out; every
+    product accumulates in fp32.  To first order each output element therefore
+    differs from the exact result by at most 4u times the same retention
+    evaluated on absolute values,
+        sum_{m<=n} gamma^(n-m) (|q_n| . |k_m|) |v_m|,
+    plus u |out| when the output itself is stored in bf16, and the fp32 state
+    by at most 2u times the absolute-value state.  u = 2^-8."""
+    import oracle
+    aq, ak, av = np.abs(q_rot), np.abs(k_rot), np.abs(v)
+    abs_out, abs_state = oracle.retention_recurrent(aq, ak, av, gammas)
+    bound = 4 * U_BF16 * abs_out + (U_BF16 * np.abs(ref_out) if out_is_bf16 else 0.0) + 1e-30
+    excess = np.abs(np.asarray(got_out, np.float64) - ref_out) - bound
+    assert excess.max() <= 0, f"output outside the bf16 rounding bound by {excess.max():.3e}"
+    if got_state is not None:
+        sb = 2 * U_BF16 * abs_state + 1e-30
+        sx = np.abs(np.asarray(got_state, np.float64) - ref_state) - sb
+        assert sx.max() <= 0, f"state outside the bf16 rounding bound by {sx.max():.3e}"

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from retention_inputs import C3, C4, C5, gamma_schedule, make_tensor
-from tests.helpers import TOL_BF16, dev, err_out, err_state, host64, max_rel_l2
+from tests.helpers import TOL_BF16, bf16_bound_check, dev, err_out, err_state, host64, max_rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -30,10 +30,15 @@ def qkv(seed, B, N, H, dk, dv, scale):
             make_tensor(seed, 3, (B, N, H, dv), "bf16"))
 
 
-def ref_of(q, k, v, g, xpos, off=0):
+def rotated(q, k, xpos, off=0):
     qf, kf = q.f64, k.f64
     if xpos:
         qf, kf = oracle.xpos_rotate(qf, off), oracle.xpos_rotate(kf, off)
+    return qf, kf
+
+
+def ref_of(q, k, v, g, xpos, off=0):
+    qf, kf = rotated(q, k, xpos, off)
     return oracle.retention_recurrent(qf, kf, v.f64, g)
 
 
@@ -52,23 +57,28 @@ def test_chunkwise_tc_small(B, N, H, dk, dv, xpos, off, out_dtype):
     out, fs = R.ret_forward_chunkwise(dev(q), dev(k), dev(v), g, 128, out_dtype=out_dtype, xpos=xpos,
                                       pos_offset=off, want_final_state=True)
     R.ret_check_device_error()
-    ref, S = ref_of(q, k, v, g, xpos, off)
-    assert err_out(host64(out), ref) < TOL_BF16
-    assert err_state(host64(fs), S) < TOL_BF16
+    qr, kr = rotated(q, k, xpos, off)
+    ref, S = oracle.retention_recurrent(qr, kr, v.f64, g)
+    # small shapes: element-wise rounding bound; >= 1024 tokens also the relative L2 bar
+    bf16_bound_check(host64(out), host64(fs), qr, kr, v.f64, g, ref, S, out_dtype == torch.bfloat16)
+    if N >= 1024:
+        assert err_out(host64(out), ref) < TOL_BF16
+        assert err_state(host64(fs), S) < TOL_BF16
 
 
-@pytest.mark.parametrize("gam", [1.0, 0.7, 0.5, 0.0])
+@pytest.mark.parametrize("gam", [1.0, 0.75, 0.6, 0.0])
 def test_chunkwise_degenerate_decays(gam):
-    """gamma 1 and 0.7 run on the tensor cores; 0.5 and 0 (gamma^128 below
-    2^-60) take another GPU kernel; all must match the oracle."""
+    """gamma 1 and 0.75 (0.75^128 = 2^-53) run on the tensor cores; 0.6 and 0
+    (gamma^128 below 2^-60) take the recurrent GPU kernel; all must match the
+    oracle."""
     q, k, v = qkv(50, 1, 260, 2, 256, 64, 1 / 16)
     g = np.array([gam, 0.99])
     out, fs = R.ret_forward_chunkwise(dev(q), dev(k), dev(v), g, 128, out_dtype=torch.float32, xpos=True,
                                       want_final_state=True)
     R.ret_check_device_error()
-    ref, S = ref_of(q, k, v, g, True)
-    assert err_out(host64(out), ref) < TOL_BF16
-    assert err_state(host64(fs), S) < TOL_BF16
+    qr, kr = rotated(q, k, True)
+    ref, S = oracle.retention_recurrent(qr, kr, v.f64, g)
+    bf16_bound_check(host64(out), host64(fs), qr, kr, v.f64, g, ref, S, False)
 
 
 def test_long_sequence_workload_all_heads():
