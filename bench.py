@@ -144,8 +144,18 @@ def run_ours(args):
             dist.barrier()
 
     w = dict(WORKLOAD)
+    if args.seq != w["N"]:
+        w["N"] = args.seq
+        w["workload"] = f"retention_bf16_1x{args.seq}x16x256x512"
     B, N, H, dk, dv, C = w["B"], w["N"], w["H"], w["dk"], w["dv"], w["chunk"]
     g = gammas(H)
+    if args.no_chunkwise:
+        peaks = load_peaks()
+        res = {"decode": bench_decode(R, torch, dev, torch.cuda.current_stream(), args, peaks, world, barrier, dist,
+                                      rank)}
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return
     gen = torch.Generator(device=dev)
     gen.manual_seed(0x5EED0003 + rank)
     sc = dk ** -0.5
@@ -396,6 +406,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--seq", type=int, default=WORKLOAD["N"],
+                    help="sequence length of the chunkwise workload (smaller values make ncu captures short)")
+    ap.add_argument("--no-chunkwise", action="store_true", help="skip the chunkwise forward (decode only)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
