@@ -105,6 +105,29 @@ ret_status ret_forward_chunkwise(const void* q, const void* k, const void* v,
                                  int64_t pos_offset, double theta_base);
 
 /*
+ * Chunkwise forward with a caller-provided device workspace: the same
+ * computation and arguments as ret_forward_chunkwise, plus `workspace`
+ * (device, 256-byte aligned, not overlapping any other buffer) of at least
+ * ret_chunkwise_workspace_bytes(...) bytes.  The workspace receives, in one
+ * bandwidth-bound pass, the rotated queries (when xpos != 0) and the rotated
+ * keys scaled by zeta = gamma^(chunk-1-j) (the decay of section 7.2 folded
+ * into the keys), so that the tensor-core kernel that follows runs TMA ->
+ * tcgen05 with no per-element work on q and k.  Its contents are scratch and
+ * undefined after the call.  When the problem does not take this path
+ * (ret_chunkwise_workspace_bytes returns 0, or some gamma_h^chunk < 2^-60)
+ * the call behaves as ret_forward_chunkwise and does not touch the workspace.
+ */
+size_t ret_chunkwise_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk, ret_dtype in_dt,
+                                     int xpos);
+
+ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
+                                    const double* gammas, int B, int N, int H, int dk, int dv,
+                                    int chunk, void* out, float* final_state, cudaStream_t stream,
+                                    ret_dtype in_dt, ret_dtype out_dt, int xpos,
+                                    int64_t pos_offset, double theta_base, void* workspace,
+                                    size_t workspace_bytes);
+
+/*
  * One recurrent decode step, state updated in place.
  * "Hybrid Architectures ...", sections 2.1 and 5.2; RetNet paper summary,
  * recurrent representation and inference protocol:

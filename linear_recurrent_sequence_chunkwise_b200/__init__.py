@@ -17,7 +17,8 @@ from typing import Optional, Sequence
 import torch
 
 __all__ = [
-    "RetentionError", "lib", "ret_xpos_rotate", "ret_forward_chunkwise", "ret_decode_step",
+    "RetentionError", "lib", "ret_xpos_rotate", "ret_forward_chunkwise", "ret_forward_chunkwise_ws",
+    "ret_chunkwise_workspace_bytes", "ret_decode_step",
     "ret_forward_parallel", "ret_forward_recurrent", "ret_check_device_error", "ret_last_error_string",
     "RET_OK", "RET_ERR_INVALID_ARG", "RET_ERR_UNSUPPORTED", "RET_ERR_CUDA", "RET_ERR_TIMEOUT",
     "RET_F32", "RET_BF16",
@@ -48,13 +49,18 @@ def _load_library():
     dp = ctypes.POINTER(ctypes.c_double)
     L.ret_xpos_rotate.argtypes = [vp, i, i, i, i, i, i64, d, vp]
     L.ret_forward_chunkwise.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d]
+    L.ret_forward_chunkwise_ws.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d, vp,
+                                           ctypes.c_size_t]
+    L.ret_chunkwise_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+    L.ret_chunkwise_workspace_bytes.restype = ctypes.c_size_t
     L.ret_decode_step.argtypes = [vp, vp, vp, dp, vp, vp, vp, i, i, i, i, i, i]
     L.ret_forward_parallel.argtypes = [vp, vp, vp, dp, i, i, i, i, i, vp, vp, i, i, i, i64, d]
     L.ret_forward_recurrent.argtypes = [vp, vp, vp, dp, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d]
     L.ret_check_device_error.argtypes = [vp]
     L.ret_last_error_string.restype = ctypes.c_char_p
     L.ret_last_error_string.argtypes = []
-    for name in ("ret_xpos_rotate", "ret_forward_chunkwise", "ret_decode_step", "ret_forward_parallel",
+    for name in ("ret_xpos_rotate", "ret_forward_chunkwise", "ret_forward_chunkwise_ws", "ret_decode_step",
+                 "ret_forward_parallel",
                  "ret_forward_recurrent", "ret_check_device_error"):
         getattr(L, name).restype = ctypes.c_int
     return L
@@ -139,6 +145,30 @@ def ret_forward_chunkwise(q, k, v, gammas, chunk: int, out=None, final_state=Non
                                      dv, int(chunk), _ptr(out, "out"), _ptr(final_state, "final_state"),
                                      _stream(stream), _dt(q.dtype), _dt(out.dtype), int(bool(xpos)),
                                      int(pos_offset), float(theta_base)))
+    return (out, final_state) if final_state is not None else out
+
+
+def ret_chunkwise_workspace_bytes(B, N, H, dk, dv, chunk, dtype=torch.bfloat16, xpos: bool = False) -> int:
+    """Workspace bytes ret_forward_chunkwise_ws needs for this shape (0: the
+    shape does not take the workspace path)."""
+    return int(lib.ret_chunkwise_workspace_bytes(B, N, H, dk, dv, int(chunk), _dt(dtype), int(bool(xpos))))
+
+
+def ret_forward_chunkwise_ws(q, k, v, gammas, chunk: int, workspace, out=None, final_state=None, out_dtype=None,
+                             xpos: bool = False, pos_offset: int = 0, theta_base: float = 10000.0,
+                             want_final_state: bool = False, stream=None):
+    """Chunkwise forward with a caller-provided workspace (a CUDA uint8 tensor
+    of at least ret_chunkwise_workspace_bytes bytes)."""
+    B, N, H, dk, dv = _seq_shapes(q, k, v)
+    if out is None:
+        out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
+    if final_state is None and want_final_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib.ret_forward_chunkwise_ws(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N, H, dk,
+                                        dv, int(chunk), _ptr(out, "out"), _ptr(final_state, "final_state"),
+                                        _stream(stream), _dt(q.dtype), _dt(out.dtype), int(bool(xpos)),
+                                        int(pos_offset), float(theta_base), _ptr(workspace, "workspace"), nbytes))
     return (out, final_state) if final_state is not None else out
 
 

@@ -31,6 +31,7 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 // host reader that returns and clears it (cudaSuccess or the CUDA error).
 constexpr int kErrTimeout = 1;
 cudaError_t read_clear_error_chunk_tc(int* flag);
+cudaError_t read_clear_error_chunk_ws(int* flag);
 
 // ---------------------------------------------------------------- device side
 

@@ -1,0 +1,464 @@
+// k_chunk_ws.cu -- chunkwise retention forward with a caller-provided
+// workspace: a bandwidth-bound prep kernel plus a warp-specialized
+// tcgen05 / TMEM / TMA kernel.
+//
+// Same mathematics as k_chunk_tc.cu ("Hybrid Architectures: RetNet and the
+// Three Computation Paradigms", section 7.2; RetNet paper summary, Eq. 7),
+// with the decay folded into a scaled key k'_c = gamma^(L-1-c) k_c (c the row
+// in its chunk of L rows), a pre-scaled state T = gamma^L R and a row scale:
+//     out_r = gamma^(r+1-L) [ sum_{c<=r} (q_r . k'_c) v_c + q_r^T T ],
+//     R     = T + K'^T V.
+//
+// 1. k_prep_qk (HBM-bound, one pass): rotates q and k once per head (xPos,
+//    consecutive pairs, angle (pos_offset + n) theta_p with the sine and
+//    cosine of each (position, pair) evaluated once for all heads), scales
+//    each rotated key row by its zeta, and writes q_rot and k' (bf16) into the
+//    workspace.  Without rotation only k' is written and q is read in place.
+// 2. k_chunkwise_ws: one CTA per (batch, head, 64 value columns), three roles:
+//      warp 0  TMA producer: per chunk, d_k in parts of 128 (Q part + K' part,
+//              64 KB) through a 2-slot ring, and the V tile (2 slots);
+//      warp 1  MMA issuer (one thread):
+//                A[b]  = Q K'^T                      (TMEM, 2 buffers)
+//                O[b]  = Q T  (+)  ... P V           (TMEM, 2 buffers)
+//                R    += K'^T V                      (TMEM, fp32 state)
+//      warps 2-5 (one warpgroup, TMEM lanes 0..127):
+//                mask:     P = tril(A) -> packed bf16 into A[b] (A operand)
+//                state:    T = gamma^L R -> TMEM (fp32) and smem (bf16)
+//                epilogue: out = gamma^(r+1-L) O -> global
+//    so the tensor core runs Q K'^T of chunk j+1 while the warpgroup writes
+//    chunk j's output, and the only serial chain between chunks is
+//    state MMA -> state rescale -> next state MMA.
+#include "kernels.h"
+#include "tc_util.cuh"
+#include "tmap.h"
+
+namespace ret {
+
+static __device__ int g_err_chunk_ws = 0;
+
+cudaError_t read_clear_error_chunk_ws(int* flag) {
+    cudaError_t e = cudaMemcpyFromSymbol(flag, g_err_chunk_ws, sizeof(int));
+    if (e == cudaSuccess && *flag) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_err_chunk_ws, &zero, sizeof(int));
+    }
+    return e;
+}
+
+namespace {
+
+constexpr int kC = 128;           // chunk rows (M of every MMA)
+constexpr int kW = 64;            // d_v columns per CTA
+constexpr int kPartDk = 128;      // d_k rows per pipeline part (one state block)
+constexpr int kPartBytes = 2 * kPartDk * kC * 2;  // Q part + K' part = 64 KB
+constexpr int kVBytes = kC * kW * 2;              // 16 KB
+constexpr int kThreads = 192;
+constexpr uint32_t kColA = 0, kColO = 256, kColS = 384;
+
+// ------------------------------------------------------------------ prep
+
+// One warp per (batch, token); lanes walk groups of 8 d_k elements (4 pairs).
+template <int DK>
+__global__ void __launch_bounds__(256) k_prep_qk(const __nv_bfloat16* __restrict__ q,
+                                                  const __nv_bfloat16* __restrict__ k,
+                                                  __nv_bfloat16* __restrict__ q_rot,
+                                                  __nv_bfloat16* __restrict__ k_out, HeadConsts hc, int B, int N,
+                                                  int H, int chunk, int xpos, long long pos0, double log2base) {
+    const int lane = threadIdx.x & 31;
+    const long long t = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);  // b * N + n
+    if (t >= (long long)B * N) return;
+    const int n = (int)(t % N);
+    const int r = n % chunk;
+    const int L = min(chunk, N - (n - r));
+    constexpr int kGroups = DK / 8;
+    for (int g = lane; g < kGroups; g += 32) {
+        float cs[4], sn[4];
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            cs[i] = 1.f;
+            sn[i] = 0.f;
+            if (xpos) {
+                const int p = 4 * g + i;
+                const double theta = exp2(-2.0 * p / DK * log2base);
+                sincosf(rot_angle(pos0 + n, theta), &sn[i], &cs[i]);
+            }
+        }
+        for (int h = 0; h < H; h++) {
+            const size_t e = ((size_t)t * H + h) * DK + 8 * g;
+            const float zeta = (float)exp2((double)(L - 1 - r) * hc.log2g[h]);
+            uint4 kw = *reinterpret_cast<const uint4*>(k + e);
+            uint32_t* kwv = reinterpret_cast<uint32_t*>(&kw);
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const float x0 = tc::bf16lo(kwv[i]), x1 = tc::bf16hi(kwv[i]);
+                const float c = cs[i] * zeta, s = sn[i] * zeta;
+                kwv[i] = tc::pack_bf16x2(x0 * c - x1 * s, x0 * s + x1 * c);
+            }
+            *reinterpret_cast<uint4*>(k_out + e) = kw;
+            if (xpos) {
+                uint4 qw = *reinterpret_cast<const uint4*>(q + e);
+                uint32_t* qwv = reinterpret_cast<uint32_t*>(&qw);
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const float x0 = tc::bf16lo(qwv[i]), x1 = tc::bf16hi(qwv[i]);
+                    qwv[i] = tc::pack_bf16x2(x0 * cs[i] - x1 * sn[i], x0 * sn[i] + x1 * cs[i]);
+                }
+                *reinterpret_cast<uint4*>(q_rot + e) = qw;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------- main kernel
+
+struct WsParams {
+    CUtensorMap tq, tk, tv;
+    void* out;
+    float* fstate;
+    int N, H, dv;
+    HeadConsts hc;
+};
+
+template <int DK>
+struct WsSmem {
+    static constexpr int kParts = DK / kPartDk;
+    static constexpr uint32_t kRing = 0;                         // 2 x 64 KB
+    static constexpr uint32_t kV = kRing + 2 * kPartBytes;       // 2 x 16 KB
+    static constexpr uint32_t kT = kV + 2 * kVBytes;             // DK x 128 B
+    static constexpr uint32_t kEnd = kT + DK * 128;
+    static constexpr uint32_t kBytes = kEnd + 1024;
+};
+
+struct Bars {
+    uint64_t full[2], empty[2], vfull[2], vempty[2], afull[2], pready[2], ofull[2], ofree[2], sdone, tready;
+};
+
+__device__ __forceinline__ void elect_arrive(uint64_t* bar, int lane) {
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(bar);
+}
+
+template <int DK, typename Tout>
+__global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_constant__ WsParams p) {
+    constexpr int kParts = DK / kPartDk;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ Bars bars;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_fail;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int j0 = blockIdx.x * kW, h = blockIdx.y, b = blockIdx.z;
+    const int N = p.N;
+    const int nchunks = (N + kC - 1) / kC;
+    const double lg = p.hc.log2g[h];
+
+    if (tid == 0) {
+        for (int i = 0; i < 2; i++) {
+            tc::mbar_init(&bars.full[i], 1);
+            tc::mbar_init(&bars.empty[i], 1);
+            tc::mbar_init(&bars.vfull[i], 1);
+            tc::mbar_init(&bars.vempty[i], 1);
+            tc::mbar_init(&bars.afull[i], 1);
+            tc::mbar_init(&bars.pready[i], 4);
+            tc::mbar_init(&bars.ofull[i], 1);
+            tc::mbar_init(&bars.ofree[i], 4);
+        }
+        tc::mbar_init(&bars.sdone, 1);
+        tc::mbar_init(&bars.tready, 4);
+        s_fail = 0;
+        tc::fence_barrier_init();
+        tc::prefetch_tmap(&p.tq);
+        tc::prefetch_tmap(&p.tk);
+        tc::prefetch_tmap(&p.tv);
+    }
+    if (warp == 1) tc::tmem_alloc(&s_tmem, 512);
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tb = s_tmem;
+    bool ok = true;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            for (int jc = 0; jc < nchunks && ok; jc++) {
+                const int n0 = jc * kC;
+                for (int part = 0; part < kParts && ok; part++) {
+                    const int g = jc * kParts + part, slot = g & 1;
+                    if (g >= 2) ok = tc::mbar_wait(&bars.empty[slot], ((g >> 1) & 1) ^ 1);
+                    if (!ok) break;
+                    uint8_t* dst = sm + WsSmem<DK>::kRing + slot * kPartBytes;
+                    tc::mbar_arrive_expect_tx(&bars.full[slot], kPartBytes);
+                    for (int s = 0; s < 2; s++) {
+                        const int dk0 = part * kPartDk + 64 * s;
+                        tc::tma_load_4d(dst + s * (kC * 128), &p.tq, &bars.full[slot], dk0, h, n0, b);
+                        tc::tma_load_4d(dst + (2 + s) * (kC * 128), &p.tk, &bars.full[slot], dk0, h, n0, b);
+                    }
+                }
+                const int vs = jc & 1;
+                if (ok && jc >= 2) ok = tc::mbar_wait(&bars.vempty[vs], ((jc >> 1) & 1) ^ 1);
+                if (!ok) break;
+                tc::mbar_arrive_expect_tx(&bars.vfull[vs], kVBytes);
+                tc::tma_load_4d(sm + WsSmem<DK>::kV + vs * kVBytes, &p.tv, &bars.vfull[vs], j0, h, n0, b);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t id_qk = tc::idesc_bf16_f32(128, 128, 0, 0);
+            const uint32_t id_qt = tc::idesc_bf16_f32(128, kW, 0, 1);
+            const uint32_t id_st = tc::idesc_bf16_f32(128, kW, 1, 1);
+            const uint32_t id_pv = tc::idesc_bf16_f32(128, kW, 0, 1);
+            const uint32_t ring0 = tc::smem_u32(sm + WsSmem<DK>::kRing);
+            const uint32_t v0 = tc::smem_u32(sm + WsSmem<DK>::kV);
+            const uint32_t t0 = tc::smem_u32(sm + WsSmem<DK>::kT);
+            for (int jc = 0; jc < nchunks && ok; jc++) {
+                const int bb = jc & 1;
+                const uint32_t dA = tb + kColA + 128 * bb, dO = tb + kColO + kW * bb;
+                // A[bb] = Q K'^T over all parts
+                for (int part = 0; part < kParts && ok; part++) {
+                    const int g = jc * kParts + part, slot = g & 1;
+                    ok = tc::mbar_wait(&bars.full[slot], (g >> 1) & 1);
+                    if (!ok) break;
+                    tc::tc_fence_after();
+                    const uint32_t qb = ring0 + slot * kPartBytes, kb = qb + 2 * (kC * 128);
+                    for (int k = 0; k < kPartDk / 16; k++) {
+                        const uint32_t off = (k / 4) * (kC * 128) + (k % 4) * 32;
+                        tc::mma_bf16_ss(dA, tc::sdesc_sw128(qb + off, 16, 1024), tc::sdesc_sw128(kb + off, 16, 1024),
+                                        id_qk, (part > 0) || (k > 0));
+                    }
+                }
+                if (!ok) break;
+                tc::mma_commit(&bars.afull[bb]);
+                // cross read-out and state update need T (rescale of chunk jc-1),
+                // a free O[bb] and this chunk's V
+                if (jc > 0) ok = tc::mbar_wait(&bars.tready, (jc - 1) & 1);
+                if (ok && jc >= 2) ok = tc::mbar_wait(&bars.ofree[bb], ((jc >> 1) & 1) ^ 1);
+                if (ok) ok = tc::mbar_wait(&bars.vfull[bb], (jc >> 1) & 1);
+                if (!ok) break;
+                tc::tc_fence_after();
+                const uint32_t vb = v0 + bb * kVBytes;
+                for (int part = 0; part < kParts; part++) {
+                    const int g = jc * kParts + part, slot = g & 1;
+                    const uint32_t qb = ring0 + slot * kPartBytes, kb = qb + 2 * (kC * 128);
+                    if (jc > 0) {
+                        for (int k = 0; k < kPartDk / 16; k++) {
+                            const uint32_t off = (k / 4) * (kC * 128) + (k % 4) * 32;
+                            tc::mma_bf16_ss(dO, tc::sdesc_sw128(qb + off, 16, 1024),
+                                            tc::sdesc_sw128(t0 + (part * kPartDk + 16 * k) * 128, DK * 128, 1024),
+                                            id_qt, (part > 0) || (k > 0));
+                        }
+                    }
+                    for (int k = 0; k < kC / 16; k++)
+                        tc::mma_bf16_ss(tb + kColS + part * kW, tc::sdesc_sw128(kb + k * 2048, kC * 128, 1024),
+                                        tc::sdesc_sw128(vb + k * 2048, kC * 128, 1024), id_st, (jc > 0) || (k > 0));
+                    tc::mma_commit(&bars.empty[slot]);
+                }
+                tc::mma_commit(&bars.sdone);
+                // O[bb] += P V
+                ok = tc::mbar_wait(&bars.pready[bb], (jc >> 1) & 1);
+                if (!ok) break;
+                tc::tc_fence_after();
+                for (int k = 0; k < kC / 16; k++)
+                    tc::mma_bf16_ts(dO, dA + 8 * k, tc::sdesc_sw128(vb + k * 2048, kC * 128, 1024), id_pv,
+                                    (jc > 0) || (k > 0));
+                tc::mma_commit(&bars.ofull[bb]);
+                tc::mma_commit(&bars.vempty[bb]);
+            }
+        }
+    } else {
+        // ------------------------------------------- transform warpgroup
+        const int quarter = warp & 3;                 // TMEM lanes 32*quarter ..
+        const int r = quarter * 32 + lane;            // chunk row / state row in a block
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        uint8_t* sT = sm + WsSmem<DK>::kT;
+        for (int jc = 0; jc < nchunks && ok; jc++) {
+            const int bb = jc & 1;
+            const int n0 = jc * kC, L = min(kC, N - n0);
+            const bool last = (jc == nchunks - 1);
+            // ---- mask: P = tril(A) as packed bf16 into A[bb] columns [0, 64)
+            ok = tc::mbar_wait(&bars.afull[bb], (jc >> 1) & 1);
+            if (!ok) break;
+            tc::tc_fence_after();
+            {
+                const uint32_t a_addr = tb + lane_off + kColA + 128 * bb;
+                uint32_t a[4][32];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; q4++) tc::tmem_ld32(a_addr + 32 * q4, a[q4]);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int half = 0; half < 2; half++) {
+                    uint32_t w[32];
+#pragma unroll
+                    for (int i = 0; i < 32; i++) {
+                        const int c = 64 * half + 2 * i;
+                        const float lo = (c <= r) ? __uint_as_float(a[2 * half + (i >> 4)][(2 * i) & 31]) : 0.f;
+                        const float hi = (c + 1 <= r) ? __uint_as_float(a[2 * half + (i >> 4)][(2 * i + 1) & 31]) : 0.f;
+                        w[i] = tc::pack_bf16x2(lo, hi);
+                    }
+                    tc::tmem_st32(a_addr + 32 * half, w);
+                }
+                tc::tmem_st_wait();
+            }
+            tc::tc_fence_before();
+            elect_arrive(&bars.pready[bb], lane);
+            // ---- state: T = gamma^L_next R (TMEM fp32 and shared bf16), or the final state
+            ok = tc::mbar_wait(&bars.sdone, jc & 1);
+            if (!ok) break;
+            tc::tc_fence_after();
+            {
+                const float gL = last ? 1.f : (float)exp2((double)min(kC, N - (n0 + kC)) * lg);
+#pragma unroll
+                for (int part = 0; part < kParts; part++) {
+                    const uint32_t s_addr = tb + lane_off + kColS + part * kW;
+                    const int d = part * kPartDk + r;
+                    uint32_t s[2][32];
+                    tc::tmem_ld32(s_addr, s[0]);
+                    tc::tmem_ld32(s_addr + 32, s[1]);
+                    tc::tmem_ld_wait();
+                    if (!last) {
+#pragma unroll
+                        for (int hh = 0; hh < 2; hh++)
+#pragma unroll
+                            for (int i = 0; i < 32; i++) s[hh][i] = __float_as_uint(__uint_as_float(s[hh][i]) * gL);
+                        tc::tmem_st32(s_addr, s[0]);
+                        tc::tmem_st32(s_addr + 32, s[1]);
+#pragma unroll
+                        for (int c16 = 0; c16 < 8; c16++) {
+                            const int hh = c16 >> 2, base = (c16 & 3) * 8;
+                            uint4 v;
+                            v.x = tc::pack_bf16x2(__uint_as_float(s[hh][base + 0]), __uint_as_float(s[hh][base + 1]));
+                            v.y = tc::pack_bf16x2(__uint_as_float(s[hh][base + 2]), __uint_as_float(s[hh][base + 3]));
+                            v.z = tc::pack_bf16x2(__uint_as_float(s[hh][base + 4]), __uint_as_float(s[hh][base + 5]));
+                            v.w = tc::pack_bf16x2(__uint_as_float(s[hh][base + 6]), __uint_as_float(s[hh][base + 7]));
+                            *reinterpret_cast<uint4*>(sT + tc::sw128_off((uint32_t)d, (uint32_t)c16)) = v;
+                        }
+                    } else if (p.fstate) {
+                        float4* dst = reinterpret_cast<float4*>(p.fstate + (((size_t)b * p.H + h) * DK + d) * p.dv + j0);
+#pragma unroll
+                        for (int c4 = 0; c4 < 16; c4++) {
+                            const int hh = c4 >> 3, base = (c4 & 7) * 4;
+                            dst[c4] = make_float4(__uint_as_float(s[hh][base]), __uint_as_float(s[hh][base + 1]),
+                                                  __uint_as_float(s[hh][base + 2]), __uint_as_float(s[hh][base + 3]));
+                        }
+                    }
+                }
+                if (!last) tc::tmem_st_wait();
+            }
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
+            elect_arrive(&bars.tready, lane);
+            // ---- epilogue: out = gamma^(r+1-L) O
+            ok = tc::mbar_wait(&bars.ofull[bb], (jc >> 1) & 1);
+            if (!ok) break;
+            tc::tc_fence_after();
+            {
+                uint32_t o[2][32];
+                const uint32_t o_addr = tb + lane_off + kColO + kW * bb;
+                tc::tmem_ld32(o_addr, o[0]);
+                tc::tmem_ld32(o_addr + 32, o[1]);
+                tc::tmem_ld_wait();
+                tc::tc_fence_before();
+                elect_arrive(&bars.ofree[bb], lane);
+                if (r < L) {
+                    const float sc = (float)exp2((double)(r + 1 - L) * lg);
+                    Tout* dst = reinterpret_cast<Tout*>(p.out) + (((size_t)b * N + n0 + r) * p.H + h) * p.dv + j0;
+                    if constexpr (sizeof(Tout) == 2) {
+#pragma unroll
+                        for (int c16 = 0; c16 < 8; c16++) {
+                            const int hh = c16 >> 2, base = (c16 & 3) * 8;
+                            uint4 v;
+                            v.x = tc::pack_bf16x2(__uint_as_float(o[hh][base + 0]) * sc, __uint_as_float(o[hh][base + 1]) * sc);
+                            v.y = tc::pack_bf16x2(__uint_as_float(o[hh][base + 2]) * sc, __uint_as_float(o[hh][base + 3]) * sc);
+                            v.z = tc::pack_bf16x2(__uint_as_float(o[hh][base + 4]) * sc, __uint_as_float(o[hh][base + 5]) * sc);
+                            v.w = tc::pack_bf16x2(__uint_as_float(o[hh][base + 6]) * sc, __uint_as_float(o[hh][base + 7]) * sc);
+                            reinterpret_cast<uint4*>(dst)[c16] = v;
+                        }
+                    } else {
+#pragma unroll
+                        for (int c4 = 0; c4 < 16; c4++) {
+                            const int hh = c4 >> 3, base = (c4 & 7) * 4;
+                            reinterpret_cast<float4*>(dst)[c4] =
+                                make_float4(__uint_as_float(o[hh][base + 0]) * sc, __uint_as_float(o[hh][base + 1]) * sc,
+                                            __uint_as_float(o[hh][base + 2]) * sc, __uint_as_float(o[hh][base + 3]) * sc);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    if (!ok) atomicExch(&s_fail, 1);
+    tc::tc_fence_before();
+    __syncthreads();
+    if (s_fail && tid == 0) atomicExch(&g_err_chunk_ws, kErrTimeout);
+    if (warp == 1) tc::tmem_dealloc(tb, 512);
+}
+
+template <int DK, typename Tout>
+ret_status launch_main(const WsParams& p, const RetArgs& a, cudaStream_t s) {
+    auto kern = k_chunkwise_ws<DK, Tout>;
+    const int smem = (int)WsSmem<DK>::kBytes;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return check_launch("chunkwise (workspace path): smem attribute");
+    dim3 grid(a.dv / kW, a.H, a.B);
+    kern<<<grid, kThreads, smem, s>>>(p);
+    return check_launch("chunkwise (workspace path)");
+}
+
+}  // namespace
+
+size_t chunkwise_ws_bytes(const RetArgs& a) {
+    const size_t qk = (size_t)a.B * a.N * a.H * a.dk * 2;
+    return a.xpos ? 2 * qk : qk;
+}
+
+bool chunkwise_ws_supported(const RetArgs& a) {
+    if (a.in_dt != RET_BF16) return false;
+    if (a.chunk != kC || !(a.dk == 128 || a.dk == 256) || a.dv % kW != 0) return false;
+    if (a.N > (1 << 30)) return false;
+    for (int h = 0; h < a.H; h++)
+        if (!(a.hc.log2g[h] * kC >= -60.0)) return false;
+    return true;
+}
+
+ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s) {
+    const size_t qk = (size_t)a.B * a.N * a.H * a.dk;
+    __nv_bfloat16* k_out = reinterpret_cast<__nv_bfloat16*>(ws);
+    __nv_bfloat16* q_rot = a.xpos ? k_out + qk : nullptr;
+    const int blocks = (int)(((long long)a.B * a.N + 7) / 8);
+    const double lb = log2(a.theta_base);
+    if (a.dk == 256)
+        k_prep_qk<256><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, q_rot, k_out,
+                                               a.hc, a.B, a.N, a.H, a.chunk, a.xpos, a.pos_offset, lb);
+    else
+        k_prep_qk<128><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, q_rot, k_out,
+                                               a.hc, a.B, a.N, a.H, a.chunk, a.xpos, a.pos_offset, lb);
+    ret_status st = check_launch("chunkwise (workspace path): prep");
+    if (st != RET_OK) return st;
+
+    WsParams p;
+    const uint64_t B = a.B, N = a.N, H = a.H, dk = a.dk, dv = a.dv;
+    const uint64_t dq[4] = {dk, H, N, B};
+    const uint64_t sq[3] = {dk * 2, H * dk * 2, N * H * dk * 2};
+    const uint32_t box[4] = {64, 1, (uint32_t)kC, 1};
+    const uint64_t dvv[4] = {dv, H, N, B};
+    const uint64_t svv[3] = {dv * 2, H * dv * 2, N * H * dv * 2};
+    const void* qsrc = a.xpos ? (const void*)q_rot : a.q;
+    if (!make_tmap_bf16(&p.tq, qsrc, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_bf16(&p.tk, k_out, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_bf16(&p.tv, a.v, 4, dvv, svv, box, CU_TENSOR_MAP_SWIZZLE_128B))
+        return RET_ERR_CUDA;
+    p.out = a.out;
+    p.fstate = a.final_state;
+    p.N = a.N;
+    p.H = a.H;
+    p.dv = a.dv;
+    p.hc = a.hc;
+    const bool f32 = a.out_dt == RET_F32;
+    if (a.dk == 256) return f32 ? launch_main<256, float>(p, a, s) : launch_main<256, __nv_bfloat16>(p, a, s);
+    return f32 ? launch_main<128, float>(p, a, s) : launch_main<128, __nv_bfloat16>(p, a, s);
+}
+
+}  // namespace ret

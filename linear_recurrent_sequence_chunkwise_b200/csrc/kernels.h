@@ -36,4 +36,10 @@ ret_status launch_decode(const void* q, const void* k, const void* v, const Head
 // Does the tensor-core chunkwise kernel take this problem?
 bool chunkwise_tc_supported(const RetArgs& a);
 
+// Workspace path: prep kernel (rotation + zeta scaling into the workspace)
+// and the warp-specialized tensor-core kernel.
+bool chunkwise_ws_supported(const RetArgs& a);
+size_t chunkwise_ws_bytes(const RetArgs& a);
+ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s);
+
 }  // namespace ret

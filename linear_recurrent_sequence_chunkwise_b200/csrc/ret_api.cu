@@ -127,6 +127,41 @@ ret_status ret_forward_chunkwise(const void* q, const void* k, const void* v, co
     return launch_recurrent_simt(a, stream);
 }
 
+size_t ret_chunkwise_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk, ret_dtype in_dt, int xpos) {
+    if (B < 1 || N < 1 || H < 1 || H > kMaxHeads || dk < 1 || dv < 1 || chunk < 1) return 0;
+    RetArgs a{};
+    a.B = B; a.N = N; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.in_dt = in_dt; a.xpos = xpos ? 1 : 0;
+    for (int h = 0; h < kMaxHeads; h++) a.hc.log2g[h] = 0.0;  // shape check only
+    return chunkwise_ws_supported(a) ? chunkwise_ws_bytes(a) : 0;
+}
+
+ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v, const double* gammas, int B, int N,
+                                    int H, int dk, int dv, int chunk, void* out, float* final_state,
+                                    cudaStream_t stream, ret_dtype in_dt, ret_dtype out_dt, int xpos,
+                                    int64_t pos_offset, double theta_base, void* workspace, size_t workspace_bytes) {
+    t_err[0] = 0;
+    RetArgs a;
+    ret_status st = make_args(&a, "ret_forward_chunkwise_ws", q, k, v, gammas, B, N, H, dk, dv, chunk, out,
+                              final_state, in_dt, out_dt, xpos, pos_offset, theta_base);
+    if (st != RET_OK) return st;
+    if (!chunkwise_ws_supported(a)) return ret_forward_chunkwise(q, k, v, gammas, B, N, H, dk, dv, chunk, out,
+                                                                 final_state, stream, in_dt, out_dt, xpos,
+                                                                 pos_offset, theta_base);
+    const size_t need = chunkwise_ws_bytes(a);
+    if (!workspace || workspace_bytes < need)
+        return fail(RET_ERR_INVALID_ARG, "ret_forward_chunkwise_ws: workspace of %zu bytes needed (got %zu)", need,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (!aligned(workspace, 256))
+        return fail(RET_ERR_INVALID_ARG, "ret_forward_chunkwise_ws: workspace must be 256-byte aligned");
+    const size_t ntok = (size_t)B * N * H;
+    const size_t bq = ntok * dk * 2, bv = ntok * dv * 2, bo = ntok * dv * (out_dt == RET_F32 ? 4 : 2);
+    if (overlaps(workspace, need, q, bq) || overlaps(workspace, need, k, bq) || overlaps(workspace, need, v, bv) ||
+        overlaps(workspace, need, out, bo) ||
+        (final_state && overlaps(workspace, need, final_state, (size_t)B * H * dk * dv * 4)))
+        return fail(RET_ERR_INVALID_ARG, "ret_forward_chunkwise_ws: workspace overlaps another buffer");
+    return launch_chunkwise_ws(a, workspace, stream);
+}
+
 ret_status ret_forward_parallel(const void* q, const void* k, const void* v, const double* gammas, int B, int N,
                                 int H, int dk, int dv, void* out, cudaStream_t stream, ret_dtype in_dt,
                                 ret_dtype out_dt, int xpos, int64_t pos_offset, double theta_base) {
@@ -176,9 +211,11 @@ ret_status ret_check_device_error(cudaStream_t stream) {
     t_err[0] = 0;
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return fail(RET_ERR_CUDA, "ret_check_device_error: %s", cudaGetErrorString(e));
-    int flag = 0;
+    int flag = 0, flag2 = 0;
     e = read_clear_error_chunk_tc(&flag);
+    if (e == cudaSuccess) e = read_clear_error_chunk_ws(&flag2);
     if (e != cudaSuccess) return fail(RET_ERR_CUDA, "ret_check_device_error: %s", cudaGetErrorString(e));
+    flag |= flag2;
     if (flag) return fail(RET_ERR_TIMEOUT, "a kernel gave up a bounded wait (device error word %d)", flag);
     return RET_OK;
 }

@@ -1,0 +1,131 @@
+"""GPU parity of the workspace path of the chunkwise forward (rotation and
+zeta scaling in one bandwidth-bound pass, then the warp-specialized
+tcgen05 kernel) against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from retention_inputs import C3, C4, gamma_schedule, make_tensor
+from tests.helpers import TOL_BF16, bf16_bound_check, dev, err_out, err_state, host64
+
+pytestmark = pytest.mark.gpu
+
+R = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    global R
+    import linear_recurrent_sequence_chunkwise_b200 as mod
+    R = mod
+    yield mod
+    mod.ret_check_device_error()
+
+
+def qkv(seed, B, N, H, dk, dv, scale):
+    return (make_tensor(seed, 1, (B, N, H, dk), "bf16", scale), make_tensor(seed, 2, (B, N, H, dk), "bf16", scale),
+            make_tensor(seed, 3, (B, N, H, dv), "bf16"))
+
+
+def rotated(q, k, xpos, off=0):
+    qf, kf = q.f64, k.f64
+    if xpos:
+        qf, kf = oracle.xpos_rotate(qf, off), oracle.xpos_rotate(kf, off)
+    return qf, kf
+
+
+def run_ws(q, k, v, g, chunk, **kw):
+    B, N, H, dk = q.shape
+    dv = v.shape[3]
+    nb = R.ret_chunkwise_workspace_bytes(B, N, H, dk, dv, chunk, torch.bfloat16, kw.get("xpos", False))
+    assert nb > 0
+    ws = torch.full((nb + 512,), 0xAB, dtype=torch.uint8, device="cuda")[256:256 + nb]
+    assert ws.data_ptr() % 256 == 0
+    return R.ret_forward_chunkwise_ws(dev(q), dev(k), dev(v), g, chunk, ws, **kw)
+
+
+@pytest.mark.parametrize("B,N,H,dk,dv,xpos,off", [
+    (1, 128, 1, 256, 64, True, 0),
+    (2, 300, 2, 256, 128, True, 0),
+    (1, 1, 2, 256, 64, True, 9),
+    (1, 77, 1, 128, 64, False, 0),
+    (2, 513, 3, 128, 192, True, 1000),
+    (1, 640, 2, 256, 512, False, 0),
+    (1, 1024, 2, 256, 512, True, 0),
+])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_chunkwise_ws_small(B, N, H, dk, dv, xpos, off, out_dtype):
+    q, k, v = qkv(70 + N, B, N, H, dk, dv, dk ** -0.5)
+    g = gamma_schedule(H)
+    out, fs = run_ws(q, k, v, g, 128, out_dtype=out_dtype, xpos=xpos, pos_offset=off, want_final_state=True)
+    R.ret_check_device_error()
+    qr, kr = rotated(q, k, xpos, off)
+    ref, S = oracle.retention_recurrent(qr, kr, v.f64, g)
+    bf16_bound_check(host64(out), host64(fs), qr, kr, v.f64, g, ref, S, out_dtype == torch.bfloat16)
+    if N >= 1024:
+        assert err_out(host64(out), ref) < TOL_BF16
+        assert err_state(host64(fs), S) < TOL_BF16
+
+
+@pytest.mark.parametrize("gam", [1.0, 0.75, 0.6])
+def test_chunkwise_ws_decays(gam):
+    q, k, v = qkv(80, 1, 390, 2, 256, 64, 1 / 16)
+    g = np.array([gam, 0.99])
+    out, fs = run_ws(q, k, v, g, 128, out_dtype=torch.float32, xpos=True, want_final_state=True)
+    R.ret_check_device_error()
+    qr, kr = rotated(q, k, True)
+    ref, S = oracle.retention_recurrent(qr, kr, v.f64, g)
+    bf16_bound_check(host64(out), host64(fs), qr, kr, v.f64, g, ref, S, False)
+
+
+def test_ws_long_sequence_workload_all_heads():
+    w = C3
+    q, k, v = w.qkv()
+    qr, kr = rotated(q, k, True)
+    ref, S = oracle.retention_recurrent(qr, kr, v.f64, w.gammas)
+    for odt in (torch.bfloat16, torch.float32):
+        out, fs = run_ws(q, k, v, w.gammas, w.chunk, out_dtype=odt, xpos=True, want_final_state=True)
+        R.ret_check_device_error()
+        assert err_out(host64(out), ref) < TOL_BF16
+        assert err_state(host64(fs), S) < TOL_BF16
+
+
+def test_ws_matches_fused_path():
+    """Workspace path and single-kernel path agree (same arithmetic up to
+    rounding order)."""
+    q, k, v = qkv(81, 2, 700, 3, 256, 128, 1 / 16)
+    g = gamma_schedule(3)
+    a, fa = run_ws(q, k, v, g, 128, out_dtype=torch.float32, xpos=True, want_final_state=True)
+    b, fb = R.ret_forward_chunkwise(dev(q), dev(k), dev(v), g, 128, out_dtype=torch.float32, xpos=True,
+                                    want_final_state=True)
+    torch.cuda.synchronize()
+    assert err_out(host64(a), host64(b)) < 1e-3
+    assert err_state(host64(fa), host64(fb)) < 1e-3
+
+
+def _picked(t, picks):
+    return np.stack([t.f64_at((b, slice(None), h)) for b, h in picks], axis=1)[None]
+
+
+def test_ws_prefill_workload_sampled():
+    w = C4
+    q, k, v = w.qkv()
+    out, fs = run_ws(q, k, v, w.gammas, w.chunk, out_dtype=torch.float32, want_final_state=True)
+    R.ret_check_device_error()
+    picks = [(0, 0), (17, 5), (63, 15), (40, 11)]
+    g = np.array([w.gammas[h] for _, h in picks])
+    ref, S = oracle.retention_recurrent(_picked(q, picks), _picked(k, picks), _picked(v, picks), g)
+    o = out.cpu().numpy()
+    got = np.stack([o[b, :, h] for b, h in picks], axis=1)[None].astype(np.float64)
+    assert err_out(got, ref) < TOL_BF16
+    f = fs.cpu().numpy()
+    assert err_state(np.stack([f[b, h] for b, h in picks])[None].astype(np.float64), S) < TOL_BF16
+
+
+def test_ws_rejects_small_workspace():
+    q, k, v = qkv(82, 1, 256, 1, 256, 64, 1 / 16)
+    nb = R.ret_chunkwise_workspace_bytes(1, 256, 1, 256, 64, 128, torch.bfloat16, True)
+    ws = torch.empty(nb - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(R.RetentionError):
+        R.ret_forward_chunkwise_ws(dev(q), dev(k), dev(v), [0.9], 128, ws, xpos=True)
