@@ -14,19 +14,22 @@
 //    cosine of each (position, pair) evaluated once for all heads), scales
 //    each rotated key row by its zeta, and writes q_rot and k' (bf16) into the
 //    workspace.  Without rotation only k' is written and q is read in place.
-// 2. k_chunkwise_ws: one CTA per (batch, head, 64 value columns), three roles:
-//      warp 0  TMA producer: per chunk, d_k in parts of 128 (Q part + K' part,
-//              64 KB) through a 2-slot ring, and the V tile (2 slots);
-//      warp 1  MMA issuer (one thread):
-//                A[b]  = Q K'^T                      (TMEM, 2 buffers)
-//                O[b]  = Q T  (+)  ... P V           (TMEM, 2 buffers)
-//                R    += K'^T V                      (TMEM, fp32 state)
+// 2. k_chunkwise_ws: one CTA per (batch, head, 64 value columns), three roles
+//      warp 0  TMA producer: per chunk the Q tile into a staging buffer, the
+//              K' tile in parts of 128 d_k rows through a 3-slot ring, and
+//              the V tile (2 slots);
+//      warp 1  MMA issuer (one thread), A operands from TMEM where possible:
+//                A  = Q K'^T          (Q from TMEM, K' from smem)
+//                O  = Q T  + P V      (Q and P from TMEM, T and V from smem)
+//                R += K'^T V          (fp32 state in TMEM)
 //      warps 2-5 (one warpgroup, TMEM lanes 0..127):
-//                mask:     P = tril(A) -> packed bf16 into A[b] (A operand)
-//                state:    T = gamma^L R -> TMEM (fp32) and smem (bf16)
-//                epilogue: out = gamma^(r+1-L) O -> global
-//    so the tensor core runs Q K'^T of chunk j+1 while the warpgroup writes
-//    chunk j's output, and the only serial chain between chunks is
+//                Q staging -> TMEM (frees the 64 KB staging buffer early),
+//                mask:     P = tril(A) -> packed bf16 in TMEM,
+//                state:    T = gamma^L R -> TMEM (fp32) and smem (bf16),
+//                epilogue: out = gamma^(r+1-L) O -> global.
+//    TMEM columns: A [0,128), P [128,192), O [192,256), Q [256,384),
+//    R [384,512).  The tensor core computes Q K'^T of chunk j+1 while the
+//    warpgroup stores chunk j's output; the serial chain between chunks is
 //    state MMA -> state rescale -> next state MMA.
 #include "kernels.h"
 #include "tc_util.cuh"
@@ -50,10 +53,8 @@ namespace {
 constexpr int kC = 128;           // chunk rows (M of every MMA)
 constexpr int kW = 64;            // d_v columns per CTA
 constexpr int kPartDk = 128;      // d_k rows per pipeline part (one state block)
-constexpr int kPartBytes = 2 * kPartDk * kC * 2;  // Q part + K' part = 64 KB
 constexpr int kVBytes = kC * kW * 2;              // 16 KB
 constexpr int kThreads = 192;
-constexpr uint32_t kColA = 0, kColO = 256, kColS = 384;
 
 // ------------------------------------------------------------------ prep
 
@@ -119,18 +120,25 @@ struct WsParams {
     HeadConsts hc;
 };
 
+constexpr int kKSlots = 3;                         // K' ring depth (parts of 128 d_k rows)
+constexpr int kKPartBytes = kPartDk * kC * 2;      // 32 KB
+
 template <int DK>
 struct WsSmem {
-    static constexpr int kParts = DK / kPartDk;
-    static constexpr uint32_t kRing = 0;                         // 2 x 64 KB
-    static constexpr uint32_t kV = kRing + 2 * kPartBytes;       // 2 x 16 KB
-    static constexpr uint32_t kT = kV + 2 * kVBytes;             // DK x 128 B
+    static constexpr uint32_t kQ = 0;                              // Q staging, DK x 128 rows
+    static constexpr uint32_t kK = kQ + DK * kC * 2;               // K' ring
+    static constexpr uint32_t kV = kK + kKSlots * kKPartBytes;     // 2 x 16 KB
+    static constexpr uint32_t kT = kV + 2 * kVBytes;               // DK x 128 B
     static constexpr uint32_t kEnd = kT + DK * 128;
     static constexpr uint32_t kBytes = kEnd + 1024;
 };
 
+// TMEM columns
+constexpr uint32_t kTA = 0, kTP = 128, kTO = 192, kTQ = 256, kTS = 384;
+
 struct Bars {
-    uint64_t full[2], empty[2], vfull[2], vempty[2], afull[2], pready[2], ofull[2], ofree[2], sdone, tready;
+    uint64_t qfull, qempty, kfull[kKSlots], kempty[kKSlots], vfull[2], vempty[2];
+    uint64_t qready, qfree, afull, aread, pready, sdone, tready, ofull, ofree;
 };
 
 __device__ __forceinline__ void elect_arrive(uint64_t* bar, int lane) {
@@ -141,6 +149,7 @@ __device__ __forceinline__ void elect_arrive(uint64_t* bar, int lane) {
 template <int DK, typename Tout>
 __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_constant__ WsParams p) {
     constexpr int kParts = DK / kPartDk;
+    constexpr int kQSlabs = DK / 64;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ Bars bars;
@@ -154,18 +163,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
     const double lg = p.hc.log2g[h];
 
     if (tid == 0) {
+        tc::mbar_init(&bars.qfull, 1);
+        tc::mbar_init(&bars.qempty, 4);
+        for (int i = 0; i < kKSlots; i++) {
+            tc::mbar_init(&bars.kfull[i], 1);
+            tc::mbar_init(&bars.kempty[i], 1);
+        }
         for (int i = 0; i < 2; i++) {
-            tc::mbar_init(&bars.full[i], 1);
-            tc::mbar_init(&bars.empty[i], 1);
             tc::mbar_init(&bars.vfull[i], 1);
             tc::mbar_init(&bars.vempty[i], 1);
-            tc::mbar_init(&bars.afull[i], 1);
-            tc::mbar_init(&bars.pready[i], 4);
-            tc::mbar_init(&bars.ofull[i], 1);
-            tc::mbar_init(&bars.ofree[i], 4);
         }
+        tc::mbar_init(&bars.qready, 4);
+        tc::mbar_init(&bars.qfree, 1);
+        tc::mbar_init(&bars.afull, 1);
+        tc::mbar_init(&bars.aread, 4);
+        tc::mbar_init(&bars.pready, 4);
         tc::mbar_init(&bars.sdone, 1);
         tc::mbar_init(&bars.tready, 4);
+        tc::mbar_init(&bars.ofull, 1);
+        tc::mbar_init(&bars.ofree, 4);
         s_fail = 0;
         tc::fence_barrier_init();
         tc::prefetch_tmap(&p.tq);
@@ -184,17 +200,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         if (lane == 0) {
             for (int jc = 0; jc < nchunks && ok; jc++) {
                 const int n0 = jc * kC;
+                if (jc > 0) ok = tc::mbar_wait(&bars.qempty, (jc - 1) & 1);
+                if (!ok) break;
+                tc::mbar_arrive_expect_tx(&bars.qfull, DK * kC * 2);
+                for (int s = 0; s < kQSlabs; s++)
+                    tc::tma_load_4d(sm + WsSmem<DK>::kQ + s * (kC * 128), &p.tq, &bars.qfull, 64 * s, h, n0, b);
                 for (int part = 0; part < kParts && ok; part++) {
-                    const int g = jc * kParts + part, slot = g & 1;
-                    if (g >= 2) ok = tc::mbar_wait(&bars.empty[slot], ((g >> 1) & 1) ^ 1);
+                    const int g = jc * kParts + part, slot = g % kKSlots, u = g / kKSlots;
+                    if (u > 0) ok = tc::mbar_wait(&bars.kempty[slot], (u - 1) & 1);
                     if (!ok) break;
-                    uint8_t* dst = sm + WsSmem<DK>::kRing + slot * kPartBytes;
-                    tc::mbar_arrive_expect_tx(&bars.full[slot], kPartBytes);
-                    for (int s = 0; s < 2; s++) {
-                        const int dk0 = part * kPartDk + 64 * s;
-                        tc::tma_load_4d(dst + s * (kC * 128), &p.tq, &bars.full[slot], dk0, h, n0, b);
-                        tc::tma_load_4d(dst + (2 + s) * (kC * 128), &p.tk, &bars.full[slot], dk0, h, n0, b);
-                    }
+                    uint8_t* dst = sm + WsSmem<DK>::kK + slot * kKPartBytes;
+                    tc::mbar_arrive_expect_tx(&bars.kfull[slot], kKPartBytes);
+                    for (int s = 0; s < 2; s++)
+                        tc::tma_load_4d(dst + s * (kC * 128), &p.tk, &bars.kfull[slot], part * kPartDk + 64 * s, h,
+                                        n0, b);
                 }
                 const int vs = jc & 1;
                 if (ok && jc >= 2) ok = tc::mbar_wait(&bars.vempty[vs], ((jc >> 1) & 1) ^ 1);
@@ -210,61 +229,59 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             const uint32_t id_qt = tc::idesc_bf16_f32(128, kW, 0, 1);
             const uint32_t id_st = tc::idesc_bf16_f32(128, kW, 1, 1);
             const uint32_t id_pv = tc::idesc_bf16_f32(128, kW, 0, 1);
-            const uint32_t ring0 = tc::smem_u32(sm + WsSmem<DK>::kRing);
+            const uint32_t k0 = tc::smem_u32(sm + WsSmem<DK>::kK);
             const uint32_t v0 = tc::smem_u32(sm + WsSmem<DK>::kV);
             const uint32_t t0 = tc::smem_u32(sm + WsSmem<DK>::kT);
             for (int jc = 0; jc < nchunks && ok; jc++) {
-                const int bb = jc & 1;
-                const uint32_t dA = tb + kColA + 128 * bb, dO = tb + kColO + kW * bb;
-                // A[bb] = Q K'^T over all parts
+                // A = Q K'^T  (A operand Q from TMEM)
+                ok = tc::mbar_wait(&bars.qready, jc & 1);
+                if (ok && jc > 0) ok = tc::mbar_wait(&bars.aread, (jc - 1) & 1);
                 for (int part = 0; part < kParts && ok; part++) {
-                    const int g = jc * kParts + part, slot = g & 1;
-                    ok = tc::mbar_wait(&bars.full[slot], (g >> 1) & 1);
+                    const int g = jc * kParts + part, slot = g % kKSlots, u = g / kKSlots;
+                    ok = tc::mbar_wait(&bars.kfull[slot], u & 1);
                     if (!ok) break;
                     tc::tc_fence_after();
-                    const uint32_t qb = ring0 + slot * kPartBytes, kb = qb + 2 * (kC * 128);
+                    const uint32_t kb = k0 + slot * kKPartBytes;
                     for (int k = 0; k < kPartDk / 16; k++) {
                         const uint32_t off = (k / 4) * (kC * 128) + (k % 4) * 32;
-                        tc::mma_bf16_ss(dA, tc::sdesc_sw128(qb + off, 16, 1024), tc::sdesc_sw128(kb + off, 16, 1024),
+                        tc::mma_bf16_ts(tb + kTA, tb + kTQ + 64 * part + 8 * k, tc::sdesc_sw128(kb + off, 16, 1024),
                                         id_qk, (part > 0) || (k > 0));
                     }
                 }
                 if (!ok) break;
-                tc::mma_commit(&bars.afull[bb]);
-                // cross read-out and state update need T (rescale of chunk jc-1),
-                // a free O[bb] and this chunk's V
+                tc::mma_commit(&bars.afull);
+                // cross read-out (needs T of the previous chunk and a free O) and state update
                 if (jc > 0) ok = tc::mbar_wait(&bars.tready, (jc - 1) & 1);
-                if (ok && jc >= 2) ok = tc::mbar_wait(&bars.ofree[bb], ((jc >> 1) & 1) ^ 1);
-                if (ok) ok = tc::mbar_wait(&bars.vfull[bb], (jc >> 1) & 1);
+                if (ok && jc > 0) ok = tc::mbar_wait(&bars.ofree, (jc - 1) & 1);
+                if (ok) ok = tc::mbar_wait(&bars.vfull[jc & 1], (jc >> 1) & 1);
                 if (!ok) break;
                 tc::tc_fence_after();
-                const uint32_t vb = v0 + bb * kVBytes;
+                const uint32_t vb = v0 + (jc & 1) * kVBytes;
                 for (int part = 0; part < kParts; part++) {
-                    const int g = jc * kParts + part, slot = g & 1;
-                    const uint32_t qb = ring0 + slot * kPartBytes, kb = qb + 2 * (kC * 128);
+                    const int g = jc * kParts + part, slot = g % kKSlots;
+                    const uint32_t kb = k0 + slot * kKPartBytes;
                     if (jc > 0) {
-                        for (int k = 0; k < kPartDk / 16; k++) {
-                            const uint32_t off = (k / 4) * (kC * 128) + (k % 4) * 32;
-                            tc::mma_bf16_ss(dO, tc::sdesc_sw128(qb + off, 16, 1024),
+                        for (int k = 0; k < kPartDk / 16; k++)
+                            tc::mma_bf16_ts(tb + kTO, tb + kTQ + 64 * part + 8 * k,
                                             tc::sdesc_sw128(t0 + (part * kPartDk + 16 * k) * 128, DK * 128, 1024),
                                             id_qt, (part > 0) || (k > 0));
-                        }
                     }
                     for (int k = 0; k < kC / 16; k++)
-                        tc::mma_bf16_ss(tb + kColS + part * kW, tc::sdesc_sw128(kb + k * 2048, kC * 128, 1024),
+                        tc::mma_bf16_ss(tb + kTS + part * kW, tc::sdesc_sw128(kb + k * 2048, kC * 128, 1024),
                                         tc::sdesc_sw128(vb + k * 2048, kC * 128, 1024), id_st, (jc > 0) || (k > 0));
-                    tc::mma_commit(&bars.empty[slot]);
+                    tc::mma_commit(&bars.kempty[slot]);
                 }
+                tc::mma_commit(&bars.qfree);
                 tc::mma_commit(&bars.sdone);
-                // O[bb] += P V
-                ok = tc::mbar_wait(&bars.pready[bb], (jc >> 1) & 1);
+                // O += P V   (A operand P from TMEM)
+                ok = tc::mbar_wait(&bars.pready, jc & 1);
                 if (!ok) break;
                 tc::tc_fence_after();
                 for (int k = 0; k < kC / 16; k++)
-                    tc::mma_bf16_ts(dO, dA + 8 * k, tc::sdesc_sw128(vb + k * 2048, kC * 128, 1024), id_pv,
+                    tc::mma_bf16_ts(tb + kTO, tb + kTP + 8 * k, tc::sdesc_sw128(vb + k * 2048, kC * 128, 1024), id_pv,
                                     (jc > 0) || (k > 0));
-                tc::mma_commit(&bars.ofull[bb]);
-                tc::mma_commit(&bars.vempty[bb]);
+                tc::mma_commit(&bars.ofull);
+                tc::mma_commit(&bars.vempty[jc & 1]);
             }
         }
     } else {
@@ -273,20 +290,52 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         const int r = quarter * 32 + lane;            // chunk row / state row in a block
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         uint8_t* sT = sm + WsSmem<DK>::kT;
+        const uint8_t* sQ = sm + WsSmem<DK>::kQ;
+
+        // Q of chunk jq from the staging buffer into TMEM columns [kTQ, kTQ + DK/2)
+        auto copy_q = [&](int jq) -> bool {
+            if (!tc::mbar_wait(&bars.qfull, jq & 1)) return false;
+            if (jq > 0 && !tc::mbar_wait(&bars.qfree, (jq - 1) & 1)) return false;
+            tc::tc_fence_after();
+#pragma unroll
+            for (int g32 = 0; g32 < DK / 64; g32++) {       // 32 packed words = 64 d_k values = one slab row
+                uint32_t w[32];
+#pragma unroll
+                for (int c16 = 0; c16 < 8; c16++) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(sQ + g32 * (kC * 128) +
+                                                                    tc::sw128_off((uint32_t)r, (uint32_t)c16));
+                    w[4 * c16 + 0] = v.x;
+                    w[4 * c16 + 1] = v.y;
+                    w[4 * c16 + 2] = v.z;
+                    w[4 * c16 + 3] = v.w;
+                }
+                tc::tmem_st32(tb + lane_off + kTQ + 32 * g32, w);
+            }
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(&bars.qready);
+                tc::mbar_arrive(&bars.qempty);
+            }
+            return true;
+        };
+
+        ok = copy_q(0);
         for (int jc = 0; jc < nchunks && ok; jc++) {
-            const int bb = jc & 1;
             const int n0 = jc * kC, L = min(kC, N - n0);
             const bool last = (jc == nchunks - 1);
-            // ---- mask: P = tril(A) as packed bf16 into A[bb] columns [0, 64)
-            ok = tc::mbar_wait(&bars.afull[bb], (jc >> 1) & 1);
+            // ---- mask: P = tril(A) as packed bf16 into TMEM columns [kTP, kTP + 64)
+            ok = tc::mbar_wait(&bars.afull, jc & 1);
             if (!ok) break;
             tc::tc_fence_after();
             {
-                const uint32_t a_addr = tb + lane_off + kColA + 128 * bb;
                 uint32_t a[4][32];
 #pragma unroll
-                for (int q4 = 0; q4 < 4; q4++) tc::tmem_ld32(a_addr + 32 * q4, a[q4]);
+                for (int q4 = 0; q4 < 4; q4++) tc::tmem_ld32(tb + lane_off + kTA + 32 * q4, a[q4]);
                 tc::tmem_ld_wait();
+                tc::tc_fence_before();
+                elect_arrive(&bars.aread, lane);
 #pragma unroll
                 for (int half = 0; half < 2; half++) {
                     uint32_t w[32];
@@ -297,12 +346,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                         const float hi = (c + 1 <= r) ? __uint_as_float(a[2 * half + (i >> 4)][(2 * i + 1) & 31]) : 0.f;
                         w[i] = tc::pack_bf16x2(lo, hi);
                     }
-                    tc::tmem_st32(a_addr + 32 * half, w);
+                    tc::tmem_st32(tb + lane_off + kTP + 32 * half, w);
                 }
                 tc::tmem_st_wait();
             }
             tc::tc_fence_before();
-            elect_arrive(&bars.pready[bb], lane);
+            elect_arrive(&bars.pready, lane);
             // ---- state: T = gamma^L_next R (TMEM fp32 and shared bf16), or the final state
             ok = tc::mbar_wait(&bars.sdone, jc & 1);
             if (!ok) break;
@@ -311,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 const float gL = last ? 1.f : (float)exp2((double)min(kC, N - (n0 + kC)) * lg);
 #pragma unroll
                 for (int part = 0; part < kParts; part++) {
-                    const uint32_t s_addr = tb + lane_off + kColS + part * kW;
+                    const uint32_t s_addr = tb + lane_off + kTS + part * kW;
                     const int d = part * kPartDk + r;
                     uint32_t s[2][32];
                     tc::tmem_ld32(s_addr, s[0]);
@@ -349,18 +398,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             tc::fence_proxy_async_smem();
             tc::tc_fence_before();
             elect_arrive(&bars.tready, lane);
+            // ---- the next chunk's Q into TMEM (its readers of this chunk are done: sdone)
+            if (!last) {
+                ok = copy_q(jc + 1);
+                if (!ok) break;
+            }
             // ---- epilogue: out = gamma^(r+1-L) O
-            ok = tc::mbar_wait(&bars.ofull[bb], (jc >> 1) & 1);
+            ok = tc::mbar_wait(&bars.ofull, jc & 1);
             if (!ok) break;
             tc::tc_fence_after();
             {
                 uint32_t o[2][32];
-                const uint32_t o_addr = tb + lane_off + kColO + kW * bb;
-                tc::tmem_ld32(o_addr, o[0]);
-                tc::tmem_ld32(o_addr + 32, o[1]);
+                tc::tmem_ld32(tb + lane_off + kTO, o[0]);
+                tc::tmem_ld32(tb + lane_off + kTO + 32, o[1]);
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
-                elect_arrive(&bars.ofree[bb], lane);
+                elect_arrive(&bars.ofree, lane);
                 if (r < L) {
                     const float sc = (float)exp2((double)(r + 1 - L) * lg);
                     Tout* dst = reinterpret_cast<Tout*>(p.out) + (((size_t)b * N + n0 + r) * p.H + h) * p.dv + j0;
