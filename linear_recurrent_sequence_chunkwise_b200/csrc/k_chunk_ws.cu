@@ -15,14 +15,15 @@
 //    each rotated key row by its zeta, and writes q_rot and k' (bf16) into the
 //    workspace.  Without rotation only k' is written and q is read in place.
 // 2. k_chunkwise_ws: one CTA per (batch, head, 64 value columns), three roles
-//      warp 0  TMA producer: per chunk the Q tile into a staging buffer, the
+//      warp 0  TMA producer: L2 prefetch two chunks ahead (the CTAs of a
+//              head split the boxes), then per chunk the Q tile into a staging buffer, the
 //              K' tile in parts of 128 d_k rows through a 3-slot ring, and
 //              the V tile (2 slots);
 //      warp 1  MMA issuer (one thread), A operands from TMEM where possible:
 //                A  = Q K'^T          (Q from TMEM, K' from smem)
 //                O  = Q T  + P V      (Q and P from TMEM, T and V from smem)
 //                R += K'^T V          (fp32 state in TMEM)
-//      warps 2-5 (one warpgroup, TMEM lanes 0..127):
+//      warps 2-9 (two warpgroups on TMEM lanes 0..127, one column half each):
 //                Q staging -> TMEM (frees the 64 KB staging buffer early),
 //                mask:     P = tril(A) -> packed bf16 in TMEM,
 //                state:    T = gamma^L R -> TMEM (fp32) and smem (bf16),
@@ -54,7 +55,7 @@ constexpr int kC = 128;           // chunk rows (M of every MMA)
 constexpr int kW = 64;            // d_v columns per CTA
 constexpr int kPartDk = 128;      // d_k rows per pipeline part (one state block)
 constexpr int kVBytes = kC * kW * 2;              // 16 KB
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;   // TMA warp, MMA warp, two transform warpgroups
 
 // ------------------------------------------------------------------ prep
 
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
 
     if (tid == 0) {
         tc::mbar_init(&bars.qfull, 1);
-        tc::mbar_init(&bars.qempty, 4);
+        tc::mbar_init(&bars.qempty, 8);
         for (int i = 0; i < kKSlots; i++) {
             tc::mbar_init(&bars.kfull[i], 1);
             tc::mbar_init(&bars.kempty[i], 1);
@@ -173,15 +174,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             tc::mbar_init(&bars.vfull[i], 1);
             tc::mbar_init(&bars.vempty[i], 1);
         }
-        tc::mbar_init(&bars.qready, 4);
+        tc::mbar_init(&bars.qready, 8);
         tc::mbar_init(&bars.qfree, 1);
         tc::mbar_init(&bars.afull, 1);
-        tc::mbar_init(&bars.aread, 4);
-        tc::mbar_init(&bars.pready, 4);
+        tc::mbar_init(&bars.aread, 8);
+        tc::mbar_init(&bars.pready, 8);
         tc::mbar_init(&bars.sdone, 1);
-        tc::mbar_init(&bars.tready, 4);
+        tc::mbar_init(&bars.tready, 8);
         tc::mbar_init(&bars.ofull, 1);
-        tc::mbar_init(&bars.ofree, 4);
+        tc::mbar_init(&bars.ofree, 8);
         s_fail = 0;
         tc::fence_barrier_init();
         tc::prefetch_tmap(&p.tq);
@@ -198,8 +199,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
+            // L2 prefetch of chunk jp: the CTAs of one head split the Q and K'
+            // boxes between them; each prefetches its own V tile.
+            auto prefetch = [&](int jp) {
+                if (jp >= nchunks) return;
+                const int n0p = jp * kC;
+                for (int i = blockIdx.x; i < 2 * kQSlabs; i += gridDim.x)
+                    tc::tma_prefetch_l2_4d(i < kQSlabs ? &p.tq : &p.tk, 64 * (i % kQSlabs), h, n0p, b);
+                tc::tma_prefetch_l2_4d(&p.tv, j0, h, n0p, b);
+            };
+            prefetch(1);
             for (int jc = 0; jc < nchunks && ok; jc++) {
                 const int n0 = jc * kC;
+                prefetch(jc + 2);
                 if (jc > 0) ok = tc::mbar_wait(&bars.qempty, (jc - 1) & 1);
                 if (!ok) break;
                 tc::mbar_arrive_expect_tx(&bars.qfull, DK * kC * 2);
@@ -285,8 +297,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             }
         }
     } else {
-        // ------------------------------------------- transform warpgroup
+        // ------------------------------------------ transform warpgroups
+        // Warps 2-5 and 6-9 form two warpgroups; each covers TMEM lanes
+        // 0..127 (a warp reaches the lane quarter warp % 4) and takes one half
+        // of the columns of every phase.
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter ..
+        const int wg = (warp - 2) >> 2;               // column half
         const int r = quarter * 32 + lane;            // chunk row / state row in a block
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         uint8_t* sT = sm + WsSmem<DK>::kT;
@@ -298,7 +314,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             if (jq > 0 && !tc::mbar_wait(&bars.qfree, (jq - 1) & 1)) return false;
             tc::tc_fence_after();
 #pragma unroll
-            for (int g32 = 0; g32 < DK / 64; g32++) {       // 32 packed words = 64 d_k values = one slab row
+            for (int gg = 0; gg < DK / 128; gg++) {        // 32 packed words = 64 d_k values = one slab row
+                const int g32 = wg * (DK / 128) + gg;
                 uint32_t w[32];
 #pragma unroll
                 for (int c16 = 0; c16 < 8; c16++) {
@@ -330,24 +347,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             if (!ok) break;
             tc::tc_fence_after();
             {
-                uint32_t a[4][32];
-#pragma unroll
-                for (int q4 = 0; q4 < 4; q4++) tc::tmem_ld32(tb + lane_off + kTA + 32 * q4, a[q4]);
+                uint32_t a[2][32];
+                tc::tmem_ld32(tb + lane_off + kTA + 64 * wg, a[0]);
+                tc::tmem_ld32(tb + lane_off + kTA + 64 * wg + 32, a[1]);
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
                 elect_arrive(&bars.aread, lane);
+                uint32_t w[32];
 #pragma unroll
-                for (int half = 0; half < 2; half++) {
-                    uint32_t w[32];
-#pragma unroll
-                    for (int i = 0; i < 32; i++) {
-                        const int c = 64 * half + 2 * i;
-                        const float lo = (c <= r) ? __uint_as_float(a[2 * half + (i >> 4)][(2 * i) & 31]) : 0.f;
-                        const float hi = (c + 1 <= r) ? __uint_as_float(a[2 * half + (i >> 4)][(2 * i + 1) & 31]) : 0.f;
-                        w[i] = tc::pack_bf16x2(lo, hi);
-                    }
-                    tc::tmem_st32(tb + lane_off + kTP + 32 * half, w);
+                for (int i = 0; i < 32; i++) {
+                    const int c = 64 * wg + 2 * i;
+                    const float lo = (c <= r) ? __uint_as_float(a[i >> 4][(2 * i) & 31]) : 0.f;
+                    const float hi = (c + 1 <= r) ? __uint_as_float(a[i >> 4][(2 * i + 1) & 31]) : 0.f;
+                    w[i] = tc::pack_bf16x2(lo, hi);
                 }
+                tc::tmem_st32(tb + lane_off + kTP + 32 * wg, w);
                 tc::tmem_st_wait();
             }
             tc::tc_fence_before();
@@ -360,37 +374,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 const float gL = last ? 1.f : (float)exp2((double)min(kC, N - (n0 + kC)) * lg);
 #pragma unroll
                 for (int part = 0; part < kParts; part++) {
-                    const uint32_t s_addr = tb + lane_off + kTS + part * kW;
+                    const uint32_t s_addr = tb + lane_off + kTS + part * kW + 32 * wg;
                     const int d = part * kPartDk + r;
-                    uint32_t s[2][32];
-                    tc::tmem_ld32(s_addr, s[0]);
-                    tc::tmem_ld32(s_addr + 32, s[1]);
+                    uint32_t s[32];
+                    tc::tmem_ld32(s_addr, s);
                     tc::tmem_ld_wait();
                     if (!last) {
 #pragma unroll
-                        for (int hh = 0; hh < 2; hh++)
+                        for (int i = 0; i < 32; i++) s[i] = __float_as_uint(__uint_as_float(s[i]) * gL);
+                        tc::tmem_st32(s_addr, s);
 #pragma unroll
-                            for (int i = 0; i < 32; i++) s[hh][i] = __float_as_uint(__uint_as_float(s[hh][i]) * gL);
-                        tc::tmem_st32(s_addr, s[0]);
-                        tc::tmem_st32(s_addr + 32, s[1]);
-#pragma unroll
-                        for (int c16 = 0; c16 < 8; c16++) {
-                            const int hh = c16 >> 2, base = (c16 & 3) * 8;
+                        for (int c4 = 0; c4 < 4; c4++) {
+                            const int base = c4 * 8;
                             uint4 v;
-                            v.x = tc::pack_bf16x2(__uint_as_float(s[hh][base + 0]), __uint_as_float(s[hh][base + 1]));
-                            v.y = tc::pack_bf16x2(__uint_as_float(s[hh][base + 2]), __uint_as_float(s[hh][base + 3]));
-                            v.z = tc::pack_bf16x2(__uint_as_float(s[hh][base + 4]), __uint_as_float(s[hh][base + 5]));
-                            v.w = tc::pack_bf16x2(__uint_as_float(s[hh][base + 6]), __uint_as_float(s[hh][base + 7]));
-                            *reinterpret_cast<uint4*>(sT + tc::sw128_off((uint32_t)d, (uint32_t)c16)) = v;
+                            v.x = tc::pack_bf16x2(__uint_as_float(s[base + 0]), __uint_as_float(s[base + 1]));
+                            v.y = tc::pack_bf16x2(__uint_as_float(s[base + 2]), __uint_as_float(s[base + 3]));
+                            v.z = tc::pack_bf16x2(__uint_as_float(s[base + 4]), __uint_as_float(s[base + 5]));
+                            v.w = tc::pack_bf16x2(__uint_as_float(s[base + 6]), __uint_as_float(s[base + 7]));
+                            *reinterpret_cast<uint4*>(sT + tc::sw128_off((uint32_t)d, (uint32_t)(4 * wg + c4))) = v;
                         }
                     } else if (p.fstate) {
-                        float4* dst = reinterpret_cast<float4*>(p.fstate + (((size_t)b * p.H + h) * DK + d) * p.dv + j0);
+                        float4* dst = reinterpret_cast<float4*>(p.fstate + (((size_t)b * p.H + h) * DK + d) * p.dv +
+                                                                j0 + 32 * wg);
 #pragma unroll
-                        for (int c4 = 0; c4 < 16; c4++) {
-                            const int hh = c4 >> 3, base = (c4 & 7) * 4;
-                            dst[c4] = make_float4(__uint_as_float(s[hh][base]), __uint_as_float(s[hh][base + 1]),
-                                                  __uint_as_float(s[hh][base + 2]), __uint_as_float(s[hh][base + 3]));
-                        }
+                        for (int c4 = 0; c4 < 8; c4++)
+                            dst[c4] = make_float4(__uint_as_float(s[4 * c4]), __uint_as_float(s[4 * c4 + 1]),
+                                                  __uint_as_float(s[4 * c4 + 2]), __uint_as_float(s[4 * c4 + 3]));
                     }
                 }
                 if (!last) tc::tmem_st_wait();
@@ -408,34 +417,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             if (!ok) break;
             tc::tc_fence_after();
             {
-                uint32_t o[2][32];
-                tc::tmem_ld32(tb + lane_off + kTO, o[0]);
-                tc::tmem_ld32(tb + lane_off + kTO + 32, o[1]);
+                uint32_t o[32];
+                tc::tmem_ld32(tb + lane_off + kTO + 32 * wg, o);
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
                 elect_arrive(&bars.ofree, lane);
                 if (r < L) {
                     const float sc = (float)exp2((double)(r + 1 - L) * lg);
-                    Tout* dst = reinterpret_cast<Tout*>(p.out) + (((size_t)b * N + n0 + r) * p.H + h) * p.dv + j0;
+                    Tout* dst = reinterpret_cast<Tout*>(p.out) + (((size_t)b * N + n0 + r) * p.H + h) * p.dv + j0 +
+                                32 * wg;
                     if constexpr (sizeof(Tout) == 2) {
 #pragma unroll
-                        for (int c16 = 0; c16 < 8; c16++) {
-                            const int hh = c16 >> 2, base = (c16 & 3) * 8;
+                        for (int c16 = 0; c16 < 4; c16++) {
+                            const int base = c16 * 8;
                             uint4 v;
-                            v.x = tc::pack_bf16x2(__uint_as_float(o[hh][base + 0]) * sc, __uint_as_float(o[hh][base + 1]) * sc);
-                            v.y = tc::pack_bf16x2(__uint_as_float(o[hh][base + 2]) * sc, __uint_as_float(o[hh][base + 3]) * sc);
-                            v.z = tc::pack_bf16x2(__uint_as_float(o[hh][base + 4]) * sc, __uint_as_float(o[hh][base + 5]) * sc);
-                            v.w = tc::pack_bf16x2(__uint_as_float(o[hh][base + 6]) * sc, __uint_as_float(o[hh][base + 7]) * sc);
+                            v.x = tc::pack_bf16x2(__uint_as_float(o[base + 0]) * sc, __uint_as_float(o[base + 1]) * sc);
+                            v.y = tc::pack_bf16x2(__uint_as_float(o[base + 2]) * sc, __uint_as_float(o[base + 3]) * sc);
+                            v.z = tc::pack_bf16x2(__uint_as_float(o[base + 4]) * sc, __uint_as_float(o[base + 5]) * sc);
+                            v.w = tc::pack_bf16x2(__uint_as_float(o[base + 6]) * sc, __uint_as_float(o[base + 7]) * sc);
                             reinterpret_cast<uint4*>(dst)[c16] = v;
                         }
                     } else {
 #pragma unroll
-                        for (int c4 = 0; c4 < 16; c4++) {
-                            const int hh = c4 >> 3, base = (c4 & 7) * 4;
+                        for (int c4 = 0; c4 < 8; c4++)
                             reinterpret_cast<float4*>(dst)[c4] =
-                                make_float4(__uint_as_float(o[hh][base + 0]) * sc, __uint_as_float(o[hh][base + 1]) * sc,
-                                            __uint_as_float(o[hh][base + 2]) * sc, __uint_as_float(o[hh][base + 3]) * sc);
-                        }
+                                make_float4(__uint_as_float(o[4 * c4 + 0]) * sc, __uint_as_float(o[4 * c4 + 1]) * sc,
+                                            __uint_as_float(o[4 * c4 + 2]) * sc, __uint_as_float(o[4 * c4 + 3]) * sc);
                     }
                 }
             }
