@@ -1,0 +1,46 @@
+// gemm.h -- internal interface of the tcgen05 GEMM (k_gemm.cu) and its
+// fused epilogues.
+#pragma once
+
+#include "common.cuh"
+
+namespace ret {
+
+enum : int {
+    kEpiStore = 0,            // out = scale * acc
+    kEpiRotate = 1,           // out = rot(scale * acc)             (queries)
+    kEpiRotateScaleZeta = 2,  // out = rot(scale * acc) * zeta      (keys)
+    kEpiSwish = 3,            // out = swish(acc)                   (gate)
+};
+
+struct GemmSegment {
+    const void* B;  // [K, N] bf16 row-major
+    int N;
+};
+
+struct GemmSegOut {
+    void* ptr;          // [M, ld] row-major destination of this segment
+    int ld;             // leading dimension (elements)
+    int kind;           // kEpi*
+    ret_dtype dtype;    // kEpiStore / kEpiSwish: RET_F32 or RET_BF16; rotations write bf16
+    float scale;
+    int head_dim;       // rotations: width of a head (pairs rotate within it)
+};
+
+struct GemmEpilogue {
+    GemmSegOut seg[4];
+    int M;                  // filled by launch_gemm
+    int seq;                // rows are (batch, token) with token = row % seq
+    int chunk;              // chunk length for the zeta of the keys
+    long long pos_offset;
+    double log2base;        // log2(theta_base)
+    double log2g[kMaxHeads];
+};
+
+// C = A B with A [M, K] bf16 row-major and B split into column segments.
+ret_status launch_gemm(const void* A, int M, int K, const GemmSegment* segs, int nseg, const GemmEpilogue& epi,
+                       cudaStream_t s);
+
+cudaError_t read_clear_error_gemm(int* flag);
+
+}  // namespace ret

@@ -134,12 +134,13 @@ struct WsSmem {
     static constexpr uint32_t kBytes = kEnd + 1024;
 };
 
-// TMEM columns
-constexpr uint32_t kTA = 0, kTP = 128, kTO = 192, kTQ = 256, kTS = 384;
+// TMEM columns: A = Q K'^T (fp32), P (packed bf16), O (fp32), Q (packed
+// bf16, the A operand of Q K'^T and of the read-out), dS = K'^T V (fp32).
+constexpr uint32_t kTA = 0, kTP = 128, kTO = 192, kTQ = 256, kTD = 384;
 
 struct Bars {
     uint64_t qfull, qempty, kfull[kKSlots], kempty[kKSlots], vfull[2], vempty[2];
-    uint64_t qready, qfree, afull, aread, pready, sdone, tready, ofull, ofree;
+    uint64_t qready, qfree, afull, aread, pready, dsdone, dsfree, tready, ofull, ofree;
 };
 
 __device__ __forceinline__ void elect_arrive(uint64_t* bar, int lane) {
@@ -162,10 +163,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
     const int N = p.N;
     const int nchunks = (N + kC - 1) / kC;
     const double lg = p.hc.log2g[h];
+    constexpr int kTG = 8;  // transform warps arriving on the warpgroup barriers
 
     if (tid == 0) {
         tc::mbar_init(&bars.qfull, 1);
-        tc::mbar_init(&bars.qempty, 8);
+        tc::mbar_init(&bars.qempty, kTG);
         for (int i = 0; i < kKSlots; i++) {
             tc::mbar_init(&bars.kfull[i], 1);
             tc::mbar_init(&bars.kempty[i], 1);
@@ -174,15 +176,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             tc::mbar_init(&bars.vfull[i], 1);
             tc::mbar_init(&bars.vempty[i], 1);
         }
-        tc::mbar_init(&bars.qready, 8);
+        tc::mbar_init(&bars.qready, kTG);
         tc::mbar_init(&bars.qfree, 1);
         tc::mbar_init(&bars.afull, 1);
-        tc::mbar_init(&bars.aread, 8);
-        tc::mbar_init(&bars.pready, 8);
-        tc::mbar_init(&bars.sdone, 1);
-        tc::mbar_init(&bars.tready, 8);
+        tc::mbar_init(&bars.aread, kTG);
+        tc::mbar_init(&bars.pready, kTG);
+        tc::mbar_init(&bars.dsdone, 1);
+        tc::mbar_init(&bars.dsfree, kTG);
+        tc::mbar_init(&bars.tready, kTG);
         tc::mbar_init(&bars.ofull, 1);
-        tc::mbar_init(&bars.ofree, 8);
+        tc::mbar_init(&bars.ofree, kTG);
         s_fail = 0;
         tc::fence_barrier_init();
         tc::prefetch_tmap(&p.tq);
@@ -245,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             const uint32_t v0 = tc::smem_u32(sm + WsSmem<DK>::kV);
             const uint32_t t0 = tc::smem_u32(sm + WsSmem<DK>::kT);
             for (int jc = 0; jc < nchunks && ok; jc++) {
-                // A = Q K'^T  (A operand Q from TMEM)
+                // ---- A = Q K'^T  (Q from TMEM)
                 ok = tc::mbar_wait(&bars.qready, jc & 1);
                 if (ok && jc > 0) ok = tc::mbar_wait(&bars.aread, (jc - 1) & 1);
                 for (int part = 0; part < kParts && ok; part++) {
@@ -262,30 +265,33 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 }
                 if (!ok) break;
                 tc::mma_commit(&bars.afull);
-                // cross read-out (needs T of the previous chunk and a free O) and state update
-                if (jc > 0) ok = tc::mbar_wait(&bars.tready, (jc - 1) & 1);
-                if (ok && jc > 0) ok = tc::mbar_wait(&bars.ofree, (jc - 1) & 1);
-                if (ok) ok = tc::mbar_wait(&bars.vfull[jc & 1], (jc >> 1) & 1);
+                // ---- O = Q T  (read-out of the state before this chunk)
+                if (jc > 0) {
+                    ok = tc::mbar_wait(&bars.tready, (jc - 1) & 1);
+                    if (ok) ok = tc::mbar_wait(&bars.ofree, (jc - 1) & 1);
+                    if (!ok) break;
+                    tc::tc_fence_after();
+                    for (int k = 0; k < DK / 16; k++)
+                        tc::mma_bf16_ts(tb + kTO, tb + kTQ + 8 * k,
+                                        tc::sdesc_sw128(t0 + 16 * k * 128, DK * 128, 1024), id_qt, k > 0);
+                }
+                tc::mma_commit(&bars.qfree);
+                // ---- dS = K'^T V
+                ok = tc::mbar_wait(&bars.vfull[jc & 1], (jc >> 1) & 1);
+                if (ok && jc > 0) ok = tc::mbar_wait(&bars.dsfree, (jc - 1) & 1);
                 if (!ok) break;
                 tc::tc_fence_after();
                 const uint32_t vb = v0 + (jc & 1) * kVBytes;
                 for (int part = 0; part < kParts; part++) {
                     const int g = jc * kParts + part, slot = g % kKSlots;
                     const uint32_t kb = k0 + slot * kKPartBytes;
-                    if (jc > 0) {
-                        for (int k = 0; k < kPartDk / 16; k++)
-                            tc::mma_bf16_ts(tb + kTO, tb + kTQ + 64 * part + 8 * k,
-                                            tc::sdesc_sw128(t0 + (part * kPartDk + 16 * k) * 128, DK * 128, 1024),
-                                            id_qt, (part > 0) || (k > 0));
-                    }
                     for (int k = 0; k < kC / 16; k++)
-                        tc::mma_bf16_ss(tb + kTS + part * kW, tc::sdesc_sw128(kb + k * 2048, kC * 128, 1024),
-                                        tc::sdesc_sw128(vb + k * 2048, kC * 128, 1024), id_st, (jc > 0) || (k > 0));
+                        tc::mma_bf16_ss(tb + kTD + part * kW, tc::sdesc_sw128(kb + k * 2048, kC * 128, 1024),
+                                        tc::sdesc_sw128(vb + k * 2048, kC * 128, 1024), id_st, k > 0);
                     tc::mma_commit(&bars.kempty[slot]);
                 }
-                tc::mma_commit(&bars.qfree);
-                tc::mma_commit(&bars.sdone);
-                // O += P V   (A operand P from TMEM)
+                tc::mma_commit(&bars.dsdone);
+                // ---- O += P V  (P from TMEM)
                 ok = tc::mbar_wait(&bars.pready, jc & 1);
                 if (!ok) break;
                 tc::tc_fence_after();
@@ -300,13 +306,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         // ------------------------------------------ transform warpgroups
         // Warps 2-5 and 6-9 form two warpgroups; each covers TMEM lanes
         // 0..127 (a warp reaches the lane quarter warp % 4) and takes one half
-        // of the columns of every phase.
+        // of the columns of every phase.  The fp32 state R lives in their
+        // registers: row r of every 128-row block, 32 columns each.
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter ..
         const int wg = (warp - 2) >> 2;               // column half
         const int r = quarter * 32 + lane;            // chunk row / state row in a block
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         uint8_t* sT = sm + WsSmem<DK>::kT;
         const uint8_t* sQ = sm + WsSmem<DK>::kQ;
+        float R[kParts][32];
+#pragma unroll
+        for (int part = 0; part < kParts; part++)
+#pragma unroll
+            for (int i = 0; i < 32; i++) R[part][i] = 0.f;
 
         // Q of chunk jq from the staging buffer into TMEM columns [kTQ, kTQ + DK/2)
         auto copy_q = [&](int jq) -> bool {
@@ -342,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         for (int jc = 0; jc < nchunks && ok; jc++) {
             const int n0 = jc * kC, L = min(kC, N - n0);
             const bool last = (jc == nchunks - 1);
-            // ---- mask: P = tril(A) as packed bf16 into TMEM columns [kTP, kTP + 64)
+            // ---- mask: P = tril(A) as packed bf16 into TMEM
             ok = tc::mbar_wait(&bars.afull, jc & 1);
             if (!ok) break;
             tc::tc_fence_after();
@@ -366,51 +378,57 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             }
             tc::tc_fence_before();
             elect_arrive(&bars.pready, lane);
-            // ---- state: T = gamma^L_next R (TMEM fp32 and shared bf16), or the final state
-            ok = tc::mbar_wait(&bars.sdone, jc & 1);
+            // ---- the next chunk's Q into TMEM once this chunk's read-out is done
+            if (!last) {
+                ok = copy_q(jc + 1);
+                if (!ok) break;
+            }
+            // ---- state: R = gamma^L R + dS; T = gamma^L_next R (bf16, read-out of the next chunk)
+            ok = tc::mbar_wait(&bars.dsdone, jc & 1);
             if (!ok) break;
             tc::tc_fence_after();
             {
-                const float gL = last ? 1.f : (float)exp2((double)min(kC, N - (n0 + kC)) * lg);
+                const float gL = (float)exp2((double)L * lg);
 #pragma unroll
                 for (int part = 0; part < kParts; part++) {
-                    const uint32_t s_addr = tb + lane_off + kTS + part * kW + 32 * wg;
-                    const int d = part * kPartDk + r;
-                    uint32_t s[32];
-                    tc::tmem_ld32(s_addr, s);
+                    uint32_t d[32];
+                    tc::tmem_ld32(tb + lane_off + kTD + part * kW + 32 * wg, d);
                     tc::tmem_ld_wait();
-                    if (!last) {
 #pragma unroll
-                        for (int i = 0; i < 32; i++) s[i] = __float_as_uint(__uint_as_float(s[i]) * gL);
-                        tc::tmem_st32(s_addr, s);
+                    for (int i = 0; i < 32; i++) R[part][i] = fmaf(gL, R[part][i], __uint_as_float(d[i]));
+                }
+                tc::tc_fence_before();
+                elect_arrive(&bars.dsfree, lane);
+                if (!last) {
+                    const float gN = (float)exp2((double)min(kC, N - (n0 + kC)) * lg);
+#pragma unroll
+                    for (int part = 0; part < kParts; part++) {
+                        const int dr = part * kPartDk + r;
 #pragma unroll
                         for (int c4 = 0; c4 < 4; c4++) {
                             const int base = c4 * 8;
                             uint4 v;
-                            v.x = tc::pack_bf16x2(__uint_as_float(s[base + 0]), __uint_as_float(s[base + 1]));
-                            v.y = tc::pack_bf16x2(__uint_as_float(s[base + 2]), __uint_as_float(s[base + 3]));
-                            v.z = tc::pack_bf16x2(__uint_as_float(s[base + 4]), __uint_as_float(s[base + 5]));
-                            v.w = tc::pack_bf16x2(__uint_as_float(s[base + 6]), __uint_as_float(s[base + 7]));
-                            *reinterpret_cast<uint4*>(sT + tc::sw128_off((uint32_t)d, (uint32_t)(4 * wg + c4))) = v;
+                            v.x = tc::pack_bf16x2(gN * R[part][base + 0], gN * R[part][base + 1]);
+                            v.y = tc::pack_bf16x2(gN * R[part][base + 2], gN * R[part][base + 3]);
+                            v.z = tc::pack_bf16x2(gN * R[part][base + 4], gN * R[part][base + 5]);
+                            v.w = tc::pack_bf16x2(gN * R[part][base + 6], gN * R[part][base + 7]);
+                            *reinterpret_cast<uint4*>(sT + tc::sw128_off((uint32_t)dr, (uint32_t)(4 * wg + c4))) = v;
                         }
-                    } else if (p.fstate) {
-                        float4* dst = reinterpret_cast<float4*>(p.fstate + (((size_t)b * p.H + h) * DK + d) * p.dv +
+                    }
+                    tc::fence_proxy_async_smem();
+                    elect_arrive(&bars.tready, lane);
+                } else if (p.fstate) {
+#pragma unroll
+                    for (int part = 0; part < kParts; part++) {
+                        const int dr = part * kPartDk + r;
+                        float4* dst = reinterpret_cast<float4*>(p.fstate + (((size_t)b * p.H + h) * DK + dr) * p.dv +
                                                                 j0 + 32 * wg);
 #pragma unroll
                         for (int c4 = 0; c4 < 8; c4++)
-                            dst[c4] = make_float4(__uint_as_float(s[4 * c4]), __uint_as_float(s[4 * c4 + 1]),
-                                                  __uint_as_float(s[4 * c4 + 2]), __uint_as_float(s[4 * c4 + 3]));
+                            dst[c4] = make_float4(R[part][4 * c4], R[part][4 * c4 + 1], R[part][4 * c4 + 2],
+                                                  R[part][4 * c4 + 3]);
                     }
                 }
-                if (!last) tc::tmem_st_wait();
-            }
-            tc::fence_proxy_async_smem();
-            tc::tc_fence_before();
-            elect_arrive(&bars.tready, lane);
-            // ---- the next chunk's Q into TMEM (its readers of this chunk are done: sdone)
-            if (!last) {
-                ok = copy_q(jc + 1);
-                if (!ok) break;
             }
             // ---- epilogue: out = gamma^(r+1-L) O
             ok = tc::mbar_wait(&bars.ofull, jc & 1);
