@@ -166,6 +166,45 @@ ret_status ret_forward_recurrent(const void* q, const void* k, const void* v,
                                  int64_t pos_offset, double theta_base);
 
 /*
+ * MultiScaleRetention layer forward ("Hybrid Architectures ...", section 9.1;
+ * RetNet paper summary, "Gated Multi-Scale Retention"):
+ *     Q = rot(X W_Q), K = rot(k_scale X W_K), V = X W_V, G = X W_G,
+ *     Y_h = Retention(Q_h, K_h, V_h; gamma_h)          (chunkwise, `chunk`)
+ *     Z = swish(G) (.) GroupNorm_H(Y),  out = Z W_O,
+ * GroupNorm per (token, head) over the head's d_v channels with biased
+ * variance, eps inside the square root and no affine term; swish(x) =
+ * x sigmoid(x).
+ * X [B, N, d_model] bf16; W_Q, W_K [d_model, H dk], W_V, W_G [d_model, H dv],
+ * W_O [H dv, d_model], all bf16 row-major as (input, output); out
+ * [B, N, d_model] of dtype out_dt.  All device, 16-byte aligned.
+ * workspace: device, 256-byte aligned, at least ret_msr_workspace_bytes(...)
+ * bytes, overlapping nothing; scratch, undefined after the call.
+ * xpos/pos_offset/theta_base as in ret_forward_chunkwise.  Requires chunk
+ * 128, dk 128 or 256, dv in {128, 256, 512, 1024}, d_model a multiple of 8
+ * and every gamma_h^128 >= 2^-60 (else RET_ERR_UNSUPPORTED).
+ * Four launches on `stream`: the projections (tcgen05 GEMM with the rotation,
+ * k_scale, the chunkwise key decay and swish fused in its epilogue), the
+ * chunkwise retention, GroupNorm with the gate, and the output projection.
+ */
+size_t ret_msr_workspace_bytes(int B, int N, int dmodel, int H, int dk, int dv);
+
+ret_status ret_msr_forward(const void* X, const void* Wq, const void* Wk, const void* Wv,
+                           const void* Wg, const void* Wo, const double* gammas, int B, int N,
+                           int dmodel, int H, int dk, int dv, int chunk, double k_scale, double eps,
+                           int xpos, int64_t pos_offset, double theta_base, void* out,
+                           ret_dtype out_dt, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
+/*
+ * Y = X W on the tensor cores (the GEMM of the MSR layer): X [M, K] bf16,
+ * W [K, N] bf16, row-major; Y [M, N] of dtype out_dt.  fp32 accumulation.
+ * N and K multiples of 8; device pointers 16-byte aligned; Y must not overlap
+ * X or W.
+ */
+ret_status ret_linear_bf16(const void* X, const void* W, void* Y, int M, int N, int K, ret_dtype out_dt,
+                           cudaStream_t stream);
+
+/*
  * Synchronises `stream`, then reports (and clears) the device-side error word
  * that kernels set when a bounded wait gives up.  RET_OK if none was set.
  */

@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "RetentionError", "lib", "ret_xpos_rotate", "ret_forward_chunkwise", "ret_forward_chunkwise_ws",
-    "ret_chunkwise_workspace_bytes", "ret_decode_step",
+    "ret_chunkwise_workspace_bytes", "ret_decode_step", "ret_msr_forward", "ret_msr_workspace_bytes",
+    "ret_linear_bf16",
     "ret_forward_parallel", "ret_forward_recurrent", "ret_check_device_error", "ret_last_error_string",
     "RET_OK", "RET_ERR_INVALID_ARG", "RET_ERR_UNSUPPORTED", "RET_ERR_CUDA", "RET_ERR_TIMEOUT",
     "RET_F32", "RET_BF16",
@@ -56,12 +57,17 @@ def _load_library():
     L.ret_decode_step.argtypes = [vp, vp, vp, dp, vp, vp, vp, i, i, i, i, i, i]
     L.ret_forward_parallel.argtypes = [vp, vp, vp, dp, i, i, i, i, i, vp, vp, i, i, i, i64, d]
     L.ret_forward_recurrent.argtypes = [vp, vp, vp, dp, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d]
+    L.ret_msr_workspace_bytes.argtypes = [i, i, i, i, i, i]
+    L.ret_msr_workspace_bytes.restype = ctypes.c_size_t
+    L.ret_msr_forward.argtypes = [vp, vp, vp, vp, vp, vp, dp, i, i, i, i, i, i, i, d, d, i, i64, d, vp, i, vp,
+                                  ctypes.c_size_t, vp]
+    L.ret_linear_bf16.argtypes = [vp, vp, vp, i, i, i, i, vp]
     L.ret_check_device_error.argtypes = [vp]
     L.ret_last_error_string.restype = ctypes.c_char_p
     L.ret_last_error_string.argtypes = []
     for name in ("ret_xpos_rotate", "ret_forward_chunkwise", "ret_forward_chunkwise_ws", "ret_decode_step",
                  "ret_forward_parallel",
-                 "ret_forward_recurrent", "ret_check_device_error"):
+                 "ret_forward_recurrent", "ret_check_device_error", "ret_msr_forward", "ret_linear_bf16"):
         getattr(L, name).restype = ctypes.c_int
     return L
 
@@ -220,3 +226,44 @@ def ret_decode_step(q, k, v, gammas, state, out=None, out_dtype=None, stream=Non
 def ret_check_device_error(stream=None):
     """Synchronise the stream and raise if a kernel gave up a bounded wait."""
     _check(lib.ret_check_device_error(_stream(stream)))
+
+
+def ret_linear_bf16(x, w, out=None, out_dtype=torch.bfloat16, stream=None):
+    """Y = X W on the tensor cores; x [..., K] bf16, w [K, N] bf16."""
+    if x.dtype != torch.bfloat16 or w.dtype != torch.bfloat16:
+        raise TypeError("x and w must be bfloat16")
+    K = x.shape[-1]
+    if w.dim() != 2 or w.shape[0] != K:
+        raise ValueError("w must be [K, N]")
+    N = w.shape[1]
+    M = x.numel() // K
+    if out is None:
+        out = torch.empty((*x.shape[:-1], N), dtype=out_dtype, device=x.device)
+    _check(lib.ret_linear_bf16(_ptr(x, "x"), _ptr(w, "w"), _ptr(out, "out"), M, N, K, _dt(out.dtype),
+                               _stream(stream)))
+    return out
+
+
+def ret_msr_workspace_bytes(B, N, dmodel, H, dk, dv) -> int:
+    return int(lib.ret_msr_workspace_bytes(B, N, dmodel, H, dk, dv))
+
+
+def ret_msr_forward(x, wq, wk, wv, wg, wo, gammas, H: int, chunk: int = 128, k_scale: float = 1.0,
+                    eps: float = 1e-5, xpos: bool = True, pos_offset: int = 0, theta_base: float = 10000.0,
+                    out=None, out_dtype=torch.bfloat16, workspace=None, stream=None):
+    """MultiScaleRetention layer forward.  x [B, N, d_model] bf16; weights
+    bf16 [in, out]; returns out [B, N, d_model]."""
+    B, N, dm = x.shape
+    dk = wq.shape[1] // H
+    dv = wv.shape[1] // H
+    if out is None:
+        out = torch.empty((B, N, dm), dtype=out_dtype, device=x.device)
+    need = ret_msr_workspace_bytes(B, N, dm, H, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib.ret_msr_forward(_ptr(x, "x"), _ptr(wq, "wq"), _ptr(wk, "wk"), _ptr(wv, "wv"), _ptr(wg, "wg"),
+                               _ptr(wo, "wo"), _gammas(gammas, H), B, N, dm, H, dk, dv, int(chunk), float(k_scale),
+                               float(eps), int(bool(xpos)), int(pos_offset), float(theta_base), _ptr(out, "out"),
+                               _dt(out.dtype), _ptr(workspace, "workspace"), nbytes, _stream(stream)))
+    return out

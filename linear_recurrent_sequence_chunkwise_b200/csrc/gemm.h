@@ -32,6 +32,7 @@ struct GemmEpilogue {
     int M;                  // filled by launch_gemm
     int seq;                // rows are (batch, token) with token = row % seq
     int chunk;              // chunk length for the zeta of the keys
+    int xpos;               // rotations: 0 leaves the pairs unrotated
     long long pos_offset;
     double log2base;        // log2(theta_base)
     double log2g[kMaxHeads];

@@ -501,6 +501,29 @@ bool chunkwise_ws_supported(const RetArgs& a) {
     return true;
 }
 
+ret_status launch_chunkwise_main(const RetArgs& a, const void* q_src, const void* k_prime, cudaStream_t s) {
+    WsParams p;
+    const uint64_t B = a.B, N = a.N, H = a.H, dk = a.dk, dv = a.dv;
+    const uint64_t dq[4] = {dk, H, N, B};
+    const uint64_t sq[3] = {dk * 2, H * dk * 2, N * H * dk * 2};
+    const uint32_t box[4] = {64, 1, (uint32_t)kC, 1};
+    const uint64_t dvv[4] = {dv, H, N, B};
+    const uint64_t svv[3] = {dv * 2, H * dv * 2, N * H * dv * 2};
+    if (!make_tmap_bf16(&p.tq, q_src, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_bf16(&p.tk, k_prime, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_bf16(&p.tv, a.v, 4, dvv, svv, box, CU_TENSOR_MAP_SWIZZLE_128B))
+        return RET_ERR_CUDA;
+    p.out = a.out;
+    p.fstate = a.final_state;
+    p.N = a.N;
+    p.H = a.H;
+    p.dv = a.dv;
+    p.hc = a.hc;
+    const bool f32 = a.out_dt == RET_F32;
+    if (a.dk == 256) return f32 ? launch_main<256, float>(p, a, s) : launch_main<256, __nv_bfloat16>(p, a, s);
+    return f32 ? launch_main<128, float>(p, a, s) : launch_main<128, __nv_bfloat16>(p, a, s);
+}
+
 ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s) {
     const size_t qk = (size_t)a.B * a.N * a.H * a.dk;
     __nv_bfloat16* k_out = reinterpret_cast<__nv_bfloat16*>(ws);
@@ -515,28 +538,7 @@ ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s) {
                                                a.hc, a.B, a.N, a.H, a.chunk, a.xpos, a.pos_offset, lb);
     ret_status st = check_launch("chunkwise (workspace path): prep");
     if (st != RET_OK) return st;
-
-    WsParams p;
-    const uint64_t B = a.B, N = a.N, H = a.H, dk = a.dk, dv = a.dv;
-    const uint64_t dq[4] = {dk, H, N, B};
-    const uint64_t sq[3] = {dk * 2, H * dk * 2, N * H * dk * 2};
-    const uint32_t box[4] = {64, 1, (uint32_t)kC, 1};
-    const uint64_t dvv[4] = {dv, H, N, B};
-    const uint64_t svv[3] = {dv * 2, H * dv * 2, N * H * dv * 2};
-    const void* qsrc = a.xpos ? (const void*)q_rot : a.q;
-    if (!make_tmap_bf16(&p.tq, qsrc, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_bf16(&p.tk, k_out, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_bf16(&p.tv, a.v, 4, dvv, svv, box, CU_TENSOR_MAP_SWIZZLE_128B))
-        return RET_ERR_CUDA;
-    p.out = a.out;
-    p.fstate = a.final_state;
-    p.N = a.N;
-    p.H = a.H;
-    p.dv = a.dv;
-    p.hc = a.hc;
-    const bool f32 = a.out_dt == RET_F32;
-    if (a.dk == 256) return f32 ? launch_main<256, float>(p, a, s) : launch_main<256, __nv_bfloat16>(p, a, s);
-    return f32 ? launch_main<128, float>(p, a, s) : launch_main<128, __nv_bfloat16>(p, a, s);
+    return launch_chunkwise_main(a, a.xpos ? (const void*)q_rot : a.q, k_out, s);
 }
 
 }  // namespace ret

@@ -93,9 +93,11 @@ __device__ __forceinline__ void epi_store(const GemmEpilogue& e, int seg, int m,
 #pragma unroll
         for (int i = 0; i < 16; i++) {
             const int pidx = (d0 >> 1) + i;
-            const double theta = exp2(-2.0 * pidx / o.head_dim * e.log2base);
-            float sn, cs;
-            sincosf(rot_angle(e.pos_offset + n, theta), &sn, &cs);
+            float sn = 0.f, cs = 1.f;
+            if (e.xpos) {
+                const double theta = exp2(-2.0 * pidx / o.head_dim * e.log2base);
+                sincosf(rot_angle(e.pos_offset + n, theta), &sn, &cs);
+            }
             cs *= mult;
             sn *= mult;
             const float x0 = v[2 * i], x1 = v[2 * i + 1];
@@ -296,6 +298,17 @@ ret_status launch_gemm(const void* A, int M, int K, const GemmSegment* segs, int
         return check_launch("gemm: smem attribute");
     k_gemm<<<grid, kThreads, kSmemBytes, s>>>(p);
     return check_launch("gemm");
+}
+
+ret_status launch_linear(const void* X, const void* W, void* Y, int M, int N, int K, ret_dtype out_dt,
+                         cudaStream_t s) {
+    GemmSegment seg[1] = {{W, N}};
+    GemmEpilogue e;
+    memset(&e, 0, sizeof(e));
+    e.seg[0] = {Y, N, kEpiStore, out_dt, 1.f, 0};
+    e.seq = 1;
+    e.chunk = 1;
+    return launch_gemm(X, M, K, seg, 1, e, s);
 }
 
 }  // namespace ret

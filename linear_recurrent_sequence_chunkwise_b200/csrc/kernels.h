@@ -41,5 +41,23 @@ bool chunkwise_tc_supported(const RetArgs& a);
 bool chunkwise_ws_supported(const RetArgs& a);
 size_t chunkwise_ws_bytes(const RetArgs& a);
 ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s);
+// The tensor-core kernel alone, on prepared q_rot (or q) and k' (zeta-scaled keys).
+ret_status launch_chunkwise_main(const RetArgs& a, const void* q_rot, const void* k_prime, cudaStream_t s);
+
+struct MsrArgs {
+    const void *X, *Wq, *Wk, *Wv, *Wg, *Wo;
+    int B, N, dmodel, H, dk, dv, chunk;
+    double k_scale, eps;
+    int xpos;
+    long long pos_offset;
+    double theta_base;
+    HeadConsts hc;
+    void* out;
+    ret_dtype out_dt;
+    void* workspace;
+};
+size_t msr_workspace_bytes(int B, int N, int dmodel, int H, int dk, int dv);
+ret_status launch_msr(const MsrArgs& m, cudaStream_t s);
+ret_status launch_linear(const void* X, const void* W, void* Y, int M, int N, int K, ret_dtype out_dt, cudaStream_t s);
 
 }  // namespace ret

@@ -4,6 +4,7 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include "gemm.h"
 #include "kernels.h"
 
 namespace ret {
@@ -207,15 +208,83 @@ ret_status ret_decode_step(const void* q, const void* k, const void* v, const do
     return launch_decode(q, k, v, hc, state, out, B, H, dk, dv, in_dt, out_dt, stream);
 }
 
+size_t ret_msr_workspace_bytes(int B, int N, int dmodel, int H, int dk, int dv) {
+    if (B < 1 || N < 1 || dmodel < 1 || H < 1 || dk < 1 || dv < 1) return 0;
+    return msr_workspace_bytes(B, N, dmodel, H, dk, dv);
+}
+
+ret_status ret_msr_forward(const void* X, const void* Wq, const void* Wk, const void* Wv, const void* Wg,
+                           const void* Wo, const double* gammas, int B, int N, int dmodel, int H, int dk, int dv,
+                           int chunk, double k_scale, double eps, int xpos, int64_t pos_offset, double theta_base,
+                           void* out, ret_dtype out_dt, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+    t_err[0] = 0;
+    const char* who = "ret_msr_forward";
+    for (const void* ptr : {X, Wq, Wk, Wv, Wg, Wo, (const void*)out, (const void*)workspace})
+        if (!ptr) return fail(RET_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
+    for (const void* ptr : {X, Wq, Wk, Wv, Wg, Wo, (const void*)out})
+        if (!aligned(ptr, 16)) return fail(RET_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    if (!aligned(workspace, 256)) return fail(RET_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+    if (B < 1 || N < 1 || dmodel < 1 || H < 1 || dk < 1 || dv < 1 || chunk < 1)
+        return fail(RET_ERR_INVALID_ARG, "%s: sizes must be >= 1", who);
+    if (!is_dtype(out_dt)) return fail(RET_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    ret_status st = check_gammas(gammas, H, who);
+    if (st != RET_OK) return st;
+    if (dmodel % 8) return fail(RET_ERR_INVALID_ARG, "%s: d_model must be a multiple of 8", who);
+    if (!(eps >= 0.0) || !isfinite(k_scale)) return fail(RET_ERR_INVALID_ARG, "%s: bad eps or k_scale", who);
+    if (xpos && !(theta_base > 0.0 && isfinite(theta_base)))
+        return fail(RET_ERR_INVALID_ARG, "%s: theta_base must be finite and > 0", who);
+    const size_t need = msr_workspace_bytes(B, N, dmodel, H, dk, dv);
+    if (workspace_bytes < need)
+        return fail(RET_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed (got %zu)", who, need, workspace_bytes);
+    const size_t M = (size_t)B * N;
+    const size_t bx = M * dmodel * 2, bo = M * dmodel * (out_dt == RET_F32 ? 4 : 2);
+    if (overlaps(out, bo, X, bx) || overlaps(workspace, need, X, bx) || overlaps(workspace, need, out, bo))
+        return fail(RET_ERR_INVALID_ARG, "%s: out or workspace overlaps another buffer", who);
+    MsrArgs m;
+    m.X = X; m.Wq = Wq; m.Wk = Wk; m.Wv = Wv; m.Wg = Wg; m.Wo = Wo;
+    m.B = B; m.N = N; m.dmodel = dmodel; m.H = H; m.dk = dk; m.dv = dv; m.chunk = chunk;
+    m.k_scale = k_scale; m.eps = eps; m.xpos = xpos ? 1 : 0; m.pos_offset = pos_offset;
+    m.theta_base = xpos ? theta_base : 10000.0;
+    make_head_consts(gammas, H, &m.hc);
+    m.out = out; m.out_dt = out_dt; m.workspace = workspace;
+    // the retention step runs on the tensor-core kernel only
+    RetArgs a;
+    a.in_dt = RET_BF16; a.chunk = chunk; a.dk = dk; a.dv = dv; a.N = N; a.H = H; a.hc = m.hc;
+    if (!chunkwise_ws_supported(a))
+        return fail(RET_ERR_UNSUPPORTED, "%s: needs chunk 128, d_k 128 or 256, d_v a multiple of 64 and "
+                    "gamma_h^128 >= 2^-60", who);
+    if (!(dv == 128 || dv == 256 || dv == 512 || dv == 1024))
+        return fail(RET_ERR_UNSUPPORTED, "%s: d_v must be 128, 256, 512 or 1024", who);
+    return launch_msr(m, stream);
+}
+
+ret_status ret_linear_bf16(const void* X, const void* W, void* Y, int M, int N, int K, ret_dtype out_dt,
+                           cudaStream_t stream) {
+    t_err[0] = 0;
+    const char* who = "ret_linear_bf16";
+    if (!X || !W || !Y) return fail(RET_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
+    if (M < 1 || N < 1 || K < 1) return fail(RET_ERR_INVALID_ARG, "%s: sizes must be >= 1", who);
+    if (N % 8 || K % 8) return fail(RET_ERR_INVALID_ARG, "%s: N and K must be multiples of 8", who);
+    if (!is_dtype(out_dt)) return fail(RET_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    for (const void* ptr : {X, W, (const void*)Y})
+        if (!aligned(ptr, 16)) return fail(RET_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    const size_t by = (size_t)M * N * (out_dt == RET_F32 ? 4 : 2);
+    if (overlaps(Y, by, X, (size_t)M * K * 2) || overlaps(Y, by, W, (size_t)K * N * 2))
+        return fail(RET_ERR_INVALID_ARG, "%s: Y overlaps an input", who);
+    return launch_linear(X, W, Y, M, N, K, out_dt, stream);
+}
+
 ret_status ret_check_device_error(cudaStream_t stream) {
     t_err[0] = 0;
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return fail(RET_ERR_CUDA, "ret_check_device_error: %s", cudaGetErrorString(e));
-    int flag = 0, flag2 = 0;
+    int flag = 0, flag2 = 0, flag3 = 0;
     e = read_clear_error_chunk_tc(&flag);
     if (e == cudaSuccess) e = read_clear_error_chunk_ws(&flag2);
+    if (e == cudaSuccess) e = read_clear_error_gemm(&flag3);
     if (e != cudaSuccess) return fail(RET_ERR_CUDA, "ret_check_device_error: %s", cudaGetErrorString(e));
-    flag |= flag2;
+    flag |= flag2 | flag3;
     if (flag) return fail(RET_ERR_TIMEOUT, "a kernel gave up a bounded wait (device error word %d)", flag);
     return RET_OK;
 }
