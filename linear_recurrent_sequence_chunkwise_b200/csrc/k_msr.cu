@@ -52,14 +52,14 @@ __global__ void __launch_bounds__(256) k_gn_gate(const float* __restrict__ Y, __
     for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
     const float rstd = rsqrtf(q / dv + eps);
 #pragma unroll
-    for (int i = 0; i < PER; i += 8) {
-        uint4 gw = *reinterpret_cast<const uint4*>(g + i);
+    for (int i = 0; i < PER; i += 4) {  // 4 bf16 = 8 bytes, aligned since PER is a multiple of 4
+        uint2 gw = *reinterpret_cast<const uint2*>(g + i);
         __nv_bfloat16* gb = reinterpret_cast<__nv_bfloat16*>(&gw);
-        uint4 zw;
+        uint2 zw;
         __nv_bfloat16* zb = reinterpret_cast<__nv_bfloat16*>(&zw);
 #pragma unroll
-        for (int e = 0; e < 8; e++) zb[e] = __float2bfloat16_rn(__bfloat162float(gb[e]) * (v[i + e] - mu) * rstd);
-        *reinterpret_cast<uint4*>(g + i) = zw;
+        for (int e = 0; e < 4; e++) zb[e] = __float2bfloat16_rn(__bfloat162float(gb[e]) * (v[i + e] - mu) * rstd);
+        *reinterpret_cast<uint2*>(g + i) = zw;
     }
 }
 
