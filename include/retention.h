@@ -128,6 +128,36 @@ ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
                                     size_t workspace_bytes);
 
 /*
+ * Allocation-free variant of ret_forward_chunkwise_ws, for callers that
+ * cannot allocate device memory at call time: for example a plug-in that runs
+ * inside a host framework which owns all device memory and hands out no
+ * allocator, or a service that fixes its memory footprint at start-up and
+ * forbids allocation afterwards.  The pages have no counterpart; this is a
+ * deployment convenience of this library.
+ * Same arguments and results as ret_forward_chunkwise (the caller still
+ * passes every input and output buffer); the scratch of the workspace path
+ * is a fixed device array inside the library, of
+ * ret_chunkwise_noalloc_max_bytes() bytes (64 MiB) on every GPU that loads
+ * the library, held until the process exits.  Problems needing more scratch
+ * than that (B*N*H*dk*4 bytes with xpos, B*N*H*dk*2 without) return
+ * RET_ERR_INVALID_ARG, shapes outside the workspace path RET_ERR_UNSUPPORTED;
+ * nothing is allocated in either case.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array and leave their scratch in it;
+ * nothing in it needs to start at zero.  Calls whose kernels overlap on the
+ * GPU (other streams, other host threads) race on the array: serialise them.
+ */
+ret_status ret_forward_chunkwise_noalloc(const void* q, const void* k, const void* v,
+                                         const double* gammas, int B, int N, int H, int dk, int dv,
+                                         int chunk, void* out, float* final_state,
+                                         cudaStream_t stream, ret_dtype in_dt, ret_dtype out_dt,
+                                         int xpos, int64_t pos_offset, double theta_base);
+
+/* Size in bytes of the fixed scratch array of ret_forward_chunkwise_noalloc. */
+size_t ret_chunkwise_noalloc_max_bytes(void);
+
+/*
  * One recurrent decode step, state updated in place.
  * "Hybrid Architectures ...", sections 2.1 and 5.2; RetNet paper summary,
  * recurrent representation and inference protocol:

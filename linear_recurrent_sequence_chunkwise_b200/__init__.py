@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "RetentionError", "lib", "ret_xpos_rotate", "ret_forward_chunkwise", "ret_forward_chunkwise_ws",
-    "ret_chunkwise_workspace_bytes", "ret_decode_step", "ret_msr_forward", "ret_msr_workspace_bytes",
+    "ret_chunkwise_workspace_bytes", "ret_forward_chunkwise_noalloc", "ret_chunkwise_noalloc_max_bytes",
+    "ret_decode_step", "ret_msr_forward", "ret_msr_workspace_bytes",
     "ret_linear_bf16",
     "ret_forward_parallel", "ret_forward_recurrent", "ret_check_device_error", "ret_last_error_string",
     "RET_OK", "RET_ERR_INVALID_ARG", "RET_ERR_UNSUPPORTED", "RET_ERR_CUDA", "RET_ERR_TIMEOUT",
@@ -52,6 +53,9 @@ def _load_library():
     L.ret_forward_chunkwise.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d]
     L.ret_forward_chunkwise_ws.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d, vp,
                                            ctypes.c_size_t]
+    L.ret_forward_chunkwise_noalloc.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d]
+    L.ret_chunkwise_noalloc_max_bytes.argtypes = []
+    L.ret_chunkwise_noalloc_max_bytes.restype = ctypes.c_size_t
     L.ret_chunkwise_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
     L.ret_chunkwise_workspace_bytes.restype = ctypes.c_size_t
     L.ret_decode_step.argtypes = [vp, vp, vp, dp, vp, vp, vp, i, i, i, i, i, i]
@@ -65,7 +69,8 @@ def _load_library():
     L.ret_check_device_error.argtypes = [vp]
     L.ret_last_error_string.restype = ctypes.c_char_p
     L.ret_last_error_string.argtypes = []
-    for name in ("ret_xpos_rotate", "ret_forward_chunkwise", "ret_forward_chunkwise_ws", "ret_decode_step",
+    for name in ("ret_xpos_rotate", "ret_forward_chunkwise", "ret_forward_chunkwise_ws",
+                 "ret_forward_chunkwise_noalloc", "ret_decode_step",
                  "ret_forward_parallel",
                  "ret_forward_recurrent", "ret_check_device_error", "ret_msr_forward", "ret_linear_bf16"):
         getattr(L, name).restype = ctypes.c_int
@@ -175,6 +180,31 @@ def ret_forward_chunkwise_ws(q, k, v, gammas, chunk: int, workspace, out=None, f
                                         dv, int(chunk), _ptr(out, "out"), _ptr(final_state, "final_state"),
                                         _stream(stream), _dt(q.dtype), _dt(out.dtype), int(bool(xpos)),
                                         int(pos_offset), float(theta_base), _ptr(workspace, "workspace"), nbytes))
+    return (out, final_state) if final_state is not None else out
+
+
+def ret_chunkwise_noalloc_max_bytes() -> int:
+    """Bytes of the library's fixed scratch array used by
+    ret_forward_chunkwise_noalloc."""
+    return int(lib.ret_chunkwise_noalloc_max_bytes())
+
+
+def ret_forward_chunkwise_noalloc(q, k, v, gammas, chunk: int, out=None, final_state=None, out_dtype=None,
+                                  xpos: bool = False, pos_offset: int = 0, theta_base: float = 10000.0,
+                                  want_final_state: bool = False, stream=None):
+    """Chunkwise forward whose scratch is a fixed device array inside the
+    library: for callers that cannot allocate device memory at call time.
+    Pass ``out`` / ``final_state`` to avoid the allocations this wrapper would
+    otherwise make for them."""
+    B, N, H, dk, dv = _seq_shapes(q, k, v)
+    if out is None:
+        out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
+    if final_state is None and want_final_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check(lib.ret_forward_chunkwise_noalloc(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N,
+                                             H, dk, dv, int(chunk), _ptr(out, "out"),
+                                             _ptr(final_state, "final_state"), _stream(stream), _dt(q.dtype),
+                                             _dt(out.dtype), int(bool(xpos)), int(pos_offset), float(theta_base)))
     return (out, final_state) if final_state is not None else out
 
 

@@ -32,6 +32,8 @@
 //    R [384,512).  The tensor core computes Q K'^T of chunk j+1 while the
 //    warpgroup stores chunk j's output; the serial chain between chunks is
 //    state MMA -> state rescale -> next state MMA.
+#include <mutex>
+
 #include "kernels.h"
 #include "tc_util.cuh"
 #include "tmap.h"
@@ -539,6 +541,57 @@ ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s) {
     ret_status st = check_launch("chunkwise (workspace path): prep");
     if (st != RET_OK) return st;
     return launch_chunkwise_main(a, a.xpos ? (const void*)q_rot : a.q, k_out, s);
+}
+
+// ------------------------------------------------- allocation-free variant
+//
+// For callers that cannot allocate device memory at call time (for example a
+// plug-in running inside a host framework that owns all device memory and
+// hands out no allocator, or a deployment that fixes its memory footprint at
+// start-up and forbids allocation afterwards), the workspace path can run on
+// a file-scope device array instead of a caller-provided buffer.  Every GPU
+// that loads the library holds this array until the process exits.
+
+constexpr size_t kStaticWsBytes = 64ull << 20;  // 64 MiB
+static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
+
+size_t chunkwise_static_ws_bytes() { return kStaticWsBytes; }
+
+// Device address of g_static_ws on the current device, looked up once per
+// device (the host-side symbol is only a stand-in for the device address).
+static ret_status static_ws_address(void** out) {
+    constexpr int kMaxDev = 64;
+    static void* addr[kMaxDev] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "static workspace: cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDev) return fail(RET_ERR_UNSUPPORTED, "static workspace: device %d out of range", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_ws);
+        if (e != cudaSuccess || !p)
+            return fail(RET_ERR_CUDA, "static workspace: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return RET_OK;
+}
+
+ret_status launch_chunkwise_static(const RetArgs& a, cudaStream_t s) {
+    const size_t need = chunkwise_ws_bytes(a);
+    if (need > kStaticWsBytes)
+        return fail(RET_ERR_INVALID_ARG,
+                    "ret_forward_chunkwise_noalloc: this problem needs %zu bytes of scratch, above the fixed %zu "
+                    "(B*N*H*dk*%d bytes must not exceed it)",
+                    need, kStaticWsBytes, a.xpos ? 4 : 2);
+    void* ws = nullptr;
+    ret_status st = static_ws_address(&ws);
+    if (st != RET_OK) return st;
+    // Nothing in the scratch needs to start at zero: the prep pass writes every
+    // byte the tensor-core kernel reads.
+    return launch_chunkwise_ws(a, ws, s);
 }
 
 }  // namespace ret

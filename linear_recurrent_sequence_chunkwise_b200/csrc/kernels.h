@@ -41,6 +41,9 @@ bool chunkwise_tc_supported(const RetArgs& a);
 bool chunkwise_ws_supported(const RetArgs& a);
 size_t chunkwise_ws_bytes(const RetArgs& a);
 ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s);
+// The workspace path on the library's fixed device array (no allocation).
+size_t chunkwise_static_ws_bytes();
+ret_status launch_chunkwise_static(const RetArgs& a, cudaStream_t s);
 // The tensor-core kernel alone, on prepared q_rot (or q) and k' (zeta-scaled keys).
 ret_status launch_chunkwise_main(const RetArgs& a, const void* q_rot, const void* k_prime, cudaStream_t s);
 

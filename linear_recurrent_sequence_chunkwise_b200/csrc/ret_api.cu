@@ -163,6 +163,24 @@ ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
     return launch_chunkwise_ws(a, workspace, stream);
 }
 
+ret_status ret_forward_chunkwise_noalloc(const void* q, const void* k, const void* v, const double* gammas, int B,
+                                         int N, int H, int dk, int dv, int chunk, void* out, float* final_state,
+                                         cudaStream_t stream, ret_dtype in_dt, ret_dtype out_dt, int xpos,
+                                         int64_t pos_offset, double theta_base) {
+    t_err[0] = 0;
+    RetArgs a;
+    ret_status st = make_args(&a, "ret_forward_chunkwise_noalloc", q, k, v, gammas, B, N, H, dk, dv, chunk, out,
+                              final_state, in_dt, out_dt, xpos, pos_offset, theta_base);
+    if (st != RET_OK) return st;
+    if (!chunkwise_ws_supported(a))
+        return fail(RET_ERR_UNSUPPORTED,
+                    "ret_forward_chunkwise_noalloc: needs bf16 inputs, chunk 128, dk 128 or 256, dv a multiple of "
+                    "64 and every gamma_h^128 >= 2^-60");
+    return launch_chunkwise_static(a, stream);
+}
+
+size_t ret_chunkwise_noalloc_max_bytes(void) { return chunkwise_static_ws_bytes(); }
+
 ret_status ret_forward_parallel(const void* q, const void* k, const void* v, const double* gammas, int B, int N,
                                 int H, int dk, int dv, void* out, cudaStream_t stream, ret_dtype in_dt,
                                 ret_dtype out_dt, int xpos, int64_t pos_offset, double theta_base) {
