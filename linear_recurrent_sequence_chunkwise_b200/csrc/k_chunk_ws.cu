@@ -14,24 +14,31 @@
 //    cosine of each (position, pair) evaluated once for all heads), scales
 //    each rotated key row by its zeta, and writes q_rot and k' (bf16) into the
 //    workspace.  Without rotation only k' is written and q is read in place.
-// 2. k_chunkwise_ws: one CTA per (batch, head, 64 value columns), three roles
+// 2. k_chunkwise_ws: one CTA per (batch, head, 64 value columns), 16 warps
+//    in four roles (registers rebalanced with setmaxnreg):
 //      warp 0  TMA producer: L2 prefetch two chunks ahead (the CTAs of a
-//              head split the boxes), then per chunk the Q tile into a staging buffer, the
-//              K' tile in parts of 128 d_k rows through a 3-slot ring, and
-//              the V tile (2 slots);
-//      warp 1  MMA issuer (one thread), A operands from TMEM where possible:
-//                A  = Q K'^T          (Q from TMEM, K' from smem)
-//                O  = Q T  + P V      (Q and P from TMEM, T and V from smem)
-//                R += K'^T V          (fp32 state in TMEM)
-//      warps 2-9 (two warpgroups on TMEM lanes 0..127, one column half each):
-//                Q staging -> TMEM (frees the 64 KB staging buffer early),
+//              head split the boxes), then per chunk the Q tile into a
+//              staging buffer, the K' tile in parts of 128 d_k rows through
+//              a 3-slot ring, and the V tile (2 slots);
+//      warp 1  tensor pipe (one elected lane issues), per chunk j
+//                A  = Q K'^T          (Q from TMEM, K' from smem), part by
+//                                     part, each part but the last followed
+//                                     by its dS = K'^T V (frees the K' slot)
+//                O  = Q T             (read-out of the state before chunk j)
+//                dS of the last part, then O += P V (P from TMEM);
+//      warps 4-7 (Q warpgroup): the staged Q of chunk j+1 -> registers as
+//                soon as it lands, -> TMEM once the read-out of chunk j is
+//                done; a plain smem read keeps the load traffic on the TMA
+//                path (per-row global loads from these threads measurably
+//                slow the tensor pipe down);
+//      warps 8-15 (two warpgroups on TMEM lanes 0..127, one column half each):
 //                mask:     P = tril(A) -> packed bf16 in TMEM,
-//                state:    T = gamma^L R -> TMEM (fp32) and smem (bf16),
+//                state:    R = gamma^L R + dS in registers (fp32), then the
+//                          bf16 T = gamma^L' R into smem for the next read-out,
 //                epilogue: out = gamma^(r+1-L) O -> global.
 //    TMEM columns: A [0,128), P [128,192), O [192,256), Q [256,384),
-//    R [384,512).  The tensor core computes Q K'^T of chunk j+1 while the
-//    warpgroup stores chunk j's output; the serial chain between chunks is
-//    state MMA -> state rescale -> next state MMA.
+//    dS [384,512).  Every hand-off between the roles has at least one block
+//    of MMAs in between, so no role waits on another in the steady state.
 #include <mutex>
 
 #include "kernels.h"
@@ -57,7 +64,7 @@ constexpr int kC = 128;           // chunk rows (M of every MMA)
 constexpr int kW = 64;            // d_v columns per CTA
 constexpr int kPartDk = 128;      // d_k rows per pipeline part (one state block)
 constexpr int kVBytes = kC * kW * 2;              // 16 KB
-constexpr int kThreads = 320;   // TMA warp, MMA warp, two transform warpgroups
+constexpr int kThreads = 512;   // control warpgroup (TMA, MMA), Q warpgroup, two transform warpgroups
 
 // ------------------------------------------------------------------ prep
 
@@ -140,14 +147,29 @@ struct WsSmem {
 // bf16, the A operand of Q K'^T and of the read-out), dS = K'^T V (fp32).
 constexpr uint32_t kTA = 0, kTP = 128, kTO = 192, kTQ = 256, kTD = 384;
 
+// Per-thread register budgets of the three warpgroup roles.  The block is
+// launched with 512 threads x 128 registers (ptxas reports 128 for every
+// instance); the budgets add up to 128 * (72 + 136) + 256 * 152 = 65536.
+constexpr int kRegsCtl = 72, kRegsQ = 136, kRegsXf = 152;
+static_assert(128 * (kRegsCtl + kRegsQ) + 256 * kRegsXf <= 512 * 128, "register split exceeds the launch allocation");
+
 struct Bars {
     uint64_t qfull, qempty, kfull[kKSlots], kempty[kKSlots], vfull[2], vempty[2];
-    uint64_t qready, qfree, afull, aread, pready, dsdone, dsfree, tready, ofull, ofree;
+    uint64_t qready, qtm, afull, aread, pready, dsdone, dsfree, tready, ofull, ofree;
 };
 
 __device__ __forceinline__ void elect_arrive(uint64_t* bar, int lane) {
     __syncwarp();
     if (lane == 0) tc::mbar_arrive(bar);
+}
+
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 template <int DK, typename Tout>
@@ -165,11 +187,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
     const int N = p.N;
     const int nchunks = (N + kC - 1) / kC;
     const double lg = p.hc.log2g[h];
-    constexpr int kTG = 8;  // transform warps arriving on the warpgroup barriers
+    constexpr int kXfWarps = 8;  // transform warps arriving on the warpgroup barriers
 
     if (tid == 0) {
         tc::mbar_init(&bars.qfull, 1);
-        tc::mbar_init(&bars.qempty, kTG);
+        tc::mbar_init(&bars.qempty, 4);
         for (int i = 0; i < kKSlots; i++) {
             tc::mbar_init(&bars.kfull[i], 1);
             tc::mbar_init(&bars.kempty[i], 1);
@@ -178,16 +200,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             tc::mbar_init(&bars.vfull[i], 1);
             tc::mbar_init(&bars.vempty[i], 1);
         }
-        tc::mbar_init(&bars.qready, kTG);
-        tc::mbar_init(&bars.qfree, 1);
+        tc::mbar_init(&bars.qready, 4);
+        tc::mbar_init(&bars.qtm, 1);
         tc::mbar_init(&bars.afull, 1);
-        tc::mbar_init(&bars.aread, kTG);
-        tc::mbar_init(&bars.pready, kTG);
+        tc::mbar_init(&bars.aread, kXfWarps);
+        tc::mbar_init(&bars.pready, kXfWarps);
         tc::mbar_init(&bars.dsdone, 1);
-        tc::mbar_init(&bars.dsfree, kTG);
-        tc::mbar_init(&bars.tready, kTG);
+        tc::mbar_init(&bars.dsfree, kXfWarps);
+        tc::mbar_init(&bars.tready, kXfWarps);
         tc::mbar_init(&bars.ofull, 1);
-        tc::mbar_init(&bars.ofree, kTG);
+        tc::mbar_init(&bars.ofree, kXfWarps);
         s_fail = 0;
         tc::fence_barrier_init();
         tc::prefetch_tmap(&p.tq);
@@ -201,9 +223,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
     const uint32_t tb = s_tmem;
     bool ok = true;
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        if (lane == 0) {
+    if (warp < 4) {
+        regs_dec<kRegsCtl>();
+        if (warp == 0 && lane == 0) {
+            // -------------------------------------------- TMA producer
             // L2 prefetch of chunk jp: the CTAs of one head split the Q and K'
             // boxes between them; each prefetches its own V tile.
             auto prefetch = [&](int jp) {
@@ -213,6 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                     tc::tma_prefetch_l2_4d(i < kQSlabs ? &p.tq : &p.tk, 64 * (i % kQSlabs), h, n0p, b);
                 tc::tma_prefetch_l2_4d(&p.tv, j0, h, n0p, b);
             };
+            prefetch(0);
             prefetch(1);
             for (int jc = 0; jc < nchunks && ok; jc++) {
                 const int n0 = jc * kC;
@@ -238,159 +262,200 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 tc::mbar_arrive_expect_tx(&bars.vfull[vs], kVBytes);
                 tc::tma_load_4d(sm + WsSmem<DK>::kV + vs * kVBytes, &p.tv, &bars.vfull[vs], j0, h, n0, b);
             }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        } else if (warp == 1) {
+            // --------------------------------------------- tensor pipe
+            // The whole warp walks the loop (warp-uniform descriptors); one
+            // elected lane issues each tcgen05 instruction.
             const uint32_t id_qk = tc::idesc_bf16_f32(128, 128, 0, 0);
             const uint32_t id_qt = tc::idesc_bf16_f32(128, kW, 0, 1);
             const uint32_t id_st = tc::idesc_bf16_f32(128, kW, 1, 1);
             const uint32_t id_pv = tc::idesc_bf16_f32(128, kW, 0, 1);
-            const uint32_t k0 = tc::smem_u32(sm + WsSmem<DK>::kK);
-            const uint32_t v0 = tc::smem_u32(sm + WsSmem<DK>::kV);
-            const uint32_t t0 = tc::smem_u32(sm + WsSmem<DK>::kT);
+            // descriptor bases; offsets are added in 16-byte units
+            const uint64_t dk_k = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kK), 16, 1024);         // K' as B, K-major
+            const uint64_t dk_mn = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kK), kC * 128, 1024);  // K'^T as A, MN-major
+            const uint64_t dv_mn = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kV), kC * 128, 1024);  // V as B, MN-major
+            const uint64_t dt_mn = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kT), DK * 128, 1024);  // T as B, MN-major
+            // a timed-out wait must leave the warp converged for elect.sync
+            auto wait = [&](uint64_t* bar, uint32_t parity) {
+                return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity));
+            };
+            // Per chunk: A = Q K'^T part by part with dS = K'^T V of every part
+            // but the last right behind it (so each K' part is released early),
+            // then the read-out O = Q T, the last dS part, and O += P V.
             for (int jc = 0; jc < nchunks && ok; jc++) {
-                // ---- A = Q K'^T  (Q from TMEM)
-                ok = tc::mbar_wait(&bars.qready, jc & 1);
-                if (ok && jc > 0) ok = tc::mbar_wait(&bars.aread, (jc - 1) & 1);
+                const uint32_t vo = (uint32_t)((jc & 1) * kVBytes) >> 4;
+                ok = wait(&bars.qready, jc & 1);
+                if (ok && jc > 0) ok = wait(&bars.aread, (jc - 1) & 1);
+                if (!ok) break;
+                auto ds_part = [&](int part) -> bool {  // dS rows of this d_k part = K'^T V
+                    if (part == 0) {  // V landed, previous dS read out of TMEM
+                        if (!wait(&bars.vfull[jc & 1], (jc >> 1) & 1)) return false;
+                        if (jc > 0 && !wait(&bars.dsfree, (jc - 1) & 1)) return false;
+                        tc::tc_fence_after();
+                    }
+                    const int g = jc * kParts + part, slot = g % kKSlots;
+                    const uint32_t ko = (uint32_t)(slot * kKPartBytes) >> 4;
+#pragma unroll
+                    for (int k = 0; k < kC / 16; k++)
+                        tc::mma_bf16_ss_elect(tb + kTD + part * kW, dk_mn + ko + (uint32_t)((k * 2048) >> 4),
+                                              dv_mn + vo + (uint32_t)((k * 2048) >> 4), id_st, k > 0);
+                    tc::mma_commit_elect(&bars.kempty[slot]);
+                    return true;
+                };
                 for (int part = 0; part < kParts && ok; part++) {
                     const int g = jc * kParts + part, slot = g % kKSlots, u = g / kKSlots;
-                    ok = tc::mbar_wait(&bars.kfull[slot], u & 1);
+                    ok = wait(&bars.kfull[slot], u & 1);
                     if (!ok) break;
                     tc::tc_fence_after();
-                    const uint32_t kb = k0 + slot * kKPartBytes;
-                    for (int k = 0; k < kPartDk / 16; k++) {
-                        const uint32_t off = (k / 4) * (kC * 128) + (k % 4) * 32;
-                        tc::mma_bf16_ts(tb + kTA, tb + kTQ + 64 * part + 8 * k, tc::sdesc_sw128(kb + off, 16, 1024),
-                                        id_qk, (part > 0) || (k > 0));
-                    }
+                    const uint32_t ko = (uint32_t)(slot * kKPartBytes) >> 4;
+#pragma unroll
+                    for (int k = 0; k < kPartDk / 16; k++)
+                        tc::mma_bf16_ts_elect(tb + kTA, tb + kTQ + 64 * part + 8 * k,
+                                              dk_k + ko + (uint32_t)(((k / 4) * (kC * 128) + (k % 4) * 32) >> 4),
+                                              id_qk, (part > 0) || (k > 0));
+                    if (part + 1 < kParts) ok = ds_part(part);
                 }
                 if (!ok) break;
-                tc::mma_commit(&bars.afull);
+                tc::mma_commit_elect(&bars.afull);
                 // ---- O = Q T  (read-out of the state before this chunk)
                 if (jc > 0) {
-                    ok = tc::mbar_wait(&bars.tready, (jc - 1) & 1);
-                    if (ok) ok = tc::mbar_wait(&bars.ofree, (jc - 1) & 1);
+                    ok = wait(&bars.tready, (jc - 1) & 1);
+                    if (ok) ok = wait(&bars.ofree, (jc - 1) & 1);
                     if (!ok) break;
                     tc::tc_fence_after();
+#pragma unroll 4
                     for (int k = 0; k < DK / 16; k++)
-                        tc::mma_bf16_ts(tb + kTO, tb + kTQ + 8 * k,
-                                        tc::sdesc_sw128(t0 + 16 * k * 128, DK * 128, 1024), id_qt, k > 0);
+                        tc::mma_bf16_ts_elect(tb + kTO, tb + kTQ + 8 * k, dt_mn + (uint32_t)((16 * k * 128) >> 4),
+                                              id_qt, k > 0);
                 }
-                tc::mma_commit(&bars.qfree);
-                // ---- dS = K'^T V
-                ok = tc::mbar_wait(&bars.vfull[jc & 1], (jc >> 1) & 1);
-                if (ok && jc > 0) ok = tc::mbar_wait(&bars.dsfree, (jc - 1) & 1);
+                tc::mma_commit_elect(&bars.qtm);  // Q in TMEM and T in smem are read
+                ok = ds_part(kParts - 1);
                 if (!ok) break;
-                tc::tc_fence_after();
-                const uint32_t vb = v0 + (jc & 1) * kVBytes;
-                for (int part = 0; part < kParts; part++) {
-                    const int g = jc * kParts + part, slot = g % kKSlots;
-                    const uint32_t kb = k0 + slot * kKPartBytes;
-                    for (int k = 0; k < kC / 16; k++)
-                        tc::mma_bf16_ss(tb + kTD + part * kW, tc::sdesc_sw128(kb + k * 2048, kC * 128, 1024),
-                                        tc::sdesc_sw128(vb + k * 2048, kC * 128, 1024), id_st, k > 0);
-                    tc::mma_commit(&bars.kempty[slot]);
-                }
-                tc::mma_commit(&bars.dsdone);
+                tc::mma_commit_elect(&bars.dsdone);
                 // ---- O += P V  (P from TMEM)
-                ok = tc::mbar_wait(&bars.pready, jc & 1);
+                ok = wait(&bars.pready, jc & 1);
                 if (!ok) break;
                 tc::tc_fence_after();
+#pragma unroll
                 for (int k = 0; k < kC / 16; k++)
-                    tc::mma_bf16_ts(tb + kTO, tb + kTP + 8 * k, tc::sdesc_sw128(vb + k * 2048, kC * 128, 1024), id_pv,
-                                    (jc > 0) || (k > 0));
-                tc::mma_commit(&bars.ofull);
-                tc::mma_commit(&bars.vempty[jc & 1]);
+                    tc::mma_bf16_ts_elect(tb + kTO, tb + kTP + 8 * k, dv_mn + vo + (uint32_t)((k * 2048) >> 4), id_pv,
+                                          (jc > 0) || (k > 0));
+                tc::mma_commit_elect(&bars.ofull);
+                tc::mma_commit_elect(&bars.vempty[jc & 1]);
             }
+        }
+    } else if (warp < 8) {
+        // ------------------------------------------------- Q warpgroup
+        // Thread r copies row r of the next chunk's Q from the staging buffer
+        // into registers as soon as it lands (freeing the buffer for the
+        // chunk after), and writes it into TMEM columns [kTQ, kTQ + DK/2)
+        // once the read-out of the current chunk has consumed the previous
+        // one.  Rows past the end arrive as zeros from the TMA fill.
+        regs_inc<kRegsQ>();
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const uint8_t* sQ = sm + WsSmem<DK>::kQ;
+        uint4 qv[DK / 8];
+        for (int jq = 0; jq < nchunks && ok; jq++) {
+            ok = tc::mbar_wait(&bars.qfull, jq & 1);
+            if (!ok) break;
+#pragma unroll
+            for (int s = 0; s < kQSlabs; s++)
+#pragma unroll
+                for (int c16 = 0; c16 < 8; c16++)
+                    qv[8 * s + c16] = *reinterpret_cast<const uint4*>(sQ + s * (kC * 128) +
+                                                                      tc::sw128_off((uint32_t)r, (uint32_t)c16));
+            // The buffer is handed back to the TMA only once every load has
+            // landed in registers: an arrive right behind the loads can let
+            // the next tile's bulk copy overwrite data a load has not read
+            // yet.  Consuming one word of each load makes the warp wait for
+            // them; the proxy fence orders them before the async-proxy write.
+            {
+                uint32_t dep = 0;
+#pragma unroll
+                for (int i = 0; i < DK / 8; i++) dep ^= qv[i].x;
+                asm volatile("" ::"r"(dep));
+            }
+            tc::fence_proxy_async_smem();
+            elect_arrive(&bars.qempty, lane);
+            if (jq > 0) ok = tc::mbar_wait(&bars.qtm, (jq - 1) & 1);
+            if (!ok) break;
+            tc::tc_fence_after();
+#pragma unroll
+            for (int g = 0; g < DK / 64; g++) {
+                uint32_t w[32];
+#pragma unroll
+                for (int k = 0; k < 8; k++) {
+                    w[4 * k + 0] = qv[8 * g + k].x;
+                    w[4 * k + 1] = qv[8 * g + k].y;
+                    w[4 * k + 2] = qv[8 * g + k].z;
+                    w[4 * k + 3] = qv[8 * g + k].w;
+                }
+                tc::tmem_st32(tb + lane_off + kTQ + 32 * g, w);
+            }
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            elect_arrive(&bars.qready, lane);
         }
     } else {
         // ------------------------------------------ transform warpgroups
-        // Warps 2-5 and 6-9 form two warpgroups; each covers TMEM lanes
+        // Warps 8-11 and 12-15 form two warpgroups; each covers TMEM lanes
         // 0..127 (a warp reaches the lane quarter warp % 4) and takes one half
         // of the columns of every phase.  The fp32 state R lives in their
         // registers: row r of every 128-row block, 32 columns each.
+        regs_inc<kRegsXf>();
         const int quarter = warp & 3;                 // TMEM lanes 32*quarter ..
-        const int wg = (warp - 2) >> 2;               // column half
+        const int wg = (warp - 8) >> 2;               // column half
         const int r = quarter * 32 + lane;            // chunk row / state row in a block
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         uint8_t* sT = sm + WsSmem<DK>::kT;
-        const uint8_t* sQ = sm + WsSmem<DK>::kQ;
         float R[kParts][32];
 #pragma unroll
         for (int part = 0; part < kParts; part++)
 #pragma unroll
             for (int i = 0; i < 32; i++) R[part][i] = 0.f;
+        // decay powers of a full chunk and of the (possibly shorter) last one
+        const int L_last = N - (nchunks - 1) * kC;
+        const float g_full = (float)exp2((double)kC * lg);
+        const float sc_full = (float)exp2((double)(r + 1 - kC) * lg);
+        const float g_last = (float)exp2((double)L_last * lg);
+        const float sc_last = (float)exp2((double)(r + 1 - L_last) * lg);
 
-        // Q of chunk jq from the staging buffer into TMEM columns [kTQ, kTQ + DK/2)
-        auto copy_q = [&](int jq) -> bool {
-            if (!tc::mbar_wait(&bars.qfull, jq & 1)) return false;
-            if (jq > 0 && !tc::mbar_wait(&bars.qfree, (jq - 1) & 1)) return false;
-            tc::tc_fence_after();
-#pragma unroll
-            for (int gg = 0; gg < DK / 128; gg++) {        // 32 packed words = 64 d_k values = one slab row
-                const int g32 = wg * (DK / 128) + gg;
-                uint32_t w[32];
-#pragma unroll
-                for (int c16 = 0; c16 < 8; c16++) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(sQ + g32 * (kC * 128) +
-                                                                    tc::sw128_off((uint32_t)r, (uint32_t)c16));
-                    w[4 * c16 + 0] = v.x;
-                    w[4 * c16 + 1] = v.y;
-                    w[4 * c16 + 2] = v.z;
-                    w[4 * c16 + 3] = v.w;
-                }
-                tc::tmem_st32(tb + lane_off + kTQ + 32 * g32, w);
-            }
-            tc::tmem_st_wait();
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                tc::mbar_arrive(&bars.qready);
-                tc::mbar_arrive(&bars.qempty);
-            }
-            return true;
-        };
-
-        ok = copy_q(0);
         for (int jc = 0; jc < nchunks && ok; jc++) {
             const int n0 = jc * kC, L = min(kC, N - n0);
             const bool last = (jc == nchunks - 1);
-            // ---- mask: P = tril(A) as packed bf16 into TMEM
+            // ---- mask: P = tril(A) as packed bf16 into TMEM, 32 A columns at a time
             ok = tc::mbar_wait(&bars.afull, jc & 1);
             if (!ok) break;
             tc::tc_fence_after();
             {
-                uint32_t a[2][32];
-                tc::tmem_ld32(tb + lane_off + kTA + 64 * wg, a[0]);
-                tc::tmem_ld32(tb + lane_off + kTA + 64 * wg + 32, a[1]);
-                tc::tmem_ld_wait();
+#pragma unroll
+                for (int hh = 0; hh < 2; hh++) {
+                    uint32_t a[32], w[16];
+                    tc::tmem_ld32(tb + lane_off + kTA + 64 * wg + 32 * hh, a);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; i++) {
+                        const int c = 64 * wg + 32 * hh + 2 * i;
+                        const float lo = (c <= r) ? __uint_as_float(a[2 * i]) : 0.f;
+                        const float hi = (c + 1 <= r) ? __uint_as_float(a[2 * i + 1]) : 0.f;
+                        w[i] = tc::pack_bf16x2(lo, hi);
+                    }
+                    tc::tmem_st16(tb + lane_off + kTP + 32 * wg + 16 * hh, w);
+                }
                 tc::tc_fence_before();
                 elect_arrive(&bars.aread, lane);
-                uint32_t w[32];
-#pragma unroll
-                for (int i = 0; i < 32; i++) {
-                    const int c = 64 * wg + 2 * i;
-                    const float lo = (c <= r) ? __uint_as_float(a[i >> 4][(2 * i) & 31]) : 0.f;
-                    const float hi = (c + 1 <= r) ? __uint_as_float(a[i >> 4][(2 * i + 1) & 31]) : 0.f;
-                    w[i] = tc::pack_bf16x2(lo, hi);
-                }
-                tc::tmem_st32(tb + lane_off + kTP + 32 * wg, w);
                 tc::tmem_st_wait();
             }
             tc::tc_fence_before();
             elect_arrive(&bars.pready, lane);
-            // ---- the next chunk's Q into TMEM once this chunk's read-out is done
-            if (!last) {
-                ok = copy_q(jc + 1);
-                if (!ok) break;
-            }
             // ---- state: R = gamma^L R + dS; T = gamma^L_next R (bf16, read-out of the next chunk)
             ok = tc::mbar_wait(&bars.dsdone, jc & 1);
             if (!ok) break;
             tc::tc_fence_after();
             {
-                const float gL = (float)exp2((double)L * lg);
+                const float gL = last ? g_last : g_full;
 #pragma unroll
                 for (int part = 0; part < kParts; part++) {
                     uint32_t d[32];
@@ -402,7 +467,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 tc::tc_fence_before();
                 elect_arrive(&bars.dsfree, lane);
                 if (!last) {
-                    const float gN = (float)exp2((double)min(kC, N - (n0 + kC)) * lg);
+                    const float gN = (jc + 1 == nchunks - 1) ? g_last : g_full;
+                    // T is overwritten only once this chunk's read-out has consumed it
+                    ok = tc::mbar_wait(&bars.qtm, jc & 1);
+                    if (!ok) break;
 #pragma unroll
                     for (int part = 0; part < kParts; part++) {
                         const int dr = part * kPartDk + r;
@@ -443,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 tc::tc_fence_before();
                 elect_arrive(&bars.ofree, lane);
                 if (r < L) {
-                    const float sc = (float)exp2((double)(r + 1 - L) * lg);
+                    const float sc = last ? sc_last : sc_full;
                     Tout* dst = reinterpret_cast<Tout*>(p.out) + (((size_t)b * N + n0 + r) * p.H + h) * p.dv + j0 +
                                 32 * wg;
                     if constexpr (sizeof(Tout) == 2) {
