@@ -128,6 +128,47 @@ ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
                                     size_t workspace_bytes);
 
 /*
+ * The two passes of ret_forward_chunkwise_ws as separate calls, on the same
+ * workspace, in stream order (prepare, then prepared).  Shapes outside the
+ * workspace path (ret_chunkwise_workspace_bytes returns 0, or some
+ * gamma_h^chunk < 2^-60) return RET_ERR_UNSUPPORTED from both; use
+ * ret_forward_chunkwise for them.
+ *
+ * ret_chunkwise_prepare reads q and k (device [B, N, H, dk], bf16, 16-byte
+ * aligned) and fills the workspace with the rotated queries (xpos != 0) and
+ * the rotated, zeta-scaled keys.  Its arguments mean what they mean for
+ * ret_forward_chunkwise_ws; dv only selects the path (a multiple of 64).
+ *
+ * ret_forward_chunkwise_prepared runs the tensor-core kernel on a workspace
+ * that ret_chunkwise_prepare filled with the same q, k, gammas, B, N, H, dk,
+ * chunk, xpos, pos_offset and theta_base (the workspace is only read).  It
+ * can continue a sequence: initial_state (device fp32 [B, H, dk, dv], 16-byte
+ * aligned, or NULL for the zero state) is the state S after every token
+ * before this call's first one, and the call computes
+ *     S_n = gamma_h S_{n-1} + k_n v_n^T from S = initial_state,  o_n = q_n^T S_n,
+ * i.e. the chunkwise recurrence with R_0 = initial_state ("Hybrid
+ * Architectures: RetNet and the Three Computation Paradigms", section 7.2;
+ * RetNet paper summary, chunkwise representation, Eq. 7, and inference
+ * protocol).  With pos_offset set to the number of earlier tokens, splitting
+ * a sequence into calls that pass each call's final_state on as the next
+ * call's initial_state gives the single call's outputs and final state up
+ * to rounding.  final_state may be the same buffer as initial_state (updated
+ * in place); any other overlap is RET_ERR_INVALID_ARG.
+ */
+ret_status ret_chunkwise_prepare(const void* q, const void* k, const double* gammas, int B, int N,
+                                 int H, int dk, int dv, int chunk, cudaStream_t stream,
+                                 ret_dtype in_dt, int xpos, int64_t pos_offset, double theta_base,
+                                 void* workspace, size_t workspace_bytes);
+
+ret_status ret_forward_chunkwise_prepared(const void* q, const void* k, const void* v,
+                                          const double* gammas, int B, int N, int H, int dk,
+                                          int dv, int chunk, void* out, float* final_state,
+                                          const float* initial_state, cudaStream_t stream,
+                                          ret_dtype in_dt, ret_dtype out_dt, int xpos,
+                                          int64_t pos_offset, double theta_base,
+                                          const void* workspace, size_t workspace_bytes);
+
+/*
  * Allocation-free variant of ret_forward_chunkwise_ws, for callers that
  * cannot allocate device memory at call time: for example a plug-in that runs
  * inside a host framework which owns all device memory and hands out no

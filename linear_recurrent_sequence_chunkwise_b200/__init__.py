@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "RetentionError", "lib", "ret_xpos_rotate", "ret_forward_chunkwise", "ret_forward_chunkwise_ws",
-    "ret_chunkwise_workspace_bytes", "ret_forward_chunkwise_noalloc", "ret_chunkwise_noalloc_max_bytes",
+    "ret_chunkwise_workspace_bytes", "ret_chunkwise_prepare", "ret_forward_chunkwise_prepared",
+    "ret_forward_chunkwise_noalloc", "ret_chunkwise_noalloc_max_bytes",
     "ret_decode_step", "ret_msr_forward", "ret_msr_workspace_bytes",
     "ret_linear_bf16",
     "ret_forward_parallel", "ret_forward_recurrent", "ret_check_device_error", "ret_last_error_string",
@@ -54,6 +55,9 @@ def _load_library():
     L.ret_forward_chunkwise_ws.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d, vp,
                                            ctypes.c_size_t]
     L.ret_forward_chunkwise_noalloc.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d]
+    L.ret_chunkwise_prepare.argtypes = [vp, vp, dp, i, i, i, i, i, i, vp, i, i, i64, d, vp, ctypes.c_size_t]
+    L.ret_forward_chunkwise_prepared.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, vp, vp, vp, vp, i, i, i, i64, d,
+                                                 vp, ctypes.c_size_t]
     L.ret_chunkwise_noalloc_max_bytes.argtypes = []
     L.ret_chunkwise_noalloc_max_bytes.restype = ctypes.c_size_t
     L.ret_chunkwise_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
@@ -70,7 +74,8 @@ def _load_library():
     L.ret_last_error_string.restype = ctypes.c_char_p
     L.ret_last_error_string.argtypes = []
     for name in ("ret_xpos_rotate", "ret_forward_chunkwise", "ret_forward_chunkwise_ws",
-                 "ret_forward_chunkwise_noalloc", "ret_decode_step",
+                 "ret_forward_chunkwise_noalloc", "ret_chunkwise_prepare", "ret_forward_chunkwise_prepared",
+                 "ret_decode_step",
                  "ret_forward_parallel",
                  "ret_forward_recurrent", "ret_check_device_error", "ret_msr_forward", "ret_linear_bf16"):
         getattr(L, name).restype = ctypes.c_int
@@ -180,6 +185,43 @@ def ret_forward_chunkwise_ws(q, k, v, gammas, chunk: int, workspace, out=None, f
                                         dv, int(chunk), _ptr(out, "out"), _ptr(final_state, "final_state"),
                                         _stream(stream), _dt(q.dtype), _dt(out.dtype), int(bool(xpos)),
                                         int(pos_offset), float(theta_base), _ptr(workspace, "workspace"), nbytes))
+    return (out, final_state) if final_state is not None else out
+
+
+def ret_chunkwise_prepare(q, k, gammas, chunk: int, workspace, dv: int, xpos: bool = False, pos_offset: int = 0,
+                          theta_base: float = 10000.0, stream=None):
+    """First pass of the workspace path: rotated queries (xpos) and rotated,
+    zeta-scaled keys into ``workspace``."""
+    if q.shape != k.shape or q.dim() != 4:
+        raise ValueError("q and k must both be [B, N, H, dk]")
+    B, N, H, dk = q.shape
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib.ret_chunkwise_prepare(_ptr(q, "q"), _ptr(k, "k"), _gammas(gammas, H), B, N, H, dk, int(dv),
+                                     int(chunk), _stream(stream), _dt(q.dtype), int(bool(xpos)), int(pos_offset),
+                                     float(theta_base), _ptr(workspace, "workspace"), nbytes))
+
+
+def ret_forward_chunkwise_prepared(q, k, v, gammas, chunk: int, workspace, out=None, final_state=None,
+                                   initial_state=None, out_dtype=None, xpos: bool = False, pos_offset: int = 0,
+                                   theta_base: float = 10000.0, want_final_state: bool = False, stream=None):
+    """Second pass of the workspace path on a workspace filled by
+    ret_chunkwise_prepare with the same arguments; ``initial_state`` (fp32
+    [B, H, dk, dv], or None for zero) continues a sequence."""
+    B, N, H, dk, dv = _seq_shapes(q, k, v)
+    if out is None:
+        out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
+    if final_state is None and want_final_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    if initial_state is not None and (initial_state.dtype != torch.float32 or
+                                      tuple(initial_state.shape) != (B, H, dk, dv)):
+        raise ValueError("initial_state must be fp32 [B, H, dk, dv]")
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib.ret_forward_chunkwise_prepared(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N,
+                                              H, dk, dv, int(chunk), _ptr(out, "out"),
+                                              _ptr(final_state, "final_state"),
+                                              _ptr(initial_state, "initial_state"), _stream(stream), _dt(q.dtype),
+                                              _dt(out.dtype), int(bool(xpos)), int(pos_offset), float(theta_base),
+                                              _ptr(workspace, "workspace"), nbytes))
     return (out, final_state) if final_state is not None else out
 
 

@@ -126,6 +126,7 @@ struct WsParams {
     CUtensorMap tq, tk, tv;
     void* out;
     float* fstate;
+    const float* istate;  // state before the first token, [B, H, DK, dv] fp32, or null (zero)
     int N, H, dv;
     HeadConsts hc;
 };
@@ -187,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
     const int N = p.N;
     const int nchunks = (N + kC - 1) / kC;
     const double lg = p.hc.log2g[h];
+    const int has_init = p.istate != nullptr;
     constexpr int kXfWarps = 8;  // transform warps arriving on the warpgroup barriers
 
     if (tid == 0) {
@@ -317,10 +319,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 }
                 if (!ok) break;
                 tc::mma_commit_elect(&bars.afull);
-                // ---- O = Q T  (read-out of the state before this chunk)
-                if (jc > 0) {
-                    ok = wait(&bars.tready, (jc - 1) & 1);
-                    if (ok) ok = wait(&bars.ofree, (jc - 1) & 1);
+                // ---- O = Q T  (read-out of the state before this chunk; none for
+                // the first chunk unless the call continues from a given state)
+                if (jc > 0 || has_init) {
+                    ok = wait(&bars.tready, (jc - 1 + has_init) & 1);
+                    if (ok && jc > 0) ok = wait(&bars.ofree, (jc - 1) & 1);
                     if (!ok) break;
                     tc::tc_fence_after();
 #pragma unroll 4
@@ -339,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
 #pragma unroll
                 for (int k = 0; k < kC / 16; k++)
                     tc::mma_bf16_ts_elect(tb + kTO, tb + kTP + 8 * k, dv_mn + vo + (uint32_t)((k * 2048) >> 4), id_pv,
-                                          (jc > 0) || (k > 0));
+                                          (jc > 0) || has_init || (k > 0));
                 tc::mma_commit_elect(&bars.ofull);
                 tc::mma_commit_elect(&bars.vempty[jc & 1]);
             }
@@ -411,16 +414,48 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         uint8_t* sT = sm + WsSmem<DK>::kT;
         float R[kParts][32];
-#pragma unroll
-        for (int part = 0; part < kParts; part++)
-#pragma unroll
-            for (int i = 0; i < 32; i++) R[part][i] = 0.f;
         // decay powers of a full chunk and of the (possibly shorter) last one
         const int L_last = N - (nchunks - 1) * kC;
         const float g_full = (float)exp2((double)kC * lg);
         const float sc_full = (float)exp2((double)(r + 1 - kC) * lg);
         const float g_last = (float)exp2((double)L_last * lg);
         const float sc_last = (float)exp2((double)(r + 1 - L_last) * lg);
+        if (has_init) {
+            // Continue from the given state: R = S_init, and the first read-out
+            // uses T = gamma^L0 S_init (L0 the first chunk's length).
+            const float g0 = nchunks == 1 ? g_last : g_full;
+#pragma unroll
+            for (int part = 0; part < kParts; part++) {
+                const int dr = part * kPartDk + r;
+                const float4* src = reinterpret_cast<const float4*>(p.istate + (((size_t)b * p.H + h) * DK + dr) * p.dv +
+                                                                    j0 + 32 * wg);
+#pragma unroll
+                for (int c4 = 0; c4 < 8; c4++) {
+                    const float4 x = __ldg(src + c4);
+                    R[part][4 * c4 + 0] = x.x;
+                    R[part][4 * c4 + 1] = x.y;
+                    R[part][4 * c4 + 2] = x.z;
+                    R[part][4 * c4 + 3] = x.w;
+                }
+#pragma unroll
+                for (int c4 = 0; c4 < 4; c4++) {
+                    const int base = c4 * 8;
+                    uint4 v;
+                    v.x = tc::pack_bf16x2(g0 * R[part][base + 0], g0 * R[part][base + 1]);
+                    v.y = tc::pack_bf16x2(g0 * R[part][base + 2], g0 * R[part][base + 3]);
+                    v.z = tc::pack_bf16x2(g0 * R[part][base + 4], g0 * R[part][base + 5]);
+                    v.w = tc::pack_bf16x2(g0 * R[part][base + 6], g0 * R[part][base + 7]);
+                    *reinterpret_cast<uint4*>(sT + tc::sw128_off((uint32_t)dr, (uint32_t)(4 * wg + c4))) = v;
+                }
+            }
+            tc::fence_proxy_async_smem();
+            elect_arrive(&bars.tready, lane);
+        } else {
+#pragma unroll
+            for (int part = 0; part < kParts; part++)
+#pragma unroll
+                for (int i = 0; i < 32; i++) R[part][i] = 0.f;
+        }
 
         for (int jc = 0; jc < nchunks && ok; jc++) {
             const int n0 = jc * kC, L = min(kC, N - n0);
@@ -585,6 +620,7 @@ ret_status launch_chunkwise_main(const RetArgs& a, const void* q_src, const void
         return RET_ERR_CUDA;
     p.out = a.out;
     p.fstate = a.final_state;
+    p.istate = a.initial_state;
     p.N = a.N;
     p.H = a.H;
     p.dv = a.dv;
@@ -594,10 +630,16 @@ ret_status launch_chunkwise_main(const RetArgs& a, const void* q_src, const void
     return f32 ? launch_main<128, float>(p, a, s) : launch_main<128, __nv_bfloat16>(p, a, s);
 }
 
-ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s) {
+// Pointers into the workspace: k' first, then q_rot (rotation only).
+static void ws_parts(const RetArgs& a, void* ws, __nv_bfloat16** k_out, __nv_bfloat16** q_rot) {
     const size_t qk = (size_t)a.B * a.N * a.H * a.dk;
-    __nv_bfloat16* k_out = reinterpret_cast<__nv_bfloat16*>(ws);
-    __nv_bfloat16* q_rot = a.xpos ? k_out + qk : nullptr;
+    *k_out = reinterpret_cast<__nv_bfloat16*>(ws);
+    *q_rot = a.xpos ? *k_out + qk : nullptr;
+}
+
+ret_status launch_chunkwise_prep(const RetArgs& a, void* ws, cudaStream_t s) {
+    __nv_bfloat16 *k_out, *q_rot;
+    ws_parts(a, ws, &k_out, &q_rot);
     const int blocks = (int)(((long long)a.B * a.N + 7) / 8);
     const double lb = log2(a.theta_base);
     if (a.dk == 256)
@@ -606,9 +648,19 @@ ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s) {
     else
         k_prep_qk<128><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, q_rot, k_out,
                                                a.hc, a.B, a.N, a.H, a.chunk, a.xpos, a.pos_offset, lb);
-    ret_status st = check_launch("chunkwise (workspace path): prep");
-    if (st != RET_OK) return st;
+    return check_launch("chunkwise (workspace path): prep");
+}
+
+ret_status launch_chunkwise_prepared(const RetArgs& a, void* ws, cudaStream_t s) {
+    __nv_bfloat16 *k_out, *q_rot;
+    ws_parts(a, ws, &k_out, &q_rot);
     return launch_chunkwise_main(a, a.xpos ? (const void*)q_rot : a.q, k_out, s);
+}
+
+ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s) {
+    ret_status st = launch_chunkwise_prep(a, ws, s);
+    if (st != RET_OK) return st;
+    return launch_chunkwise_prepared(a, ws, s);
 }
 
 // ------------------------------------------------- allocation-free variant

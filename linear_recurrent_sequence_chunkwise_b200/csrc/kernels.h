@@ -13,7 +13,8 @@ struct RetArgs {
     const void* k;
     const void* v;
     void* out;
-    float* final_state;  // may be null
+    float* final_state;          // may be null
+    const float* initial_state;  // may be null (zero state); workspace path only
     int B, N, H, dk, dv, chunk;
     ret_dtype in_dt, out_dt;
     int xpos;
@@ -41,6 +42,10 @@ bool chunkwise_tc_supported(const RetArgs& a);
 bool chunkwise_ws_supported(const RetArgs& a);
 size_t chunkwise_ws_bytes(const RetArgs& a);
 ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s);
+// Its two halves: the prep pass alone, and the tensor-core kernel on a
+// workspace the prep pass has filled (a.initial_state honoured).
+ret_status launch_chunkwise_prep(const RetArgs& a, void* ws, cudaStream_t s);
+ret_status launch_chunkwise_prepared(const RetArgs& a, void* ws, cudaStream_t s);
 // The workspace path on the library's fixed device array (no allocation).
 size_t chunkwise_static_ws_bytes();
 ret_status launch_chunkwise_static(const RetArgs& a, cudaStream_t s);

@@ -1,5 +1,6 @@
 // ret_api.cu -- the C ABI: argument validation, per-head constants and
 // dispatch to the kernels.  Nothing here allocates device memory.
+#include <cstring>
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
@@ -81,7 +82,7 @@ static ret_status make_args(RetArgs* a, const char* who, const void* q, const vo
             overlaps(final_state, bs, k, bq) || overlaps(final_state, bs, v, bv))
             return fail(RET_ERR_INVALID_ARG, "%s: final_state overlaps another buffer", who);
     }
-    a->q = q; a->k = k; a->v = v; a->out = out; a->final_state = final_state;
+    a->q = q; a->k = k; a->v = v; a->out = out; a->final_state = final_state; a->initial_state = nullptr;
     a->B = B; a->N = N; a->H = H; a->dk = dk; a->dv = dv; a->chunk = chunk;
     a->in_dt = in_dt; a->out_dt = out_dt;
     a->xpos = xpos ? 1 : 0; a->pos_offset = pos_offset; a->theta_base = xpos ? theta_base : 10000.0;
@@ -161,6 +162,88 @@ ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
         (final_state && overlaps(workspace, need, final_state, (size_t)B * H * dk * dv * 4)))
         return fail(RET_ERR_INVALID_ARG, "ret_forward_chunkwise_ws: workspace overlaps another buffer");
     return launch_chunkwise_ws(a, workspace, stream);
+}
+
+// Workspace checks shared by the workspace-path entry points.
+static ret_status check_workspace(const RetArgs& a, const char* who, const void* workspace, size_t workspace_bytes,
+                                  bool with_outputs) {
+    const size_t need = chunkwise_ws_bytes(a);
+    if (!workspace || workspace_bytes < need)
+        return fail(RET_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed (got %zu)", who, need,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (!aligned(workspace, 256)) return fail(RET_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+    const size_t ntok = (size_t)a.B * a.N * a.H;
+    const size_t bq = ntok * a.dk * 2, bv = ntok * a.dv * 2, bo = ntok * a.dv * (a.out_dt == RET_F32 ? 4 : 2);
+    const size_t bs = (size_t)a.B * a.H * a.dk * a.dv * 4;
+    bool bad = overlaps(workspace, need, a.q, bq) || overlaps(workspace, need, a.k, bq);
+    if (with_outputs)
+        bad = bad || overlaps(workspace, need, a.v, bv) || overlaps(workspace, need, a.out, bo) ||
+              (a.final_state && overlaps(workspace, need, a.final_state, bs)) ||
+              (a.initial_state && overlaps(workspace, need, a.initial_state, bs));
+    if (bad) return fail(RET_ERR_INVALID_ARG, "%s: workspace overlaps another buffer", who);
+    return RET_OK;
+}
+
+ret_status ret_chunkwise_prepare(const void* q, const void* k, const double* gammas, int B, int N, int H, int dk,
+                                 int dv, int chunk, cudaStream_t stream, ret_dtype in_dt, int xpos,
+                                 int64_t pos_offset, double theta_base, void* workspace, size_t workspace_bytes) {
+    t_err[0] = 0;
+    const char* who = "ret_chunkwise_prepare";
+    if (!q || !k) return fail(RET_ERR_INVALID_ARG, "%s: NULL q or k", who);
+    if (B < 1 || N < 1 || H < 1 || dk < 1 || dv < 1 || chunk < 1)
+        return fail(RET_ERR_INVALID_ARG, "%s: sizes must be >= 1", who);
+    if (!is_dtype(in_dt)) return fail(RET_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    ret_status st = check_gammas(gammas, H, who);
+    if (st != RET_OK) return st;
+    if (xpos && (dk % 2 != 0)) return fail(RET_ERR_INVALID_ARG, "%s: xpos needs an even dk (got %d)", who, dk);
+    if (xpos && !(theta_base > 0.0 && isfinite(theta_base)))
+        return fail(RET_ERR_INVALID_ARG, "%s: theta_base must be finite and > 0", who);
+    if ((size_t)B * N * H * (size_t)(dk > dv ? dk : dv) > ((size_t)1 << 40))
+        return fail(RET_ERR_INVALID_ARG, "%s: problem too large", who);
+    if (!aligned(q, 16) || !aligned(k, 16)) return fail(RET_ERR_INVALID_ARG, "%s: q, k must be 16-byte aligned", who);
+    RetArgs a{};
+    a.q = q; a.k = k;
+    a.B = B; a.N = N; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk;
+    a.in_dt = in_dt; a.out_dt = RET_BF16;
+    a.xpos = xpos ? 1 : 0; a.pos_offset = pos_offset; a.theta_base = xpos ? theta_base : 10000.0;
+    make_head_consts(gammas, H, &a.hc);
+    if (!chunkwise_ws_supported(a))
+        return fail(RET_ERR_UNSUPPORTED, "%s: shape outside the workspace path (ret_chunkwise_workspace_bytes is 0)",
+                    who);
+    st = check_workspace(a, who, workspace, workspace_bytes, false);
+    if (st != RET_OK) return st;
+    return launch_chunkwise_prep(a, workspace, stream);
+}
+
+ret_status ret_forward_chunkwise_prepared(const void* q, const void* k, const void* v, const double* gammas, int B,
+                                          int N, int H, int dk, int dv, int chunk, void* out, float* final_state,
+                                          const float* initial_state, cudaStream_t stream, ret_dtype in_dt,
+                                          ret_dtype out_dt, int xpos, int64_t pos_offset, double theta_base,
+                                          const void* workspace, size_t workspace_bytes) {
+    t_err[0] = 0;
+    const char* who = "ret_forward_chunkwise_prepared";
+    RetArgs a;
+    ret_status st = make_args(&a, who, q, k, v, gammas, B, N, H, dk, dv, chunk, out, final_state, in_dt, out_dt,
+                              xpos, pos_offset, theta_base);
+    if (st != RET_OK) return st;
+    if (!chunkwise_ws_supported(a))
+        return fail(RET_ERR_UNSUPPORTED, "%s: shape outside the workspace path (ret_chunkwise_workspace_bytes is 0)",
+                    who);
+    if (initial_state) {
+        const size_t ntok = (size_t)B * N * H, bs = (size_t)B * H * dk * dv * 4;
+        const size_t bq = ntok * dk * 2, bv = ntok * dv * 2, bo = ntok * dv * (out_dt == RET_F32 ? 4 : 2);
+        if (!aligned(initial_state, 16)) return fail(RET_ERR_INVALID_ARG, "%s: initial_state must be 16-byte aligned", who);
+        if (overlaps(initial_state, bs, out, bo) || overlaps(initial_state, bs, q, bq) ||
+            overlaps(initial_state, bs, k, bq) || overlaps(initial_state, bs, v, bv) ||
+            (final_state && (const void*)final_state != (const void*)initial_state &&
+             overlaps(initial_state, bs, final_state, bs)))
+            return fail(RET_ERR_INVALID_ARG, "%s: initial_state overlaps another buffer (final_state may equal it)",
+                        who);
+        a.initial_state = initial_state;
+    }
+    st = check_workspace(a, who, workspace, workspace_bytes, true);
+    if (st != RET_OK) return st;
+    return launch_chunkwise_prepared(a, const_cast<void*>(workspace), stream);
 }
 
 ret_status ret_forward_chunkwise_noalloc(const void* q, const void* k, const void* v, const double* gammas, int B,

@@ -118,3 +118,48 @@ def test_binding_requires_cuda_tensors():
     q = torch.zeros(1, 4, 1, 8)
     with pytest.raises(ValueError):
         R.ret_forward_chunkwise(q, q, q, [0.9], chunk=4, out=torch.zeros(1, 4, 1, 8))
+
+
+# The two-pass workspace entry points.  Shape on the workspace path: bf16,
+# chunk 128, dk 128, dv 64 (q, k 64 KB each at the fake addresses above).
+WS = ctypes.c_void_p(0xA0000000)
+WS_BYTES = 1 * 128 * 2 * 128 * 2
+
+
+def prepare_call(q=P, k=P2, g=G2, dk=128, dv=64, ws=WS, nbytes=WS_BYTES, xpos=0):
+    return R.lib.ret_chunkwise_prepare(q, k, g, 1, 128, 2, dk, dv, 128, S0, 1, xpos, 0, 1e4, ws, nbytes)
+
+
+def prepared_call(ws=WS, nbytes=WS_BYTES, init=None, fs=None, dk=128, out=P4):
+    return R.lib.ret_forward_chunkwise_prepared(P, P2, P3, G2, 1, 128, 2, dk, 64, 128, out, fs, init, S0, 1, 1, 0, 0,
+                                                1e4, ws, nbytes)
+
+
+def test_workspace_size_matches_the_two_pass_shape():
+    assert R.ret_chunkwise_workspace_bytes(1, 128, 2, 128, 64, 128, torch.bfloat16, False) == WS_BYTES
+    assert R.ret_chunkwise_workspace_bytes(1, 128, 2, 128, 64, 128, torch.bfloat16, True) == 2 * WS_BYTES
+    assert R.ret_chunkwise_workspace_bytes(1, 128, 2, 16, 64, 128, torch.bfloat16, False) == 0
+
+
+@needs_no_gpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(ws=None), 1), (dict(nbytes=100), 1), (dict(nbytes=2 * WS_BYTES - 1, xpos=1), 1),
+    (dict(ws=ctypes.c_void_p(0xA0000010)), 1), (dict(ws=ctypes.c_void_p(0x10000)), 1),
+    (dict(g=(ctypes.c_double * 2)(0.9, 1.5)), 1), (dict(dk=16), 2), (dict(dv=48), 2),
+])
+def test_prepare_rejects_bad_arguments(kw, status):
+    assert prepare_call(**kw) == status, (kw, R.ret_last_error_string())
+    assert R.ret_last_error_string()
+
+
+@needs_no_gpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(ws=None), 1), (dict(nbytes=1000), 1), (dict(ws=ctypes.c_void_p(0x90000000)), 1),
+    (dict(init=ctypes.c_void_p(0xB0000004)), 1),                 # misaligned initial state
+    (dict(init=ctypes.c_void_p(0x90000000)), 1),                 # initial state overlaps out
+    (dict(init=ctypes.c_void_p(0xB0000000), fs=ctypes.c_void_p(0xB0000100)), 1),  # partial overlap
+    (dict(out=None), 1), (dict(dk=16), 2),
+])
+def test_prepared_rejects_bad_arguments(kw, status):
+    assert prepared_call(**kw) == status, (kw, R.ret_last_error_string())
+    assert R.ret_last_error_string()

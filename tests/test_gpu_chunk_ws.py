@@ -129,3 +129,56 @@ def test_ws_rejects_small_workspace():
     ws = torch.empty(nb - 256, dtype=torch.uint8, device="cuda")
     with pytest.raises(R.RetentionError):
         R.ret_forward_chunkwise_ws(dev(q), dev(k), dev(v), [0.9], 128, ws, xpos=True)
+
+
+def run_two_pass(qd, kd, vd, g, chunk, init=None, fs=None, pos_offset=0, xpos=True, out_dtype=torch.float32):
+    """ret_chunkwise_prepare then ret_forward_chunkwise_prepared on device tensors."""
+    B, N, H, dk = qd.shape
+    dv = vd.shape[3]
+    nb = R.ret_chunkwise_workspace_bytes(B, N, H, dk, dv, chunk, torch.bfloat16, xpos)
+    assert nb > 0
+    ws = torch.full((nb,), 0xCD, dtype=torch.uint8, device="cuda")
+    R.ret_chunkwise_prepare(qd, kd, g, chunk, ws, dv, xpos=xpos, pos_offset=pos_offset)
+    return R.ret_forward_chunkwise_prepared(qd, kd, vd, g, chunk, ws, final_state=fs, initial_state=init,
+                                            out_dtype=out_dtype, xpos=xpos, pos_offset=pos_offset,
+                                            want_final_state=True)
+
+
+def test_two_pass_equals_one_call():
+    """prepare + prepared is the workspace path split in two: identical bits."""
+    q, k, v = qkv(83, 2, 300, 3, 256, 128, 1 / 16)
+    g = gamma_schedule(3)
+    a, fa = run_ws(q, k, v, g, 128, out_dtype=torch.float32, xpos=True, pos_offset=5, want_final_state=True)
+    b, fb = run_two_pass(dev(q), dev(k), dev(v), g, 128, pos_offset=5)
+    torch.cuda.synchronize()
+    R.ret_check_device_error()
+    assert torch.equal(a, b) and torch.equal(fa, fb)
+
+
+@pytest.mark.parametrize("N,split,dk,dv,xpos,in_place", [
+    (300, 128, 256, 128, True, False),     # split on a chunk boundary
+    (300, 77, 128, 64, False, False),      # ragged: both calls end in a partial chunk
+    (1100, 513, 256, 512, True, True),     # final_state written over initial_state
+    (260, 1, 256, 64, True, False),        # a one-token first call
+])
+def test_continuation_from_state_matches_whole_sequence(N, split, dk, dv, xpos, in_place):
+    """Two calls, the second starting from the first's final state at position
+    `split`, reproduce the oracle's recurrence over the whole sequence."""
+    B, H = 2, 2
+    q, k, v = qkv(90 + split, B, N, H, dk, dv, dk ** -0.5)
+    g = gamma_schedule(H)
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    o1, s1 = run_two_pass(qd[:, :split].contiguous(), kd[:, :split].contiguous(), vd[:, :split].contiguous(), g,
+                          128, xpos=xpos)
+    s1_copy = s1.clone()
+    o2, s2 = run_two_pass(qd[:, split:].contiguous(), kd[:, split:].contiguous(), vd[:, split:].contiguous(), g,
+                          128, init=s1, fs=s1 if in_place else None, pos_offset=split, xpos=xpos)
+    torch.cuda.synchronize()
+    R.ret_check_device_error()
+    if not in_place:
+        assert torch.equal(s1, s1_copy)          # the initial state is only read
+    qr, kr = rotated(q, k, xpos)
+    ref, S = oracle.retention_recurrent(qr, kr, v.f64, g)
+    got = np.concatenate([host64(o1), host64(o2)], axis=1)
+    assert err_out(got, ref) < TOL_BF16
+    assert err_state(host64(s2), S) < TOL_BF16
