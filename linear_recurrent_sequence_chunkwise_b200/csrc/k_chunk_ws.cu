@@ -39,6 +39,7 @@
 //    TMEM columns: A [0,128), P [128,192), O [192,256), Q [256,384),
 //    dS [384,512).  Every hand-off between the roles has at least one block
 //    of MMAs in between, so no role waits on another in the steady state.
+#include <cstring>
 #include <mutex>
 
 #include "kernels.h"
@@ -75,6 +76,10 @@ __global__ void __launch_bounds__(256) k_prep_qk(const __nv_bfloat16* __restrict
                                                   __nv_bfloat16* __restrict__ q_rot,
                                                   __nv_bfloat16* __restrict__ k_out, HeadConsts hc, int B, int N,
                                                   int H, int chunk, int xpos, long long pos0, double log2base) {
+    // theta_p = base^(-2p/DK), once per block (fp64, as the rotation's reference)
+    __shared__ double s_theta[DK / 2];
+    for (int i = threadIdx.x; i < DK / 2; i += blockDim.x) s_theta[i] = exp2(-2.0 * i / DK * log2base);
+    __syncthreads();
     const int lane = threadIdx.x & 31;
     const long long t = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);  // b * N + n
     if (t >= (long long)B * N) return;
@@ -88,33 +93,44 @@ __global__ void __launch_bounds__(256) k_prep_qk(const __nv_bfloat16* __restrict
         for (int i = 0; i < 4; i++) {
             cs[i] = 1.f;
             sn[i] = 0.f;
-            if (xpos) {
-                const int p = 4 * g + i;
-                const double theta = exp2(-2.0 * p / DK * log2base);
-                sincosf(rot_angle(pos0 + n, theta), &sn[i], &cs[i]);
-            }
+            if (xpos) sincosf(rot_angle(pos0 + n, s_theta[4 * g + i]), &sn[i], &cs[i]);
         }
-        for (int h = 0; h < H; h++) {
-            const size_t e = ((size_t)t * H + h) * DK + 8 * g;
-            const float zeta = (float)exp2((double)(L - 1 - r) * hc.log2g[h]);
-            uint4 kw = *reinterpret_cast<const uint4*>(k + e);
-            uint32_t* kwv = reinterpret_cast<uint32_t*>(&kw);
+        // The loads of kHB heads are issued together (memory-level
+        // parallelism), then rotated and stored.
+        constexpr int kHB = 8;
+        for (int h0 = 0; h0 < H; h0 += kHB) {
+            uint4 kw[kHB], qw[kHB];
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const float x0 = tc::bf16lo(kwv[i]), x1 = tc::bf16hi(kwv[i]);
-                const float c = cs[i] * zeta, s = sn[i] * zeta;
-                kwv[i] = tc::pack_bf16x2(x0 * c - x1 * s, x0 * s + x1 * c);
+            for (int hh = 0; hh < kHB; hh++) {
+                if (h0 + hh < H) {
+                    const size_t e = ((size_t)t * H + h0 + hh) * DK + 8 * g;
+                    kw[hh] = __ldg(reinterpret_cast<const uint4*>(k + e));
+                    if (xpos) qw[hh] = __ldg(reinterpret_cast<const uint4*>(q + e));
+                }
             }
-            *reinterpret_cast<uint4*>(k_out + e) = kw;
-            if (xpos) {
-                uint4 qw = *reinterpret_cast<const uint4*>(q + e);
-                uint32_t* qwv = reinterpret_cast<uint32_t*>(&qw);
+#pragma unroll
+            for (int hh = 0; hh < kHB; hh++) {
+                if (h0 + hh >= H) continue;
+                const size_t e = ((size_t)t * H + h0 + hh) * DK + 8 * g;
+                // zeta = gamma^(L-1-r): the exponent in fp64, exp2 in fp32 (relative error ~1e-7)
+                const float zeta = exp2f((float)((double)(L - 1 - r) * hc.log2g[h0 + hh]));
+                uint32_t* kwv = reinterpret_cast<uint32_t*>(&kw[hh]);
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
-                    const float x0 = tc::bf16lo(qwv[i]), x1 = tc::bf16hi(qwv[i]);
-                    qwv[i] = tc::pack_bf16x2(x0 * cs[i] - x1 * sn[i], x0 * sn[i] + x1 * cs[i]);
+                    const float x0 = tc::bf16lo(kwv[i]), x1 = tc::bf16hi(kwv[i]);
+                    const float c = cs[i] * zeta, s = sn[i] * zeta;
+                    kwv[i] = tc::pack_bf16x2(x0 * c - x1 * s, x0 * s + x1 * c);
                 }
-                *reinterpret_cast<uint4*>(q_rot + e) = qw;
+                *reinterpret_cast<uint4*>(k_out + e) = kw[hh];
+                if (xpos) {
+                    uint32_t* qwv = reinterpret_cast<uint32_t*>(&qw[hh]);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) {
+                        const float x0 = tc::bf16lo(qwv[i]), x1 = tc::bf16hi(qwv[i]);
+                        qwv[i] = tc::pack_bf16x2(x0 * cs[i] - x1 * sn[i], x0 * sn[i] + x1 * cs[i]);
+                    }
+                    *reinterpret_cast<uint4*>(q_rot + e) = qw[hh];
+                }
             }
         }
     }
@@ -128,6 +144,7 @@ struct WsParams {
     float* fstate;
     const float* istate;  // state before the first token, [B, H, DK, dv] fp32, or null (zero)
     int N, H, dv;
+    int nmain;            // CTAs: B * H * (dv / 64), one per (b, h, 64 value columns)
     HeadConsts hc;
 };
 
@@ -184,7 +201,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
     __shared__ int s_fail;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int j0 = blockIdx.x * kW, h = blockIdx.y, b = blockIdx.z;
+    const int nt = p.dv / kW, jt = (int)blockIdx.x % nt;     // this CTA's 64 value columns
+    const int h = ((int)blockIdx.x / nt) % p.H, b = (int)blockIdx.x / (nt * p.H);
+    const int j0 = jt * kW;
     const int N = p.N;
     const int nchunks = (N + kC - 1) / kC;
     const double lg = p.hc.log2g[h];
@@ -234,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             auto prefetch = [&](int jp) {
                 if (jp >= nchunks) return;
                 const int n0p = jp * kC;
-                for (int i = blockIdx.x; i < 2 * kQSlabs; i += gridDim.x)
+                for (int i = jt; i < 2 * kQSlabs; i += nt)
                     tc::tma_prefetch_l2_4d(i < kQSlabs ? &p.tq : &p.tk, 64 * (i % kQSlabs), h, n0p, b);
                 tc::tma_prefetch_l2_4d(&p.tv, j0, h, n0p, b);
             };
@@ -580,18 +599,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
 }
 
 template <int DK, typename Tout>
-ret_status launch_main(const WsParams& p, const RetArgs& a, cudaStream_t s) {
+ret_status launch_main(const WsParams& p, cudaStream_t s) {
     auto kern = k_chunkwise_ws<DK, Tout>;
     const int smem = (int)WsSmem<DK>::kBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return check_launch("chunkwise (workspace path): smem attribute");
-    dim3 grid(a.dv / kW, a.H, a.B);
-    kern<<<grid, kThreads, smem, s>>>(p);
+    kern<<<p.nmain, kThreads, smem, s>>>(p);
     return check_launch("chunkwise (workspace path)");
 }
 
 }  // namespace
 
+// Workspace layout: k' [B, N, H, dk] bf16, then q_rot (rotation only).
 size_t chunkwise_ws_bytes(const RetArgs& a) {
     const size_t qk = (size_t)a.B * a.N * a.H * a.dk * 2;
     return a.xpos ? 2 * qk : qk;
@@ -601,33 +620,43 @@ bool chunkwise_ws_supported(const RetArgs& a) {
     if (a.in_dt != RET_BF16) return false;
     if (a.chunk != kC || !(a.dk == 128 || a.dk == 256) || a.dv % kW != 0) return false;
     if (a.N > (1 << 30)) return false;
+    if ((long long)a.B * a.H * (a.dv / kW) > (1ll << 30)) return false;
     for (int h = 0; h < a.H; h++)
         if (!(a.hc.log2g[h] * kC >= -60.0)) return false;
     return true;
 }
 
-ret_status launch_chunkwise_main(const RetArgs& a, const void* q_src, const void* k_prime, cudaStream_t s) {
-    WsParams p;
+// Tensor maps and per-launch fields shared by both kernel variants.
+static ret_status fill_params(WsParams* p, const RetArgs& a, const void* q_src, const void* k_prime) {
+    memset(p, 0, sizeof(*p));
     const uint64_t B = a.B, N = a.N, H = a.H, dk = a.dk, dv = a.dv;
     const uint64_t dq[4] = {dk, H, N, B};
     const uint64_t sq[3] = {dk * 2, H * dk * 2, N * H * dk * 2};
     const uint32_t box[4] = {64, 1, (uint32_t)kC, 1};
     const uint64_t dvv[4] = {dv, H, N, B};
     const uint64_t svv[3] = {dv * 2, H * dv * 2, N * H * dv * 2};
-    if (!make_tmap_bf16(&p.tq, q_src, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_bf16(&p.tk, k_prime, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_bf16(&p.tv, a.v, 4, dvv, svv, box, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_tmap_bf16(&p->tq, q_src, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_bf16(&p->tk, k_prime, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_bf16(&p->tv, a.v, 4, dvv, svv, box, CU_TENSOR_MAP_SWIZZLE_128B))
         return RET_ERR_CUDA;
-    p.out = a.out;
-    p.fstate = a.final_state;
-    p.istate = a.initial_state;
-    p.N = a.N;
-    p.H = a.H;
-    p.dv = a.dv;
-    p.hc = a.hc;
+    p->out = a.out;
+    p->fstate = a.final_state;
+    p->istate = a.initial_state;
+    p->N = a.N;
+    p->H = a.H;
+    p->dv = a.dv;
+    p->hc = a.hc;
+    p->nmain = a.B * a.H * (a.dv / kW);
+    return RET_OK;
+}
+
+ret_status launch_chunkwise_main(const RetArgs& a, const void* q_src, const void* k_prime, cudaStream_t s) {
+    WsParams p;
+    ret_status st = fill_params(&p, a, q_src, k_prime);
+    if (st != RET_OK) return st;
     const bool f32 = a.out_dt == RET_F32;
-    if (a.dk == 256) return f32 ? launch_main<256, float>(p, a, s) : launch_main<256, __nv_bfloat16>(p, a, s);
-    return f32 ? launch_main<128, float>(p, a, s) : launch_main<128, __nv_bfloat16>(p, a, s);
+    if (a.dk == 256) return f32 ? launch_main<256, float>(p, s) : launch_main<256, __nv_bfloat16>(p, s);
+    return f32 ? launch_main<128, float>(p, s) : launch_main<128, __nv_bfloat16>(p, s);
 }
 
 // Pointers into the workspace: k' first, then q_rot (rotation only).

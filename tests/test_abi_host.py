@@ -123,7 +123,8 @@ def test_binding_requires_cuda_tensors():
 # The two-pass workspace entry points.  Shape on the workspace path: bf16,
 # chunk 128, dk 128, dv 64 (q, k 64 KB each at the fake addresses above).
 WS = ctypes.c_void_p(0xA0000000)
-WS_BYTES = 1 * 128 * 2 * 128 * 2
+QK_BYTES = 1 * 128 * 2 * 128 * 2          # one bf16 [B, N, H, dk] tensor
+WS_BYTES = QK_BYTES                       # k' alone (no rotation)
 
 
 def prepare_call(q=P, k=P2, g=G2, dk=128, dv=64, ws=WS, nbytes=WS_BYTES, xpos=0):
@@ -137,13 +138,14 @@ def prepared_call(ws=WS, nbytes=WS_BYTES, init=None, fs=None, dk=128, out=P4):
 
 def test_workspace_size_matches_the_two_pass_shape():
     assert R.ret_chunkwise_workspace_bytes(1, 128, 2, 128, 64, 128, torch.bfloat16, False) == WS_BYTES
-    assert R.ret_chunkwise_workspace_bytes(1, 128, 2, 128, 64, 128, torch.bfloat16, True) == 2 * WS_BYTES
+    assert R.ret_chunkwise_workspace_bytes(1, 128, 2, 128, 64, 128, torch.bfloat16, True) == 2 * QK_BYTES
+    assert R.ret_chunkwise_workspace_bytes(3, 1000, 2, 128, 64, 128, torch.bfloat16, True) == 2 * 3 * 1000 * 2 * 128 * 2
     assert R.ret_chunkwise_workspace_bytes(1, 128, 2, 16, 64, 128, torch.bfloat16, False) == 0
 
 
 @needs_no_gpu
 @pytest.mark.parametrize("kw,status", [
-    (dict(q=None), 1), (dict(ws=None), 1), (dict(nbytes=100), 1), (dict(nbytes=2 * WS_BYTES - 1, xpos=1), 1),
+    (dict(q=None), 1), (dict(ws=None), 1), (dict(nbytes=100), 1), (dict(nbytes=2 * QK_BYTES - 1, xpos=1), 1),
     (dict(ws=ctypes.c_void_p(0xA0000010)), 1), (dict(ws=ctypes.c_void_p(0x10000)), 1),
     (dict(g=(ctypes.c_double * 2)(0.9, 1.5)), 1), (dict(dk=16), 2), (dict(dv=48), 2),
 ])
