@@ -37,6 +37,22 @@ UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 
 
+def max_over_ranks(x: float, world: int, dist=None, device="cpu") -> float:
+    """The maximum of ``x`` over all ranks (device time of the slowest rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput under weak scaling: every rank processes
+    ``units_per_rank`` per step and the job takes the slowest rank's time."""
+    return world * units_per_rank / (ms_max / 1e3)
+
+
 def gammas(H):
     return [1.0 - 2.0 ** (-5 - h) for h in range(H)]
 
@@ -202,12 +218,9 @@ def run_ours(args):
     t_prep = statistics.mean(a.elapsed_time(b) for a, b, c in evs) / 1e3
     t_main = statistics.mean(b.elapsed_time(c) for a, b, c in evs) / 1e3
     total_ms = sum(times)
-    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dist, dev)
     ms_per_step = total_ms / args.steps
-    value = world * B * N / (ms_per_step / 1e3)
+    value = job_throughput(B * N, world, ms_per_step)
 
     peaks = load_peaks()
     # Dominant kernel: k_chunkwise_ws, timed alone (CUDA events around its
@@ -259,6 +272,9 @@ def run_ours(args):
         result["e2e"] = e2e_ours(R, torch, dev, stream, w, g, args, world, barrier, dist)
     if not args.no_decode:
         result["decode"] = bench_decode(R, torch, dev, stream, args, peaks, world, barrier, dist, rank)
+    if not args.no_layer:
+        result["msr_layer"] = bench_msr(R, torch, dev, stream, args, peaks, world, dist)
+        result["fp32_small"] = bench_fp32_small(R, torch, dev, stream, args, world, dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
     if rank == 0:
@@ -299,10 +315,7 @@ def e2e_ours(R, torch, dev, stream, w, g, args, world, barrier, dist):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    t = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item()) / steps
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev) / steps
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
     return {"value": round(world * B * N / (ms / 1e3), 1), "unit": UNIT, "ms_per_step": round(ms, 3),
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho.numel() * ho.element_size(), "steps": steps}
@@ -342,10 +355,7 @@ def bench_decode(R, torch, dev, stream, args, peaks, world, barrier, dist, rank)
     torch.cuda.synchronize()
     R.ret_check_device_error()
     ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
+    ms = max_over_ranks(ms, world, dist, dev)
     nbytes = 2 * B * H * dk * dv * 4 + B * H * (2 * dk * 2 + dv * 2 + dv * 4)
     gbs = nbytes / (ms / 1e3) / 1e9
     return {"workload": d["workload"], "metric": "decode-step state HBM GB/s", "value": round(gbs * world, 1),
@@ -355,6 +365,74 @@ def bench_decode(R, torch, dev, stream, args, peaks, world, barrier, dist, rank)
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "kernel": "k_decode_step",
                          "traffic": (load_traffic("k_decode_step") or {}).get("bytes_per_launch")},
             "l2": "state (537 MB) larger than L2"}
+
+
+def _timed(torch, stream, fn, steps, warmup, world, dist, dev):
+    """Mean CUDA-event time (ms) of fn() over `steps` calls after `warmup`,
+    max over ranks."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world, dist, dev)
+
+
+def bench_msr(R, torch, dev, stream, args, peaks, world, dist):
+    """The MultiScaleRetention layer forward on X [2, 4096, 2048] (H 8, d_k 256,
+    d_v 512, xPos, chunk 128): four projections, retention, GroupNorm + swish
+    gate and the output projection.  Tensor-bound: 549.8 GFLOP of GEMMs plus
+    47.2 GFLOP of retention."""
+    B, N, dm, H, dk, dv = 2, 4096, 2048, 8, 256, 512
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0x5EED0005)
+    x = torch.randn((B, N, dm), generator=gen, device=dev).to(torch.bfloat16)
+    w = {n: (torch.randn(shape, generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+         for n, shape in (("wq", (dm, H * dk)), ("wk", (dm, H * dk)), ("wv", (dm, H * dv)), ("wg", (dm, H * dv)),
+                          ("wo", (H * dv, dm)))}
+    out = torch.empty((B, N, dm), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(R.ret_msr_workspace_bytes(B, N, dm, H, dk, dv), dtype=torch.uint8, device=dev)
+    g = gammas(H)
+
+    def fn():
+        R.ret_msr_forward(x, w["wq"], w["wk"], w["wv"], w["wg"], w["wo"], g, H=H, chunk=128, k_scale=dk ** -0.5,
+                          xpos=True, out=out, workspace=ws, stream=stream)
+
+    ms = _timed(torch, stream, fn, max(5, min(args.steps, 20)), 3, world, dist, dev)
+    R.ret_check_device_error()
+    M = B * N
+    gemm = 2 * M * dm * (2 * H * dk + 2 * H * dv) + 2 * M * H * dv * dm
+    ret = flops_per_token_head(128, dk, dv) * B * N * H
+    tf = (gemm + ret) / (ms / 1e3) / 1e12
+    return {"workload": "msr_layer_bf16_2x4096x2048_h8_256_512", "ms_per_step": round(ms, 4),
+            "tokens_per_s": round(world * M / (ms / 1e3), 1), "algo_flops": gemm + ret,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
+                         "kernels": "k_gemm (the 4 projections, fused rotation/zeta/swish epilogue), "
+                                    "k_chunkwise_ws, k_gn_gate, k_gemm (W_O)"}}
+
+
+def bench_fp32_small(R, torch, dev, stream, args, world, dist):
+    """The fp32 path at the exercise shape [1, 64, 8, 16], chunk 16 (CUDA cores;
+    136 KB of I/O, so the figure is launch latency)."""
+    B, N, H, d = 1, 64, 8, 16
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0x5EED0001)
+    q, k, v = (torch.randn((B, N, H, d), generator=gen, device=dev) for _ in range(3))
+    out = torch.empty((B, N, H, d), dtype=torch.float32, device=dev)
+    g = gammas(H)
+
+    def fn():
+        R.ret_forward_chunkwise(q, k, v, g, 16, out=out, stream=stream)
+
+    ms = _timed(torch, stream, fn, 50, 5, world, dist, dev)
+    R.ret_check_device_error()
+    return {"workload": "retention_f32_1x64x8x16", "us_per_call": round(ms * 1e3, 2),
+            "bound": "latency", "kernel": "k_chunkwise_simt"}
 
 
 # ---------------------------------------------------------- the oracle ---
@@ -431,6 +509,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-layer", action="store_true", help="skip the MSR-layer and fp32 small-shape timings")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--seq", type=int, default=WORKLOAD["N"],
                     help="sequence length of the chunkwise workload (smaller values make ncu captures short)")
