@@ -7,7 +7,8 @@ code.  Inputs arrive as float64 numpy arrays (the bf16- or fp32-rounded
 values, widened exactly), outputs are float64.
 
 The retention core (rotation, recurrent definition, parallel and chunkwise
-cross-check forms, decode step) is plain C in ``retention_oracle.c``; the
+cross-check forms, decode step, the gradients of the definition) is plain C
+in ``retention_oracle.c``; the
 MultiScaleRetention layer pieces (projections, per-head GroupNorm, swish gate,
 output projection) are in ``msr.py`` on numpy fp64.  Each function cites the
 passage of the pages it follows.
@@ -48,6 +49,7 @@ def _configure(lib):
     lib.orc_retention_parallel.argtypes = [dp, dp, dp, dp, i, i, i, i, i, dp, i]
     lib.orc_retention_chunkwise.argtypes = [dp, dp, dp, dp, i, i, i, i, i, i, dp, dp, i]
     lib.orc_decode_step.argtypes = [dp, dp, dp, dp, i, i, i, i, dp, dp, i]
+    lib.orc_retention_backward.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, dp, dp, dp, i]
     return lib
 
 
@@ -98,6 +100,44 @@ def xpos_rotate(x, pos_offset: int = 0, theta_base: float = 10000.0):
     assert d % 2 == 0
     _load().orc_xpos_rotate(_p(y), B, N, H, d, int(pos_offset), float(theta_base))
     return y
+
+
+def xpos_unrotate(x, pos_offset: int = 0, theta_base: float = 10000.0):
+    """Inverse of xpos_rotate (the transpose of each 2x2 rotation): pair
+    (2p, 2p+1) of position n turned by -n * theta_base^(-2p/d).  The
+    gradient of a rotated vector flows back through this."""
+    y = _f64(x).copy()
+    B, N, H, d = y.shape
+    assert d % 2 == 0
+    p = np.arange(d // 2)
+    theta = np.power(float(theta_base), -2.0 * p / d)
+    ang = (int(pos_offset) + np.arange(N))[:, None] * theta[None, :]      # [N, d/2]
+    c, s = np.cos(ang)[None, :, None, :], np.sin(ang)[None, :, None, :]
+    x0, x1 = y[..., 0::2].copy(), y[..., 1::2].copy()
+    y[..., 0::2] = x0 * c + x1 * s
+    y[..., 1::2] = -x0 * s + x1 * c
+    return y
+
+
+def retention_backward(q, k, v, dout, gammas, xpos: bool = False, pos_offset: int = 0,
+                       theta_base: float = 10000.0, nthreads: int = 0):
+    """Gradients (dq, dk, dv) of sum(out * dout) for out = retention of the
+    (optionally xPos-rotated) q, k and v: the derivatives of the definition
+    (P1 section 2.1, P3 Eq. 6) summed by brute force in C; with xpos the
+    gradients of the rotated q, k are turned back by the inverse rotation
+    (P1 sections 6.6 and 6.8)."""
+    q, k, v, do, g = _f64(q), _f64(k), _f64(v), _f64(dout), _f64(gammas)
+    if xpos:
+        q, k = xpos_rotate(q, pos_offset, theta_base), xpos_rotate(k, pos_offset, theta_base)
+    B, N, H, dk = q.shape
+    dv = v.shape[3]
+    assert k.shape == q.shape and v.shape[:3] == q.shape[:3] and do.shape == v.shape and g.shape == (H,)
+    dq, dkk, dvv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    _load().orc_retention_backward(_p(q), _p(k), _p(v), _p(do), _p(g), B, N, H, dk, dv, _p(dq), _p(dkk),
+                                   _p(dvv), int(nthreads))
+    if xpos:
+        dq, dkk = xpos_unrotate(dq, pos_offset, theta_base), xpos_unrotate(dkk, pos_offset, theta_base)
+    return dq, dkk, dvv
 
 
 def retention_recurrent(q, k, v, gammas, init_state=None, nthreads: int = 0):

@@ -251,3 +251,52 @@ void orc_decode_step(const double *q, const double *k, const double *v,
             for (int j = 0; j < dv; j++) ob[j] += qb[i] * S[(size_t)i * dv + j];
     }
 }
+
+/*
+ * Gradients of the definition (the recurrent form above, [P1] section 2.1,
+ * [P3] Eq. 6) with respect to q, k and v, for an upstream gradient dout of
+ * the output.  The pages train through the chunkwise form ([P3] training
+ * protocol) but print no backward pass; these are the derivatives of the
+ * unrolled definition o_n = sum_{m<=n} gamma^(n-m) (q_n . k_m) v_m, summed
+ * straight from it over every pair m <= n (brute force, O(N^2)):
+ *     dq_n += gamma^(n-m) (dout_n . v_m) k_m
+ *     dk_m += gamma^(n-m) (dout_n . v_m) q_n
+ *     dv_m += gamma^(n-m) (q_n . k_m)   dout_n
+ * q and k are the vectors the definition multiplies (rotated ones when the
+ * caller rotates); dq, dk, dv are overwritten.
+ */
+void orc_retention_backward(const double *q, const double *k, const double *v, const double *dout,
+                            const double *gammas, int B, int N, int H, int dk, int dv,
+                            double *dq, double *dkk, double *dvv, int nthreads) {
+    set_threads(nthreads);
+    int BH = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < BH; bh++) {
+        int b = bh / H, h = bh % H;
+        double gamma = gammas[h];
+        for (int n = 0; n < N; n++) {
+            for (int i = 0; i < dk; i++) {
+                dq[IDX4(b, n, h, i, N, H, dk)] = 0.0;
+                dkk[IDX4(b, n, h, i, N, H, dk)] = 0.0;
+            }
+            for (int j = 0; j < dv; j++) dvv[IDX4(b, n, h, j, N, H, dv)] = 0.0;
+        }
+        for (int n = 0; n < N; n++) {
+            const double *qn = q + IDX4(b, n, h, 0, N, H, dk);
+            const double *gn = dout + IDX4(b, n, h, 0, N, H, dv);
+            for (int m = 0; m <= n; m++) {
+                const double *km = k + IDX4(b, m, h, 0, N, H, dk);
+                const double *vm = v + IDX4(b, m, h, 0, N, H, dv);
+                double w = orc_gamma_pow(gamma, n - m);
+                double a = 0.0, g = 0.0;
+                for (int i = 0; i < dk; i++) a += qn[i] * km[i];
+                for (int j = 0; j < dv; j++) g += gn[j] * vm[j];
+                for (int i = 0; i < dk; i++) {
+                    dq[IDX4(b, n, h, i, N, H, dk)] += w * g * km[i];
+                    dkk[IDX4(b, m, h, i, N, H, dk)] += w * g * qn[i];
+                }
+                for (int j = 0; j < dv; j++) dvv[IDX4(b, m, h, j, N, H, dv)] += w * a * gn[j];
+            }
+        }
+    }
+}

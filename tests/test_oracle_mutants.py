@@ -29,6 +29,11 @@ MUTANTS = {
     "decode_no_decay": ("S[(size_t)i * dv + j] = gamma * S[(size_t)i * dv + j] + kb[i] * vb[j];",
                         "S[(size_t)i * dv + j] = S[(size_t)i * dv + j] + kb[i] * vb[j];"),
     "gamma_pow_zero_exponent": ("if (e == 0) return 1.0;", "if (e == 0) return gamma;"),
+    "backward_dk_on_the_query_row": ("dkk[IDX4(b, m, h, i, N, H, dk)] += w * g * qn[i];",
+                                     "dkk[IDX4(b, n, h, i, N, H, dk)] += w * g * qn[i];"),
+    "backward_dv_with_the_wrong_score": ("+= w * a * gn[j];", "+= w * g * gn[j];"),
+    "backward_dq_with_the_wrong_score": ("dq[IDX4(b, n, h, i, N, H, dk)] += w * g * km[i];",
+                                         "dq[IDX4(b, n, h, i, N, H, dk)] += w * a * km[i];"),
 }
 
 

@@ -303,3 +303,74 @@ def test_msr_layer_invariants():
     np.testing.assert_allclose(z1[:, :, 0], z[:, :, 1], atol=1e-12)
     # output = Z W_O
     np.testing.assert_allclose(out, z.reshape(1, 10, H * dv) @ W["wo"], atol=1e-12)
+
+
+# ---- gradients of the definition (oracle.retention_backward)
+
+def _loss(q, k, v, dout, g, xpos, off):
+    if xpos:
+        q, k = oracle.xpos_rotate(q, off), oracle.xpos_rotate(k, off)
+    out, _ = oracle.retention_recurrent(q, k, v, g)
+    return float((out * dout).sum())
+
+
+@pytest.mark.parametrize("xpos", [False, True])
+def test_backward_matches_finite_differences(xpos):
+    """<grad, d> equals the central difference of sum(out * dout) along a
+    random direction d, for each of q, k, v (the loss is cubic in the inputs,
+    so the difference is exact up to eps^2 and rounding)."""
+    rng = np.random.default_rng(11 + xpos)
+    B, N, H, dk, dv, off = 2, 7, 2, 6, 5, 3
+    q, k = rng.standard_normal((B, N, H, dk)), rng.standard_normal((B, N, H, dk))
+    v, dout = rng.standard_normal((B, N, H, dv)), rng.standard_normal((B, N, H, dv))
+    g = np.array([0.9, 0.55])
+    grads = oracle.retention_backward(q, k, v, dout, g, xpos=xpos, pos_offset=off)
+    eps = 1e-6
+    for idx, base in enumerate((q, k, v)):
+        d = rng.standard_normal(base.shape)
+        args_p = [q, k, v]
+        args_m = [q, k, v]
+        args_p[idx] = base + eps * d
+        args_m[idx] = base - eps * d
+        fd = (_loss(*args_p, dout, g, xpos, off) - _loss(*args_m, dout, g, xpos, off)) / (2 * eps)
+        an = float((grads[idx] * d).sum())
+        assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (idx, fd, an)
+
+
+def test_backward_single_entries_match_finite_differences():
+    """Entry by entry on a tiny case: every element of every gradient."""
+    rng = np.random.default_rng(5)
+    B, N, H, dk, dv = 1, 4, 1, 2, 3
+    q, k = rng.standard_normal((B, N, H, dk)), rng.standard_normal((B, N, H, dk))
+    v, dout = rng.standard_normal((B, N, H, dv)), rng.standard_normal((B, N, H, dv))
+    g = np.array([0.8])
+    grads = oracle.retention_backward(q, k, v, dout, g)
+    eps = 1e-6
+    for idx, base in enumerate((q, k, v)):
+        for pos in np.ndindex(base.shape):
+            d = np.zeros_like(base)
+            d[pos] = 1.0
+            a_p, a_m = [q, k, v], [q, k, v]
+            a_p[idx], a_m[idx] = base + eps * d, base - eps * d
+            fd = (_loss(*a_p, dout, g, False, 0) - _loss(*a_m, dout, g, False, 0)) / (2 * eps)
+            assert abs(fd - grads[idx][pos]) <= 1e-7 * max(1.0, abs(fd)), (idx, pos)
+
+
+def test_backward_gamma_zero_closed_form():
+    """gamma = 0: o_n = (q_n . k_n) v_n, so dq_n = (dout_n . v_n) k_n,
+    dk_n = (dout_n . v_n) q_n and dv_n = (q_n . k_n) dout_n."""
+    rng = np.random.default_rng(8)
+    q, k = rng.standard_normal((1, 5, 1, 3)), rng.standard_normal((1, 5, 1, 3))
+    v, dout = rng.standard_normal((1, 5, 1, 4)), rng.standard_normal((1, 5, 1, 4))
+    dq, dk, dv = oracle.retention_backward(q, k, v, dout, np.array([0.0]))
+    gv = (dout * v).sum(-1, keepdims=True)
+    qk = (q * k).sum(-1, keepdims=True)
+    assert np.allclose(dq, gv * k, rtol=0, atol=1e-14)
+    assert np.allclose(dk, gv * q, rtol=0, atol=1e-14)
+    assert np.allclose(dv, qk * dout, rtol=0, atol=1e-14)
+
+
+def test_unrotate_inverts_rotate():
+    x = np.random.default_rng(9).standard_normal((2, 6, 3, 8))
+    assert np.allclose(oracle.xpos_unrotate(oracle.xpos_rotate(x, 4), 4), x, rtol=0, atol=1e-14)
+    assert np.allclose(oracle.xpos_rotate(oracle.xpos_unrotate(x, 4), 4), x, rtol=0, atol=1e-14)
