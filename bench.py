@@ -273,6 +273,7 @@ def run_ours(args):
     if not args.no_decode:
         result["decode"] = bench_decode(R, torch, dev, stream, args, peaks, world, barrier, dist, rank)
     if not args.no_layer:
+        result["backward"] = bench_backward(R, torch, dev, stream, w, g, args, peaks, world, dist)
         result["msr_layer"] = bench_msr(R, torch, dev, stream, args, peaks, world, dist)
         result["fp32_small"] = bench_fp32_small(R, torch, dev, stream, args, world, dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -380,6 +381,39 @@ def _timed(torch, stream, fn, steps, warmup, world, dist, dev):
         b.record(stream)
     torch.cuda.synchronize()
     return max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world, dist, dev)
+
+
+def bench_backward(R, torch, dev, stream, w, g, args, peaks, world, dist):
+    """Gradients of the chunkwise forward (dq, dk, dv in fp32) on the same
+    workload: three tensor-core retention passes (dq and dk in two d_v slices
+    each), the anti-causal two on the time-reversed sequence.  Algorithmic
+    FLOPs: three times the forward's."""
+    B, N, H, dk, dv, C = w["B"], w["N"], w["H"], w["dk"], w["dv"], w["chunk"]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0x5EED0006)
+    sc = dk ** -0.5
+    q = (torch.randn((B, N, H, dk), generator=gen, device=dev) * sc).to(torch.bfloat16)
+    k = (torch.randn((B, N, H, dk), generator=gen, device=dev) * sc).to(torch.bfloat16)
+    v = torch.randn((B, N, H, dv), generator=gen, device=dev).to(torch.bfloat16)
+    do = torch.randn((B, N, H, dv), generator=gen, device=dev).to(torch.bfloat16)
+    dq = torch.empty((B, N, H, dk), dtype=torch.float32, device=dev)
+    dkk = torch.empty_like(dq)
+    dvv = torch.empty((B, N, H, dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(R.ret_backward_workspace_bytes(B, N, H, dk, dv, C, torch.bfloat16, True), dtype=torch.uint8,
+                     device=dev)
+
+    def fn():
+        R.ret_backward_chunkwise(q, k, v, do, g, C, workspace=ws, dq=dq, dk=dkk, dv=dvv, xpos=True, stream=stream)
+
+    ms = _timed(torch, stream, fn, max(3, min(args.steps, 10)), 2, world, dist, dev)
+    R.ret_check_device_error()
+    flops = 3 * flops_per_token_head(C, dk, dv) * B * N * H
+    tf = flops / (ms / 1e3) / 1e12
+    return {"workload": w["workload"], "ms_per_step": round(ms, 4), "tokens_per_s": round(world * B * N / (ms / 1e3), 1),
+            "algo_flops": flops,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(tf / peaks["bf16_tflops"], 4),
+                         "kernels": "5 x (k_prep_qk + k_chunkwise_ws), k_reverse_rows, k_xpos_rotate"}}
 
 
 def bench_msr(R, torch, dev, stream, args, peaks, world, dist):

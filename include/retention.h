@@ -169,6 +169,39 @@ ret_status ret_forward_chunkwise_prepared(const void* q, const void* k, const vo
                                           const void* workspace, size_t workspace_bytes);
 
 /*
+ * Gradients of the chunkwise forward: given dout = dL/d(out), the gradients
+ * of L with respect to q, k and v of ret_forward_chunkwise (same q, k, v,
+ * gammas, sizes, xpos, pos_offset, theta_base).  They are the derivatives of
+ * the definition o_n = sum_{m<=n} gamma^(n-m) (q'_n . k'_m) v_m ("Hybrid
+ * Architectures ...", section 2.1; RetNet paper summary, Eq. 6), with
+ * q' = R q and k' = R k the rotated vectors (section 6.8; identity when
+ * xpos = 0):
+ *     dq = R^T sum_{m<=n} gamma^(n-m) (dout_n . v_m) k'_m
+ *     dk = R^T sum_{n>=m} gamma^(n-m) (dout_n . v_m) q'_n
+ *     dv =     sum_{n>=m} gamma^(n-m) (q'_n . k'_m)  dout_n
+ * The pages train through the chunkwise form but print no backward pass;
+ * these are its plain derivatives.  Each sum is computed as a tensor-core
+ * chunkwise retention pass (the two anti-causal ones on the time-reversed
+ * sequence), so the same path constraints apply: bf16 q, k, v, dout
+ * (device [B, N, H, d], 16-byte aligned), chunk = 128, dk 128 or 256, dv a
+ * multiple of 128 and every gamma_h^128 >= 2^-60, else RET_ERR_UNSUPPORTED.
+ * dq, dk: device fp32 [B, N, H, dk]; dv: device fp32 [B, N, H, dv]; written,
+ * 16-byte aligned, overlapping nothing else.
+ * workspace: device, 256-byte aligned, at least
+ * ret_backward_workspace_bytes(...) bytes (about 2x(q, k, v, dout) in bf16
+ * plus k and v gradients in fp32), scratch, overlapping nothing else.
+ */
+size_t ret_backward_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk, ret_dtype in_dt,
+                                    int xpos);
+
+ret_status ret_backward_chunkwise(const void* q, const void* k, const void* v, const void* dout,
+                                  const double* gammas, int B, int N, int H, int dk, int dv,
+                                  int chunk, float* dq, float* dk_out, float* dv_out,
+                                  cudaStream_t stream, ret_dtype in_dt, int xpos,
+                                  int64_t pos_offset, double theta_base, void* workspace,
+                                  size_t workspace_bytes);
+
+/*
  * Allocation-free variant of ret_forward_chunkwise_ws, for callers that
  * cannot allocate device memory at call time: for example a plug-in that runs
  * inside a host framework which owns all device memory and hands out no

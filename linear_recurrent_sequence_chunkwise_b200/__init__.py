@@ -19,6 +19,7 @@ import torch
 __all__ = [
     "RetentionError", "lib", "ret_xpos_rotate", "ret_forward_chunkwise", "ret_forward_chunkwise_ws",
     "ret_chunkwise_workspace_bytes", "ret_chunkwise_prepare", "ret_forward_chunkwise_prepared",
+    "ret_backward_chunkwise", "ret_backward_workspace_bytes",
     "ret_forward_chunkwise_noalloc", "ret_chunkwise_noalloc_max_bytes",
     "ret_decode_step", "ret_msr_forward", "ret_msr_workspace_bytes",
     "ret_linear_bf16",
@@ -55,6 +56,10 @@ def _load_library():
     L.ret_forward_chunkwise_ws.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d, vp,
                                            ctypes.c_size_t]
     L.ret_forward_chunkwise_noalloc.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d]
+    L.ret_backward_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+    L.ret_backward_workspace_bytes.restype = ctypes.c_size_t
+    L.ret_backward_chunkwise.argtypes = [vp, vp, vp, vp, dp, i, i, i, i, i, i, vp, vp, vp, vp, i, i, i64, d, vp,
+                                         ctypes.c_size_t]
     L.ret_chunkwise_prepare.argtypes = [vp, vp, dp, i, i, i, i, i, i, vp, i, i, i64, d, vp, ctypes.c_size_t]
     L.ret_forward_chunkwise_prepared.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, vp, vp, vp, vp, i, i, i, i64, d,
                                                  vp, ctypes.c_size_t]
@@ -75,7 +80,7 @@ def _load_library():
     L.ret_last_error_string.argtypes = []
     for name in ("ret_xpos_rotate", "ret_forward_chunkwise", "ret_forward_chunkwise_ws",
                  "ret_forward_chunkwise_noalloc", "ret_chunkwise_prepare", "ret_forward_chunkwise_prepared",
-                 "ret_decode_step",
+                 "ret_backward_chunkwise", "ret_decode_step",
                  "ret_forward_parallel",
                  "ret_forward_recurrent", "ret_check_device_error", "ret_msr_forward", "ret_linear_bf16"):
         getattr(L, name).restype = ctypes.c_int
@@ -223,6 +228,33 @@ def ret_forward_chunkwise_prepared(q, k, v, gammas, chunk: int, workspace, out=N
                                               _dt(out.dtype), int(bool(xpos)), int(pos_offset), float(theta_base),
                                               _ptr(workspace, "workspace"), nbytes))
     return (out, final_state) if final_state is not None else out
+
+
+def ret_backward_workspace_bytes(B, N, H, dk, dv, chunk, in_dtype=torch.bfloat16, xpos: bool = False) -> int:
+    """Workspace bytes of ret_backward_chunkwise (0: shape not supported)."""
+    return int(lib.ret_backward_workspace_bytes(B, N, H, dk, dv, int(chunk), _dt(in_dtype), int(bool(xpos))))
+
+
+def ret_backward_chunkwise(q, k, v, dout, gammas, chunk: int, workspace=None, dq=None, dk=None, dv=None,
+                           xpos: bool = False, pos_offset: int = 0, theta_base: float = 10000.0, stream=None):
+    """Gradients (dq, dk, dv) in fp32 of sum(out * dout) for the chunkwise
+    forward of the same arguments."""
+    B, N, H, dk_, dv_ = _seq_shapes(q, k, v)
+    if tuple(dout.shape) != (B, N, H, dv_):
+        raise ValueError("dout must be [B, N, H, dv]")
+    dq = torch.empty((B, N, H, dk_), dtype=torch.float32, device=q.device) if dq is None else dq
+    dk = torch.empty((B, N, H, dk_), dtype=torch.float32, device=q.device) if dk is None else dk
+    dv = torch.empty((B, N, H, dv_), dtype=torch.float32, device=q.device) if dv is None else dv
+    if workspace is None:
+        nb = ret_backward_workspace_bytes(B, N, H, dk_, dv_, chunk, q.dtype, xpos)
+        workspace = torch.empty(max(nb, 1), dtype=torch.uint8, device=q.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib.ret_backward_chunkwise(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(dout, "dout"),
+                                      _gammas(gammas, H), B, N, H, dk_, dv_, int(chunk), _ptr(dq, "dq"),
+                                      _ptr(dk, "dk"), _ptr(dv, "dv"), _stream(stream), _dt(q.dtype),
+                                      int(bool(xpos)), int(pos_offset), float(theta_base),
+                                      _ptr(workspace, "workspace"), nbytes))
+    return dq, dk, dv
 
 
 def ret_chunkwise_noalloc_max_bytes() -> int:

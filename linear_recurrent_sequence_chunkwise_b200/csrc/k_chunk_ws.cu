@@ -75,7 +75,8 @@ __global__ void __launch_bounds__(256) k_prep_qk(const __nv_bfloat16* __restrict
                                                   const __nv_bfloat16* __restrict__ k,
                                                   __nv_bfloat16* __restrict__ q_rot,
                                                   __nv_bfloat16* __restrict__ k_out, HeadConsts hc, int B, int N,
-                                                  int H, int chunk, int xpos, long long pos0, double log2base) {
+                                                  int H, int chunk, int xpos, long long pos0, double log2base,
+                                                  int q_ld, int k_ld) {
     // theta_p = base^(-2p/DK), once per block (fp64, as the rotation's reference)
     __shared__ double s_theta[DK / 2];
     for (int i = threadIdx.x; i < DK / 2; i += blockDim.x) s_theta[i] = exp2(-2.0 * i / DK * log2base);
@@ -103,9 +104,9 @@ __global__ void __launch_bounds__(256) k_prep_qk(const __nv_bfloat16* __restrict
 #pragma unroll
             for (int hh = 0; hh < kHB; hh++) {
                 if (h0 + hh < H) {
-                    const size_t e = ((size_t)t * H + h0 + hh) * DK + 8 * g;
-                    kw[hh] = __ldg(reinterpret_cast<const uint4*>(k + e));
-                    if (xpos) qw[hh] = __ldg(reinterpret_cast<const uint4*>(q + e));
+                    const size_t row = (size_t)t * H + h0 + hh;
+                    kw[hh] = __ldg(reinterpret_cast<const uint4*>(k + row * k_ld + 8 * g));
+                    if (xpos) qw[hh] = __ldg(reinterpret_cast<const uint4*>(q + row * q_ld + 8 * g));
                 }
             }
 #pragma unroll
@@ -144,6 +145,7 @@ struct WsParams {
     float* fstate;
     const float* istate;  // state before the first token, [B, H, DK, dv] fp32, or null (zero)
     int N, H, dv;
+    int accumulate;       // fp32 out only: out += result
     int nmain;            // CTAs: B * H * (dv / 64), one per (b, h, 64 value columns)
     HeadConsts hc;
 };
@@ -581,10 +583,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                         }
                     } else {
 #pragma unroll
-                        for (int c4 = 0; c4 < 8; c4++)
-                            reinterpret_cast<float4*>(dst)[c4] =
-                                make_float4(__uint_as_float(o[4 * c4 + 0]) * sc, __uint_as_float(o[4 * c4 + 1]) * sc,
-                                            __uint_as_float(o[4 * c4 + 2]) * sc, __uint_as_float(o[4 * c4 + 3]) * sc);
+                        for (int c4 = 0; c4 < 8; c4++) {
+                            float4 y = make_float4(__uint_as_float(o[4 * c4 + 0]) * sc, __uint_as_float(o[4 * c4 + 1]) * sc,
+                                                   __uint_as_float(o[4 * c4 + 2]) * sc, __uint_as_float(o[4 * c4 + 3]) * sc);
+                            if (p.accumulate) {
+                                const float4 x = reinterpret_cast<const float4*>(dst)[c4];
+                                y.x += x.x;
+                                y.y += x.y;
+                                y.z += x.z;
+                                y.w += x.w;
+                            }
+                            reinterpret_cast<float4*>(dst)[c4] = y;
+                        }
                     }
                 }
             }
@@ -627,15 +637,16 @@ bool chunkwise_ws_supported(const RetArgs& a) {
 }
 
 // Tensor maps and per-launch fields shared by both kernel variants.
-static ret_status fill_params(WsParams* p, const RetArgs& a, const void* q_src, const void* k_prime) {
+static ret_status fill_params(WsParams* p, const RetArgs& a, const void* q_src, int q_pitch, const void* k_prime) {
     memset(p, 0, sizeof(*p));
-    const uint64_t B = a.B, N = a.N, H = a.H, dk = a.dk, dv = a.dv;
+    const uint64_t B = a.B, N = a.N, H = a.H, dk = a.dk, dv = a.dv, qp = (uint64_t)q_pitch;
     const uint64_t dq[4] = {dk, H, N, B};
     const uint64_t sq[3] = {dk * 2, H * dk * 2, N * H * dk * 2};
+    const uint64_t sqq[3] = {qp * 2, H * qp * 2, N * H * qp * 2};
     const uint32_t box[4] = {64, 1, (uint32_t)kC, 1};
     const uint64_t dvv[4] = {dv, H, N, B};
     const uint64_t svv[3] = {dv * 2, H * dv * 2, N * H * dv * 2};
-    if (!make_tmap_bf16(&p->tq, q_src, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!make_tmap_bf16(&p->tq, q_src, 4, dq, sqq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_bf16(&p->tk, k_prime, 4, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_bf16(&p->tv, a.v, 4, dvv, svv, box, CU_TENSOR_MAP_SWIZZLE_128B))
         return RET_ERR_CUDA;
@@ -647,12 +658,14 @@ static ret_status fill_params(WsParams* p, const RetArgs& a, const void* q_src, 
     p->dv = a.dv;
     p->hc = a.hc;
     p->nmain = a.B * a.H * (a.dv / kW);
+    p->accumulate = a.accumulate;
     return RET_OK;
 }
 
-ret_status launch_chunkwise_main(const RetArgs& a, const void* q_src, const void* k_prime, cudaStream_t s) {
+ret_status launch_chunkwise_main(const RetArgs& a, const void* q_src, int q_pitch, const void* k_prime,
+                                 cudaStream_t s) {
     WsParams p;
-    ret_status st = fill_params(&p, a, q_src, k_prime);
+    ret_status st = fill_params(&p, a, q_src, q_pitch, k_prime);
     if (st != RET_OK) return st;
     const bool f32 = a.out_dt == RET_F32;
     if (a.dk == 256) return f32 ? launch_main<256, float>(p, s) : launch_main<256, __nv_bfloat16>(p, s);
@@ -673,17 +686,20 @@ ret_status launch_chunkwise_prep(const RetArgs& a, void* ws, cudaStream_t s) {
     const double lb = log2(a.theta_base);
     if (a.dk == 256)
         k_prep_qk<256><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, q_rot, k_out,
-                                               a.hc, a.B, a.N, a.H, a.chunk, a.xpos, a.pos_offset, lb);
+                                               a.hc, a.B, a.N, a.H, a.chunk, a.xpos, a.pos_offset, lb,
+                                               a.q_ld ? a.q_ld : a.dk, a.k_ld ? a.k_ld : a.dk);
     else
         k_prep_qk<128><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, q_rot, k_out,
-                                               a.hc, a.B, a.N, a.H, a.chunk, a.xpos, a.pos_offset, lb);
+                                               a.hc, a.B, a.N, a.H, a.chunk, a.xpos, a.pos_offset, lb,
+                                               a.q_ld ? a.q_ld : a.dk, a.k_ld ? a.k_ld : a.dk);
     return check_launch("chunkwise (workspace path): prep");
 }
 
 ret_status launch_chunkwise_prepared(const RetArgs& a, void* ws, cudaStream_t s) {
     __nv_bfloat16 *k_out, *q_rot;
     ws_parts(a, ws, &k_out, &q_rot);
-    return launch_chunkwise_main(a, a.xpos ? (const void*)q_rot : a.q, k_out, s);
+    // q_rot in the workspace is contiguous; a raw q keeps its row pitch
+    return launch_chunkwise_main(a, a.xpos ? (const void*)q_rot : a.q, a.xpos || !a.q_ld ? a.dk : a.q_ld, k_out, s);
 }
 
 ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s) {

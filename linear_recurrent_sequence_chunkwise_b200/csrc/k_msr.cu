@@ -111,7 +111,7 @@ ret_status launch_msr(const MsrArgs& m, cudaStream_t s) {
     a.B = m.B; a.N = m.N; a.H = m.H; a.dk = m.dk; a.dv = m.dv; a.chunk = m.chunk;
     a.in_dt = RET_BF16; a.out_dt = RET_F32; a.xpos = 0; a.pos_offset = 0; a.theta_base = 10000.0;
     a.hc = m.hc;
-    st = launch_chunkwise_main(a, q_rot, k_pr, s);
+    st = launch_chunkwise_main(a, q_rot, m.dk, k_pr, s);
     if (st != RET_OK) return st;
 
     // 3. GroupNorm per (token, head) times swish(G), written over swish(G)

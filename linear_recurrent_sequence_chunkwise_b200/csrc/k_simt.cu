@@ -17,7 +17,7 @@ namespace ret {
 
 template <typename T>
 __global__ void k_xpos_rotate(T* __restrict__ x, int N, int H, int d, size_t total_pairs,
-                              long long pos_offset, double log2base) {
+                              long long pos_offset, double log2base, float sign) {
     extern __shared__ double s_theta[];
     const int half = d / 2;
     for (int p = threadIdx.x; p < half; p += blockDim.x) s_theta[p] = exp2(-2.0 * p / d * log2base);
@@ -29,6 +29,7 @@ __global__ void k_xpos_rotate(T* __restrict__ x, int N, int H, int d, size_t tot
         const int n = (int)((row / H) % N);
         float sn, cs;
         sincosf(rot_angle(pos_offset + n, s_theta[p]), &sn, &cs);
+        sn *= sign;  // -1: the inverse (transposed) rotation
         const size_t e = row * d + 2 * p;
         const float x0 = ld_as_float(x, e), x1 = ld_as_float(x, e + 1);
         st_from_float(x, e, x0 * cs - x1 * sn);
@@ -37,7 +38,7 @@ __global__ void k_xpos_rotate(T* __restrict__ x, int N, int H, int d, size_t tot
 }
 
 ret_status launch_xpos_rotate(void* x, ret_dtype dt, int B, int N, int H, int d, long long pos_offset,
-                              double theta_base, cudaStream_t s) {
+                              double theta_base, cudaStream_t s, bool inverse) {
     const size_t total = (size_t)B * N * H * (d / 2);
     const int threads = 256;
     const int blocks = (int)std::min<size_t>((total + threads - 1) / threads, 148 * 16);
@@ -45,9 +46,10 @@ ret_status launch_xpos_rotate(void* x, ret_dtype dt, int B, int N, int H, int d,
     if (smem > 48 * 1024) return fail(RET_ERR_UNSUPPORTED, "ret_xpos_rotate: d too large");
     const double lb = log2(theta_base);
     if (dt == RET_BF16)
-        k_xpos_rotate<<<blocks, threads, smem, s>>>((__nv_bfloat16*)x, N, H, d, total, pos_offset, lb);
+        k_xpos_rotate<<<blocks, threads, smem, s>>>((__nv_bfloat16*)x, N, H, d, total, pos_offset, lb,
+                                                    inverse ? -1.f : 1.f);
     else
-        k_xpos_rotate<<<blocks, threads, smem, s>>>((float*)x, N, H, d, total, pos_offset, lb);
+        k_xpos_rotate<<<blocks, threads, smem, s>>>((float*)x, N, H, d, total, pos_offset, lb, inverse ? -1.f : 1.f);
     return check_launch("ret_xpos_rotate");
 }
 

@@ -15,6 +15,11 @@ struct RetArgs {
     void* out;
     float* final_state;          // may be null
     const float* initial_state;  // may be null (zero state); workspace path only
+    // Workspace path only: elements between consecutive (token, head) rows of
+    // q and of k (0: dk, i.e. contiguous), so that a column slice of a wider
+    // tensor can serve as q or k; and accumulate = 1 adds the result into an
+    // fp32 out instead of storing it.
+    int q_ld, k_ld, accumulate;
     int B, N, H, dk, dv, chunk;
     ret_dtype in_dt, out_dt;
     int xpos;
@@ -24,8 +29,9 @@ struct RetArgs {
     double gamma[kMaxHeads];
 };
 
+// inverse: turn by -angle (the transpose of each rotation).
 ret_status launch_xpos_rotate(void* x, ret_dtype dt, int B, int N, int H, int d, long long pos_offset,
-                              double theta_base, cudaStream_t s);
+                              double theta_base, cudaStream_t s, bool inverse = false);
 ret_status launch_chunkwise_simt(const RetArgs& a, cudaStream_t s);
 ret_status launch_chunkwise_tc(const RetArgs& a, cudaStream_t s);
 ret_status launch_parallel_simt(const RetArgs& a, cudaStream_t s);
@@ -50,7 +56,25 @@ ret_status launch_chunkwise_prepared(const RetArgs& a, void* ws, cudaStream_t s)
 size_t chunkwise_static_ws_bytes();
 ret_status launch_chunkwise_static(const RetArgs& a, cudaStream_t s);
 // The tensor-core kernel alone, on prepared q_rot (or q) and k' (zeta-scaled keys).
-ret_status launch_chunkwise_main(const RetArgs& a, const void* q_rot, const void* k_prime, cudaStream_t s);
+// q_rot: [B, N, H, dk] rows q_pitch elements apart.
+ret_status launch_chunkwise_main(const RetArgs& a, const void* q_rot, int q_pitch, const void* k_prime,
+                                 cudaStream_t s);
+
+// Gradients of chunkwise retention (k_backward.cu): bf16 q, k, v, dout
+// [B, N, H, d], fp32 dq, dk, dv.
+struct BwdArgs {
+    const void *q, *k, *v, *dout;
+    float *dq, *dkk, *dvv;
+    int B, N, H, dk, dv, chunk;
+    int xpos;
+    long long pos_offset;
+    double theta_base;
+    HeadConsts hc;
+    void* workspace;
+};
+bool backward_supported(const BwdArgs& a);
+size_t backward_ws_bytes(const BwdArgs& a);
+ret_status launch_backward(const BwdArgs& a, cudaStream_t s);
 
 struct MsrArgs {
     const void *X, *Wq, *Wk, *Wv, *Wg, *Wo;

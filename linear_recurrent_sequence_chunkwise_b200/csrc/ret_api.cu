@@ -83,6 +83,7 @@ static ret_status make_args(RetArgs* a, const char* who, const void* q, const vo
             return fail(RET_ERR_INVALID_ARG, "%s: final_state overlaps another buffer", who);
     }
     a->q = q; a->k = k; a->v = v; a->out = out; a->final_state = final_state; a->initial_state = nullptr;
+    a->q_ld = 0; a->k_ld = 0; a->accumulate = 0;
     a->B = B; a->N = N; a->H = H; a->dk = dk; a->dv = dv; a->chunk = chunk;
     a->in_dt = in_dt; a->out_dt = out_dt;
     a->xpos = xpos ? 1 : 0; a->pos_offset = pos_offset; a->theta_base = xpos ? theta_base : 10000.0;
@@ -244,6 +245,78 @@ ret_status ret_forward_chunkwise_prepared(const void* q, const void* k, const vo
     st = check_workspace(a, who, workspace, workspace_bytes, true);
     if (st != RET_OK) return st;
     return launch_chunkwise_prepared(a, const_cast<void*>(workspace), stream);
+}
+
+static void fill_bwd(BwdArgs* b, const void* q, const void* k, const void* v, const void* dout, int B, int N, int H,
+                     int dk, int dv, int chunk, int xpos, int64_t pos_offset, double theta_base) {
+    memset(b, 0, sizeof(*b));
+    b->q = q; b->k = k; b->v = v; b->dout = dout;
+    b->B = B; b->N = N; b->H = H; b->dk = dk; b->dv = dv; b->chunk = chunk;
+    b->xpos = xpos ? 1 : 0; b->pos_offset = pos_offset; b->theta_base = xpos ? theta_base : 10000.0;
+}
+
+size_t ret_backward_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk, ret_dtype in_dt, int xpos) {
+    if (B < 1 || N < 1 || H < 1 || H > kMaxHeads || dk < 1 || dv < 1 || chunk < 1 || in_dt != RET_BF16) return 0;
+    BwdArgs b;
+    fill_bwd(&b, nullptr, nullptr, nullptr, nullptr, B, N, H, dk, dv, chunk, xpos, 0, 10000.0);
+    return backward_supported(b) ? backward_ws_bytes(b) : 0;
+}
+
+ret_status ret_backward_chunkwise(const void* q, const void* k, const void* v, const void* dout,
+                                  const double* gammas, int B, int N, int H, int dk, int dv, int chunk, float* dq,
+                                  float* dk_out, float* dv_out, cudaStream_t stream, ret_dtype in_dt, int xpos,
+                                  int64_t pos_offset, double theta_base, void* workspace, size_t workspace_bytes) {
+    t_err[0] = 0;
+    const char* who = "ret_backward_chunkwise";
+    if (!q || !k || !v || !dout || !dq || !dk_out || !dv_out)
+        return fail(RET_ERR_INVALID_ARG, "%s: NULL q, k, v, dout, dq, dk or dv", who);
+    if (B < 1 || N < 1 || H < 1 || dk < 1 || dv < 1 || chunk < 1)
+        return fail(RET_ERR_INVALID_ARG, "%s: sizes must be >= 1", who);
+    if (!is_dtype(in_dt)) return fail(RET_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    ret_status st = check_gammas(gammas, H, who);
+    if (st != RET_OK) return st;
+    if (xpos && (dk % 2 != 0)) return fail(RET_ERR_INVALID_ARG, "%s: xpos needs an even dk", who);
+    if (xpos && !(theta_base > 0.0 && isfinite(theta_base)))
+        return fail(RET_ERR_INVALID_ARG, "%s: theta_base must be finite and > 0", who);
+    if ((size_t)B * N * H * (size_t)(dk > dv ? dk : dv) > ((size_t)1 << 40))
+        return fail(RET_ERR_INVALID_ARG, "%s: problem too large", who);
+    for (const void* p : {q, k, v, dout, (const void*)dq, (const void*)dk_out, (const void*)dv_out})
+        if (!aligned(p, 16)) return fail(RET_ERR_INVALID_ARG, "%s: device pointers must be 16-byte aligned", who);
+    BwdArgs b;
+    fill_bwd(&b, q, k, v, dout, B, N, H, dk, dv, chunk, xpos, pos_offset, theta_base);
+    b.dq = dq; b.dkk = dk_out; b.dvv = dv_out;
+    make_head_consts(gammas, H, &b.hc);
+    if (in_dt != RET_BF16 || !backward_supported(b))
+        return fail(RET_ERR_UNSUPPORTED,
+                    "%s: needs bf16 inputs, chunk 128, dk 128 or 256, dv a multiple of 128 and every "
+                    "gamma_h^128 >= 2^-60",
+                    who);
+    const size_t need = backward_ws_bytes(b);
+    if (!workspace || workspace_bytes < need)
+        return fail(RET_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed (got %zu)", who, need,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (!aligned(workspace, 256)) return fail(RET_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+    const size_t ntok = (size_t)B * N * H;
+    const size_t bq = ntok * dk * 2, bv = ntok * dv * 2, gq = ntok * dk * 4, gv = ntok * dv * 4;
+    const void* ins[4] = {q, k, v, dout};
+    const size_t insz[4] = {bq, bq, bv, bv};
+    const void* outs[3] = {dq, dk_out, dv_out};
+    const size_t outsz[3] = {gq, gq, gv};
+    for (int i = 0; i < 3; i++) {
+        if (overlaps(outs[i], outsz[i], workspace, need))
+            return fail(RET_ERR_INVALID_ARG, "%s: an output overlaps the workspace", who);
+        for (int j = 0; j < 4; j++)
+            if (overlaps(outs[i], outsz[i], ins[j], insz[j]))
+                return fail(RET_ERR_INVALID_ARG, "%s: an output overlaps an input", who);
+        for (int j = i + 1; j < 3; j++)
+            if (overlaps(outs[i], outsz[i], outs[j], outsz[j]))
+                return fail(RET_ERR_INVALID_ARG, "%s: outputs overlap", who);
+    }
+    for (int j = 0; j < 4; j++)
+        if (overlaps(workspace, need, ins[j], insz[j]))
+            return fail(RET_ERR_INVALID_ARG, "%s: workspace overlaps an input", who);
+    b.workspace = workspace;
+    return launch_backward(b, stream);
 }
 
 ret_status ret_forward_chunkwise_noalloc(const void* q, const void* k, const void* v, const double* gammas, int B,

@@ -165,3 +165,35 @@ def test_prepare_rejects_bad_arguments(kw, status):
 def test_prepared_rejects_bad_arguments(kw, status):
     assert prepared_call(**kw) == status, (kw, R.ret_last_error_string())
     assert R.ret_last_error_string()
+
+
+def backward_call(q=P, k=P2, v=P3, do=ctypes.c_void_p(0x40000), dq=ctypes.c_void_p(0xC0000000),
+                  dk_=ctypes.c_void_p(0xD0000000), dv_=ctypes.c_void_p(0xE0000000), dk=128, dv=128, in_dt=1,
+                  ws=WS, nbytes=None):
+    if nbytes is None:   # exactly the workspace this shape needs: [WS, WS + nbytes) overlaps nothing above
+        nbytes = R.ret_backward_workspace_bytes(1, 64, 2, 128, 128, 128, torch.bfloat16, False)
+        assert 0 < nbytes < 0x20000000
+    return R.lib.ret_backward_chunkwise(q, k, v, do, G2, 1, 64, 2, dk, dv, 128, dq, dk_, dv_, S0, in_dt, 0, 0, 1e4,
+                                        ws, nbytes)
+
+
+def test_backward_workspace_size():
+    assert R.ret_backward_workspace_bytes(1, 64, 2, 128, 128, 128, torch.bfloat16, False) > 0
+    assert R.ret_backward_workspace_bytes(1, 64, 2, 128, 192, 128, torch.bfloat16, False) == 0   # dv % 128
+    assert R.ret_backward_workspace_bytes(1, 64, 2, 64, 128, 128, torch.bfloat16, False) == 0    # dk
+    assert R.ret_backward_workspace_bytes(1, 64, 2, 128, 128, 64, torch.bfloat16, False) == 0    # chunk
+    assert R.ret_backward_workspace_bytes(1, 64, 2, 128, 128, 128, torch.float32, False) == 0    # fp32 inputs
+
+
+@needs_no_gpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(dq=None), 1), (dict(ws=None), 1), (dict(nbytes=1000), 1),
+    (dict(dq=ctypes.c_void_p(0xC0000004)), 1),                    # misaligned gradient
+    (dict(dk_=ctypes.c_void_p(0xC0000000)), 1),                   # dk overlaps dq
+    (dict(dq=ctypes.c_void_p(0x10000)), 1),                       # dq overlaps q
+    (dict(ws=ctypes.c_void_p(0xC0000000)), 1),                    # workspace overlaps dq
+    (dict(dk=64), 2), (dict(dv=192), 2), (dict(in_dt=0), 2),
+])
+def test_backward_rejects_bad_arguments(kw, status):
+    assert backward_call(**kw) == status, (kw, R.ret_last_error_string())
+    assert R.ret_last_error_string()
