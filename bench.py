@@ -413,7 +413,7 @@ def bench_backward(R, torch, dev, stream, w, g, args, peaks, world, dist):
             "algo_flops": flops,
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": round(tf / peaks["bf16_tflops"], 4),
-                         "kernels": "5 x (k_prep_qk + k_chunkwise_ws), 7 x k_row_transform"}}
+                         "kernels": "5 x (k_prep_qk + k_chunkwise_ws), 6 x k_row_transform"}}
 
 
 def bench_msr(R, torch, dev, stream, args, peaks, world, dist):

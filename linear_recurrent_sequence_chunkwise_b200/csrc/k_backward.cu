@@ -12,12 +12,14 @@
 // dO, key v and value k'; dk' and dv are anti-causal, i.e. causal on the
 // time-reversed sequence (query v, key dO, value q' and query k', key q',
 // value dO).  dq' and dk' contract over d_v, which the tensor-core kernel
-// takes in column slices of 128 or 256 (strided views of v and dO), adding
-// the slices in fp32.  With xPos, q' = R q and k' = R k, so dq = R^T dq' and
-// dk = R^T dk' (the inverse rotation, section 6.8).  The dq passes run on the
-// caller's stream and the dk passes beside them on a second stream of the
-// library's, joined back before the call returns: each pass fills only
-// B * H * dk / 64 SMs.
+// takes in column slices of 128 or 256 (strided views of v and dO), each
+// slice's result added into the fp32 gradient by the kernel's epilogue; the
+// anti-causal passes store row n of their output at row N-1-n, i.e. back in
+// time order.  With xPos, q' = R q and k' = R k, so dq = R^T dq' and
+// dk = R^T dk' (the inverse rotation, section 6.8), applied in place at the
+// end.  The dq and dv passes run on the caller's stream and the dk passes
+// beside them on a second stream of the library's, joined back before the
+// call returns: a pass of d_v slice width fills only B * H * dk / 64 SMs.
 #include <algorithm>
 #include <cstring>
 #include <mutex>
@@ -61,11 +63,12 @@ __device__ __forceinline__ void store8(float* p, const float* x) {
 // them, turns each pair (2p, 2p+1) of every head by sign * (pos0 + t) *
 // theta_p (sign 0: no rotation; -1: the inverse rotation), and writes the
 // row to dst at (rev_dst ? N-1-t : t) and, if dst2 is set, to dst2 at N-1-t.
+// With nsrc = 1 and rev_src == rev_dst, src and dst may be the same tensor.
 // The sine and cosine of each (token, pair) are evaluated once for all
 // heads; the loads of kHB heads are issued together.
 template <typename Tin, typename Tout>
-__global__ void __launch_bounds__(256) k_row_transform(const Tin* __restrict__ src, int nsrc, size_t nsrc_stride,
-                                                       Tout* __restrict__ dst, Tout* __restrict__ dst2, int B, int N,
+__global__ void __launch_bounds__(256) k_row_transform(const Tin* src, int nsrc, size_t nsrc_stride, Tout* dst,
+                                                       Tout* __restrict__ dst2, int B, int N,
                                                        int H, int d, int rev_src, int rev_dst, float sign,
                                                        long long pos0, double log2base) {
     constexpr int kHB = 4;
@@ -134,12 +137,11 @@ ret_status row_transform(const void* src, int nsrc, size_t nsrc_stride, void* ds
 int dv_slice(int dv) { return dv % 256 == 0 ? 256 : 128; }
 
 struct BwdLayout {
-    size_t kr, kr_rev, qr_rev, v_rev, do_rev, inner, inner2, dq_parts, dk_parts, dv_rev, total;
+    size_t kr, kr_rev, qr_rev, v_rev, do_rev, inner, inner2, total;
 };
 
 BwdLayout bwd_layout(const BwdArgs& a) {
     const size_t tok = (size_t)a.B * a.N * a.H, qk = tok * a.dk * 2, vv = tok * a.dv * 2;
-    const int nsl = a.dv / dv_slice(a.dv);
     auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
     BwdLayout L;
     size_t o = 0;
@@ -150,18 +152,17 @@ BwdLayout bwd_layout(const BwdArgs& a) {
     L.do_rev = o; o += al(vv);
     const size_t inner = al(std::max(qk, tok * dv_slice(a.dv) * 2));  // k' of one pass
     L.inner = o; o += inner;
-    L.inner2 = o; o += inner;                    // the second stream's passes
-    L.dq_parts = o; o += nsl * al(2 * qk);       // fp32, one per d_v slice
-    L.dk_parts = o; o += nsl * al(2 * qk);       // fp32, reversed order
-    L.dv_rev = o; o += al(2 * vv);               // fp32, reversed order
+    L.inner2 = o; o += inner;  // the second stream's passes
     L.total = o;
     return L;
 }
 
 // One causal retention pass of the workspace path (prep, then the
-// tensor-core kernel) with query/key rows q_ld / k_ld elements apart.
+// tensor-core kernel) with query/key rows q_ld / k_ld elements apart; its
+// fp32 output is stored (or added, `accumulate`) at row n, or at row N-1-n
+// (`out_rev`).
 ret_status pass(const BwdArgs& b, const void* q, int q_ld, const void* k, int k_ld, int dk, const void* v, int dv,
-                float* out, void* inner, cudaStream_t s) {
+                float* out, bool accumulate, bool out_rev, void* inner, cudaStream_t s) {
     RetArgs a;
     memset(&a, 0, sizeof(a));
     a.q = q; a.k = k; a.v = v; a.out = out;
@@ -169,7 +170,7 @@ ret_status pass(const BwdArgs& b, const void* q, int q_ld, const void* k, int k_
     a.in_dt = RET_BF16; a.out_dt = RET_F32;
     a.xpos = 0; a.theta_base = 10000.0;
     a.hc = b.hc;
-    a.q_ld = q_ld; a.k_ld = k_ld; a.accumulate = 0;
+    a.q_ld = q_ld; a.k_ld = k_ld; a.accumulate = accumulate ? 1 : 0; a.out_rev = out_rev ? 1 : 0;
     if (!chunkwise_ws_supported(a)) return fail(RET_ERR_UNSUPPORTED, "backward: pass shape outside the tensor-core path");
     ret_status st = launch_chunkwise_prep(a, inner, s);
     if (st != RET_OK) return st;
@@ -218,50 +219,52 @@ ret_status launch_backward(const BwdArgs& a, cudaStream_t s) {
     const BwdLayout L = bwd_layout(a);
     uint8_t* ws = reinterpret_cast<uint8_t*>(a.workspace);
     auto at = [&](size_t off) { return reinterpret_cast<void*>(ws + off); };
-    const size_t part = (((size_t)a.B * a.N * a.H * a.dk * 4 + 255) & ~(size_t)255) / 4;  // floats between parts
     using bf = __nv_bfloat16;
     ret_status st;
-
-    // k' = R k in both time orders, q' = R q reversed, v and dO reversed.
-    if ((st = row_transform<bf, bf>(a.k, 1, 0, at(L.kr), at(L.kr_rev), a, a.dk, false, false, 1.f, s)) != RET_OK ||
-        (st = row_transform<bf, bf>(a.q, 1, 0, at(L.qr_rev), nullptr, a, a.dk, false, true, 1.f, s)) != RET_OK ||
-        (st = row_transform<bf, bf>(a.v, 1, 0, at(L.v_rev), nullptr, a, a.dv, false, true, 0.f, s)) != RET_OK ||
-        (st = row_transform<bf, bf>(a.dout, 1, 0, at(L.do_rev), nullptr, a, a.dv, false, true, 0.f, s)) != RET_OK)
-        return st;
-
     cudaStream_t s2;
     if ((st = side_stream(&s2)) != RET_OK || (st = join(s, s2)) != RET_OK) return st;
+
+    // Caller's stream: k' = R k in both time orders, then the dq passes.
+    // Second stream: q' = R q, v and dO reversed, then the dk passes.
+    if ((st = row_transform<bf, bf>(a.k, 1, 0, at(L.kr), at(L.kr_rev), a, a.dk, false, false, 1.f, s)) != RET_OK ||
+        (st = row_transform<bf, bf>(a.q, 1, 0, at(L.qr_rev), nullptr, a, a.dk, false, true, 1.f, s2)) != RET_OK ||
+        (st = row_transform<bf, bf>(a.dout, 1, 0, at(L.do_rev), nullptr, a, a.dv, false, true, 0.f, s2)) != RET_OK)
+        return st;
+    cudaEvent_t reversed;  // q' and dO reversed: what the dv pass takes from the second stream
+    if (cudaEventCreateWithFlags(&reversed, cudaEventDisableTiming) != cudaSuccess)
+        return check_launch("backward: event");
+    const bool rec = cudaEventRecord(reversed, s2) == cudaSuccess;
+    if (!rec || (st = row_transform<bf, bf>(a.v, 1, 0, at(L.v_rev), nullptr, a, a.dv, false, true, 0.f, s2)) != RET_OK) {
+        cudaEventDestroy(reversed);
+        return rec ? st : check_launch("backward: event record");
+    }
+
     const int S = dv_slice(a.dv), nsl = a.dv / S;
     const bf* dout = reinterpret_cast<const bf*>(a.dout);
     const bf* v = reinterpret_cast<const bf*>(a.v);
     const bf* v_rev = reinterpret_cast<const bf*>(at(L.v_rev));
     const bf* do_rev = reinterpret_cast<const bf*>(at(L.do_rev));
-    float* dq_parts = reinterpret_cast<float*>(at(L.dq_parts));
-    float* dk_parts = reinterpret_cast<float*>(at(L.dk_parts));
-    for (int i = 0; i < nsl; i++) {
+    for (int i = 0; i < nsl && st == RET_OK; i++) {
         const int s0 = i * S;
         // dq' = causal retention (query dO, key v, value k'), d_v slice [s0, s0 + S)
-        if ((st = pass(a, dout + s0, a.dv, v + s0, a.dv, S, at(L.kr), a.dk, dq_parts + i * part, at(L.inner), s)) !=
-            RET_OK)
-            return st;
-        // reversed dk' = causal retention (query v, key dO, value q') on the reversed sequence (second stream)
-        if ((st = pass(a, v_rev + s0, a.dv, do_rev + s0, a.dv, S, at(L.qr_rev), a.dk, dk_parts + i * part,
-                       at(L.inner2), s2)) != RET_OK)
+        st = pass(a, dout + s0, a.dv, v + s0, a.dv, S, at(L.kr), a.dk, a.dq, i > 0, false, at(L.inner), s);
+        // dk' = causal retention (query v, key dO, value q') on the reversed sequence, stored back in time order
+        if (st == RET_OK)
+            st = pass(a, v_rev + s0, a.dv, do_rev + s0, a.dv, S, at(L.qr_rev), a.dk, a.dkk, i > 0, true, at(L.inner2),
+                      s2);
+    }
+    // dv = causal retention (query k', key q', value dO) on the reversed sequence, stored back in time order
+    if (st == RET_OK && cudaStreamWaitEvent(s, reversed, 0) != cudaSuccess) st = check_launch("backward: stream wait");
+    cudaEventDestroy(reversed);  // released once it has completed
+    if (st == RET_OK)
+        st = pass(a, at(L.kr_rev), a.dk, at(L.qr_rev), a.dk, a.dk, at(L.do_rev), a.dv, a.dvv, false, true, at(L.inner),
+                  s);
+    if (st != RET_OK) return st;
+    if (a.xpos) {  // dq = R^T dq', dk = R^T dk', in place
+        if ((st = row_transform<float, float>(a.dkk, 1, 0, a.dkk, nullptr, a, a.dk, false, false, -1.f, s2)) != RET_OK ||
+            (st = row_transform<float, float>(a.dq, 1, 0, a.dq, nullptr, a, a.dk, false, false, -1.f, s)) != RET_OK)
             return st;
     }
-    // dk = R^T (sum of the slices), back in time order
-    if ((st = row_transform<float, float>(dk_parts, nsl, part, a.dkk, nullptr, a, a.dk, true, false, -1.f, s2)) !=
-        RET_OK)
-        return st;
-    // reversed dv = causal retention (query k', key q', value dO) on the reversed sequence
-    if ((st = pass(a, at(L.kr_rev), a.dk, at(L.qr_rev), a.dk, a.dk, at(L.do_rev), a.dv,
-                   reinterpret_cast<float*>(at(L.dv_rev)), at(L.inner), s)) != RET_OK)
-        return st;
-    // dq = R^T (sum of the slices); dv back in time order
-    if ((st = row_transform<float, float>(dq_parts, nsl, part, a.dq, nullptr, a, a.dk, false, false, -1.f, s)) !=
-            RET_OK ||
-        (st = row_transform<float, float>(at(L.dv_rev), 1, 0, a.dvv, nullptr, a, a.dv, true, false, 0.f, s)) != RET_OK)
-        return st;
     return join(s2, s);  // the caller's stream covers the second stream's work
 }
 

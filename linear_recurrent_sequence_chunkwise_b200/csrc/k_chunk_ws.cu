@@ -146,6 +146,7 @@ struct WsParams {
     const float* istate;  // state before the first token, [B, H, DK, dv] fp32, or null (zero)
     int N, H, dv;
     int accumulate;       // fp32 out only: out += result
+    int out_rev;          // output of token n goes to row N-1-n
     int nmain;            // CTAs: B * H * (dv / 64), one per (b, h, 64 value columns)
     HeadConsts hc;
 };
@@ -568,8 +569,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 elect_arrive(&bars.ofree, lane);
                 if (r < L) {
                     const float sc = last ? sc_last : sc_full;
-                    Tout* dst = reinterpret_cast<Tout*>(p.out) + (((size_t)b * N + n0 + r) * p.H + h) * p.dv + j0 +
-                                32 * wg;
+                    const int n = p.out_rev ? N - 1 - (n0 + r) : n0 + r;
+                    Tout* dst = reinterpret_cast<Tout*>(p.out) + (((size_t)b * N + n) * p.H + h) * p.dv + j0 + 32 * wg;
                     if constexpr (sizeof(Tout) == 2) {
 #pragma unroll
                         for (int c16 = 0; c16 < 4; c16++) {
@@ -659,6 +660,7 @@ static ret_status fill_params(WsParams* p, const RetArgs& a, const void* q_src, 
     p->hc = a.hc;
     p->nmain = a.B * a.H * (a.dv / kW);
     p->accumulate = a.accumulate;
+    p->out_rev = a.out_rev;
     return RET_OK;
 }
 

@@ -17,9 +17,10 @@ struct RetArgs {
     const float* initial_state;  // may be null (zero state); workspace path only
     // Workspace path only: elements between consecutive (token, head) rows of
     // q and of k (0: dk, i.e. contiguous), so that a column slice of a wider
-    // tensor can serve as q or k; and accumulate = 1 adds the result into an
-    // fp32 out instead of storing it.
-    int q_ld, k_ld, accumulate;
+    // tensor can serve as q or k; accumulate = 1 adds the result into an
+    // fp32 out instead of storing it; out_rev = 1 writes the output of token n
+    // to row N-1-n.
+    int q_ld, k_ld, accumulate, out_rev;
     int B, N, H, dk, dv, chunk;
     ret_dtype in_dt, out_dt;
     int xpos;

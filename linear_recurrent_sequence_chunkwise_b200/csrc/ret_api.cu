@@ -83,7 +83,7 @@ static ret_status make_args(RetArgs* a, const char* who, const void* q, const vo
             return fail(RET_ERR_INVALID_ARG, "%s: final_state overlaps another buffer", who);
     }
     a->q = q; a->k = k; a->v = v; a->out = out; a->final_state = final_state; a->initial_state = nullptr;
-    a->q_ld = 0; a->k_ld = 0; a->accumulate = 0;
+    a->q_ld = 0; a->k_ld = 0; a->accumulate = 0; a->out_rev = 0;
     a->B = B; a->N = N; a->H = H; a->dk = dk; a->dv = dv; a->chunk = chunk;
     a->in_dt = in_dt; a->out_dt = out_dt;
     a->xpos = xpos ? 1 : 0; a->pos_offset = pos_offset; a->theta_base = xpos ? theta_base : 10000.0;
