@@ -165,6 +165,16 @@ def run_ours(args):
         w["workload"] = f"retention_bf16_1x{args.seq}x16x256x512"
     B, N, H, dk, dv, C = w["B"], w["N"], w["H"], w["dk"], w["dv"], w["chunk"]
     g = gammas(H)
+    if args.only:
+        peaks = load_peaks()
+        stream = torch.cuda.current_stream()
+        if args.only == "backward":
+            res = {"backward": bench_backward(R, torch, dev, stream, w, g, args, peaks, world, dist)}
+        else:
+            res = {"msr_layer": bench_msr(R, torch, dev, stream, args, peaks, world, dist)}
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return
     if args.no_chunkwise:
         peaks = load_peaks()
         res = {"decode": bench_decode(R, torch, dev, torch.cuda.current_stream(), args, peaks, world, barrier, dist,
@@ -405,7 +415,7 @@ def bench_backward(R, torch, dev, stream, w, g, args, peaks, world, dist):
     def fn():
         R.ret_backward_chunkwise(q, k, v, do, g, C, workspace=ws, dq=dq, dk=dkk, dv=dvv, xpos=True, stream=stream)
 
-    ms = _timed(torch, stream, fn, max(3, min(args.steps, 10)), 2, world, dist, dev)
+    ms = _timed(torch, stream, fn, max(3, min(args.steps, 10)), 3, world, dist, dev)
     R.ret_check_device_error()
     flops = 3 * flops_per_token_head(C, dk, dv) * B * N * H
     tf = flops / (ms / 1e3) / 1e12
@@ -548,6 +558,8 @@ def main():
     ap.add_argument("--seq", type=int, default=WORKLOAD["N"],
                     help="sequence length of the chunkwise workload (smaller values make ncu captures short)")
     ap.add_argument("--no-chunkwise", action="store_true", help="skip the chunkwise forward (decode only)")
+    ap.add_argument("--only", choices=["backward", "msr"],
+                    help="time only the backward or only the MSR layer (for ncu launch lists of one part)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
