@@ -50,6 +50,7 @@ def _configure(lib):
     lib.orc_retention_chunkwise.argtypes = [dp, dp, dp, dp, i, i, i, i, i, i, dp, dp, i]
     lib.orc_decode_step.argtypes = [dp, dp, dp, dp, i, i, i, i, dp, dp, i]
     lib.orc_retention_backward.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, dp, dp, dp, i]
+    lib.orc_retention_normalized.argtypes = [dp, dp, dp, dp, i, i, i, i, i, i, dp, i]
     return lib
 
 
@@ -138,6 +139,27 @@ def retention_backward(q, k, v, dout, gammas, xpos: bool = False, pos_offset: in
     if xpos:
         dq, dkk = xpos_unrotate(dq, pos_offset, theta_base), xpos_unrotate(dkk, pos_offset, theta_base)
     return dq, dkk, dvv
+
+
+NORM_DECAY = 1  # score normalization 2: D_nm / sqrt(sum_i D_ni)
+NORM_SCORE = 2  # score normalization 3: R_nm / max(|sum_i R_ni|, 1)
+
+
+def retention_normalized(q, k, v, gammas, flags: int = NORM_DECAY | NORM_SCORE, xpos: bool = False,
+                         pos_offset: int = 0, theta_base: float = 10000.0, nthreads: int = 0):
+    """Parallel form with the score normalizations 2 and 3 (P1 section 8.5;
+    P3 "Retention Score Normalization"), brute force in C over the whole
+    sequence; with xpos, q and k are rotated first (P1 sections 6.6, 6.8)."""
+    q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(gammas)
+    if xpos:
+        q, k = xpos_rotate(q, pos_offset, theta_base), xpos_rotate(k, pos_offset, theta_base)
+    B, N, H, dk = q.shape
+    dv = v.shape[3]
+    assert k.shape == q.shape and v.shape[:3] == q.shape[:3] and g.shape == (H,)
+    out = np.zeros((B, N, H, dv))
+    _load().orc_retention_normalized(_p(q), _p(k), _p(v), _p(g), B, N, H, dk, dv, int(flags), _p(out),
+                                     int(nthreads))
+    return out
 
 
 def retention_recurrent(q, k, v, gammas, init_state=None, nthreads: int = 0):

@@ -300,3 +300,53 @@ void orc_retention_backward(const double *q, const double *k, const double *v, c
         }
     }
 }
+
+/*
+ * Retention with the score normalizations 2 and 3, parallel form by brute
+ * force.  [P1] section 8.5 and [P3] "Retention Score Normalization":
+ *   2. the decay matrix row-normalized:  Dt_nm = D_nm / sqrt(sum_{i<=n} D_ni)
+ *   3. the scores row-normalized:        Rt_nm = R_nm / max(|sum_{i<=n} R_ni|, 1)
+ *      with R = (Q K^T) (.) Dt (the scores after normalization 2)
+ * and out = Rt V.  Normalization 1 (the 1/sqrt(d) on Q K^T) is the caller's
+ * scaling of q.  The row sums are taken as written: the absolute value of the
+ * sum, not the sum of absolute values.  flags bit 0 turns on normalization
+ * 2, bit 1 normalization 3; flags = 0 is orc_retention_parallel.
+ */
+void orc_retention_normalized(const double *q, const double *k, const double *v,
+                              const double *gammas, int B, int N, int H, int dk, int dv,
+                              int flags, double *out, int nthreads) {
+    set_threads(nthreads);
+    int BH = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int bh = 0; bh < BH; bh++) {
+        int b = bh / H, h = bh % H;
+        double gamma = gammas[h];
+        double *row = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1)); /* R_n. */
+        for (int n = 0; n < N; n++) {
+            const double *qn = q + IDX4(b, n, h, 0, N, H, dk);
+            /* sum_{i<=n} D_ni */
+            double dsum = 0.0;
+            for (int i = 0; i <= n; i++) dsum += orc_gamma_pow(gamma, n - i);
+            double dscale = (flags & 1) ? 1.0 / sqrt(dsum) : 1.0;
+            /* R_nm = (Q K^T)_nm Dt_nm */
+            double rsum = 0.0;
+            for (int m = 0; m <= n; m++) {
+                const double *km = k + IDX4(b, m, h, 0, N, H, dk);
+                double qk = 0.0;
+                for (int i = 0; i < dk; i++) qk += qn[i] * km[i];
+                row[m] = qk * orc_gamma_pow(gamma, n - m) * dscale;
+                rsum += row[m];
+            }
+            double den = 1.0;
+            if (flags & 2) den = fabs(rsum) > 1.0 ? fabs(rsum) : 1.0;
+            double *on = out + IDX4(b, n, h, 0, N, H, dv);
+            for (int j = 0; j < dv; j++) on[j] = 0.0;
+            for (int m = 0; m <= n; m++) {
+                const double *vm = v + IDX4(b, m, h, 0, N, H, dv);
+                double w = row[m] / den;
+                for (int j = 0; j < dv; j++) on[j] += w * vm[j];
+            }
+        }
+        free(row);
+    }
+}

@@ -34,6 +34,11 @@ MUTANTS = {
     "backward_dv_with_the_wrong_score": ("+= w * a * gn[j];", "+= w * g * gn[j];"),
     "backward_dq_with_the_wrong_score": ("dq[IDX4(b, n, h, i, N, H, dk)] += w * g * km[i];",
                                          "dq[IDX4(b, n, h, i, N, H, dk)] += w * a * km[i];"),
+    "decay_norm_without_sqrt": ("double dscale = (flags & 1) ? 1.0 / sqrt(dsum) : 1.0;",
+                                "double dscale = (flags & 1) ? 1.0 / dsum : 1.0;"),
+    "score_norm_sum_of_abs": ("rsum += row[m];", "rsum += fabs(row[m]);"),
+    "score_norm_before_decay_norm": ("rsum += row[m];", "rsum += row[m] / dscale;"),
+    "score_norm_without_clamp": ("den = fabs(rsum) > 1.0 ? fabs(rsum) : 1.0;", "den = fabs(rsum);"),
 }
 
 

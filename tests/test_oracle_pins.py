@@ -374,3 +374,94 @@ def test_unrotate_inverts_rotate():
     x = np.random.default_rng(9).standard_normal((2, 6, 3, 8))
     assert np.allclose(oracle.xpos_unrotate(oracle.xpos_rotate(x, 4), 4), x, rtol=0, atol=1e-14)
     assert np.allclose(oracle.xpos_rotate(oracle.xpos_unrotate(x, 4), 4), x, rtol=0, atol=1e-14)
+
+
+# ------------------------------------------------ score normalizations 2 and 3
+
+def test_normalized_hand_example():
+    """Two tokens, d = 1, gamma = 0.5, worked by hand from the definitions
+    (P1 section 8.5): D = [[1, 0], [0.5, 1]], row sums of D 1 and 1.5, so
+    Dt = [[1, 0], [0.5, 1] / sqrt(1.5)]; Q K^T = [[2, .], [3, 6]], so
+    R = [[2, 0], [1.5, 6] / sqrt(1.5)] with row sums 2 and 7.5 / sqrt(1.5);
+    Rt = [[1, 0], [0.2, 0.8]] and with v = (1, 10): out = (1, 8.2)."""
+    q = np.array([2.0, 3.0]).reshape(1, 2, 1, 1)
+    k = np.array([1.0, 2.0]).reshape(1, 2, 1, 1)
+    v = np.array([1.0, 10.0]).reshape(1, 2, 1, 1)
+    out = oracle.retention_normalized(q, k, v, [0.5])
+    np.testing.assert_allclose(out.ravel(), [1.0, 8.2], rtol=1e-14)
+    # normalization 2 alone: row 1 is (1.5 + 60) / sqrt(1.5)
+    out2 = oracle.retention_normalized(q, k, v, [0.5], flags=oracle.NORM_DECAY)
+    np.testing.assert_allclose(out2.ravel(), [2.0, 61.5 / math.sqrt(1.5)], rtol=1e-14)
+    # normalization 3 alone: row 1 scores (1.5, 6) over 7.5
+    out3 = oracle.retention_normalized(q, k, v, [0.5], flags=oracle.NORM_SCORE)
+    np.testing.assert_allclose(out3.ravel(), [1.0, 8.2], rtol=1e-14)
+
+
+@pytest.mark.parametrize("gamma", [0.5, 0.9, 1 - 2.0 ** -5, 1.0])
+def test_decay_normalization_closed_form(gamma):
+    """Unit scores (q = k = e_1) and v = 1 make out_n the row sum of Dt, i.e.
+    sum_i D_ni / sqrt(sum_i D_ni) = sqrt of the geometric series
+    (1 - gamma^(n+1)) / (1 - gamma)  (n + 1 at gamma = 1)."""
+    N = 40
+    q = np.zeros((1, N, 1, 3))
+    q[..., 0] = 1.0
+    v = np.ones((1, N, 1, 2))
+    out = oracle.retention_normalized(q, q, v, [gamma], flags=oracle.NORM_DECAY)
+    n = np.arange(N)
+    geo = n + 1.0 if gamma == 1.0 else (1 - gamma ** (n + 1)) / (1 - gamma)
+    np.testing.assert_allclose(out[0, :, 0, 0] ** 2, geo, rtol=1e-12)
+    np.testing.assert_allclose(out[0, :, 0, 1], out[0, :, 0, 0], rtol=0)
+
+
+@pytest.mark.parametrize("flags", [oracle.NORM_SCORE, oracle.NORM_DECAY | oracle.NORM_SCORE])
+def test_score_normalization_row_sums(flags):
+    """With v = 1 the output is the row sum of Rt: sum_m R_nm divided by
+    max(|sum_m R_nm|, 1), i.e. sign(s) where |s| >= 1 and s itself where
+    |s| < 1.  s comes from the plain oracle (pinned above) with v = 1,
+    times 1 / sqrt(sum_i D_ni) when normalization 2 is on."""
+    rng = np.random.default_rng(31)
+    B, N, H, d = 2, 37, 3, 5
+    q = rng.standard_normal((B, N, H, d)) * 0.6
+    k = rng.standard_normal((B, N, H, d)) * 0.6
+    g = np.array([0.5, 0.9, 0.99])
+    ones = np.ones((B, N, H, 1))
+    s, _ = oracle.retention_recurrent(q, k, ones, g)
+    s = s[..., 0]
+    if flags & oracle.NORM_DECAY:
+        n = np.arange(N)[None, :, None]
+        s = s / np.sqrt((1 - g[None, None, :] ** (n + 1)) / (1 - g[None, None, :]))
+    expect = s / np.maximum(np.abs(s), 1.0)
+    out = oracle.retention_normalized(q, k, ones, g, flags=flags)[..., 0]
+    np.testing.assert_allclose(out, expect, rtol=1e-12, atol=1e-14)
+    # both branches of the max occur in this sample
+    assert (np.abs(s) < 1).any() and (np.abs(s) > 1).any()
+
+
+def test_normalizations_vanish_under_group_norm():
+    """GroupNorm per head is scale-invariant (P1 section 8.4), and both
+    normalizations scale each (token, head) output row by a positive scalar,
+    so GroupNorm of the normalized output equals GroupNorm of the plain one
+    (P1 section 8.5: they do not change the model's output)."""
+    rng = np.random.default_rng(32)
+    B, N, H, dk, dv = 1, 29, 2, 6, 8
+    q = rng.standard_normal((B, N, H, dk))
+    k = rng.standard_normal((B, N, H, dk))
+    v = rng.standard_normal((B, N, H, dv))
+    g = np.array([0.8, 0.97])
+    plain = oracle.retention_parallel(q, k, v, g)
+    for flags in (oracle.NORM_DECAY, oracle.NORM_SCORE, oracle.NORM_DECAY | oracle.NORM_SCORE):
+        out = oracle.retention_normalized(q, k, v, g, flags=flags)
+        np.testing.assert_allclose(omsr.group_norm_heads(out, 0.0), omsr.group_norm_heads(plain, 0.0), atol=1e-9)
+        # and the scale is a per-row positive scalar, not the identity
+        alpha = (out * plain).sum(-1) / (plain * plain).sum(-1)
+        np.testing.assert_allclose(out, alpha[..., None] * plain, rtol=0,
+                                   atol=1e-12 * np.abs(plain).max())
+        assert (alpha > 0).all() and not np.allclose(alpha, 1.0)
+
+
+def test_normalized_without_flags_is_the_parallel_form():
+    rng = np.random.default_rng(33)
+    q, k, v = (rng.standard_normal((1, 11, 2, 4)) for _ in range(3))
+    g = [0.7, 0.95]
+    np.testing.assert_allclose(oracle.retention_normalized(q, k, v, g, flags=0),
+                               oracle.retention_parallel(q, k, v, g), rtol=1e-13, atol=1e-13)
