@@ -202,6 +202,72 @@ ret_status ret_backward_chunkwise(const void* q, const void* k, const void* v, c
                                   size_t workspace_bytes);
 
 /*
+ * Retention with the score normalizations 2 and 3 ("Hybrid Architectures
+ * ...", section 8.5; RetNet paper summary, "Retention Score
+ * Normalization"), selected by norm_flags:
+ *   RET_NORM_DECAY  the decay matrix row-normalized,
+ *                   D~_nm = D_nm / sqrt(sum_{i<=n} D_ni);
+ *   RET_NORM_SCORE  the scores row-normalized,
+ *                   R~_nm = R_nm / max(|sum_{i<=n} R_ni|, 1),
+ *                   R = (Q K^T) (.) D~ (or D without RET_NORM_DECAY);
+ * out = R~ V.  Normalization 1 (the 1/sqrt(d) on Q K^T) is the caller's
+ * scaling of q.  The row sums run over the whole sequence: position pos_offset
+ * + n is row pos_offset + n of D, and the score row sum is q_n . z_n with
+ * z_n = gamma_h z_{n-1} + k_n, the decayed key sum (rotated keys with xpos).
+ * Both normalizations multiply output row n by a positive scalar and leave
+ * the state S unchanged.  The pages take the absolute value of the sum (not
+ * the sum of absolute values); so does this library, which keeps the
+ * chunkwise and recurrent forms exact.
+ */
+#define RET_NORM_DECAY 1
+#define RET_NORM_SCORE 2
+
+/*
+ * Chunkwise forward with the normalizations: arguments as
+ * ret_forward_chunkwise_prepared (same path constraints: bf16 inputs, chunk
+ * 128, dk 128 or 256, dv a multiple of 64, every gamma_h^128 >= 2^-60, else
+ * RET_ERR_UNSUPPORTED), plus
+ *   norm_flags  a combination of RET_NORM_DECAY and RET_NORM_SCORE (0: the
+ *               plain retention);
+ *   initial_z   device fp32 [B, H, dk], 16-byte aligned, or NULL (zero): z
+ *               after every token before this call's first one;
+ *   final_z     device fp32 [B, H, dk], 16-byte aligned, or NULL: z after
+ *               the last token (may be the same buffer as initial_z);
+ *   workspace   device, 256-byte aligned, at least
+ *               ret_normalized_workspace_bytes(...) bytes, scratch.
+ * Splitting a sequence into calls that hand final_state and final_z on, with
+ * pos_offset the number of earlier tokens, gives the single call's result.
+ * No buffer may overlap another except final_state = initial_state and
+ * final_z = initial_z.
+ */
+size_t ret_normalized_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk,
+                                      ret_dtype in_dt, int xpos);
+
+ret_status ret_forward_chunkwise_normalized(const void* q, const void* k, const void* v,
+                                            const double* gammas, int B, int N, int H, int dk,
+                                            int dv, int chunk, int norm_flags, void* out,
+                                            const float* initial_state, float* final_state,
+                                            const float* initial_z, float* final_z,
+                                            cudaStream_t stream, ret_dtype in_dt,
+                                            ret_dtype out_dt, int xpos, int64_t pos_offset,
+                                            double theta_base, void* workspace,
+                                            size_t workspace_bytes);
+
+/*
+ * One decode step with the normalizations: as ret_decode_step, then the
+ * output multiplied by c / max(|c q.z|, 1) (RET_NORM_SCORE; c = 1 without
+ * RET_NORM_DECAY), c = 1 / sqrt(sum_{i<=position} gamma_h^i), after
+ * z <- gamma_h z + k.  position: the token's 0-based position in its
+ * sequence, >= 0.  z: device fp32 [B, H, dk], 16-byte aligned, updated in
+ * place; required with RET_NORM_SCORE, ignored (may be NULL) without.
+ */
+ret_status ret_decode_step_normalized(const void* q, const void* k, const void* v,
+                                      const double* gammas, float* state, float* z, void* out,
+                                      int64_t position, int norm_flags, cudaStream_t stream,
+                                      int B, int H, int dk, int dv, ret_dtype in_dt,
+                                      ret_dtype out_dt);
+
+/*
  * Allocation-free variant of ret_forward_chunkwise_ws, for callers that
  * cannot allocate device memory at call time: for example a plug-in that runs
  * inside a host framework which owns all device memory and hands out no

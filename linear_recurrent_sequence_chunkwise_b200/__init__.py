@@ -22,6 +22,8 @@ __all__ = [
     "ret_backward_chunkwise", "ret_backward_workspace_bytes",
     "ret_forward_chunkwise_noalloc", "ret_chunkwise_noalloc_max_bytes",
     "ret_decode_step", "ret_msr_forward", "ret_msr_workspace_bytes",
+    "ret_forward_chunkwise_normalized", "ret_normalized_workspace_bytes", "ret_decode_step_normalized",
+    "NORM_DECAY", "NORM_SCORE",
     "ret_linear_bf16",
     "ret_forward_parallel", "ret_forward_recurrent", "ret_check_device_error", "ret_last_error_string",
     "RET_OK", "RET_ERR_INVALID_ARG", "RET_ERR_UNSUPPORTED", "RET_ERR_CUDA", "RET_ERR_TIMEOUT",
@@ -68,6 +70,11 @@ def _load_library():
     L.ret_chunkwise_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
     L.ret_chunkwise_workspace_bytes.restype = ctypes.c_size_t
     L.ret_decode_step.argtypes = [vp, vp, vp, dp, vp, vp, vp, i, i, i, i, i, i]
+    L.ret_normalized_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+    L.ret_normalized_workspace_bytes.restype = ctypes.c_size_t
+    L.ret_forward_chunkwise_normalized.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, i,
+                                                   i, i, i64, d, vp, ctypes.c_size_t]
+    L.ret_decode_step_normalized.argtypes = [vp, vp, vp, dp, vp, vp, vp, i64, i, vp, i, i, i, i, i, i]
     L.ret_forward_parallel.argtypes = [vp, vp, vp, dp, i, i, i, i, i, vp, vp, i, i, i, i64, d]
     L.ret_forward_recurrent.argtypes = [vp, vp, vp, dp, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d]
     L.ret_msr_workspace_bytes.argtypes = [i, i, i, i, i, i]
@@ -324,6 +331,63 @@ def ret_decode_step(q, k, v, gammas, state, out=None, out_dtype=None, stream=Non
     _check(lib.ret_decode_step(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H),
                                _ptr(state, "state"), _ptr(out, "out"), _stream(stream), B, H, dk, dv,
                                _dt(q.dtype), _dt(out.dtype)))
+    return out
+
+
+NORM_DECAY = 1  # RET_NORM_DECAY
+NORM_SCORE = 2  # RET_NORM_SCORE
+
+
+def ret_normalized_workspace_bytes(B, N, H, dk, dv, chunk, in_dtype=torch.bfloat16, xpos: bool = False) -> int:
+    """Workspace bytes of ret_forward_chunkwise_normalized (0: shape not supported)."""
+    return int(lib.ret_normalized_workspace_bytes(B, N, H, dk, dv, int(chunk), _dt(in_dtype), int(bool(xpos))))
+
+
+def ret_forward_chunkwise_normalized(q, k, v, gammas, chunk: int, norm_flags: int = NORM_DECAY | NORM_SCORE,
+                                     workspace=None, out=None, out_dtype=None, initial_state=None,
+                                     final_state=None, initial_z=None, final_z=None, xpos: bool = False,
+                                     pos_offset: int = 0, theta_base: float = 10000.0, stream=None):
+    """Chunkwise forward with the score normalizations (norm_flags: NORM_DECAY,
+    NORM_SCORE); states S [B, H, dk, dv] and z [B, H, dk] fp32, optional."""
+    B, N, H, dk, dv = _seq_shapes(q, k, v)
+    if out is None:
+        out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
+    for name, t, shape in (("initial_state", initial_state, (B, H, dk, dv)), ("final_state", final_state, (B, H, dk, dv)),
+                           ("initial_z", initial_z, (B, H, dk)), ("final_z", final_z, (B, H, dk))):
+        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != shape):
+            raise ValueError(f"{name} must be fp32 {list(shape)}")
+    if workspace is None:
+        nb = ret_normalized_workspace_bytes(B, N, H, dk, dv, chunk, q.dtype, xpos)
+        workspace = torch.empty(max(nb, 1), dtype=torch.uint8, device=q.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib.ret_forward_chunkwise_normalized(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N,
+                                                H, dk, dv, int(chunk), int(norm_flags), _ptr(out, "out"),
+                                                _ptr(initial_state, "initial_state"), _ptr(final_state, "final_state"),
+                                                _ptr(initial_z, "initial_z"), _ptr(final_z, "final_z"),
+                                                _stream(stream), _dt(q.dtype), _dt(out.dtype), int(bool(xpos)),
+                                                int(pos_offset), float(theta_base), _ptr(workspace, "workspace"),
+                                                nbytes))
+    return out
+
+
+def ret_decode_step_normalized(q, k, v, gammas, state, z, position: int, norm_flags: int = NORM_DECAY | NORM_SCORE,
+                               out=None, out_dtype=None, stream=None):
+    """One decode step with the score normalizations at 0-based ``position``:
+    state [B, H, dk, dv] and z [B, H, dk] (fp32) updated in place."""
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("expected q, k [B, H, dk] and v [B, H, dv]")
+    B, H, dk = q.shape
+    dv = v.shape[2]
+    if state.shape != (B, H, dk, dv) or state.dtype != torch.float32:
+        raise ValueError("state must be float32 [B, H, dk, dv]")
+    if z is not None and (z.shape != (B, H, dk) or z.dtype != torch.float32):
+        raise ValueError("z must be float32 [B, H, dk]")
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=out_dtype or torch.float32, device=q.device)
+    _check(lib.ret_decode_step_normalized(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H),
+                                          _ptr(state, "state"), _ptr(z, "z"), _ptr(out, "out"), int(position),
+                                          int(norm_flags), _stream(stream), B, H, dk, dv, _dt(q.dtype),
+                                          _dt(out.dtype)))
     return out
 
 

@@ -147,6 +147,7 @@ struct WsParams {
     int N, H, dv;
     int accumulate;       // fp32 out only: out += result
     int out_rev;          // output of token n goes to row N-1-n
+    const float* rowscale;  // [B, N, H] factor of each output row, or null
     int nmain;            // CTAs: B * H * (dv / 64), one per (b, h, 64 value columns)
     HeadConsts hc;
 };
@@ -482,6 +483,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         for (int jc = 0; jc < nchunks && ok; jc++) {
             const int n0 = jc * kC, L = min(kC, N - n0);
             const bool last = (jc == nchunks - 1);
+            // the row's normalization factor, loaded now and used by the epilogue
+            const float rs = (p.rowscale && r < L) ? __ldg(p.rowscale + ((size_t)b * N + n0 + r) * p.H + h) : 1.f;
             // ---- mask: P = tril(A) as packed bf16 into TMEM, 32 A columns at a time
             ok = tc::mbar_wait(&bars.afull, jc & 1);
             if (!ok) break;
@@ -568,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 tc::tc_fence_before();
                 elect_arrive(&bars.ofree, lane);
                 if (r < L) {
-                    const float sc = last ? sc_last : sc_full;
+                    const float sc = (last ? sc_last : sc_full) * rs;
                     const int n = p.out_rev ? N - 1 - (n0 + r) : n0 + r;
                     Tout* dst = reinterpret_cast<Tout*>(p.out) + (((size_t)b * N + n) * p.H + h) * p.dv + j0 + 32 * wg;
                     if constexpr (sizeof(Tout) == 2) {
@@ -661,6 +664,7 @@ static ret_status fill_params(WsParams* p, const RetArgs& a, const void* q_src, 
     p->nmain = a.B * a.H * (a.dv / kW);
     p->accumulate = a.accumulate;
     p->out_rev = a.out_rev;
+    p->rowscale = a.rowscale;
     return RET_OK;
 }
 

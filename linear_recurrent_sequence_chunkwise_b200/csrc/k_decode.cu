@@ -20,10 +20,14 @@ constexpr int kDecBatch = 16;   // row vectors in flight per thread
 __device__ __forceinline__ float4 ld_stream(const float4* p) { return __ldcs(p); }
 __device__ __forceinline__ void st_stream(float4* p, float4 x) { __stcs(p, x); }
 
+// With flags (the score normalizations 2 and 3 of section 8.5), the output
+// is multiplied by f = c / max(|c q.z|, 1), c = 1 / sqrt(sum_{i<=pos}
+// gamma^i), where z is the decayed key sum already updated for this token.
 template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(256) k_decode_step(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                                      const Tin* __restrict__ v, HeadConsts hc, int H, int dk,
-                                                     int dv, float* __restrict__ state, Tout* __restrict__ out) {
+                                                     int dv, float* __restrict__ state, Tout* __restrict__ out,
+                                                     const float* __restrict__ z, long long pos, int flags) {
     extern __shared__ float smf[];
     float* qs = smf;            // [dk]
     float* ks = smf + dk;       // [dk]
@@ -37,6 +41,31 @@ __global__ void __launch_bounds__(256) k_decode_step(const Tin* __restrict__ q, 
     }
     const float g = (float)exp2(hc.log2g[h]);
     __syncthreads();
+    float fscale = 1.f;
+    if (flags) {
+        __shared__ float s_part[kDecWarps], s_f;
+        float part = 0.f;
+        if (flags & kNormScore)
+            for (int i = threadIdx.x; i < dk; i += blockDim.x) part = fmaf(qs[i], z[(size_t)bh * dk + i], part);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) s_part[w] = part;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float sn = 0.f;
+            for (int ww = 0; ww < kDecWarps; ww++) sn += s_part[ww];
+            const double lg = hc.log2g[h];
+            double f = 1.0;
+            if (flags & kNormDecay) {
+                const double ln_g = lg * 0.69314718055994530942, cnt = (double)(pos + 1);
+                f = 1.0 / sqrt(lg == 0.0 ? cnt : expm1(cnt * ln_g) / expm1(ln_g));
+            }
+            if (flags & kNormScore) f /= fmax(fabs(f * (double)sn), 1.0);
+            s_f = (float)f;
+        }
+        __syncthreads();
+        fscale = s_f;
+    }
 
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (j < dv) {
@@ -80,6 +109,7 @@ __global__ void __launch_bounds__(256) k_decode_step(const Tin* __restrict__ q, 
             const float4 r = red[ww * 32 + lane];
             o.x += r.x; o.y += r.y; o.z += r.z; o.w += r.w;
         }
+        o.x *= fscale; o.y *= fscale; o.z *= fscale; o.w *= fscale;
         const size_t ob = (size_t)bh * dv + j;
         st_from_float(out, ob, o.x);
         st_from_float(out, ob + 1, o.y);
@@ -88,15 +118,49 @@ __global__ void __launch_bounds__(256) k_decode_step(const Tin* __restrict__ q, 
     }
 }
 
+// z <- gamma z + k, one thread per element of z [B, H, dk].
+template <typename Tin>
+__global__ void k_keysum_update(float* __restrict__ z, const Tin* __restrict__ k, HeadConsts hc, int H, int dk,
+                                long long total) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= total) return;
+    const int h = (int)((i / dk) % H);
+    z[i] = fmaf((float)exp2(hc.log2g[h]), z[i], ld_as_float(k, (size_t)i));
+}
+
+static ret_status decode_launch(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
+                                const float* z, void* out, int B, int H, int dk, int dv, ret_dtype in_dt,
+                                ret_dtype out_dt, long long pos, int flags, cudaStream_t s);
+
 ret_status launch_decode(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
                          void* out, int B, int H, int dk, int dv, ret_dtype in_dt, ret_dtype out_dt,
                          cudaStream_t s) {
+    return decode_launch(q, k, v, hc, state, nullptr, out, B, H, dk, dv, in_dt, out_dt, 0, 0, s);
+}
+
+ret_status launch_decode_normalized(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
+                                    float* z, void* out, int B, int H, int dk, int dv, ret_dtype in_dt,
+                                    ret_dtype out_dt, long long pos, int flags, cudaStream_t s) {
+    if (flags & kNormScore) {
+        const long long total = (long long)B * H * dk;
+        const int blocks = (int)((total + 255) / 256);
+        if (in_dt == RET_F32) k_keysum_update<float><<<blocks, 256, 0, s>>>(z, (const float*)k, hc, H, dk, total);
+        else k_keysum_update<__nv_bfloat16><<<blocks, 256, 0, s>>>(z, (const __nv_bfloat16*)k, hc, H, dk, total);
+        ret_status st = check_launch("ret_decode_step_normalized: key sum");
+        if (st != RET_OK) return st;
+    }
+    return decode_launch(q, k, v, hc, state, z, out, B, H, dk, dv, in_dt, out_dt, pos, flags, s);
+}
+
+static ret_status decode_launch(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
+                                const float* z, void* out, int B, int H, int dk, int dv, ret_dtype in_dt,
+                                ret_dtype out_dt, long long pos, int flags, cudaStream_t s) {
     dim3 grid((dv + kDecCols - 1) / kDecCols, B * H);
     const size_t smem = (size_t)((2 * dk + 3) & ~3) * sizeof(float) + kDecWarps * 32 * sizeof(float4);
     if (smem > 48 * 1024) return fail(RET_ERR_UNSUPPORTED, "ret_decode_step: dk too large");
 #define RET_LAUNCH_DEC(TI, TO)                                                                               \
     k_decode_step<TI, TO><<<grid, 256, smem, s>>>((const TI*)q, (const TI*)k, (const TI*)v, hc, H, dk, dv, \
-                                                  state, (TO*)out)
+                                                  state, (TO*)out, z, pos, flags)
     if (in_dt == RET_F32 && out_dt == RET_F32) RET_LAUNCH_DEC(float, float);
     else if (in_dt == RET_F32) RET_LAUNCH_DEC(float, __nv_bfloat16);
     else if (out_dt == RET_F32) RET_LAUNCH_DEC(__nv_bfloat16, float);

@@ -1,0 +1,264 @@
+// k_norm.cu -- retention with the score normalizations 2 and 3
+// ("Hybrid Architectures: RetNet and the Three Computation Paradigms",
+// section 8.5; RetNet paper summary, "Retention Score Normalization"):
+//   2. D~_nm = D_nm / sqrt(sum_{i<=n} D_ni)
+//   3. R~_nm = R_nm / max(|sum_{i<=n} R_ni|, 1),   R = (Q K^T) (.) D~
+// Both divide row n of the score matrix by a scalar, so they scale output
+// row n by f_n = c_n / max(|c_n s_n|, 1), with c_n = 1 / sqrt(sum_{i<=n}
+// gamma^(n-i)) (a geometric series in closed form) and s_n = sum_{m<=n}
+// gamma^(n-m) q_n . k_m = q_n . z_n, where z_n = gamma z_{n-1} + k_n is the
+// decayed key sum: a recurrent d_k vector beside the state S, so the
+// normalized retention keeps its chunkwise and recurrent forms.  The state S
+// itself is unchanged.
+//
+// Chunkwise: three bandwidth-bound passes over the prepared q and k' (the
+// keys already scaled by zeta = gamma^(L-1-c) within their chunk) fill a
+// factor per (token, head) that the tensor-core kernel's epilogue applies:
+//   k_keysum     sum of k' over each 32-row block,
+//   k_keycarry   z before every chunk: z_j = gamma^L z_{j-1} + sum_c k'_c,
+//   k_rowscale   s_n = gamma^(r+1-L) q_n . sum_{c<=r} k'_c + gamma^(r+1) q_n . z_{j-1}
+//                for row r of chunk j, then f_n.
+#include <cstring>
+
+#include "kernels.h"
+
+namespace ret {
+
+namespace {
+
+constexpr int kSub = 32;    // rows per key-sum block
+constexpr int kChunk = 128;  // the workspace path's chunk
+
+__device__ __forceinline__ void add_bf16x8(const uint4& u, float* acc) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const float2 f = __bfloat1622float2(h[i]);
+        acc[2 * i] += f.x;
+        acc[2 * i + 1] += f.y;
+    }
+}
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* x) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const float2 f = __bfloat1622float2(h[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+}
+
+// One warp per (batch, head, 32-row block); lane g sums elements 8g..8g+7.
+template <int DK>
+__global__ void __launch_bounds__(256) k_keysum(const __nv_bfloat16* __restrict__ kp, float* __restrict__ subsum,
+                                                int B, int N, int H, int nsub) {
+    const int lane = threadIdx.x & 31;
+    const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);  // (b * H + h) * nsub + s
+    if (w >= (long long)B * H * nsub) return;
+    const int s = (int)(w % nsub);
+    const int bh = (int)(w / nsub), h = bh % H, b = bh / H;
+    const int n0 = s * kSub, n1 = min(N, n0 + kSub);
+    for (int g = lane; g < DK / 8; g += 32) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int n = n0; n < n1; n += 8) {
+            uint4 x[8];
+#pragma unroll
+            for (int u = 0; u < 8; u++)
+                if (n + u < n1)
+                    x[u] = __ldg(reinterpret_cast<const uint4*>(kp + (((size_t)b * N + n + u) * H + h) * DK + 8 * g));
+#pragma unroll
+            for (int u = 0; u < 8; u++)
+                if (n + u < n1) add_bf16x8(x[u], acc);
+        }
+        float4* dst = reinterpret_cast<float4*>(subsum + (size_t)w * DK + 8 * g);
+        dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+}
+
+// One block per (batch, head), one thread per key component: the decayed key
+// sum before each chunk (zstart) and after the last one (z1).
+template <int DK>
+__global__ void __launch_bounds__(DK) k_keycarry(const float* __restrict__ subsum, const float* z0, float* zstart,
+                                                 float* z1, HeadConsts hc, int H, int N, int nsub, int nch) {
+    const int bh = blockIdx.x, h = bh % H, d = threadIdx.x;
+    const double lg = hc.log2g[h];
+    const float g_full = (float)exp2(kChunk * lg);
+    const int L_last = N - (nch - 1) * kChunk;
+    const float g_last = (float)exp2(L_last * lg);
+    float Z = z0 ? z0[(size_t)bh * DK + d] : 0.f;
+    const float* ss = subsum + (size_t)bh * nsub * DK + d;
+    for (int j = 0; j < nch; j++) {
+        zstart[((size_t)bh * nch + j) * DK + d] = Z;
+        const int s0 = j * (kChunk / kSub), s1 = min(nsub, s0 + kChunk / kSub);
+        float cs = 0.f;
+        for (int s = s0; s < s1; s++) cs += ss[(size_t)s * DK];
+        Z = fmaf(j == nch - 1 ? g_last : g_full, Z, cs);
+    }
+    if (z1) z1[(size_t)bh * DK + d] = Z;
+}
+
+// 32 values per lane in, lane l out with the sum over the warp of value l
+// (a butterfly that halves the values each lane carries at every step).
+template <int O>
+__device__ __forceinline__ void butterfly_step(float* v, int lane) {
+    const bool up = (lane & O) != 0;
+#pragma unroll
+    for (int i = 0; i < O; i++) {
+        const float send = up ? v[i] : v[i + O];
+        const float keep = up ? v[i + O] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+    }
+}
+
+__device__ __forceinline__ float transpose_reduce32(float* v, int lane) {
+    butterfly_step<16>(v, lane);
+    butterfly_step<8>(v, lane);
+    butterfly_step<4>(v, lane);
+    butterfly_step<2>(v, lane);
+    butterfly_step<1>(v, lane);
+    return v[0];
+}
+
+// One warp per (batch, head, 32-row block): the row sums s_n of its rows and
+// the factors f_n.
+template <int DK>
+__global__ void __launch_bounds__(256) k_rowscale(const __nv_bfloat16* __restrict__ qe,
+                                                  const __nv_bfloat16* __restrict__ kp,
+                                                  const float* __restrict__ subsum, const float* __restrict__ zstart,
+                                                  float* __restrict__ rowscale, HeadConsts hc, int B, int N, int H,
+                                                  int nsub, int nch, long long pos0, int flags) {
+    static_assert(DK / 8 <= 32, "one 8-element group per lane");
+    const int lane = threadIdx.x & 31;
+    const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (w >= (long long)B * H * nsub) return;
+    const int s = (int)(w % nsub);
+    const int bh = (int)(w / nsub), h = bh % H, b = bh / H;
+    const int j = s / (kChunk / kSub), n0c = j * kChunk, L = min(kChunk, N - n0c);
+    const int r0 = (s % (kChunk / kSub)) * kSub;  // first row of the block within its chunk
+    const int nrows = min(kSub, N - (n0c + r0));
+    const bool act = (flags & kNormScore) && lane < DK / 8;  // without it only c_n is needed
+    const double lg = hc.log2g[h];
+
+    float Z[8], P[8];
+#pragma unroll
+    for (int e = 0; e < 8; e++) Z[e] = P[e] = 0.f;
+    if (act) {
+        const float* zs = zstart + ((size_t)bh * nch + j) * DK + 8 * lane;
+#pragma unroll
+        for (int e = 0; e < 8; e++) Z[e] = zs[e];
+        for (int s2 = j * (kChunk / kSub); s2 < s; s2++) {
+            const float* ps = subsum + ((size_t)bh * nsub + s2) * DK + 8 * lane;
+#pragma unroll
+            for (int e = 0; e < 8; e++) P[e] += ps[e];
+        }
+    }
+    float vals[kSub];
+#pragma unroll
+    for (int rb = 0; rb < kSub; rb += 8) {
+        uint4 kx[8], qx[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            if (act && rb + u < nrows) {
+                const size_t row = ((size_t)b * N + n0c + r0 + rb + u) * H + h;
+                kx[u] = __ldg(reinterpret_cast<const uint4*>(kp + row * DK + 8 * lane));
+                qx[u] = __ldg(reinterpret_cast<const uint4*>(qe + row * DK + 8 * lane));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; u++) {
+            float val = 0.f;
+            if (act && rb + u < nrows) {
+                const int r = r0 + rb + u;
+                const float a = exp2f((float)((r + 1 - L) * lg));  // gamma^(r+1-L)
+                const float c = exp2f((float)((r + 1) * lg));      // gamma^(r+1)
+                float kf[8], qf[8];
+                unpack_bf16x8(kx[u], kf);
+                unpack_bf16x8(qx[u], qf);
+#pragma unroll
+                for (int e = 0; e < 8; e++) {
+                    P[e] += kf[e];
+                    val = fmaf(qf[e], fmaf(a, P[e], c * Z[e]), val);
+                }
+            }
+            vals[rb + u] = val;
+        }
+    }
+    const float sn = transpose_reduce32(vals, lane);  // row r0 + lane
+    if (lane < nrows) {
+        const long long n = n0c + r0 + lane;
+        double f = 1.0;
+        if (flags & kNormDecay) {
+            // sum_{i<=n} gamma^(n-i) over the whole sequence, position pos0 + n
+            const double ln_g = lg * 0.69314718055994530942;
+            const double cnt = (double)(pos0 + n + 1);
+            const double geo = (lg == 0.0) ? cnt : expm1(cnt * ln_g) / expm1(ln_g);
+            f = 1.0 / sqrt(geo);
+        }
+        if (flags & kNormScore) f /= fmax(fabs(f * (double)sn), 1.0);
+        rowscale[((size_t)b * N + n) * H + h] = (float)f;
+    }
+}
+
+struct NormLayout {
+    size_t rowscale, subsum, zstart, total;
+    int nsub, nch;
+};
+
+NormLayout norm_layout(const RetArgs& a) {
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    NormLayout L;
+    L.nsub = (a.N + kSub - 1) / kSub;
+    L.nch = (a.N + kChunk - 1) / kChunk;
+    size_t o = al(chunkwise_ws_bytes(a));
+    L.rowscale = o; o += al((size_t)a.B * a.N * a.H * 4);
+    L.subsum = o; o += al((size_t)a.B * a.H * L.nsub * a.dk * 4);
+    L.zstart = o; o += al((size_t)a.B * a.H * L.nch * a.dk * 4);
+    L.total = o;
+    return L;
+}
+
+}  // namespace
+
+size_t normalized_ws_bytes(const RetArgs& a) { return norm_layout(a).total; }
+
+ret_status launch_chunkwise_normalized(const RetArgs& a0, int flags, const float* z0, float* z1, void* ws,
+                                       cudaStream_t s) {
+    const NormLayout L = norm_layout(a0);
+    uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+    float* rowscale = reinterpret_cast<float*>(base + L.rowscale);
+    float* subsum = reinterpret_cast<float*>(base + L.subsum);
+    float* zstart = reinterpret_cast<float*>(base + L.zstart);
+    ret_status st = launch_chunkwise_prep(a0, ws, s);
+    if (st != RET_OK) return st;
+    // the prepared k' opens the workspace; the rotated q follows it (xpos) or is q itself
+    const size_t qk = (size_t)a0.B * a0.N * a0.H * a0.dk;
+    const __nv_bfloat16* kp = reinterpret_cast<const __nv_bfloat16*>(ws);
+    const __nv_bfloat16* qe = a0.xpos ? kp + qk : reinterpret_cast<const __nv_bfloat16*>(a0.q);
+    const long long warps = (long long)a0.B * a0.H * L.nsub;
+    const int blocks = (int)((warps + 7) / 8);
+    const bool keys = (flags & kNormScore) || z1;  // the key sums are needed
+    if (a0.dk == 256) {
+        if (keys) {
+            k_keysum<256><<<blocks, 256, 0, s>>>(kp, subsum, a0.B, a0.N, a0.H, L.nsub);
+            k_keycarry<256><<<a0.B * a0.H, 256, 0, s>>>(subsum, z0, zstart, z1, a0.hc, a0.H, a0.N, L.nsub, L.nch);
+        }
+        k_rowscale<256><<<blocks, 256, 0, s>>>(qe, kp, subsum, zstart, rowscale, a0.hc, a0.B, a0.N, a0.H, L.nsub,
+                                               L.nch, a0.pos_offset, flags);
+    } else {
+        if (keys) {
+            k_keysum<128><<<blocks, 256, 0, s>>>(kp, subsum, a0.B, a0.N, a0.H, L.nsub);
+            k_keycarry<128><<<a0.B * a0.H, 128, 0, s>>>(subsum, z0, zstart, z1, a0.hc, a0.H, a0.N, L.nsub, L.nch);
+        }
+        k_rowscale<128><<<blocks, 256, 0, s>>>(qe, kp, subsum, zstart, rowscale, a0.hc, a0.B, a0.N, a0.H, L.nsub,
+                                               L.nch, a0.pos_offset, flags);
+    }
+    st = check_launch("chunkwise normalized: row factors");
+    if (st != RET_OK) return st;
+    RetArgs a = a0;
+    a.rowscale = rowscale;
+    return launch_chunkwise_prepared(a, ws, s);
+}
+
+}  // namespace ret

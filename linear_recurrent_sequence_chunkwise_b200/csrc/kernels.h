@@ -21,6 +21,9 @@ struct RetArgs {
     // fp32 out instead of storing it; out_rev = 1 writes the output of token n
     // to row N-1-n.
     int q_ld, k_ld, accumulate, out_rev;
+    // Workspace path only: fp32 [B, N, H] factors the output row of each
+    // (token, head) is multiplied by (the score normalizations), or null.
+    const float* rowscale;
     int B, N, H, dk, dv, chunk;
     ret_dtype in_dt, out_dt;
     int xpos;
@@ -56,6 +59,20 @@ ret_status launch_chunkwise_prepared(const RetArgs& a, void* ws, cudaStream_t s)
 // The workspace path on the library's fixed device array (no allocation).
 size_t chunkwise_static_ws_bytes();
 ret_status launch_chunkwise_static(const RetArgs& a, cudaStream_t s);
+// Score normalizations 2 and 3 on the workspace path: flags bit 0 divides
+// row n of the decay matrix by sqrt(sum_i D_ni), bit 1 the scores by
+// max(|sum_i R_ni|, 1); z0 / z1 the decayed key sum before / after the
+// call ([B, H, dk] fp32, either may be null).
+constexpr int kNormDecay = RET_NORM_DECAY, kNormScore = RET_NORM_SCORE;
+size_t normalized_ws_bytes(const RetArgs& a);
+ret_status launch_chunkwise_normalized(const RetArgs& a, int flags, const float* z0, float* z1, void* ws,
+                                       cudaStream_t s);
+// The decode step with the same normalizations at absolute position pos;
+// z [B, H, dk] updated in place (may be null without kNormScore).
+ret_status launch_decode_normalized(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
+                                    float* z, void* out, int B, int H, int dk, int dv, ret_dtype in_dt,
+                                    ret_dtype out_dt, long long pos, int flags, cudaStream_t s);
+
 // The tensor-core kernel alone, on prepared q_rot (or q) and k' (zeta-scaled keys).
 // q_rot: [B, N, H, dk] rows q_pitch elements apart.
 ret_status launch_chunkwise_main(const RetArgs& a, const void* q_rot, int q_pitch, const void* k_prime,

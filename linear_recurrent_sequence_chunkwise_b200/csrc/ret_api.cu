@@ -83,7 +83,7 @@ static ret_status make_args(RetArgs* a, const char* who, const void* q, const vo
             return fail(RET_ERR_INVALID_ARG, "%s: final_state overlaps another buffer", who);
     }
     a->q = q; a->k = k; a->v = v; a->out = out; a->final_state = final_state; a->initial_state = nullptr;
-    a->q_ld = 0; a->k_ld = 0; a->accumulate = 0; a->out_rev = 0;
+    a->q_ld = 0; a->k_ld = 0; a->accumulate = 0; a->out_rev = 0; a->rowscale = nullptr;
     a->B = B; a->N = N; a->H = H; a->dk = dk; a->dv = dv; a->chunk = chunk;
     a->in_dt = in_dt; a->out_dt = out_dt;
     a->xpos = xpos ? 1 : 0; a->pos_offset = pos_offset; a->theta_base = xpos ? theta_base : 10000.0;
@@ -185,6 +185,22 @@ static ret_status check_workspace(const RetArgs& a, const char* who, const void*
     return RET_OK;
 }
 
+// initial_state (may be null) against the other buffers of a; final_state
+// may be the same buffer.  Sets a->initial_state.
+static ret_status check_initial_state(RetArgs* a, const char* who, const float* initial_state) {
+    if (!initial_state) return RET_OK;
+    const size_t ntok = (size_t)a->B * a->N * a->H, bs = (size_t)a->B * a->H * a->dk * a->dv * 4;
+    const size_t bq = ntok * a->dk * 2, bv = ntok * a->dv * 2, bo = ntok * a->dv * (a->out_dt == RET_F32 ? 4 : 2);
+    if (!aligned(initial_state, 16)) return fail(RET_ERR_INVALID_ARG, "%s: initial_state must be 16-byte aligned", who);
+    if (overlaps(initial_state, bs, a->out, bo) || overlaps(initial_state, bs, a->q, bq) ||
+        overlaps(initial_state, bs, a->k, bq) || overlaps(initial_state, bs, a->v, bv) ||
+        (a->final_state && (const void*)a->final_state != (const void*)initial_state &&
+         overlaps(initial_state, bs, a->final_state, bs)))
+        return fail(RET_ERR_INVALID_ARG, "%s: initial_state overlaps another buffer (final_state may equal it)", who);
+    a->initial_state = initial_state;
+    return RET_OK;
+}
+
 ret_status ret_chunkwise_prepare(const void* q, const void* k, const double* gammas, int B, int N, int H, int dk,
                                  int dv, int chunk, cudaStream_t stream, ret_dtype in_dt, int xpos,
                                  int64_t pos_offset, double theta_base, void* workspace, size_t workspace_bytes) {
@@ -230,21 +246,65 @@ ret_status ret_forward_chunkwise_prepared(const void* q, const void* k, const vo
     if (!chunkwise_ws_supported(a))
         return fail(RET_ERR_UNSUPPORTED, "%s: shape outside the workspace path (ret_chunkwise_workspace_bytes is 0)",
                     who);
-    if (initial_state) {
-        const size_t ntok = (size_t)B * N * H, bs = (size_t)B * H * dk * dv * 4;
-        const size_t bq = ntok * dk * 2, bv = ntok * dv * 2, bo = ntok * dv * (out_dt == RET_F32 ? 4 : 2);
-        if (!aligned(initial_state, 16)) return fail(RET_ERR_INVALID_ARG, "%s: initial_state must be 16-byte aligned", who);
-        if (overlaps(initial_state, bs, out, bo) || overlaps(initial_state, bs, q, bq) ||
-            overlaps(initial_state, bs, k, bq) || overlaps(initial_state, bs, v, bv) ||
-            (final_state && (const void*)final_state != (const void*)initial_state &&
-             overlaps(initial_state, bs, final_state, bs)))
-            return fail(RET_ERR_INVALID_ARG, "%s: initial_state overlaps another buffer (final_state may equal it)",
-                        who);
-        a.initial_state = initial_state;
-    }
+    st = check_initial_state(&a, who, initial_state);
+    if (st != RET_OK) return st;
     st = check_workspace(a, who, workspace, workspace_bytes, true);
     if (st != RET_OK) return st;
     return launch_chunkwise_prepared(a, const_cast<void*>(workspace), stream);
+}
+
+size_t ret_normalized_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk, ret_dtype in_dt, int xpos) {
+    if (B < 1 || N < 1 || H < 1 || H > kMaxHeads || dk < 1 || dv < 1 || chunk < 1) return 0;
+    RetArgs a{};
+    a.B = B; a.N = N; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.in_dt = in_dt; a.xpos = xpos ? 1 : 0;
+    for (int h = 0; h < kMaxHeads; h++) a.hc.log2g[h] = 0.0;  // shape check only
+    return chunkwise_ws_supported(a) ? normalized_ws_bytes(a) : 0;
+}
+
+ret_status ret_forward_chunkwise_normalized(const void* q, const void* k, const void* v, const double* gammas, int B,
+                                            int N, int H, int dk, int dv, int chunk, int norm_flags, void* out,
+                                            const float* initial_state, float* final_state, const float* initial_z,
+                                            float* final_z, cudaStream_t stream, ret_dtype in_dt, ret_dtype out_dt,
+                                            int xpos, int64_t pos_offset, double theta_base, void* workspace,
+                                            size_t workspace_bytes) {
+    t_err[0] = 0;
+    const char* who = "ret_forward_chunkwise_normalized";
+    RetArgs a;
+    ret_status st = make_args(&a, who, q, k, v, gammas, B, N, H, dk, dv, chunk, out, final_state, in_dt, out_dt,
+                              xpos, pos_offset, theta_base);
+    if (st != RET_OK) return st;
+    if (norm_flags & ~(RET_NORM_DECAY | RET_NORM_SCORE))
+        return fail(RET_ERR_INVALID_ARG, "%s: norm_flags must combine RET_NORM_DECAY and RET_NORM_SCORE", who);
+    if (pos_offset < 0) return fail(RET_ERR_INVALID_ARG, "%s: pos_offset must be >= 0", who);
+    if (!chunkwise_ws_supported(a))
+        return fail(RET_ERR_UNSUPPORTED,
+                    "%s: needs bf16 inputs, chunk 128, dk 128 or 256, dv a multiple of 64 and every "
+                    "gamma_h^128 >= 2^-60",
+                    who);
+    st = check_initial_state(&a, who, initial_state);
+    if (st != RET_OK) return st;
+    const size_t ntok = (size_t)B * N * H, bz = (size_t)B * H * dk * 4, bs = (size_t)B * H * dk * dv * 4;
+    const size_t bq = ntok * dk * 2, bv = ntok * dv * 2, bo = ntok * dv * (out_dt == RET_F32 ? 4 : 2);
+    for (const float* z : {initial_z, (const float*)final_z}) {
+        if (!z) continue;
+        if (!aligned(z, 16)) return fail(RET_ERR_INVALID_ARG, "%s: initial_z and final_z must be 16-byte aligned", who);
+        if (overlaps(z, bz, q, bq) || overlaps(z, bz, k, bq) || overlaps(z, bz, v, bv) || overlaps(z, bz, out, bo) ||
+            (final_state && overlaps(z, bz, final_state, bs)) || (initial_state && overlaps(z, bz, initial_state, bs)))
+            return fail(RET_ERR_INVALID_ARG, "%s: initial_z or final_z overlaps another buffer", who);
+    }
+    if (initial_z && final_z && initial_z != final_z && overlaps(initial_z, bz, final_z, bz))
+        return fail(RET_ERR_INVALID_ARG, "%s: initial_z and final_z overlap (they may be the same buffer)", who);
+    const size_t need = normalized_ws_bytes(a);
+    if (!workspace || workspace_bytes < need)
+        return fail(RET_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed (got %zu)", who, need,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (!aligned(workspace, 256)) return fail(RET_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+    if (overlaps(workspace, need, q, bq) || overlaps(workspace, need, k, bq) || overlaps(workspace, need, v, bv) ||
+        overlaps(workspace, need, out, bo) || (final_state && overlaps(workspace, need, final_state, bs)) ||
+        (initial_state && overlaps(workspace, need, initial_state, bs)) ||
+        (initial_z && overlaps(workspace, need, initial_z, bz)) || (final_z && overlaps(workspace, need, final_z, bz)))
+        return fail(RET_ERR_INVALID_ARG, "%s: workspace overlaps another buffer", who);
+    return launch_chunkwise_normalized(a, norm_flags, initial_z, final_z, workspace, stream);
 }
 
 static void fill_bwd(BwdArgs* b, const void* q, const void* k, const void* v, const void* dout, int B, int N, int H,
@@ -380,6 +440,41 @@ ret_status ret_decode_step(const void* q, const void* k, const void* v, const do
     HeadConsts hc;
     make_head_consts(gammas, H, &hc);
     return launch_decode(q, k, v, hc, state, out, B, H, dk, dv, in_dt, out_dt, stream);
+}
+
+ret_status ret_decode_step_normalized(const void* q, const void* k, const void* v, const double* gammas,
+                                      float* state, float* z, void* out, int64_t position, int norm_flags,
+                                      cudaStream_t stream, int B, int H, int dk, int dv, ret_dtype in_dt,
+                                      ret_dtype out_dt) {
+    t_err[0] = 0;
+    const char* who = "ret_decode_step_normalized";
+    if (!q || !k || !v || !state || !out) return fail(RET_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
+    if (B < 1 || H < 1 || dk < 1 || dv < 1)
+        return fail(RET_ERR_INVALID_ARG, "%s: sizes must be >= 1 (B=%d H=%d dk=%d dv=%d)", who, B, H, dk, dv);
+    if (!is_dtype(in_dt) || !is_dtype(out_dt)) return fail(RET_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    if (norm_flags & ~(RET_NORM_DECAY | RET_NORM_SCORE))
+        return fail(RET_ERR_INVALID_ARG, "%s: norm_flags must combine RET_NORM_DECAY and RET_NORM_SCORE", who);
+    if ((norm_flags & RET_NORM_SCORE) && !z)
+        return fail(RET_ERR_INVALID_ARG, "%s: RET_NORM_SCORE needs the key-sum state z", who);
+    if (position < 0) return fail(RET_ERR_INVALID_ARG, "%s: position must be >= 0", who);
+    ret_status st = check_gammas(gammas, H, who);
+    if (st != RET_OK) return st;
+    if (dv % 4 != 0) return fail(RET_ERR_INVALID_ARG, "%s: dv must be a multiple of 4 (got %d)", who, dv);
+    if (!aligned(state, 16)) return fail(RET_ERR_INVALID_ARG, "%s: state must be 16-byte aligned", who);
+    for (const void* p : {q, k, v, (const void*)out})
+        if (!aligned(p, 4)) return fail(RET_ERR_INVALID_ARG, "%s: q, k, v, out must be 4-byte aligned", who);
+    const size_t bs = (size_t)B * H * dk * dv * 4, bo = (size_t)B * H * dv * esize(out_dt);
+    const size_t bz = (size_t)B * H * dk * 4, bq = (size_t)B * H * dk * esize(in_dt);
+    if (overlaps(out, bo, state, bs)) return fail(RET_ERR_INVALID_ARG, "%s: out overlaps state", who);
+    if (z && (norm_flags & RET_NORM_SCORE)) {
+        if (!aligned(z, 16)) return fail(RET_ERR_INVALID_ARG, "%s: z must be 16-byte aligned", who);
+        if (overlaps(z, bz, state, bs) || overlaps(z, bz, out, bo) || overlaps(z, bz, q, bq) || overlaps(z, bz, k, bq))
+            return fail(RET_ERR_INVALID_ARG, "%s: z overlaps another buffer", who);
+    }
+    HeadConsts hc;
+    make_head_consts(gammas, H, &hc);
+    return launch_decode_normalized(q, k, v, hc, state, (norm_flags & RET_NORM_SCORE) ? z : nullptr, out, B, H, dk,
+                                    dv, in_dt, out_dt, position, norm_flags, stream);
 }
 
 size_t ret_msr_workspace_bytes(int B, int N, int dmodel, int H, int dk, int dv) {

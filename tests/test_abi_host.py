@@ -197,3 +197,52 @@ def test_backward_workspace_size():
 def test_backward_rejects_bad_arguments(kw, status):
     assert backward_call(**kw) == status, (kw, R.ret_last_error_string())
     assert R.ret_last_error_string()
+
+
+def test_normalized_workspace_size():
+    nb = R.ret_normalized_workspace_bytes(1, 200, 2, 128, 64, 128, torch.bfloat16, True)
+    ws = R.ret_chunkwise_workspace_bytes(1, 200, 2, 128, 64, 128, torch.bfloat16, True)
+    # the prepared q, k, then row factors [B, N, H], key sums per 32 rows and per chunk start
+    al = lambda x: (x + 255) // 256 * 256
+    assert nb == al(ws) + al(200 * 2 * 4) + al(2 * 7 * 128 * 4) + al(2 * 2 * 128 * 4)
+    assert R.ret_normalized_workspace_bytes(1, 200, 2, 16, 64, 128, torch.bfloat16, True) == 0
+    assert R.ret_normalized_workspace_bytes(1, 200, 2, 128, 64, 128, torch.float32, True) == 0
+
+
+def normalized_call(flags=3, out=P4, init=None, fs=None, z0=None, z1=None, ws=WS, nbytes=None, dk=128, pos=0):
+    if nbytes is None:
+        nbytes = R.ret_normalized_workspace_bytes(1, 128, 2, 128, 64, 128, torch.bfloat16, False)
+        assert 0 < nbytes < 0x20000000
+    return R.lib.ret_forward_chunkwise_normalized(P, P2, P3, G2, 1, 128, 2, dk, 64, 128, flags, out, init, fs, z0, z1,
+                                                  S0, 1, 1, 0, pos, 1e4, ws, nbytes)
+
+
+@needs_no_gpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(flags=4), 1), (dict(flags=-1), 1), (dict(pos=-1), 1), (dict(out=None), 1),
+    (dict(ws=None), 1), (dict(nbytes=1000), 1),
+    (dict(z0=ctypes.c_void_p(0xB0000004)), 1),                              # misaligned z
+    (dict(z1=ctypes.c_void_p(0x90000000)), 1),                              # z overlaps out
+    (dict(z0=ctypes.c_void_p(0xB0000000), z1=ctypes.c_void_p(0xB0000100)), 1),  # partial overlap
+    (dict(ws=ctypes.c_void_p(0x90000000)), 1),                              # workspace overlaps out
+    (dict(dk=16), 2),
+])
+def test_normalized_rejects_bad_arguments(kw, status):
+    assert normalized_call(**kw) == status, (kw, R.ret_last_error_string())
+    assert R.ret_last_error_string()
+
+
+def decode_normalized_call(z=ctypes.c_void_p(0xB0000000), pos=5, flags=3, state=ctypes.c_void_p(0xC0000000), dv=64):
+    return R.lib.ret_decode_step_normalized(P, P2, P3, G2, state, z, P4, pos, flags, S0, 1, 2, 16, dv, 1, 1)
+
+
+@needs_no_gpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(z=None), 1), (dict(pos=-1), 1), (dict(flags=8), 1), (dict(state=None), 1),
+    (dict(z=ctypes.c_void_p(0xB0000008)), 1),                    # misaligned z
+    (dict(z=ctypes.c_void_p(0xC0000000)), 1),                    # z overlaps the state
+    (dict(dv=6), 1),
+])
+def test_decode_normalized_rejects_bad_arguments(kw, status):
+    assert decode_normalized_call(**kw) == status, (kw, R.ret_last_error_string())
+    assert R.ret_last_error_string()
