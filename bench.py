@@ -170,6 +170,8 @@ def run_ours(args):
         stream = torch.cuda.current_stream()
         if args.only == "backward":
             res = {"backward": bench_backward(R, torch, dev, stream, w, g, args, peaks, world, dist)}
+        elif args.only == "normalized":
+            res = {"normalized": bench_normalized(R, torch, dev, stream, w, g, args, peaks, world, dist)}
         else:
             res = {"msr_layer": bench_msr(R, torch, dev, stream, args, peaks, world, dist)}
         if rank == 0:
@@ -284,6 +286,7 @@ def run_ours(args):
         result["decode"] = bench_decode(R, torch, dev, stream, args, peaks, world, barrier, dist, rank)
     if not args.no_layer:
         result["backward"] = bench_backward(R, torch, dev, stream, w, g, args, peaks, world, dist)
+        result["normalized"] = bench_normalized(R, torch, dev, stream, w, g, args, peaks, world, dist)
         result["msr_layer"] = bench_msr(R, torch, dev, stream, args, peaks, world, dist)
         result["fp32_small"] = bench_fp32_small(R, torch, dev, stream, args, world, dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -426,6 +429,42 @@ def bench_backward(R, torch, dev, stream, w, g, args, peaks, world, dist):
                          "kernels": "5 x (k_prep_qk + k_chunkwise_ws), 6 x k_row_transform"}}
 
 
+def bench_normalized(R, torch, dev, stream, w, g, args, peaks, world, dist):
+    """The chunkwise forward with the score normalizations 2 and 3 on the same
+    workload (one call: the rotation + zeta pass, three passes for the row
+    factors, the tensor-core kernel with the factors in its epilogue), final
+    S and z written.  Compared with the plain forward of the same call
+    shape, timed the same way."""
+    B, N, H, dk, dv, C = w["B"], w["N"], w["H"], w["dk"], w["dv"], w["chunk"]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0x5EED0007)
+    sc = dk ** -0.5
+    q = (torch.randn((B, N, H, dk), generator=gen, device=dev) * sc).to(torch.bfloat16)
+    k = (torch.randn((B, N, H, dk), generator=gen, device=dev) * sc).to(torch.bfloat16)
+    v = torch.randn((B, N, H, dv), generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty((B, N, H, dv), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    fz = torch.empty((B, H, dk), dtype=torch.float32, device=dev)
+    ws = torch.empty(R.ret_normalized_workspace_bytes(B, N, H, dk, dv, C, torch.bfloat16, True), dtype=torch.uint8,
+                     device=dev)
+
+    def norm():
+        R.ret_forward_chunkwise_normalized(q, k, v, g, C, norm_flags=R.NORM_DECAY | R.NORM_SCORE, workspace=ws,
+                                           out=out, final_state=fs, final_z=fz, xpos=True, stream=stream)
+
+    def plain():
+        R.ret_forward_chunkwise_ws(q, k, v, g, C, ws, out=out, final_state=fs, xpos=True, stream=stream)
+
+    steps = max(5, min(args.steps, 20))
+    ms = _timed(torch, stream, norm, steps, 3, world, dist, dev)
+    ms_plain = _timed(torch, stream, plain, steps, 3, world, dist, dev)
+    R.ret_check_device_error()
+    return {"workload": w["workload"], "flags": "decay + score", "ms_per_step": round(ms, 4),
+            "tokens_per_s": round(world * B * N / (ms / 1e3), 1), "plain_ms_per_step": round(ms_plain, 4),
+            "overhead": round(ms / ms_plain - 1.0, 4),
+            "kernels": "k_prep_qk, k_keysum, k_keycarry, k_rowscale, k_chunkwise_ws (row factors in the epilogue)"}
+
+
 def bench_msr(R, torch, dev, stream, args, peaks, world, dist):
     """The MultiScaleRetention layer forward on X [2, 4096, 2048] (H 8, d_k 256,
     d_v 512, xPos, chunk 128): four projections, retention, GroupNorm + swish
@@ -558,7 +597,7 @@ def main():
     ap.add_argument("--seq", type=int, default=WORKLOAD["N"],
                     help="sequence length of the chunkwise workload (smaller values make ncu captures short)")
     ap.add_argument("--no-chunkwise", action="store_true", help="skip the chunkwise forward (decode only)")
-    ap.add_argument("--only", choices=["backward", "msr"],
+    ap.add_argument("--only", choices=["backward", "msr", "normalized"],
                     help="time only the backward or only the MSR layer (for ncu launch lists of one part)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -77,61 +77,84 @@ __global__ void __launch_bounds__(256) k_keysum(const __nv_bfloat16* __restrict_
     }
 }
 
-// One block per (batch, head), one thread per key component: the decayed key
-// sum before each chunk (zstart) and after the last one (z1).
-template <int DK>
-__global__ void __launch_bounds__(DK) k_keycarry(const float* __restrict__ subsum, const float* z0, float* zstart,
-                                                 float* z1, HeadConsts hc, int H, int N, int nsub, int nch) {
-    const int bh = blockIdx.x, h = bh % H, d = threadIdx.x;
+// The decayed key sum before each chunk (zstart) and after the last one
+// (z1).  Block (batch, head, half of d_k), thread (segment t, component d):
+// the chunks are cut into kSeg segments; each thread carries its segment
+// from zero, the segments' end values are combined in order through shared
+// memory, and each thread carries its segment again from its true start.
+constexpr int kSeg = 8, kCarryD = 128;
+__global__ void __launch_bounds__(kSeg * kCarryD) k_keycarry(const float* __restrict__ subsum, const float* z0,
+                                                             float* zstart, float* z1, HeadConsts hc, int H, int DK,
+                                                             int N, int nsub, int nch) {
+    __shared__ float s_end[kSeg][kCarryD];
+    const int halves = DK / kCarryD;
+    const int bh = blockIdx.x / halves, h = bh % H;
+    const int d = (blockIdx.x % halves) * kCarryD + threadIdx.x % kCarryD, t = threadIdx.x / kCarryD;
     const double lg = hc.log2g[h];
     const float g_full = (float)exp2(kChunk * lg);
-    const int L_last = N - (nch - 1) * kChunk;
-    const float g_last = (float)exp2(L_last * lg);
-    float Z = z0 ? z0[(size_t)bh * DK + d] : 0.f;
+    const float g_last = (float)exp2((N - (nch - 1) * kChunk) * lg);
+    const int per = (nch + kSeg - 1) / kSeg, j0 = t * per, j1 = min(nch, j0 + per);
     const float* ss = subsum + (size_t)bh * nsub * DK + d;
-    for (int j = 0; j < nch; j++) {
-        zstart[((size_t)bh * nch + j) * DK + d] = Z;
-        const int s0 = j * (kChunk / kSub), s1 = min(nsub, s0 + kChunk / kSub);
-        float cs = 0.f;
-        for (int s = s0; s < s1; s++) cs += ss[(size_t)s * DK];
-        Z = fmaf(j == nch - 1 ? g_last : g_full, Z, cs);
-    }
-    if (z1) z1[(size_t)bh * DK + d] = Z;
-}
-
-// 32 values per lane in, lane l out with the sum over the warp of value l
-// (a butterfly that halves the values each lane carries at every step).
-template <int O>
-__device__ __forceinline__ void butterfly_step(float* v, int lane) {
-    const bool up = (lane & O) != 0;
+    constexpr int kPer = kChunk / kSub;
+    auto chunk_sum = [&](int j) {
+        float c = 0.f;
 #pragma unroll
-    for (int i = 0; i < O; i++) {
-        const float send = up ? v[i] : v[i + O];
-        const float keep = up ? v[i + O] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+        for (int i = 0; i < kPer; i++) {
+            const int sb = j * kPer + i;
+            if (sb < nsub) c += ss[(size_t)sb * DK];
+        }
+        return c;
+    };
+    // read before anything is written: z1 may be the same buffer as z0
+    float Z = z0 ? z0[(size_t)bh * DK + d] : 0.f;
+    // the segment's chunk sums, loaded together (segments of up to kHeld
+    // chunks stay in registers for the second pass)
+    constexpr int kHeld = 8;
+    const bool held = j1 - j0 <= kHeld;
+    float cs[kHeld];
+#pragma unroll
+    for (int u = 0; u < kHeld; u++) cs[u] = (held && j0 + u < j1) ? chunk_sum(j0 + u) : 0.f;
+    auto sum_at = [&](int j) {
+        if (held) {
+            float c = 0.f;
+#pragma unroll
+            for (int u = 0; u < kHeld; u++) c = (j - j0 == u) ? cs[u] : c;
+            return c;
+        }
+        return chunk_sum(j);
+    };
+    // pass 1: this segment from zero
+    float E = 0.f;
+    for (int j = j0; j < j1; j++) E = fmaf(j == nch - 1 ? g_last : g_full, E, sum_at(j));
+    s_end[t][threadIdx.x % kCarryD] = E;
+    __syncthreads();
+    // the value entering this segment: earlier segments in order (all but the
+    // last chunk of the sequence span full chunks)
+    for (int u = 0; u < t; u++) {
+        const int len = min(nch, (u + 1) * per) - u * per;
+        Z = fmaf((float)exp2((double)len * kChunk * lg), Z, s_end[u][threadIdx.x % kCarryD]);
     }
-}
-
-__device__ __forceinline__ float transpose_reduce32(float* v, int lane) {
-    butterfly_step<16>(v, lane);
-    butterfly_step<8>(v, lane);
-    butterfly_step<4>(v, lane);
-    butterfly_step<2>(v, lane);
-    butterfly_step<1>(v, lane);
-    return v[0];
+    // pass 2: this segment from its true start
+    for (int j = j0; j < j1; j++) {
+        zstart[((size_t)bh * nch + j) * DK + d] = Z;
+        Z = fmaf(j == nch - 1 ? g_last : g_full, Z, sum_at(j));
+    }
+    __syncthreads();  // every thread has read z0
+    if (z1 && j1 == nch && j0 < j1) z1[(size_t)bh * DK + d] = Z;
 }
 
 // One warp per (batch, head, 32-row block): the row sums s_n of its rows and
 // the factors f_n.
+constexpr int kRsWarps = 4;  // warps per block of k_rowscale
 template <int DK>
-__global__ void __launch_bounds__(256) k_rowscale(const __nv_bfloat16* __restrict__ qe,
+__global__ void __launch_bounds__(kRsWarps * 32, 4) k_rowscale(const __nv_bfloat16* __restrict__ qe,
                                                   const __nv_bfloat16* __restrict__ kp,
                                                   const float* __restrict__ subsum, const float* __restrict__ zstart,
                                                   float* __restrict__ rowscale, HeadConsts hc, int B, int N, int H,
                                                   int nsub, int nch, long long pos0, int flags) {
     static_assert(DK / 8 <= 32, "one 8-element group per lane");
     const int lane = threadIdx.x & 31;
-    const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const long long w = (long long)blockIdx.x * kRsWarps + (threadIdx.x >> 5);
     if (w >= (long long)B * H * nsub) return;
     const int s = (int)(w % nsub);
     const int bh = (int)(w / nsub), h = bh % H, b = bh / H;
@@ -154,7 +177,10 @@ __global__ void __launch_bounds__(256) k_rowscale(const __nv_bfloat16* __restric
             for (int e = 0; e < 8; e++) P[e] += ps[e];
         }
     }
-    float vals[kSub];
+    // lane partials of each row, summed per row through shared memory (padded
+    // rows: lane l reading row l touches 32 different banks)
+    __shared__ float part[kRsWarps][kSub][33];
+    float (*pw)[33] = part[threadIdx.x >> 5];
 #pragma unroll
     for (int rb = 0; rb < kSub; rb += 8) {
         uint4 kx[8], qx[8];
@@ -182,10 +208,13 @@ __global__ void __launch_bounds__(256) k_rowscale(const __nv_bfloat16* __restric
                     val = fmaf(qf[e], fmaf(a, P[e], c * Z[e]), val);
                 }
             }
-            vals[rb + u] = val;
+            pw[rb + u][lane] = val;
         }
     }
-    const float sn = transpose_reduce32(vals, lane);  // row r0 + lane
+    __syncwarp();
+    float sn = 0.f;  // row r0 + lane
+#pragma unroll 8
+    for (int i = 0; i < 32; i++) sn += pw[lane][i];
     if (lane < nrows) {
         const long long n = n0c + r0 + lane;
         double f = 1.0;
@@ -238,20 +267,23 @@ ret_status launch_chunkwise_normalized(const RetArgs& a0, int flags, const float
     const __nv_bfloat16* qe = a0.xpos ? kp + qk : reinterpret_cast<const __nv_bfloat16*>(a0.q);
     const long long warps = (long long)a0.B * a0.H * L.nsub;
     const int blocks = (int)((warps + 7) / 8);
+    const int rs_blocks = (int)((warps + kRsWarps - 1) / kRsWarps);
     const bool keys = (flags & kNormScore) || z1;  // the key sums are needed
     if (a0.dk == 256) {
         if (keys) {
             k_keysum<256><<<blocks, 256, 0, s>>>(kp, subsum, a0.B, a0.N, a0.H, L.nsub);
-            k_keycarry<256><<<a0.B * a0.H, 256, 0, s>>>(subsum, z0, zstart, z1, a0.hc, a0.H, a0.N, L.nsub, L.nch);
+            k_keycarry<<<a0.B * a0.H * 2, kSeg * kCarryD, 0, s>>>(subsum, z0, zstart, z1, a0.hc, a0.H, 256, a0.N,
+                                                                  L.nsub, L.nch);
         }
-        k_rowscale<256><<<blocks, 256, 0, s>>>(qe, kp, subsum, zstart, rowscale, a0.hc, a0.B, a0.N, a0.H, L.nsub,
+        k_rowscale<256><<<rs_blocks, kRsWarps * 32, 0, s>>>(qe, kp, subsum, zstart, rowscale, a0.hc, a0.B, a0.N, a0.H, L.nsub,
                                                L.nch, a0.pos_offset, flags);
     } else {
         if (keys) {
             k_keysum<128><<<blocks, 256, 0, s>>>(kp, subsum, a0.B, a0.N, a0.H, L.nsub);
-            k_keycarry<128><<<a0.B * a0.H, 128, 0, s>>>(subsum, z0, zstart, z1, a0.hc, a0.H, a0.N, L.nsub, L.nch);
+            k_keycarry<<<a0.B * a0.H, kSeg * kCarryD, 0, s>>>(subsum, z0, zstart, z1, a0.hc, a0.H, 128, a0.N, L.nsub,
+                                                              L.nch);
         }
-        k_rowscale<128><<<blocks, 256, 0, s>>>(qe, kp, subsum, zstart, rowscale, a0.hc, a0.B, a0.N, a0.H, L.nsub,
+        k_rowscale<128><<<rs_blocks, kRsWarps * 32, 0, s>>>(qe, kp, subsum, zstart, rowscale, a0.hc, a0.B, a0.N, a0.H, L.nsub,
                                                L.nch, a0.pos_offset, flags);
     }
     st = check_launch("chunkwise normalized: row factors");
