@@ -366,6 +366,37 @@ ret_status ret_msr_forward(const void* X, const void* Wq, const void* Wk, const 
                            cudaStream_t stream);
 
 /*
+ * One RetNet block, pre-LayerNorm residual layout ("Hybrid Architectures
+ * ...", section 9.2; RetNet paper summary, "Overall RetNet Architecture"):
+ *     Y   = MSR(LN1(X)) + X
+ *     out = gelu(LN2(Y) W1) W2 + Y
+ * MSR as ret_msr_forward (same weights, shapes, k_scale, gn_eps, xpos and
+ * path constraints); LN(x) = (x - mean) / sqrt(var + ln_eps) * gain + bias
+ * per token over d_model (biased variance); gelu(x) = x Phi(x) with the exact
+ * normal CDF.  The pages' RetNet uses d_ff = 2 d_model.
+ * X [B, N, d_model] bf16; W1 [d_model, d_ff], W2 [d_ff, d_model] bf16
+ * row-major as (input, output); ln*_gain, ln*_bias: bf16 [d_model], or NULL
+ * (gain 1, bias 0); out [B, N, d_model] of dtype out_dt.  Y, the LayerNorm
+ * outputs and the FFN hidden layer are held in bf16 in the workspace
+ * (device, 256-byte aligned, at least ret_retnet_block_workspace_bytes(...)
+ * bytes, overlapping nothing).  d_model and d_ff multiples of 8.
+ * Seven launches: LayerNorm, the MSR's four (the residual added in the output
+ * projection's epilogue), LayerNorm, and the two FFN GEMMs (gelu and the
+ * residual in their epilogues).
+ */
+size_t ret_retnet_block_workspace_bytes(int B, int N, int dmodel, int H, int dk, int dv, int dff);
+
+ret_status ret_retnet_block_forward(const void* X, const void* ln1_gain, const void* ln1_bias,
+                                    const void* Wq, const void* Wk, const void* Wv, const void* Wg,
+                                    const void* Wo, const void* ln2_gain, const void* ln2_bias,
+                                    const void* W1, const void* W2, const double* gammas, int B,
+                                    int N, int dmodel, int H, int dk, int dv, int dff, int chunk,
+                                    double k_scale, double gn_eps, double ln_eps, int xpos,
+                                    int64_t pos_offset, double theta_base, void* out,
+                                    ret_dtype out_dt, void* workspace, size_t workspace_bytes,
+                                    cudaStream_t stream);
+
+/*
  * Y = X W on the tensor cores (the GEMM of the MSR layer): X [M, K] bf16,
  * W [K, N] bf16, row-major; Y [M, N] of dtype out_dt.  fp32 accumulation.
  * N and K multiples of 8; device pointers 16-byte aligned; Y must not overlap

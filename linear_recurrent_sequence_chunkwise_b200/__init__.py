@@ -24,7 +24,7 @@ __all__ = [
     "ret_decode_step", "ret_msr_forward", "ret_msr_workspace_bytes",
     "ret_forward_chunkwise_normalized", "ret_normalized_workspace_bytes", "ret_decode_step_normalized",
     "NORM_DECAY", "NORM_SCORE",
-    "ret_linear_bf16",
+    "ret_linear_bf16", "ret_retnet_block_forward", "ret_retnet_block_workspace_bytes",
     "ret_forward_parallel", "ret_forward_recurrent", "ret_check_device_error", "ret_last_error_string",
     "RET_OK", "RET_ERR_INVALID_ARG", "RET_ERR_UNSUPPORTED", "RET_ERR_CUDA", "RET_ERR_TIMEOUT",
     "RET_F32", "RET_BF16",
@@ -82,6 +82,10 @@ def _load_library():
     L.ret_msr_forward.argtypes = [vp, vp, vp, vp, vp, vp, dp, i, i, i, i, i, i, i, d, d, i, i64, d, vp, i, vp,
                                   ctypes.c_size_t, vp]
     L.ret_linear_bf16.argtypes = [vp, vp, vp, i, i, i, i, vp]
+    L.ret_retnet_block_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+    L.ret_retnet_block_workspace_bytes.restype = ctypes.c_size_t
+    L.ret_retnet_block_forward.argtypes = [vp] * 12 + [dp, i, i, i, i, i, i, i, i, d, d, d, i, i64, d, vp, i, vp,
+                                                       ctypes.c_size_t, vp]
     L.ret_check_device_error.argtypes = [vp]
     L.ret_last_error_string.restype = ctypes.c_char_p
     L.ret_last_error_string.argtypes = []
@@ -394,6 +398,38 @@ def ret_decode_step_normalized(q, k, v, gammas, state, z, position: int, norm_fl
 def ret_check_device_error(stream=None):
     """Synchronise the stream and raise if a kernel gave up a bounded wait."""
     _check(lib.ret_check_device_error(_stream(stream)))
+
+
+def ret_retnet_block_workspace_bytes(B, N, dmodel, H, dk, dv, dff) -> int:
+    return int(lib.ret_retnet_block_workspace_bytes(B, N, dmodel, H, dk, dv, dff))
+
+
+def ret_retnet_block_forward(x, wq, wk, wv, wg, wo, w1, w2, gammas, H: int, ln1_gain=None, ln1_bias=None,
+                             ln2_gain=None, ln2_bias=None, chunk: int = 128, k_scale: float = 1.0,
+                             gn_eps: float = 1e-5, ln_eps: float = 1e-5, xpos: bool = True, pos_offset: int = 0,
+                             theta_base: float = 10000.0, out=None, out_dtype=torch.bfloat16, workspace=None,
+                             stream=None):
+    """One pre-LayerNorm RetNet block: Y = MSR(LN1(x)) + x, out = gelu(LN2(Y) W1) W2 + Y.
+    x [B, N, d_model] bf16; weights bf16 [in, out]; LayerNorm gains/biases bf16
+    [d_model] or None (1 / 0)."""
+    B, N, dm = x.shape
+    dk = wq.shape[1] // H
+    dv = wv.shape[1] // H
+    dff = w1.shape[1]
+    if out is None:
+        out = torch.empty((B, N, dm), dtype=out_dtype, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(ret_retnet_block_workspace_bytes(B, N, dm, H, dk, dv, dff), dtype=torch.uint8,
+                                device=x.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib.ret_retnet_block_forward(_ptr(x, "x"), _ptr(ln1_gain, "ln1_gain"), _ptr(ln1_bias, "ln1_bias"),
+                                        _ptr(wq, "wq"), _ptr(wk, "wk"), _ptr(wv, "wv"), _ptr(wg, "wg"),
+                                        _ptr(wo, "wo"), _ptr(ln2_gain, "ln2_gain"), _ptr(ln2_bias, "ln2_bias"),
+                                        _ptr(w1, "w1"), _ptr(w2, "w2"), _gammas(gammas, H), B, N, dm, H, dk, dv,
+                                        dff, int(chunk), float(k_scale), float(gn_eps), float(ln_eps),
+                                        int(bool(xpos)), int(pos_offset), float(theta_base), _ptr(out, "out"),
+                                        _dt(out.dtype), _ptr(workspace, "workspace"), nbytes, _stream(stream)))
+    return out
 
 
 def ret_linear_bf16(x, w, out=None, out_dtype=torch.bfloat16, stream=None):

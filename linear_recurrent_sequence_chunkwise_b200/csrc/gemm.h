@@ -11,6 +11,8 @@ enum : int {
     kEpiRotate = 1,           // out = rot(scale * acc)             (queries)
     kEpiRotateScaleZeta = 2,  // out = rot(scale * acc) * zeta      (keys)
     kEpiSwish = 3,            // out = swish(acc)                   (gate)
+    kEpiGelu = 4,             // out = gelu(acc)                    (FFN hidden layer)
+    kEpiResidual = 5,         // out = scale * acc + res            (a residual branch)
 };
 
 struct GemmSegment {
@@ -25,6 +27,8 @@ struct GemmSegOut {
     ret_dtype dtype;    // kEpiStore / kEpiSwish: RET_F32 or RET_BF16; rotations write bf16
     float scale;
     int head_dim;       // rotations: width of a head (pairs rotate within it)
+    const __nv_bfloat16* res;  // kEpiResidual: [M, res_ld] bf16 added to the result
+    int res_ld;
 };
 
 struct GemmEpilogue {

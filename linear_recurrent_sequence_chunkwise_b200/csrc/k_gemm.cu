@@ -69,6 +69,9 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int t, int& tm,
 
 __device__ __forceinline__ float swish(float x) { return x / (1.f + expf(-x)); }
 
+// gelu(x) = x Phi(x) with the exact normal CDF, Phi(x) = (1 + erf(x / sqrt 2)) / 2.
+__device__ __forceinline__ float gelu(float x) { return 0.5f * x * (1.f + erff(x * 0.70710678118654752f)); }
+
 // Store 32 consecutive fp32 values of row m, starting at segment column c0.
 __device__ __forceinline__ void epi_store(const GemmEpilogue& e, int seg, int m, int c0, const float (&v)[32],
                                           int ncols_valid) {
@@ -117,8 +120,34 @@ __device__ __forceinline__ void epi_store(const GemmEpilogue& e, int seg, int m,
         return;
     }
     float w[32];
+    if (o.kind == kEpiSwish) {
 #pragma unroll
-    for (int i = 0; i < 32; i++) w[i] = (o.kind == kEpiSwish) ? swish(v[i]) : v[i] * o.scale;
+        for (int i = 0; i < 32; i++) w[i] = swish(v[i]);
+    } else if (o.kind == kEpiGelu) {
+#pragma unroll
+        for (int i = 0; i < 32; i++) w[i] = gelu(v[i]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; i++) w[i] = v[i] * o.scale;
+    }
+    if (o.kind == kEpiResidual) {
+        const __nv_bfloat16* r = o.res + (size_t)m * o.res_ld + c0;
+        if (ncols_valid >= 32) {
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                const uint4 u = reinterpret_cast<const uint4*>(r)[c];
+                const __nv_bfloat162* hp = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const float2 f = __bfloat1622float2(hp[e]);
+                    w[8 * c + 2 * e] += f.x;
+                    w[8 * c + 2 * e + 1] += f.y;
+                }
+            }
+        } else {
+            for (int i = 0; i < ncols_valid; i++) w[i] += __bfloat162float(r[i]);
+        }
+    }
     if (o.dtype == RET_F32) {
         float* dst = reinterpret_cast<float*>(o.ptr) + (size_t)m * o.ld + c0;
         if (ncols_valid >= 32) {
@@ -305,7 +334,7 @@ ret_status launch_linear(const void* X, const void* W, void* Y, int M, int N, in
     GemmSegment seg[1] = {{W, N}};
     GemmEpilogue e;
     memset(&e, 0, sizeof(e));
-    e.seg[0] = {Y, N, kEpiStore, out_dt, 1.f, 0};
+    e.seg[0] = {Y, N, kEpiStore, out_dt, 1.f, 0, nullptr, 0};
     e.seq = 1;
     e.chunk = 1;
     return launch_gemm(X, M, K, seg, 1, e, s);

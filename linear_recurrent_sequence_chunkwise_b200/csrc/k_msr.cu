@@ -131,7 +131,8 @@ ret_status launch_msr(const MsrArgs& m, cudaStream_t s) {
     GemmSegment so[1] = {{m.Wo, m.dmodel}};
     GemmEpilogue eo;
     memset(&eo, 0, sizeof(eo));
-    eo.seg[0] = {m.out, m.dmodel, kEpiStore, m.out_dt, 1.f, 0};
+    eo.seg[0] = {m.out, m.dmodel, m.residual ? kEpiResidual : kEpiStore, m.out_dt, 1.f, 0,
+                 reinterpret_cast<const __nv_bfloat16*>(m.residual), m.dmodel};
     eo.seq = m.N;
     eo.chunk = m.chunk;
     return launch_gemm(g, (int)M, HV, so, 1, eo, s);

@@ -105,9 +105,27 @@ struct MsrArgs {
     void* out;
     ret_dtype out_dt;
     void* workspace;
+    const void* residual;  // bf16 [B*N, dmodel] added to the output, or null
 };
 size_t msr_workspace_bytes(int B, int N, int dmodel, int H, int dk, int dv);
 ret_status launch_msr(const MsrArgs& m, cudaStream_t s);
 ret_status launch_linear(const void* X, const void* W, void* Y, int M, int N, int K, ret_dtype out_dt, cudaStream_t s);
+
+// One pre-norm RetNet block: Y = MSR(LN1(X)) + X, out = gelu(LN2(Y) W1) W2 + Y.
+struct BlockArgs {
+    MsrArgs msr;            // X, the MSR weights and shapes; out / residual / workspace unused
+    const void *ln1_g, *ln1_b, *ln2_g, *ln2_b;  // bf16 [dmodel] each, or null (gain 1, bias 0)
+    const void *W1, *W2;    // bf16 [dmodel, dff], [dff, dmodel]
+    int dff;
+    double ln_eps;
+    void* out;
+    ret_dtype out_dt;
+    void* workspace;
+};
+size_t block_workspace_bytes(int B, int N, int dmodel, int H, int dk, int dv, int dff);
+ret_status launch_block(const BlockArgs& a, cudaStream_t s);
+// LayerNorm of the rows of x [M, d] (bf16) into y (bf16).
+ret_status launch_layernorm(const void* x, const void* gain, const void* bias, void* y, int M, int d, double eps,
+                            cudaStream_t s);
 
 }  // namespace ret

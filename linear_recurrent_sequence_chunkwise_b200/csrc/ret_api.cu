@@ -516,16 +516,76 @@ ret_status ret_msr_forward(const void* X, const void* Wq, const void* Wk, const 
     m.k_scale = k_scale; m.eps = eps; m.xpos = xpos ? 1 : 0; m.pos_offset = pos_offset;
     m.theta_base = xpos ? theta_base : 10000.0;
     make_head_consts(gammas, H, &m.hc);
-    m.out = out; m.out_dt = out_dt; m.workspace = workspace;
+    m.out = out; m.out_dt = out_dt; m.workspace = workspace; m.residual = nullptr;
     // the retention step runs on the tensor-core kernel only
-    RetArgs a;
-    a.in_dt = RET_BF16; a.chunk = chunk; a.dk = dk; a.dv = dv; a.N = N; a.H = H; a.hc = m.hc;
+    RetArgs a{};
+    a.B = B; a.in_dt = RET_BF16; a.chunk = chunk; a.dk = dk; a.dv = dv; a.N = N; a.H = H; a.hc = m.hc;
     if (!chunkwise_ws_supported(a))
         return fail(RET_ERR_UNSUPPORTED, "%s: needs chunk 128, d_k 128 or 256, d_v a multiple of 64 and "
                     "gamma_h^128 >= 2^-60", who);
     if (!(dv == 128 || dv == 256 || dv == 512 || dv == 1024))
         return fail(RET_ERR_UNSUPPORTED, "%s: d_v must be 128, 256, 512 or 1024", who);
     return launch_msr(m, stream);
+}
+
+size_t ret_retnet_block_workspace_bytes(int B, int N, int dmodel, int H, int dk, int dv, int dff) {
+    if (B < 1 || N < 1 || dmodel < 1 || H < 1 || dk < 1 || dv < 1 || dff < 1) return 0;
+    return block_workspace_bytes(B, N, dmodel, H, dk, dv, dff);
+}
+
+ret_status ret_retnet_block_forward(const void* X, const void* ln1_gain, const void* ln1_bias, const void* Wq,
+                                    const void* Wk, const void* Wv, const void* Wg, const void* Wo,
+                                    const void* ln2_gain, const void* ln2_bias, const void* W1, const void* W2,
+                                    const double* gammas, int B, int N, int dmodel, int H, int dk, int dv, int dff,
+                                    int chunk, double k_scale, double gn_eps, double ln_eps, int xpos,
+                                    int64_t pos_offset, double theta_base, void* out, ret_dtype out_dt,
+                                    void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    t_err[0] = 0;
+    const char* who = "ret_retnet_block_forward";
+    for (const void* ptr : {X, Wq, Wk, Wv, Wg, Wo, W1, W2, (const void*)out, (const void*)workspace})
+        if (!ptr) return fail(RET_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
+    for (const void* ptr : {X, Wq, Wk, Wv, Wg, Wo, W1, W2, (const void*)out})
+        if (!aligned(ptr, 16)) return fail(RET_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+    for (const void* ptr : {ln1_gain, ln1_bias, ln2_gain, ln2_bias})
+        if (ptr && !aligned(ptr, 4)) return fail(RET_ERR_INVALID_ARG, "%s: LayerNorm parameters must be 4-byte aligned", who);
+    if (!aligned(workspace, 256)) return fail(RET_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
+    if (B < 1 || N < 1 || dmodel < 1 || H < 1 || dk < 1 || dv < 1 || dff < 1 || chunk < 1)
+        return fail(RET_ERR_INVALID_ARG, "%s: sizes must be >= 1", who);
+    if (!is_dtype(out_dt)) return fail(RET_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    ret_status st = check_gammas(gammas, H, who);
+    if (st != RET_OK) return st;
+    if (dmodel % 8 || dff % 8) return fail(RET_ERR_INVALID_ARG, "%s: d_model and d_ff must be multiples of 8", who);
+    if (!(gn_eps >= 0.0) || !(ln_eps >= 0.0) || !isfinite(k_scale))
+        return fail(RET_ERR_INVALID_ARG, "%s: bad eps or k_scale", who);
+    if (xpos && !(theta_base > 0.0 && isfinite(theta_base)))
+        return fail(RET_ERR_INVALID_ARG, "%s: theta_base must be finite and > 0", who);
+    const size_t need = block_workspace_bytes(B, N, dmodel, H, dk, dv, dff);
+    if (workspace_bytes < need)
+        return fail(RET_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed (got %zu)", who, need, workspace_bytes);
+    const size_t M = (size_t)B * N;
+    const size_t bx = M * dmodel * 2, bo = M * dmodel * (out_dt == RET_F32 ? 4 : 2);
+    if (overlaps(out, bo, X, bx) || overlaps(workspace, need, X, bx) || overlaps(workspace, need, out, bo))
+        return fail(RET_ERR_INVALID_ARG, "%s: out or workspace overlaps another buffer", who);
+    RetArgs a{};
+    a.B = B; a.in_dt = RET_BF16; a.chunk = chunk; a.dk = dk; a.dv = dv; a.N = N; a.H = H;
+    make_head_consts(gammas, H, &a.hc);
+    if (!chunkwise_ws_supported(a))
+        return fail(RET_ERR_UNSUPPORTED, "%s: needs chunk 128, d_k 128 or 256, d_v a multiple of 64 and "
+                    "gamma_h^128 >= 2^-60", who);
+    if (!(dv == 128 || dv == 256 || dv == 512 || dv == 1024))
+        return fail(RET_ERR_UNSUPPORTED, "%s: d_v must be 128, 256, 512 or 1024", who);
+    BlockArgs b;
+    memset(&b, 0, sizeof(b));
+    MsrArgs& m = b.msr;
+    m.X = X; m.Wq = Wq; m.Wk = Wk; m.Wv = Wv; m.Wg = Wg; m.Wo = Wo;
+    m.B = B; m.N = N; m.dmodel = dmodel; m.H = H; m.dk = dk; m.dv = dv; m.chunk = chunk;
+    m.k_scale = k_scale; m.eps = gn_eps; m.xpos = xpos ? 1 : 0; m.pos_offset = pos_offset;
+    m.theta_base = xpos ? theta_base : 10000.0;
+    m.hc = a.hc;
+    b.ln1_g = ln1_gain; b.ln1_b = ln1_bias; b.ln2_g = ln2_gain; b.ln2_b = ln2_bias;
+    b.W1 = W1; b.W2 = W2; b.dff = dff; b.ln_eps = ln_eps;
+    b.out = out; b.out_dt = out_dt; b.workspace = workspace;
+    return launch_block(b, stream);
 }
 
 ret_status ret_linear_bf16(const void* X, const void* W, void* Y, int M, int N, int K, ret_dtype out_dt,

@@ -1,14 +1,17 @@
 """The pins catch plausible mistakes: each test plants one mistake in a copy
 of the C oracle (on the CPU), loads it in place of the real one, runs the
-pin suite and requires at least one pin to fail."""
+pin suite and requires at least one pin to fail.  Mistakes in the numpy
+parts are planted by swapping one function for the duration of a run."""
 import inspect
 import json
 import os
 import subprocess
 
+import numpy as np
 import pytest
 
 import oracle
+from oracle import msr as omsr
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "retention_oracle.c")
@@ -96,3 +99,49 @@ def test_pins_catch_mutant(mutant, tmp_path, golden_data):
     finally:
         oracle.swap_library(prev)
     assert failed, f"no pin caught mutant {mutant}"
+
+
+# Plausible mistakes in the numpy parts of the oracle (the RetNet block),
+# planted by replacing one function of oracle.msr for the duration of a run.
+def _ln_unbiased(x, gain=None, bias=None, eps=1e-5):
+    x = np.asarray(x, np.float64)
+    y = (x - x.mean(-1, keepdims=True)) / np.sqrt(x.var(-1, ddof=1, keepdims=True) + eps)
+    return y * (1.0 if gain is None else gain) + (0.0 if bias is None else bias)
+
+
+def _gelu_tanh(x):
+    x = np.asarray(x, np.float64)
+    return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
+
+
+def _block_post_norm(x, wq, wk, wv, wg, wo, w1, w2, gammas, H, k_scale, gn_eps=1e-5, ln_eps=1e-5,
+                     ln1=(None, None), ln2=(None, None), theta_base=10000.0, return_y=False):
+    y = omsr.layer_norm(omsr.msr_forward(x, wq, wk, wv, wg, wo, gammas, H, k_scale, gn_eps, theta_base) + x,
+                        ln1[0], ln1[1], ln_eps)
+    out = omsr.layer_norm(omsr.ffn(y, w1, w2) + y, ln2[0], ln2[1], ln_eps)
+    return (out, y) if return_y else out
+
+
+def _block_residual_of_the_normed_input(x, wq, wk, wv, wg, wo, w1, w2, gammas, H, k_scale, gn_eps=1e-5,
+                                        ln_eps=1e-5, ln1=(None, None), ln2=(None, None), theta_base=10000.0,
+                                        return_y=False):
+    xn = omsr.layer_norm(x, ln1[0], ln1[1], ln_eps)
+    y = omsr.msr_forward(xn, wq, wk, wv, wg, wo, gammas, H, k_scale, gn_eps, theta_base) + xn
+    yn = omsr.layer_norm(y, ln2[0], ln2[1], ln_eps)
+    out = omsr.ffn(yn, w1, w2) + yn
+    return (out, y) if return_y else out
+
+
+PY_MUTANTS = {
+    "layer_norm_unbiased_variance": ("layer_norm", _ln_unbiased),
+    "gelu_tanh_approximation": ("gelu", _gelu_tanh),
+    "block_post_norm": ("retnet_block", _block_post_norm),
+    "block_residual_of_the_normed_input": ("retnet_block", _block_residual_of_the_normed_input),
+}
+
+
+@pytest.mark.parametrize("mutant", sorted(PY_MUTANTS))
+def test_pins_catch_numpy_mutant(mutant, golden_data, monkeypatch):
+    name, fn = PY_MUTANTS[mutant]
+    monkeypatch.setattr(omsr, name, fn)
+    assert _run_pins(golden_data), f"no pin caught mutant {mutant}"

@@ -465,3 +465,83 @@ def test_normalized_without_flags_is_the_parallel_form():
     g = [0.7, 0.95]
     np.testing.assert_allclose(oracle.retention_normalized(q, k, v, g, flags=0),
                                oracle.retention_parallel(q, k, v, g), rtol=1e-13, atol=1e-13)
+
+
+# ------------------------------------------------ RetNet block pieces
+
+def test_layer_norm_invariants():
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((3, 7, 32)) * 5.0 + 2.0
+    y = omsr.layer_norm(x, eps=1e-5)
+    np.testing.assert_allclose(y.mean(-1), 0.0, atol=1e-12)
+    np.testing.assert_allclose((y ** 2).mean(-1), x.var(-1) / (x.var(-1) + 1e-5), rtol=1e-12)
+    # invariant to a per-row shift and positive scale (eps = 0)
+    np.testing.assert_allclose(omsr.layer_norm(x * 3.5 - 7.0, eps=0.0), omsr.layer_norm(x, eps=0.0), atol=1e-12)
+    # gain and bias act per feature
+    g, b = rng.standard_normal(32), rng.standard_normal(32)
+    np.testing.assert_allclose(omsr.layer_norm(x, g, b, 1e-5), y * g + b, atol=1e-12)
+    # a row of two values +-a normalises to +-1 (eps = 0)
+    np.testing.assert_allclose(omsr.layer_norm(np.array([[5.0, -1.0]]), eps=0.0), [[1.0, -1.0]], atol=1e-15)
+
+
+def test_gelu_values():
+    """gelu(x) = x Phi(x): textbook values of the standard normal CDF,
+    Phi(1) = 0.8413447460685429, Phi(2) = 0.9772498680518208, Phi(0) = 1/2,
+    and the identity gelu(x) - gelu(-x) = x (Phi(x) + Phi(-x) = 1)."""
+    np.testing.assert_allclose(omsr.gelu(np.array([1.0, 2.0, -1.0, 0.0])),
+                               [0.8413447460685429, 2 * 0.9772498680518208, -(1 - 0.8413447460685429), 0.0],
+                               rtol=1e-14, atol=1e-16)
+    x = np.linspace(-6, 6, 101)
+    np.testing.assert_allclose(omsr.gelu(x) - omsr.gelu(-x), x, atol=1e-14)
+    from scipy.stats import norm
+    np.testing.assert_allclose(omsr.gelu(x), x * norm.cdf(x), rtol=1e-13, atol=1e-15)
+
+
+def _block_case(seed, B=1, N=5, dm=8, H=2, dk=2, dv=4, dff=16):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((B, N, dm))
+    W = dict(wq=rng.standard_normal((dm, H * dk)) * 0.3, wk=rng.standard_normal((dm, H * dk)) * 0.3,
+             wv=rng.standard_normal((dm, H * dv)) * 0.3, wg=rng.standard_normal((dm, H * dv)) * 0.3,
+             wo=rng.standard_normal((H * dv, dm)) * 0.3, w1=rng.standard_normal((dm, dff)) * 0.3,
+             w2=rng.standard_normal((dff, dm)) * 0.3)
+    return x, W
+
+
+def test_block_with_zero_branches_is_the_identity():
+    x, W = _block_case(42)
+    W["wo"][:] = 0.0
+    W["w2"][:] = 0.0
+    out = omsr.retnet_block(x, *(W[n] for n in ("wq", "wk", "wv", "wg", "wo", "w1", "w2")), gammas=[0.9, 0.5],
+                            H=2, k_scale=0.5)
+    np.testing.assert_array_equal(out, x)
+
+
+def test_block_brute_force_tiny():
+    """Every step of the block written out with loops on a tiny case (LayerNorm
+    per token, the MSR through the oracle's pinned retention, the FFN with
+    math.erf), in the pre-norm residual order of P1 section 9.2."""
+    import math
+    x, W = _block_case(43)
+    B, N, dm = x.shape
+    H, dk, dv, g = 2, 2, 4, [0.9, 0.5]
+    ln1 = (np.linspace(0.5, 1.5, dm), np.linspace(-0.2, 0.3, dm))
+    ln2 = (np.linspace(1.2, 0.8, dm), np.linspace(0.1, -0.1, dm))
+    eps = 1e-5
+
+    def ln(row, gb):
+        mu = sum(row) / len(row)
+        var = sum((r - mu) ** 2 for r in row) / len(row)
+        return [(r - mu) / math.sqrt(var + eps) * gb[0][i] + gb[1][i] for i, r in enumerate(row)]
+
+    def mm(rows, w):
+        return [[sum(r[i] * w[i][j] for i in range(len(r))) for j in range(w.shape[1])] for r in rows]
+
+    xn = np.array([[ln(list(x[0, n]), ln1) for n in range(N)]])
+    msr = omsr.msr_forward(xn, *(W[n] for n in ("wq", "wk", "wv", "wg", "wo")), gammas=g, H=H, k_scale=0.5, eps=1e-5)
+    y = msr + x
+    yn = [ln(list(y[0, n]), ln2) for n in range(N)]
+    hid = [[0.5 * v * (1 + math.erf(v / math.sqrt(2))) for v in r] for r in mm(yn, W["w1"])]
+    out = np.array(mm(hid, W["w2"])) + y[0]
+    got = omsr.retnet_block(x, *(W[n] for n in ("wq", "wk", "wv", "wg", "wo", "w1", "w2")), gammas=g, H=H,
+                            k_scale=0.5, ln1=ln1, ln2=ln2)
+    np.testing.assert_allclose(got[0], out, rtol=1e-12, atol=1e-12)
