@@ -170,6 +170,8 @@ def run_ours(args):
         stream = torch.cuda.current_stream()
         if args.only == "backward":
             res = {"backward": bench_backward(R, torch, dev, stream, w, g, args, peaks, world, dist)}
+        elif args.only == "block":
+            res = {"retnet_block": bench_block(R, torch, dev, stream, args, peaks, world, dist)}
         elif args.only == "normalized":
             res = {"normalized": bench_normalized(R, torch, dev, stream, w, g, args, peaks, world, dist)}
         else:
@@ -288,6 +290,7 @@ def run_ours(args):
         result["backward"] = bench_backward(R, torch, dev, stream, w, g, args, peaks, world, dist)
         result["normalized"] = bench_normalized(R, torch, dev, stream, w, g, args, peaks, world, dist)
         result["msr_layer"] = bench_msr(R, torch, dev, stream, args, peaks, world, dist)
+        result["retnet_block"] = bench_block(R, torch, dev, stream, args, peaks, world, dist)
         result["fp32_small"] = bench_fp32_small(R, torch, dev, stream, args, world, dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
@@ -499,6 +502,40 @@ def bench_msr(R, torch, dev, stream, args, peaks, world, dist):
                                     "k_chunkwise_ws, k_gn_gate, k_gemm (W_O)"}}
 
 
+def bench_block(R, torch, dev, stream, args, peaks, world, dist):
+    """One RetNet block on the MSR layer's shapes plus the FFN (d_ff = 2
+    d_model = 4096): LayerNorm, the MSR layer with the residual fused in
+    W_O, LayerNorm, gelu(Y W1) W2 + Y.  Tensor-bound: the MSR's FLOPs plus
+    2 x 2 M d_model d_ff for the FFN."""
+    B, N, dm, H, dk, dv, dff = 2, 4096, 2048, 8, 256, 512, 4096
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0x5EED0008)
+    x = torch.randn((B, N, dm), generator=gen, device=dev).to(torch.bfloat16)
+    w = {n: (torch.randn(shape, generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+         for n, shape in (("wq", (dm, H * dk)), ("wk", (dm, H * dk)), ("wv", (dm, H * dv)), ("wg", (dm, H * dv)),
+                          ("wo", (H * dv, dm)), ("w1", (dm, dff)), ("w2", (dff, dm)))}
+    out = torch.empty((B, N, dm), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(R.ret_retnet_block_workspace_bytes(B, N, dm, H, dk, dv, dff), dtype=torch.uint8, device=dev)
+    g = gammas(H)
+
+    def fn():
+        R.ret_retnet_block_forward(x, w["wq"], w["wk"], w["wv"], w["wg"], w["wo"], w["w1"], w["w2"], g, H=H,
+                                   chunk=128, k_scale=dk ** -0.5, xpos=True, out=out, workspace=ws, stream=stream)
+
+    ms = _timed(torch, stream, fn, max(5, min(args.steps, 20)), 3, world, dist, dev)
+    R.ret_check_device_error()
+    M = B * N
+    gemm = 2 * M * dm * (2 * H * dk + 2 * H * dv) + 2 * M * H * dv * dm + 2 * 2 * M * dm * dff
+    ret = flops_per_token_head(128, dk, dv) * B * N * H
+    tf = (gemm + ret) / (ms / 1e3) / 1e12
+    return {"workload": "retnet_block_bf16_2x4096x2048_h8_256_512_ff4096", "ms_per_step": round(ms, 4),
+            "tokens_per_s": round(world * M / (ms / 1e3), 1), "algo_flops": gemm + ret,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
+                         "kernels": "k_layernorm, the MSR layer's four, k_layernorm, k_gemm (W1, gelu), "
+                                    "k_gemm (W2, residual)"}}
+
+
 def bench_fp32_small(R, torch, dev, stream, args, world, dist):
     """The fp32 path at the exercise shape [1, 64, 8, 16], chunk 16 (CUDA cores;
     136 KB of I/O, so the figure is launch latency)."""
@@ -597,7 +634,7 @@ def main():
     ap.add_argument("--seq", type=int, default=WORKLOAD["N"],
                     help="sequence length of the chunkwise workload (smaller values make ncu captures short)")
     ap.add_argument("--no-chunkwise", action="store_true", help="skip the chunkwise forward (decode only)")
-    ap.add_argument("--only", choices=["backward", "msr", "normalized"],
+    ap.add_argument("--only", choices=["backward", "msr", "normalized", "block"],
                     help="time only the backward or only the MSR layer (for ncu launch lists of one part)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -99,6 +99,7 @@ SEED_BASE = 0x5EED0000
 # sub-streams of a workload's seed
 STREAM_Q, STREAM_K, STREAM_V = 1, 2, 3
 STREAM_X, STREAM_WQ, STREAM_WK, STREAM_WV, STREAM_WG, STREAM_WO = 4, 5, 6, 7, 8, 9
+STREAM_W1, STREAM_W2 = 10, 11     # the RetNet block's FFN
 STREAM_DECODE0 = 1000   # decode step s draws q, k, v from streams 1000 + 3s + {0, 1, 2}
 
 
@@ -184,6 +185,16 @@ def msr_weights(w: Workload, dmodel=None, H=None, dk=None, dv=None, seed=None):
         "wg": make_tensor(s, STREAM_WG, (dm, H * dv), "bf16", w.w_std),
         "wo": make_tensor(s, STREAM_WO, (H * dv, dm), "bf16", w.w_std),
     }
+
+
+def ffn_weights(w: Workload, dmodel=None, dff=None, seed=None):
+    """W1 [d_model, d_ff] and W2 [d_ff, d_model] of the RetNet block's FFN,
+    bf16, with the layer's weight scale; d_ff = 2 d_model unless given."""
+    dm = w.dmodel if dmodel is None else dmodel
+    dff = 2 * dm if dff is None else dff
+    s = w.seed if seed is None else seed
+    return {"w1": make_tensor(s, STREAM_W1, (dm, dff), "bf16", w.w_std),
+            "w2": make_tensor(s, STREAM_W2, (dff, dm), "bf16", w.w_std)}
 
 
 def msr_input(w: Workload, B=None, N=None, dmodel=None, seed=None):
