@@ -95,6 +95,15 @@ def gamma_schedule(H: int) -> np.ndarray:
     return 1.0 - np.exp2(-5.0 - np.arange(H, dtype=np.float64))
 
 
+def gamma_schedule_scaled(H: int) -> np.ndarray:
+    """The schedule of the larger models: gamma = 1 - exp(linspace(log 1/32,
+    log 1/512, H)), 1 - gamma log-spaced from 1/32 to 1/512 (RetNet paper
+    summary, multi-scale decay).  H = 1 takes the first end point."""
+    if H == 1:
+        return np.array([1.0 - 1.0 / 32])
+    return 1.0 - np.exp(np.linspace(np.log(1.0 / 32), np.log(1.0 / 512), H))
+
+
 SEED_BASE = 0x5EED0000
 # sub-streams of a workload's seed
 STREAM_Q, STREAM_K, STREAM_V = 1, 2, 3

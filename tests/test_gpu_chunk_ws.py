@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import oracle
-from retention_inputs import C3, C4, gamma_schedule, make_tensor
+from retention_inputs import C3, C4, gamma_schedule, gamma_schedule_scaled, make_tensor
 from tests.helpers import TOL_BF16, bf16_bound_check, dev, err_out, err_state, host64
 
 pytestmark = pytest.mark.gpu
@@ -182,3 +182,16 @@ def test_continuation_from_state_matches_whole_sequence(N, split, dk, dv, xpos, 
     got = np.concatenate([host64(o1), host64(o2)], axis=1)
     assert err_out(got, ref) < TOL_BF16
     assert err_state(host64(s2), S) < TOL_BF16
+
+
+def test_ws_scaled_gamma_schedule():
+    """The larger models' decay schedule (1 - gamma log-spaced from 1/32 to
+    1/512) through the same path, 16 heads."""
+    q, k, v = qkv(83, 1, 1000, 16, 256, 128, 256 ** -0.5)
+    g = gamma_schedule_scaled(16)
+    out, fs = run_ws(q, k, v, g, 128, out_dtype=torch.float32, xpos=True, want_final_state=True)
+    R.ret_check_device_error()
+    qr, kr = rotated(q, k, True)
+    ref, S = oracle.retention_recurrent(qr, kr, v.f64, g)
+    assert err_out(host64(out), ref) < TOL_BF16
+    assert err_state(host64(fs), S) < TOL_BF16

@@ -123,6 +123,18 @@ def test_gamma_schedule(golden):
     np.testing.assert_allclose(win, t["window"], rtol=2e-3)
 
 
+def test_scaled_gamma_schedule():
+    """1 - gamma runs from 1/32 to 1/512 with a constant ratio between heads
+    (log spacing): for 5 heads the ratio is (1/16)^(1/4) = 1/2 exactly."""
+    from retention_inputs import gamma_schedule_scaled
+    g = gamma_schedule_scaled(5)
+    np.testing.assert_allclose(1 - g, [1 / 32, 1 / 64, 1 / 128, 1 / 256, 1 / 512], rtol=1e-13)
+    g16 = gamma_schedule_scaled(16)
+    r = (1 - g16[1:]) / (1 - g16[:-1])
+    np.testing.assert_allclose(r, (1 / 16) ** (1 / 15), rtol=1e-12)
+    assert g16[0] == pytest.approx(1 - 1 / 32) and g16[-1] == pytest.approx(1 - 1 / 512)
+
+
 # --------------------------------------------- forms agree, special cases
 
 def rand_qkv(rng, B, N, H, dk, dv):
