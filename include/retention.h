@@ -268,6 +268,23 @@ ret_status ret_decode_step_normalized(const void* q, const void* k, const void* 
                                       ret_dtype out_dt);
 
 /*
+ * One decode step for a batch of sequences that sit at different positions
+ * (serving: "Hybrid Architectures ...", section 5.2; RetNet paper summary,
+ * inference protocol).  positions: device int64 [B], 8-byte aligned, the
+ * 0-based position of this token in sequence b (>= 0; not read back on the
+ * host).  With xpos != 0, q and k of sequence b are turned by the xPos
+ * rotation at positions[b] (section 6.8, theta_base as in ret_xpos_rotate;
+ * dk even) inside the step.  norm_flags and z as in
+ * ret_decode_step_normalized, at each sequence's own position (0: none,
+ * z may be NULL).  Otherwise as ret_decode_step.
+ */
+ret_status ret_decode_step_positions(const void* q, const void* k, const void* v,
+                                     const double* gammas, float* state, float* z, void* out,
+                                     const int64_t* positions, int xpos, double theta_base,
+                                     int norm_flags, cudaStream_t stream, int B, int H, int dk,
+                                     int dv, ret_dtype in_dt, ret_dtype out_dt);
+
+/*
  * Allocation-free variant of ret_forward_chunkwise_ws, for callers that
  * cannot allocate device memory at call time: for example a plug-in that runs
  * inside a host framework which owns all device memory and hands out no

@@ -23,6 +23,7 @@ __all__ = [
     "ret_forward_chunkwise_noalloc", "ret_chunkwise_noalloc_max_bytes",
     "ret_decode_step", "ret_msr_forward", "ret_msr_workspace_bytes",
     "ret_forward_chunkwise_normalized", "ret_normalized_workspace_bytes", "ret_decode_step_normalized",
+    "ret_decode_step_positions",
     "NORM_DECAY", "NORM_SCORE",
     "ret_linear_bf16", "ret_retnet_block_forward", "ret_retnet_block_workspace_bytes",
     "ret_forward_parallel", "ret_forward_recurrent", "ret_check_device_error", "ret_last_error_string",
@@ -75,6 +76,7 @@ def _load_library():
     L.ret_forward_chunkwise_normalized.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, i,
                                                    i, i, i64, d, vp, ctypes.c_size_t]
     L.ret_decode_step_normalized.argtypes = [vp, vp, vp, dp, vp, vp, vp, i64, i, vp, i, i, i, i, i, i]
+    L.ret_decode_step_positions.argtypes = [vp, vp, vp, dp, vp, vp, vp, vp, i, d, i, vp, i, i, i, i, i, i]
     L.ret_forward_parallel.argtypes = [vp, vp, vp, dp, i, i, i, i, i, vp, vp, i, i, i, i64, d]
     L.ret_forward_recurrent.argtypes = [vp, vp, vp, dp, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d]
     L.ret_msr_workspace_bytes.argtypes = [i, i, i, i, i, i]
@@ -392,6 +394,30 @@ def ret_decode_step_normalized(q, k, v, gammas, state, z, position: int, norm_fl
                                           _ptr(state, "state"), _ptr(z, "z"), _ptr(out, "out"), int(position),
                                           int(norm_flags), _stream(stream), B, H, dk, dv, _dt(q.dtype),
                                           _dt(out.dtype)))
+    return out
+
+
+def ret_decode_step_positions(q, k, v, gammas, state, positions, z=None, xpos: bool = True,
+                              theta_base: float = 10000.0, norm_flags: int = 0, out=None, out_dtype=None,
+                              stream=None):
+    """One decode step with each sequence at its own position: positions int64
+    [B] on the device; xPos rotation of q, k inside the step; optional score
+    normalizations with z [B, H, dk] fp32 (in place)."""
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("expected q, k [B, H, dk] and v [B, H, dv]")
+    B, H, dk = q.shape
+    dv = v.shape[2]
+    if state.shape != (B, H, dk, dv) or state.dtype != torch.float32:
+        raise ValueError("state must be float32 [B, H, dk, dv]")
+    if positions.dtype != torch.int64 or tuple(positions.shape) != (B,):
+        raise ValueError("positions must be int64 [B]")
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=out_dtype or torch.float32, device=q.device)
+    _check(lib.ret_decode_step_positions(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H),
+                                         _ptr(state, "state"), _ptr(z, "z"), _ptr(out, "out"),
+                                         _ptr(positions, "positions"), int(bool(xpos)), float(theta_base),
+                                         int(norm_flags), _stream(stream), B, H, dk, dv, _dt(q.dtype),
+                                         _dt(out.dtype)))
     return out
 
 

@@ -20,14 +20,18 @@ constexpr int kDecBatch = 16;   // row vectors in flight per thread
 __device__ __forceinline__ float4 ld_stream(const float4* p) { return __ldcs(p); }
 __device__ __forceinline__ void st_stream(float4* p, float4 x) { __stcs(p, x); }
 
-// With flags (the score normalizations 2 and 3 of section 8.5), the output
-// is multiplied by f = c / max(|c q.z|, 1), c = 1 / sqrt(sum_{i<=pos}
-// gamma^i), where z is the decayed key sum already updated for this token.
+// With xpos, q and k of sequence b are first turned by the xPos rotation at
+// its position (section 6.8).  With flags (the score normalizations 2 and 3
+// of section 8.5), the output is multiplied by f = c / max(|c q.z|, 1),
+// c = 1 / sqrt(sum_{i<=pos} gamma^i), where z is the decayed key sum already
+// updated for this token.
 template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(256) k_decode_step(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                                      const Tin* __restrict__ v, HeadConsts hc, int H, int dk,
                                                      int dv, float* __restrict__ state, Tout* __restrict__ out,
-                                                     const float* __restrict__ z, long long pos, int flags) {
+                                                     DecodeOpts o) {
+    const float* __restrict__ z = o.z;
+    const int flags = o.flags;
     extern __shared__ float smf[];
     float* qs = smf;            // [dk]
     float* ks = smf + dk;       // [dk]
@@ -40,6 +44,19 @@ __global__ void __launch_bounds__(256) k_decode_step(const Tin* __restrict__ q, 
         ks[i] = ld_as_float(k, (size_t)bh * dk + i);
     }
     const float g = (float)exp2(hc.log2g[h]);
+    const long long pos = o.positions ? o.positions[bh / H] : o.pos;
+    if (o.xpos) {
+        __syncthreads();
+        for (int p = threadIdx.x; p < dk / 2; p += blockDim.x) {
+            float sn, cs;
+            sincosf(rot_angle(pos, exp2(-2.0 * p / dk * o.log2base)), &sn, &cs);
+            const float q0 = qs[2 * p], q1 = qs[2 * p + 1], k0 = ks[2 * p], k1 = ks[2 * p + 1];
+            qs[2 * p] = q0 * cs - q1 * sn;
+            qs[2 * p + 1] = q0 * sn + q1 * cs;
+            ks[2 * p] = k0 * cs - k1 * sn;
+            ks[2 * p + 1] = k0 * sn + k1 * cs;
+        }
+    }
     __syncthreads();
     float fscale = 1.f;
     if (flags) {
@@ -118,49 +135,69 @@ __global__ void __launch_bounds__(256) k_decode_step(const Tin* __restrict__ q, 
     }
 }
 
-// z <- gamma z + k, one thread per element of z [B, H, dk].
+// z <- gamma z + k (k rotated at its sequence's position with xpos), one
+// thread per pair of elements of z [B, H, dk].
 template <typename Tin>
 __global__ void k_keysum_update(float* __restrict__ z, const Tin* __restrict__ k, HeadConsts hc, int H, int dk,
-                                long long total) {
+                                long long total_pairs, DecodeOpts o) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= total) return;
-    const int h = (int)((i / dk) % H);
-    z[i] = fmaf((float)exp2(hc.log2g[h]), z[i], ld_as_float(k, (size_t)i));
+    if (i >= total_pairs) return;
+    const int half = (dk + 1) / 2;  // an odd dk (no rotation then) leaves a last single element
+    const int p = (int)(i % half);
+    const long long bh = i / half;
+    const int h = (int)(bh % H);
+    const size_t e = (size_t)bh * dk + 2 * p;
+    const bool pair = 2 * p + 1 < dk;
+    float k0 = ld_as_float(k, e), k1 = pair ? ld_as_float(k, e + 1) : 0.f;
+    if (o.xpos) {
+        const long long pos = o.positions ? o.positions[bh / H] : o.pos;
+        float sn, cs;
+        sincosf(rot_angle(pos, exp2(-2.0 * p / dk * o.log2base)), &sn, &cs);
+        const float r0 = k0 * cs - k1 * sn, r1 = k0 * sn + k1 * cs;
+        k0 = r0;
+        k1 = r1;
+    }
+    const float g = (float)exp2(hc.log2g[h]);
+    z[e] = fmaf(g, z[e], k0);
+    if (pair) z[e + 1] = fmaf(g, z[e + 1], k1);
 }
 
 static ret_status decode_launch(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
-                                const float* z, void* out, int B, int H, int dk, int dv, ret_dtype in_dt,
-                                ret_dtype out_dt, long long pos, int flags, cudaStream_t s);
+                                void* out, int B, int H, int dk, int dv, ret_dtype in_dt, ret_dtype out_dt,
+                                const DecodeOpts& o, cudaStream_t s);
 
 ret_status launch_decode(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
                          void* out, int B, int H, int dk, int dv, ret_dtype in_dt, ret_dtype out_dt,
                          cudaStream_t s) {
-    return decode_launch(q, k, v, hc, state, nullptr, out, B, H, dk, dv, in_dt, out_dt, 0, 0, s);
+    DecodeOpts o{};
+    return decode_launch(q, k, v, hc, state, out, B, H, dk, dv, in_dt, out_dt, o, s);
 }
 
-ret_status launch_decode_normalized(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
-                                    float* z, void* out, int B, int H, int dk, int dv, ret_dtype in_dt,
-                                    ret_dtype out_dt, long long pos, int flags, cudaStream_t s) {
-    if (flags & kNormScore) {
-        const long long total = (long long)B * H * dk;
+ret_status launch_decode_ex(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
+                            void* out, int B, int H, int dk, int dv, ret_dtype in_dt, ret_dtype out_dt,
+                            const DecodeOpts& o, cudaStream_t s) {
+    if (o.flags & kNormScore) {
+        const long long total = (long long)B * H * ((dk + 1) / 2);
         const int blocks = (int)((total + 255) / 256);
-        if (in_dt == RET_F32) k_keysum_update<float><<<blocks, 256, 0, s>>>(z, (const float*)k, hc, H, dk, total);
-        else k_keysum_update<__nv_bfloat16><<<blocks, 256, 0, s>>>(z, (const __nv_bfloat16*)k, hc, H, dk, total);
-        ret_status st = check_launch("ret_decode_step_normalized: key sum");
+        if (in_dt == RET_F32)
+            k_keysum_update<float><<<blocks, 256, 0, s>>>(o.z, (const float*)k, hc, H, dk, total, o);
+        else
+            k_keysum_update<__nv_bfloat16><<<blocks, 256, 0, s>>>(o.z, (const __nv_bfloat16*)k, hc, H, dk, total, o);
+        ret_status st = check_launch("decode: key sum");
         if (st != RET_OK) return st;
     }
-    return decode_launch(q, k, v, hc, state, z, out, B, H, dk, dv, in_dt, out_dt, pos, flags, s);
+    return decode_launch(q, k, v, hc, state, out, B, H, dk, dv, in_dt, out_dt, o, s);
 }
 
 static ret_status decode_launch(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
-                                const float* z, void* out, int B, int H, int dk, int dv, ret_dtype in_dt,
-                                ret_dtype out_dt, long long pos, int flags, cudaStream_t s) {
+                                void* out, int B, int H, int dk, int dv, ret_dtype in_dt, ret_dtype out_dt,
+                                const DecodeOpts& o, cudaStream_t s) {
     dim3 grid((dv + kDecCols - 1) / kDecCols, B * H);
     const size_t smem = (size_t)((2 * dk + 3) & ~3) * sizeof(float) + kDecWarps * 32 * sizeof(float4);
     if (smem > 48 * 1024) return fail(RET_ERR_UNSUPPORTED, "ret_decode_step: dk too large");
 #define RET_LAUNCH_DEC(TI, TO)                                                                               \
     k_decode_step<TI, TO><<<grid, 256, smem, s>>>((const TI*)q, (const TI*)k, (const TI*)v, hc, H, dk, dv, \
-                                                  state, (TO*)out, z, pos, flags)
+                                                  state, (TO*)out, o)
     if (in_dt == RET_F32 && out_dt == RET_F32) RET_LAUNCH_DEC(float, float);
     else if (in_dt == RET_F32) RET_LAUNCH_DEC(float, __nv_bfloat16);
     else if (out_dt == RET_F32) RET_LAUNCH_DEC(__nv_bfloat16, float);

@@ -67,11 +67,21 @@ constexpr int kNormDecay = RET_NORM_DECAY, kNormScore = RET_NORM_SCORE;
 size_t normalized_ws_bytes(const RetArgs& a);
 ret_status launch_chunkwise_normalized(const RetArgs& a, int flags, const float* z0, float* z1, void* ws,
                                        cudaStream_t s);
-// The decode step with the same normalizations at absolute position pos;
-// z [B, H, dk] updated in place (may be null without kNormScore).
-ret_status launch_decode_normalized(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
-                                    float* z, void* out, int B, int H, int dk, int dv, ret_dtype in_dt,
-                                    ret_dtype out_dt, long long pos, int flags, cudaStream_t s);
+// Options of the decode step: the xPos rotation of q and k and the score
+// normalizations at each sequence's position (positions[b] on the device, or
+// pos for all when positions is null); z [B, H, dk] updated in place (needed
+// with kNormScore).
+struct DecodeOpts {
+    float* z;
+    const long long* positions;
+    long long pos;
+    int flags;
+    int xpos;
+    double log2base;
+};
+ret_status launch_decode_ex(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
+                            void* out, int B, int H, int dk, int dv, ret_dtype in_dt, ret_dtype out_dt,
+                            const DecodeOpts& o, cudaStream_t s);
 
 // The tensor-core kernel alone, on prepared q_rot (or q) and k' (zeta-scaled keys).
 // q_rot: [B, N, H, dk] rows q_pitch elements apart.

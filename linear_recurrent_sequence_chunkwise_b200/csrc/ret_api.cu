@@ -473,8 +473,58 @@ ret_status ret_decode_step_normalized(const void* q, const void* k, const void* 
     }
     HeadConsts hc;
     make_head_consts(gammas, H, &hc);
-    return launch_decode_normalized(q, k, v, hc, state, (norm_flags & RET_NORM_SCORE) ? z : nullptr, out, B, H, dk,
-                                    dv, in_dt, out_dt, position, norm_flags, stream);
+    DecodeOpts o{};
+    o.z = (norm_flags & RET_NORM_SCORE) ? z : nullptr;
+    o.pos = position;
+    o.flags = norm_flags;
+    return launch_decode_ex(q, k, v, hc, state, out, B, H, dk, dv, in_dt, out_dt, o, stream);
+}
+
+ret_status ret_decode_step_positions(const void* q, const void* k, const void* v, const double* gammas,
+                                     float* state, float* z, void* out, const int64_t* positions, int xpos,
+                                     double theta_base, int norm_flags, cudaStream_t stream, int B, int H, int dk,
+                                     int dv, ret_dtype in_dt, ret_dtype out_dt) {
+    t_err[0] = 0;
+    const char* who = "ret_decode_step_positions";
+    if (!q || !k || !v || !state || !out || !positions)
+        return fail(RET_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
+    if (B < 1 || H < 1 || dk < 1 || dv < 1)
+        return fail(RET_ERR_INVALID_ARG, "%s: sizes must be >= 1 (B=%d H=%d dk=%d dv=%d)", who, B, H, dk, dv);
+    if (!is_dtype(in_dt) || !is_dtype(out_dt)) return fail(RET_ERR_INVALID_ARG, "%s: unknown dtype", who);
+    if (norm_flags & ~(RET_NORM_DECAY | RET_NORM_SCORE))
+        return fail(RET_ERR_INVALID_ARG, "%s: norm_flags must combine RET_NORM_DECAY and RET_NORM_SCORE", who);
+    if ((norm_flags & RET_NORM_SCORE) && !z)
+        return fail(RET_ERR_INVALID_ARG, "%s: RET_NORM_SCORE needs the key-sum state z", who);
+    if (xpos && dk % 2) return fail(RET_ERR_INVALID_ARG, "%s: xpos needs an even dk (got %d)", who, dk);
+    if (xpos && !(theta_base > 0.0 && isfinite(theta_base)))
+        return fail(RET_ERR_INVALID_ARG, "%s: theta_base must be finite and > 0", who);
+    ret_status st = check_gammas(gammas, H, who);
+    if (st != RET_OK) return st;
+    if (dv % 4 != 0) return fail(RET_ERR_INVALID_ARG, "%s: dv must be a multiple of 4 (got %d)", who, dv);
+    if (!aligned(state, 16)) return fail(RET_ERR_INVALID_ARG, "%s: state must be 16-byte aligned", who);
+    if (!aligned(positions, 8)) return fail(RET_ERR_INVALID_ARG, "%s: positions must be 8-byte aligned", who);
+    for (const void* p : {q, k, v, (const void*)out})
+        if (!aligned(p, 4)) return fail(RET_ERR_INVALID_ARG, "%s: q, k, v, out must be 4-byte aligned", who);
+    const size_t bs = (size_t)B * H * dk * dv * 4, bo = (size_t)B * H * dv * esize(out_dt);
+    const size_t bz = (size_t)B * H * dk * 4, bq = (size_t)B * H * dk * esize(in_dt);
+    if (overlaps(out, bo, state, bs)) return fail(RET_ERR_INVALID_ARG, "%s: out overlaps state", who);
+    if (overlaps(positions, (size_t)B * 8, state, bs) || overlaps(positions, (size_t)B * 8, out, bo))
+        return fail(RET_ERR_INVALID_ARG, "%s: positions overlap another buffer", who);
+    if (z && (norm_flags & RET_NORM_SCORE)) {
+        if (!aligned(z, 16)) return fail(RET_ERR_INVALID_ARG, "%s: z must be 16-byte aligned", who);
+        if (overlaps(z, bz, state, bs) || overlaps(z, bz, out, bo) || overlaps(z, bz, q, bq) ||
+            overlaps(z, bz, k, bq) || overlaps(z, bz, positions, (size_t)B * 8))
+            return fail(RET_ERR_INVALID_ARG, "%s: z overlaps another buffer", who);
+    }
+    HeadConsts hc;
+    make_head_consts(gammas, H, &hc);
+    DecodeOpts o{};
+    o.z = (norm_flags & RET_NORM_SCORE) ? z : nullptr;
+    o.positions = reinterpret_cast<const long long*>(positions);
+    o.flags = norm_flags;
+    o.xpos = xpos ? 1 : 0;
+    o.log2base = log2(xpos ? theta_base : 10000.0);
+    return launch_decode_ex(q, k, v, hc, state, out, B, H, dk, dv, in_dt, out_dt, o, stream);
 }
 
 size_t ret_msr_workspace_bytes(int B, int N, int dmodel, int H, int dk, int dv) {

@@ -246,3 +246,19 @@ def decode_normalized_call(z=ctypes.c_void_p(0xB0000000), pos=5, flags=3, state=
 def test_decode_normalized_rejects_bad_arguments(kw, status):
     assert decode_normalized_call(**kw) == status, (kw, R.ret_last_error_string())
     assert R.ret_last_error_string()
+
+
+def decode_positions_call(pos=ctypes.c_void_p(0xD0000000), z=ctypes.c_void_p(0xB0000000), xpos=1, flags=3, dk=16,
+                          theta=1e4):
+    return R.lib.ret_decode_step_positions(P, P2, P3, G2, ctypes.c_void_p(0xC0000000), z, P4, pos, xpos, theta, flags,
+                                           S0, 1, 2, dk, 64, 1, 1)
+
+
+@needs_no_gpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(pos=None), 1), (dict(pos=ctypes.c_void_p(0xD0000004)), 1), (dict(z=None), 1), (dict(dk=15), 1),
+    (dict(theta=0.0), 1), (dict(flags=4), 1), (dict(pos=ctypes.c_void_p(0xC0000000)), 1),   # positions in the state
+])
+def test_decode_positions_rejects_bad_arguments(kw, status):
+    assert decode_positions_call(**kw) == status, (kw, R.ret_last_error_string())
+    assert R.ret_last_error_string()

@@ -172,3 +172,30 @@ def test_normalized_workload_all_heads():
     f = c / np.maximum(np.abs(c * s), 1.0)
     out = run(q, k, v, w.gammas, BOTH, xpos=True, out_dtype=torch.bfloat16)
     assert err_out(host64(out), f * plain) < TOL_BF16
+
+
+@pytest.mark.parametrize("xpos,flags", [(True, 0), (True, BOTH), (False, BOTH)])
+def test_decode_at_per_sequence_positions(xpos, flags):
+    """Three sequences at positions 0, 37 and 1000 take T decode steps in one
+    batch.  Each equals the oracle on its own sequence with that many leading
+    zero tokens (zero keys add nothing to S or z; the positions still count
+    for the rotation and the decay row sums)."""
+    pos0 = [0, 37, 1000]
+    B, T, H, dk, dv = len(pos0), 6, 2, 64, 64
+    q, k, v = qkv(316, B, T, H, dk, dv, dk ** -0.25)
+    g = gamma_schedule(H)
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    S = torch.zeros((B, H, dk, dv), dtype=torch.float32, device="cuda")
+    z = torch.zeros((B, H, dk), dtype=torch.float32, device="cuda")
+    outs = []
+    for t in range(T):
+        pos = torch.tensor([p + t for p in pos0], dtype=torch.int64, device="cuda")
+        outs.append(R.ret_decode_step_positions(qd[:, t].contiguous(), kd[:, t].contiguous(), vd[:, t].contiguous(),
+                                                g, S, pos, z=z if flags else None, xpos=xpos, norm_flags=flags))
+    torch.cuda.synchronize()
+    R.ret_check_device_error()
+    got = np.stack([host64(o) for o in outs], axis=1)    # [B, T, H, dv]
+    for b, P in enumerate(pos0):
+        pad = lambda x: np.concatenate([np.zeros((1, P) + x.shape[2:]), x[b:b + 1]], axis=1)
+        ref = oracle.retention_normalized(pad(q.f64), pad(k.f64), pad(v.f64), g, flags=flags, xpos=xpos)[:, P:]
+        assert err_out(got[b:b + 1], ref) < TOL_BF16, b
