@@ -141,6 +141,8 @@ __global__ void __launch_bounds__(256) k_prep_qk(const __nv_bfloat16* __restrict
 
 struct WsParams {
     CUtensorMap tq, tk, tv;
+    CUtensorMap to;       // bf16 out, stored by TMA from the staged tile (tma_out)
+    int tma_out;
     void* out;
     float* fstate;
     const float* istate;  // state before the first token, [B, H, DK, dv] fp32, or null (zero)
@@ -177,7 +179,7 @@ static_assert(128 * (kRegsCtl + kRegsQ) + 256 * kRegsXf <= 512 * 128, "register 
 
 struct Bars {
     uint64_t qfull, qempty, kfull[kKSlots], kempty[kKSlots], vfull[2], vempty[2];
-    uint64_t qready, qtm, afull, aread, pready, dsdone, dsfree, tready, ofull, ofree;
+    uint64_t qready, qtm, afull, aread, pready, dsdone, dsfree, tready, ofull, ofree, ostaged[2];
 };
 
 __device__ __forceinline__ void elect_arrive(uint64_t* bar, int lane) {
@@ -235,6 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         tc::mbar_init(&bars.tready, kXfWarps);
         tc::mbar_init(&bars.ofull, 1);
         tc::mbar_init(&bars.ofree, kXfWarps);
+        for (int i = 0; i < 2; i++) tc::mbar_init(&bars.ostaged[i], kXfWarps);
         s_fail = 0;
         tc::fence_barrier_init();
         tc::prefetch_tmap(&p.tq);
@@ -286,6 +289,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 if (!ok) break;
                 tc::mbar_arrive_expect_tx(&bars.vfull[vs], kVBytes);
                 tc::tma_load_4d(sm + WsSmem<DK>::kV + vs * kVBytes, &p.tv, &bars.vfull[vs], j0, h, n0, b);
+            }
+        } else if (warp == 2) {
+            // ------------------------------------------ output store (bf16)
+            // Each chunk's tile, staged by the transform warpgroups in the V
+            // slot it used, goes out in one TMA store; the slot returns to the
+            // producer once the store has read it.  One barrier per slot, so
+            // the staging of chunk jc + 2 (which needs that slot's next V)
+            // cannot complete a phase before this warp has seen chunk jc's.
+            if (p.tma_out) {
+                for (int jc = 0; jc < nchunks && ok; jc++) {
+                    const int vs = jc & 1;
+                    ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars.ostaged[vs], (jc >> 1) & 1));
+                    if (!ok) break;
+                    if (lane == 0) {
+                        tc::tma_store_4d(&p.to, sm + WsSmem<DK>::kV + vs * kVBytes, j0, h, jc * kC, b);
+                        tc::bulk_commit_group();
+                        tc::bulk_wait_group_read<0>();
+                        tc::mbar_arrive(&bars.vempty[vs]);
+                    }
+                    __syncwarp();
+                }
+                if (lane == 0) tc::bulk_wait_group<0>();  // the last tile is in global memory
             }
         } else if (warp == 1) {
             // --------------------------------------------- tensor pipe
@@ -367,7 +392,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                     tc::mma_bf16_ts_elect(tb + kTO, tb + kTP + 8 * k, dv_mn + vo + (uint32_t)((k * 2048) >> 4), id_pv,
                                           (jc > 0) || has_init || (k > 0));
                 tc::mma_commit_elect(&bars.ofull);
-                tc::mma_commit_elect(&bars.vempty[jc & 1]);
+                // with the TMA-store epilogue the output tile is staged in this
+                // V slot, which the epilogue hands back once the store has read it
+                if (!p.tma_out) tc::mma_commit_elect(&bars.vempty[jc & 1]);
             }
         }
     } else if (warp < 8) {
@@ -570,6 +597,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
                 elect_arrive(&bars.ofree, lane);
+                if constexpr (sizeof(Tout) == 2) {
+                    if (p.tma_out) {
+                        // Stage the bf16 tile in the V slot of this chunk (free since
+                        // P V completed) in the TMA's 128-byte swizzle, then one
+                        // thread stores it: rows past N are clipped by the TMA.
+                        uint8_t* sO = sm + WsSmem<DK>::kV + (jc & 1) * kVBytes;
+                        const float sc = (last ? sc_last : sc_full) * rs;
+#pragma unroll
+                        for (int c16 = 0; c16 < 4; c16++) {
+                            const int base = c16 * 8;
+                            uint4 v;
+                            v.x = tc::pack_bf16x2(__uint_as_float(o[base + 0]) * sc, __uint_as_float(o[base + 1]) * sc);
+                            v.y = tc::pack_bf16x2(__uint_as_float(o[base + 2]) * sc, __uint_as_float(o[base + 3]) * sc);
+                            v.z = tc::pack_bf16x2(__uint_as_float(o[base + 4]) * sc, __uint_as_float(o[base + 5]) * sc);
+                            v.w = tc::pack_bf16x2(__uint_as_float(o[base + 6]) * sc, __uint_as_float(o[base + 7]) * sc);
+                            *reinterpret_cast<uint4*>(sO + tc::sw128_off((uint32_t)r, (uint32_t)(4 * wg + c16))) = v;
+                        }
+                        tc::fence_proxy_async_smem();
+                        elect_arrive(&bars.ostaged[jc & 1], lane);
+                        continue;
+                    }
+                }
                 if (r < L) {
                     const float sc = (last ? sc_last : sc_full) * rs;
                     const int n = p.out_rev ? N - 1 - (n0 + r) : n0 + r;
@@ -665,6 +714,11 @@ static ret_status fill_params(WsParams* p, const RetArgs& a, const void* q_src, 
     p->accumulate = a.accumulate;
     p->out_rev = a.out_rev;
     p->rowscale = a.rowscale;
+    p->tma_out = 0;
+    if (a.out_dt == RET_BF16 && !a.accumulate && !a.out_rev) {
+        if (!make_tmap_bf16(&p->to, a.out, 4, dvv, svv, box, CU_TENSOR_MAP_SWIZZLE_128B)) return RET_ERR_CUDA;
+        p->tma_out = 1;
+    }
     return RET_OK;
 }
 
