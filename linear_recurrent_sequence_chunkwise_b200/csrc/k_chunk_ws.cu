@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(256) k_prep_qk(const __nv_bfloat16* __restrict
 
 struct WsParams {
     CUtensorMap tq, tk, tv;
-    CUtensorMap to;       // bf16 out, stored by TMA from the staged tile (tma_out)
+    CUtensorMap to;       // out, stored by TMA from the staged tile (tma_out); fp32 in two column halves
     int tma_out;
     void* out;
     float* fstate;
@@ -179,7 +179,7 @@ static_assert(128 * (kRegsCtl + kRegsQ) + 256 * kRegsXf <= 512 * 128, "register 
 
 struct Bars {
     uint64_t qfull, qempty, kfull[kKSlots], kempty[kKSlots], vfull[2], vempty[2];
-    uint64_t qready, qtm, afull, aread, pready, dsdone, dsfree, tready, ofull, ofree, ostaged[2];
+    uint64_t qready, qtm, afull, aread, pready, dsdone, dsfree, tready, ofull, ofree, ostaged[2], ostaged2[2], ohalf[2];
 };
 
 __device__ __forceinline__ void elect_arrive(uint64_t* bar, int lane) {
@@ -237,7 +237,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         tc::mbar_init(&bars.tready, kXfWarps);
         tc::mbar_init(&bars.ofull, 1);
         tc::mbar_init(&bars.ofree, kXfWarps);
-        for (int i = 0; i < 2; i++) tc::mbar_init(&bars.ostaged[i], kXfWarps);
+        for (int i = 0; i < 2; i++) {
+            // bf16: both column halves staged at once; fp32: one half per round
+            tc::mbar_init(&bars.ostaged[i], sizeof(Tout) == 2 ? kXfWarps : kXfWarps / 2);
+            tc::mbar_init(&bars.ostaged2[i], kXfWarps / 2);
+            tc::mbar_init(&bars.ohalf[i], 1);
+        }
         s_fail = 0;
         tc::fence_barrier_init();
         tc::prefetch_tmap(&p.tq);
@@ -298,17 +303,40 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             // the staging of chunk jc + 2 (which needs that slot's next V)
             // cannot complete a phase before this warp has seen chunk jc's.
             if (p.tma_out) {
+                // the store (or add, with accumulate) of one staged tile at
+                // column c0; reversed output: the tile's rows run backwards
+                // from row N - n0 - 1, staged that way round
+                auto put = [&](const uint8_t* slot, int c0, int jc) {
+                    const int row0 = p.out_rev ? N - jc * kC - kC : jc * kC;
+                    if (p.accumulate) tc::tma_reduce_add_4d(&p.to, slot, c0, h, row0, b);
+                    else tc::tma_store_4d(&p.to, slot, c0, h, row0, b);
+                    tc::bulk_commit_group();
+                    tc::bulk_wait_group_read<0>();
+                };
                 for (int jc = 0; jc < nchunks && ok; jc++) {
                     const int vs = jc & 1;
-                    ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars.ostaged[vs], (jc >> 1) & 1));
+                    const uint32_t par = (jc >> 1) & 1;
+                    // a reversed partial last chunk would start before row 0: the
+                    // transform warps store it directly
+                    const bool direct = p.out_rev && jc == nchunks - 1 && N - jc * kC < kC;
+                    uint8_t* slot = sm + WsSmem<DK>::kV + vs * kVBytes;
+                    ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars.ostaged[vs], par));
                     if (!ok) break;
                     if (lane == 0) {
-                        tc::tma_store_4d(&p.to, sm + WsSmem<DK>::kV + vs * kVBytes, j0, h, jc * kC, b);
-                        tc::bulk_commit_group();
-                        tc::bulk_wait_group_read<0>();
-                        tc::mbar_arrive(&bars.vempty[vs]);
+                        if (!direct) put(slot, j0, jc);
+                        // fp32: the second column half goes through the same slot
+                        tc::mbar_arrive(sizeof(Tout) == 2 ? &bars.vempty[vs] : &bars.ohalf[vs]);
                     }
                     __syncwarp();
+                    if constexpr (sizeof(Tout) == 4) {
+                        ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars.ostaged2[vs], par));
+                        if (!ok) break;
+                        if (lane == 0) {
+                            if (!direct) put(slot, j0 + kW / 2, jc);
+                            tc::mbar_arrive(&bars.vempty[vs]);
+                        }
+                        __syncwarp();
+                    }
                 }
                 if (lane == 0) tc::bulk_wait_group<0>();  // the last tile is in global memory
             }
@@ -618,6 +646,35 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                         elect_arrive(&bars.ostaged[jc & 1], lane);
                         continue;
                     }
+                } else {
+                    if (p.tma_out) {
+                        // fp32: column half wg of the tile, one half at a time
+                        // through the V slot (the second waits for the first
+                        // to be read by its store); reversed output stages row r
+                        // at 127 - r.  A reversed partial last chunk is stored
+                        // directly below, the store warp only told it is staged.
+                        const bool direct = p.out_rev && last && L < kC;
+                        if (!direct) {
+                            uint8_t* sO = sm + WsSmem<DK>::kV + (jc & 1) * kVBytes;
+                            const float sc = (last ? sc_last : sc_full) * rs;
+                            const uint32_t srow = p.out_rev ? (uint32_t)(kC - 1 - r) : (uint32_t)r;
+                            if (wg == 1) {
+                                ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars.ohalf[jc & 1], (jc >> 1) & 1));
+                                if (!ok) break;
+                            }
+#pragma unroll
+                            for (int c4 = 0; c4 < 8; c4++) {
+                                const float4 y = make_float4(
+                                    __uint_as_float(o[4 * c4 + 0]) * sc, __uint_as_float(o[4 * c4 + 1]) * sc,
+                                    __uint_as_float(o[4 * c4 + 2]) * sc, __uint_as_float(o[4 * c4 + 3]) * sc);
+                                *reinterpret_cast<float4*>(sO + tc::sw128_off(srow, (uint32_t)c4)) = y;
+                            }
+                            tc::fence_proxy_async_smem();
+                            elect_arrive(wg == 0 ? &bars.ostaged[jc & 1] : &bars.ostaged2[jc & 1], lane);
+                            continue;
+                        }
+                        elect_arrive(wg == 0 ? &bars.ostaged[jc & 1] : &bars.ostaged2[jc & 1], lane);
+                    }
                 }
                 if (r < L) {
                     const float sc = (last ? sc_last : sc_full) * rs;
@@ -715,8 +772,15 @@ static ret_status fill_params(WsParams* p, const RetArgs& a, const void* q_src, 
     p->out_rev = a.out_rev;
     p->rowscale = a.rowscale;
     p->tma_out = 0;
-    if (a.out_dt == RET_BF16 && !a.accumulate && !a.out_rev) {
-        if (!make_tmap_bf16(&p->to, a.out, 4, dvv, svv, box, CU_TENSOR_MAP_SWIZZLE_128B)) return RET_ERR_CUDA;
+    // bf16 out: plain stores only; fp32 out: stores or adds, rows forward or reversed
+    if (a.out_dt == RET_F32 || (!a.accumulate && !a.out_rev)) {
+        if (a.out_dt == RET_BF16) {
+            if (!make_tmap_bf16(&p->to, a.out, 4, dvv, svv, box, CU_TENSOR_MAP_SWIZZLE_128B)) return RET_ERR_CUDA;
+        } else {
+            const uint64_t sf[3] = {dv * 4, H * dv * 4, N * H * dv * 4};
+            const uint32_t bf[4] = {(uint32_t)kW / 2, 1, (uint32_t)kC, 1};
+            if (!make_tmap_f32(&p->to, a.out, 4, dvv, sf, bf, CU_TENSOR_MAP_SWIZZLE_128B)) return RET_ERR_CUDA;
+        }
         p->tma_out = 1;
     }
     return RET_OK;
