@@ -15,17 +15,20 @@
 //    each rotated key row by its zeta, and writes q_rot and k' (bf16) into the
 //    workspace.  Without rotation only k' is written and q is read in place.
 // 2. k_chunkwise_ws: one CTA per (batch, head, 64 value columns), 16 warps
-//    in four roles (registers rebalanced with setmaxnreg):
+//    in five roles (registers rebalanced with setmaxnreg):
 //      warp 0  TMA producer: L2 prefetch two chunks ahead (the CTAs of a
 //              head split the boxes), then per chunk the Q tile into a
 //              staging buffer, the K' tile in parts of 128 d_k rows through
 //              a 3-slot ring, and the V tile (2 slots);
-//      warp 1  tensor pipe (one elected lane issues), per chunk j
-//                A  = Q K'^T          (Q from TMEM, K' from smem), part by
-//                                     part, each part but the last followed
-//                                     by its dS = K'^T V (frees the K' slot)
-//                O  = Q T             (read-out of the state before chunk j)
-//                dS of the last part, then O += P V (P from TMEM);
+//      warp 1  tensor pipe, first issuer (one elected lane), per chunk j
+//                A  = Q K'^T          (Q from TMEM, K' from smem), part by part,
+//                O  = Q T             (read-out of the state before chunk j),
+//                O += P V             (P from TMEM);
+//      warp 3  tensor pipe, second issuer: the state update dS = K'^T V of
+//              each K' part, beside warp 1's stream (each K' slot is free
+//              once both issuers have read it);
+//      warp 2  output store: one TMA store (or reduce-add) of each staged
+//              output tile;
 //      warps 4-7 (Q warpgroup): the staged Q of chunk j+1 -> registers as
 //                soon as it lands, -> TMEM once the read-out of chunk j is
 //                done; a plain smem read keeps the load traffic on the TMA
@@ -35,7 +38,7 @@
 //                mask:     P = tril(A) -> packed bf16 in TMEM,
 //                state:    R = gamma^L R + dS in registers (fp32), then the
 //                          bf16 T = gamma^L' R into smem for the next read-out,
-//                epilogue: out = gamma^(r+1-L) O -> global.
+//                epilogue: out = gamma^(r+1-L) O staged in the chunk's V slot.
 //    TMEM columns: A [0,128), P [128,192), O [192,256), Q [256,384),
 //    dS [384,512).  Every hand-off between the roles has at least one block
 //    of MMAs in between, so no role waits on another in the steady state.
@@ -221,11 +224,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         tc::mbar_init(&bars.qempty, 4);
         for (int i = 0; i < kKSlots; i++) {
             tc::mbar_init(&bars.kfull[i], 1);
-            tc::mbar_init(&bars.kempty[i], 1);
+            tc::mbar_init(&bars.kempty[i], 2);  // read by both issuers
         }
         for (int i = 0; i < 2; i++) {
             tc::mbar_init(&bars.vfull[i], 1);
-            tc::mbar_init(&bars.vempty[i], 1);
+            tc::mbar_init(&bars.vempty[i], p.tma_out ? 1 : 2);
         }
         tc::mbar_init(&bars.qready, 4);
         tc::mbar_init(&bars.qtm, 1);
@@ -340,17 +343,45 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 }
                 if (lane == 0) tc::bulk_wait_group<0>();  // the last tile is in global memory
             }
+        } else if (warp == 3) {
+            // ------------------------------------ state-update issuer
+            const uint32_t id_st = tc::idesc_bf16_f32(128, kW, 1, 1);
+            const uint64_t dk_mn = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kK), kC * 128, 1024);
+            const uint64_t dv_mn = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kV), kC * 128, 1024);
+            auto wait = [&](uint64_t* bar, uint32_t parity) {
+                return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity));
+            };
+            for (int jc = 0; jc < nchunks && ok; jc++) {
+                const uint32_t vo = (uint32_t)((jc & 1) * kVBytes) >> 4;
+                ok = wait(&bars.vfull[jc & 1], (jc >> 1) & 1);
+                if (ok && jc > 0) ok = wait(&bars.dsfree, (jc - 1) & 1);
+                if (!ok) break;
+                tc::tc_fence_after();
+                for (int part = 0; part < kParts && ok; part++) {
+                    const int g = jc * kParts + part, slot = g % kKSlots, u = g / kKSlots;
+                    ok = wait(&bars.kfull[slot], u & 1);
+                    if (!ok) break;
+                    tc::tc_fence_after();
+                    const uint32_t ko = (uint32_t)(slot * kKPartBytes) >> 4;
+#pragma unroll
+                    for (int k = 0; k < kC / 16; k++)
+                        tc::mma_bf16_ss_elect(tb + kTD + part * kW, dk_mn + ko + (uint32_t)((k * 2048) >> 4),
+                                              dv_mn + vo + (uint32_t)((k * 2048) >> 4), id_st, k > 0);
+                    tc::mma_commit_elect(&bars.kempty[slot]);
+                }
+                if (!ok) break;
+                tc::mma_commit_elect(&bars.dsdone);
+                if (!p.tma_out) tc::mma_commit_elect(&bars.vempty[jc & 1]);
+            }
         } else if (warp == 1) {
             // --------------------------------------------- tensor pipe
             // The whole warp walks the loop (warp-uniform descriptors); one
             // elected lane issues each tcgen05 instruction.
             const uint32_t id_qk = tc::idesc_bf16_f32(128, 128, 0, 0);
             const uint32_t id_qt = tc::idesc_bf16_f32(128, kW, 0, 1);
-            const uint32_t id_st = tc::idesc_bf16_f32(128, kW, 1, 1);
             const uint32_t id_pv = tc::idesc_bf16_f32(128, kW, 0, 1);
             // descriptor bases; offsets are added in 16-byte units
             const uint64_t dk_k = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kK), 16, 1024);         // K' as B, K-major
-            const uint64_t dk_mn = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kK), kC * 128, 1024);  // K'^T as A, MN-major
             const uint64_t dv_mn = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kV), kC * 128, 1024);  // V as B, MN-major
             const uint64_t dt_mn = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kT), DK * 128, 1024);  // T as B, MN-major
             // a timed-out wait must leave the warp converged for elect.sync
@@ -365,21 +396,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 ok = wait(&bars.qready, jc & 1);
                 if (ok && jc > 0) ok = wait(&bars.aread, (jc - 1) & 1);
                 if (!ok) break;
-                auto ds_part = [&](int part) -> bool {  // dS rows of this d_k part = K'^T V
-                    if (part == 0) {  // V landed, previous dS read out of TMEM
-                        if (!wait(&bars.vfull[jc & 1], (jc >> 1) & 1)) return false;
-                        if (jc > 0 && !wait(&bars.dsfree, (jc - 1) & 1)) return false;
-                        tc::tc_fence_after();
-                    }
-                    const int g = jc * kParts + part, slot = g % kKSlots;
-                    const uint32_t ko = (uint32_t)(slot * kKPartBytes) >> 4;
-#pragma unroll
-                    for (int k = 0; k < kC / 16; k++)
-                        tc::mma_bf16_ss_elect(tb + kTD + part * kW, dk_mn + ko + (uint32_t)((k * 2048) >> 4),
-                                              dv_mn + vo + (uint32_t)((k * 2048) >> 4), id_st, k > 0);
-                    tc::mma_commit_elect(&bars.kempty[slot]);
-                    return true;
-                };
                 for (int part = 0; part < kParts && ok; part++) {
                     const int g = jc * kParts + part, slot = g % kKSlots, u = g / kKSlots;
                     ok = wait(&bars.kfull[slot], u & 1);
@@ -391,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                         tc::mma_bf16_ts_elect(tb + kTA, tb + kTQ + 64 * part + 8 * k,
                                               dk_k + ko + (uint32_t)(((k / 4) * (kC * 128) + (k % 4) * 32) >> 4),
                                               id_qk, (part > 0) || (k > 0));
-                    if (part + 1 < kParts) ok = ds_part(part);
+                    tc::mma_commit_elect(&bars.kempty[slot]);
                 }
                 if (!ok) break;
                 tc::mma_commit_elect(&bars.afull);
@@ -408,9 +424,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                                               id_qt, k > 0);
                 }
                 tc::mma_commit_elect(&bars.qtm);  // Q in TMEM and T in smem are read
-                ok = ds_part(kParts - 1);
-                if (!ok) break;
-                tc::mma_commit_elect(&bars.dsdone);
                 // ---- O += P V  (P from TMEM)
                 ok = wait(&bars.pready, jc & 1);
                 if (!ok) break;
