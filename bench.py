@@ -291,6 +291,7 @@ def run_ours(args):
         result["normalized"] = bench_normalized(R, torch, dev, stream, w, g, args, peaks, world, dist)
         result["msr_layer"] = bench_msr(R, torch, dev, stream, args, peaks, world, dist)
         result["retnet_block"] = bench_block(R, torch, dev, stream, args, peaks, world, dist)
+        result["c2_d64"] = bench_c2(R, torch, dev, stream, args, peaks, world, dist)
         result["fp32_small"] = bench_fp32_small(R, torch, dev, stream, args, world, dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
@@ -563,6 +564,36 @@ def bench_block(R, torch, dev, stream, args, peaks, world, dist):
                          "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
                          "kernels": "k_layernorm, the MSR layer's four, k_layernorm, k_gemm (W1, gelu), "
                                     "k_gemm (W2, residual)"}}
+
+
+def bench_c2(R, torch, dev, stream, args, peaks, world, dist):
+    """The pages' cost-analysis shape [4, 2048, 8 heads of 64], bf16, xPos,
+    chunk 64: the workspace path (d_k padded to 128 on the tensor cores)
+    beside the single-call path (CUDA cores, fp32 arithmetic)."""
+    B, N, H, dk, dv, C = 4, 2048, 8, 64, 64, 64
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0x5EED0009)
+    q = (torch.randn((B, N, H, dk), generator=gen, device=dev) * dk ** -0.5).to(torch.bfloat16)
+    k = (torch.randn((B, N, H, dk), generator=gen, device=dev) * dk ** -0.5).to(torch.bfloat16)
+    v = torch.randn((B, N, H, dv), generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty((B, N, H, dv), dtype=torch.bfloat16, device=dev)
+    g = gammas(H)
+    ws = torch.empty(R.ret_chunkwise_workspace_bytes(B, N, H, dk, dv, C, torch.bfloat16, True), dtype=torch.uint8,
+                     device=dev)
+
+    def tc():
+        R.ret_forward_chunkwise_ws(q, k, v, g, C, ws, out=out, xpos=True, stream=stream)
+
+    def cc():
+        R.ret_forward_chunkwise(q, k, v, g, C, out=out, xpos=True, stream=stream)
+
+    steps = max(5, min(args.steps, 20))
+    ms_tc = _timed(torch, stream, tc, steps, 3, world, dist, dev)
+    ms_cc = _timed(torch, stream, cc, steps, 3, world, dist, dev)
+    R.ret_check_device_error()
+    return {"workload": "retention_bf16_4x2048x8x64", "tokens_per_s": round(world * B * N / (ms_tc / 1e3), 1),
+            "ms_per_step": round(ms_tc, 4), "single_call_cuda_cores_ms": round(ms_cc, 4),
+            "path": "ret_forward_chunkwise_ws: k_prep_qk + k_chunkwise_ws<128>, d_k padded to 128, 128-token blocks"}
 
 
 def bench_fp32_small(R, torch, dev, stream, args, world, dist):

@@ -116,6 +116,10 @@ ret_status ret_forward_chunkwise(const void* q, const void* k, const void* v,
  * undefined after the call.  When the problem does not take this path
  * (ret_chunkwise_workspace_bytes returns 0, or some gamma_h^chunk < 2^-60)
  * the call behaves as ret_forward_chunkwise and does not touch the workspace.
+ * The path takes bf16 inputs with chunk 128, dk 128 or 256 and dv a multiple
+ * of 64; dk = 64 with chunk 64 or 128 also runs on it, zero-padded to dk 128
+ * in the workspace and blocked by 128 tokens (the result is the
+ * recurrence's for any block length; states keep 64 rows).
  */
 size_t ret_chunkwise_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk, ret_dtype in_dt,
                                      int xpos);

@@ -73,16 +73,19 @@ constexpr int kThreads = 512;   // control warpgroup (TMA, MMA), Q warpgroup, tw
 // ------------------------------------------------------------------ prep
 
 // One warp per (batch, token); lanes walk groups of 8 d_k elements (4 pairs).
+// Rows have dkr elements in memory (dkr <= DK); groups past dkr are written
+// as zeros (a smaller d_k padded to the kernel's).  With qcopy the queries
+// are written to q_rot, turned only with xpos.
 template <int DK>
 __global__ void __launch_bounds__(256) k_prep_qk(const __nv_bfloat16* __restrict__ q,
                                                   const __nv_bfloat16* __restrict__ k,
                                                   __nv_bfloat16* __restrict__ q_rot,
                                                   __nv_bfloat16* __restrict__ k_out, HeadConsts hc, int B, int N,
                                                   int H, int chunk, int xpos, long long pos0, double log2base,
-                                                  int q_ld, int k_ld) {
-    // theta_p = base^(-2p/DK), once per block (fp64, as the rotation's reference)
+                                                  int q_ld, int k_ld, int dkr, int qcopy) {
+    // theta_p = base^(-2p/dkr), once per block (fp64, as the rotation's reference)
     __shared__ double s_theta[DK / 2];
-    for (int i = threadIdx.x; i < DK / 2; i += blockDim.x) s_theta[i] = exp2(-2.0 * i / DK * log2base);
+    for (int i = threadIdx.x; i < DK / 2; i += blockDim.x) s_theta[i] = exp2(-2.0 * i / dkr * log2base);
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const long long t = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);  // b * N + n
@@ -92,6 +95,14 @@ __global__ void __launch_bounds__(256) k_prep_qk(const __nv_bfloat16* __restrict
     const int L = min(chunk, N - (n - r));
     constexpr int kGroups = DK / 8;
     for (int g = lane; g < kGroups; g += 32) {
+        if (8 * g >= dkr) {  // padding
+            for (int hh = 0; hh < H; hh++) {
+                const size_t e = ((size_t)t * H + hh) * DK + 8 * g;
+                *reinterpret_cast<uint4*>(k_out + e) = make_uint4(0, 0, 0, 0);
+                if (qcopy) *reinterpret_cast<uint4*>(q_rot + e) = make_uint4(0, 0, 0, 0);
+            }
+            continue;
+        }
         float cs[4], sn[4];
 #pragma unroll
         for (int i = 0; i < 4; i++) {
@@ -109,7 +120,7 @@ __global__ void __launch_bounds__(256) k_prep_qk(const __nv_bfloat16* __restrict
                 if (h0 + hh < H) {
                     const size_t row = (size_t)t * H + h0 + hh;
                     kw[hh] = __ldg(reinterpret_cast<const uint4*>(k + row * k_ld + 8 * g));
-                    if (xpos) qw[hh] = __ldg(reinterpret_cast<const uint4*>(q + row * q_ld + 8 * g));
+                    if (qcopy) qw[hh] = __ldg(reinterpret_cast<const uint4*>(q + row * q_ld + 8 * g));
                 }
             }
 #pragma unroll
@@ -126,7 +137,7 @@ __global__ void __launch_bounds__(256) k_prep_qk(const __nv_bfloat16* __restrict
                     kwv[i] = tc::pack_bf16x2(x0 * c - x1 * s, x0 * s + x1 * c);
                 }
                 *reinterpret_cast<uint4*>(k_out + e) = kw[hh];
-                if (xpos) {
+                if (qcopy) {
                     uint32_t* qwv = reinterpret_cast<uint32_t*>(&qw[hh]);
 #pragma unroll
                     for (int i = 0; i < 4; i++) {
@@ -152,6 +163,7 @@ struct WsParams {
     int N, H, dv;
     int accumulate;       // fp32 out only: out += result
     int out_rev;          // output of token n goes to row N-1-n
+    int dks;              // rows of the states (d_k before padding)
     const float* rowscale;  // [B, N, H] factor of each output row, or null
     int nmain;            // CTAs: B * H * (dv / 64), one per (b, h, 64 value columns)
     HeadConsts hc;
@@ -518,11 +530,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
 #pragma unroll
             for (int part = 0; part < kParts; part++) {
                 const int dr = part * kPartDk + r;
-                const float4* src = reinterpret_cast<const float4*>(p.istate + (((size_t)b * p.H + h) * DK + dr) * p.dv +
+                const float4* src = reinterpret_cast<const float4*>(p.istate + (((size_t)b * p.H + h) * p.dks + dr) * p.dv +
                                                                     j0 + 32 * wg);
 #pragma unroll
                 for (int c4 = 0; c4 < 8; c4++) {
-                    const float4 x = __ldg(src + c4);
+                    // rows past the caller's d_k (padding) start at zero
+                    const float4 x = dr < p.dks ? __ldg(src + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
                     R[part][4 * c4 + 0] = x.x;
                     R[part][4 * c4 + 1] = x.y;
                     R[part][4 * c4 + 2] = x.z;
@@ -619,7 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
 #pragma unroll
                     for (int part = 0; part < kParts; part++) {
                         const int dr = part * kPartDk + r;
-                        float4* dst = reinterpret_cast<float4*>(p.fstate + (((size_t)b * p.H + h) * DK + dr) * p.dv +
+                        if (dr >= p.dks) continue;  // padding rows are not part of the state
+                        float4* dst = reinterpret_cast<float4*>(p.fstate + (((size_t)b * p.H + h) * p.dks + dr) * p.dv +
                                                                 j0 + 32 * wg);
 #pragma unroll
                         for (int c4 = 0; c4 < 8; c4++)
@@ -743,10 +757,14 @@ ret_status launch_main(const WsParams& p, cudaStream_t s) {
 
 }  // namespace
 
-// Workspace layout: k' [B, N, H, dk] bf16, then q_rot (rotation only).
+// The workspace holds a copy of q (q_rot) when the queries are rotated or
+// padded to the kernel's d_k.
+static bool q_copied(const RetArgs& a) { return a.xpos || (a.dk_real && a.dk_real != a.dk); }
+
+// Workspace layout: k' [B, N, H, dk] bf16, then q_rot (rotated or padded q).
 size_t chunkwise_ws_bytes(const RetArgs& a) {
     const size_t qk = (size_t)a.B * a.N * a.H * a.dk * 2;
-    return a.xpos ? 2 * qk : qk;
+    return q_copied(a) ? 2 * qk : qk;
 }
 
 bool chunkwise_ws_supported(const RetArgs& a) {
@@ -783,6 +801,7 @@ static ret_status fill_params(WsParams* p, const RetArgs& a, const void* q_src, 
     p->nmain = a.B * a.H * (a.dv / kW);
     p->accumulate = a.accumulate;
     p->out_rev = a.out_rev;
+    p->dks = a.dk_real ? a.dk_real : a.dk;
     p->rowscale = a.rowscale;
     p->tma_out = 0;
     // bf16 out: plain stores only; fp32 out: stores or adds, rows forward or reversed
@@ -809,11 +828,11 @@ ret_status launch_chunkwise_main(const RetArgs& a, const void* q_src, int q_pitc
     return f32 ? launch_main<128, float>(p, s) : launch_main<128, __nv_bfloat16>(p, s);
 }
 
-// Pointers into the workspace: k' first, then q_rot (rotation only).
+// Pointers into the workspace: k' first, then q_rot (rotated or padded q).
 static void ws_parts(const RetArgs& a, void* ws, __nv_bfloat16** k_out, __nv_bfloat16** q_rot) {
     const size_t qk = (size_t)a.B * a.N * a.H * a.dk;
     *k_out = reinterpret_cast<__nv_bfloat16*>(ws);
-    *q_rot = a.xpos ? *k_out + qk : nullptr;
+    *q_rot = q_copied(a) ? *k_out + qk : nullptr;
 }
 
 ret_status launch_chunkwise_prep(const RetArgs& a, void* ws, cudaStream_t s) {
@@ -821,14 +840,16 @@ ret_status launch_chunkwise_prep(const RetArgs& a, void* ws, cudaStream_t s) {
     ws_parts(a, ws, &k_out, &q_rot);
     const int blocks = (int)(((long long)a.B * a.N + 7) / 8);
     const double lb = log2(a.theta_base);
+    const int dkr = a.dk_real ? a.dk_real : a.dk, qcopy = q_copied(a) ? 1 : 0;
+    const int qld = a.q_ld ? a.q_ld : dkr, kld = a.k_ld ? a.k_ld : dkr;
     if (a.dk == 256)
         k_prep_qk<256><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, q_rot, k_out,
-                                               a.hc, a.B, a.N, a.H, a.chunk, a.xpos, a.pos_offset, lb,
-                                               a.q_ld ? a.q_ld : a.dk, a.k_ld ? a.k_ld : a.dk);
+                                               a.hc, a.B, a.N, a.H, a.chunk, a.xpos, a.pos_offset, lb, qld, kld, dkr,
+                                               qcopy);
     else
         k_prep_qk<128><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, q_rot, k_out,
-                                               a.hc, a.B, a.N, a.H, a.chunk, a.xpos, a.pos_offset, lb,
-                                               a.q_ld ? a.q_ld : a.dk, a.k_ld ? a.k_ld : a.dk);
+                                               a.hc, a.B, a.N, a.H, a.chunk, a.xpos, a.pos_offset, lb, qld, kld, dkr,
+                                               qcopy);
     return check_launch("chunkwise (workspace path): prep");
 }
 
@@ -836,7 +857,8 @@ ret_status launch_chunkwise_prepared(const RetArgs& a, void* ws, cudaStream_t s)
     __nv_bfloat16 *k_out, *q_rot;
     ws_parts(a, ws, &k_out, &q_rot);
     // q_rot in the workspace is contiguous; a raw q keeps its row pitch
-    return launch_chunkwise_main(a, a.xpos ? (const void*)q_rot : a.q, a.xpos || !a.q_ld ? a.dk : a.q_ld, k_out, s);
+    const bool qc = q_copied(a);
+    return launch_chunkwise_main(a, qc ? (const void*)q_rot : a.q, qc || !a.q_ld ? a.dk : a.q_ld, k_out, s);
 }
 
 ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s) {

@@ -24,6 +24,10 @@ struct RetArgs {
     // Workspace path only: fp32 [B, N, H] factors the output row of each
     // (token, head) is multiplied by (the score normalizations), or null.
     const float* rowscale;
+    // Workspace path only: the caller's d_k when it is below the tensor-core
+    // kernel's (0: dk).  The rows are then zero-padded to dk in the
+    // workspace, the rotation uses dk_real, and the states have dk_real rows.
+    int dk_real;
     int B, N, H, dk, dv, chunk;
     ret_dtype in_dt, out_dt;
     int xpos;

@@ -83,7 +83,7 @@ static ret_status make_args(RetArgs* a, const char* who, const void* q, const vo
             return fail(RET_ERR_INVALID_ARG, "%s: final_state overlaps another buffer", who);
     }
     a->q = q; a->k = k; a->v = v; a->out = out; a->final_state = final_state; a->initial_state = nullptr;
-    a->q_ld = 0; a->k_ld = 0; a->accumulate = 0; a->out_rev = 0; a->rowscale = nullptr;
+    a->q_ld = 0; a->k_ld = 0; a->accumulate = 0; a->out_rev = 0; a->rowscale = nullptr; a->dk_real = 0;
     a->B = B; a->N = N; a->H = H; a->dk = dk; a->dv = dv; a->chunk = chunk;
     a->in_dt = in_dt; a->out_dt = out_dt;
     a->xpos = xpos ? 1 : 0; a->pos_offset = pos_offset; a->theta_base = xpos ? theta_base : 10000.0;
@@ -130,11 +130,28 @@ ret_status ret_forward_chunkwise(const void* q, const void* k, const void* v, co
     return launch_recurrent_simt(a, stream);
 }
 
+// The workspace path's kernel takes d_k = 128 or 256.  A d_k of 64 runs on it
+// zero-padded to 128: the padded components add nothing to q . k and leave
+// the padded state rows at zero.  Its kernel blocks the sequence by 128
+// tokens, so a chunk of 64 is computed in blocks of 128 (the chunkwise form
+// gives the recurrence's result for any block length).
+static void pad_small_dk(RetArgs* a) {
+    if (a->in_dt == RET_BF16 && a->dk == 64 && (a->chunk == 64 || a->chunk == 128)) {
+        a->dk_real = 64;
+        a->dk = 128;
+        a->chunk = 128;
+    }
+}
+
+// The caller's d_k (before padding).
+static int dk_of(const RetArgs& a) { return a.dk_real ? a.dk_real : a.dk; }
+
 size_t ret_chunkwise_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk, ret_dtype in_dt, int xpos) {
     if (B < 1 || N < 1 || H < 1 || H > kMaxHeads || dk < 1 || dv < 1 || chunk < 1) return 0;
     RetArgs a{};
     a.B = B; a.N = N; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.in_dt = in_dt; a.xpos = xpos ? 1 : 0;
     for (int h = 0; h < kMaxHeads; h++) a.hc.log2g[h] = 0.0;  // shape check only
+    pad_small_dk(&a);
     return chunkwise_ws_supported(a) ? chunkwise_ws_bytes(a) : 0;
 }
 
@@ -147,6 +164,7 @@ ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
     ret_status st = make_args(&a, "ret_forward_chunkwise_ws", q, k, v, gammas, B, N, H, dk, dv, chunk, out,
                               final_state, in_dt, out_dt, xpos, pos_offset, theta_base);
     if (st != RET_OK) return st;
+    pad_small_dk(&a);
     if (!chunkwise_ws_supported(a)) return ret_forward_chunkwise(q, k, v, gammas, B, N, H, dk, dv, chunk, out,
                                                                  final_state, stream, in_dt, out_dt, xpos,
                                                                  pos_offset, theta_base);
@@ -174,8 +192,8 @@ static ret_status check_workspace(const RetArgs& a, const char* who, const void*
                     workspace ? workspace_bytes : (size_t)0);
     if (!aligned(workspace, 256)) return fail(RET_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", who);
     const size_t ntok = (size_t)a.B * a.N * a.H;
-    const size_t bq = ntok * a.dk * 2, bv = ntok * a.dv * 2, bo = ntok * a.dv * (a.out_dt == RET_F32 ? 4 : 2);
-    const size_t bs = (size_t)a.B * a.H * a.dk * a.dv * 4;
+    const size_t bq = ntok * dk_of(a) * 2, bv = ntok * a.dv * 2, bo = ntok * a.dv * (a.out_dt == RET_F32 ? 4 : 2);
+    const size_t bs = (size_t)a.B * a.H * dk_of(a) * a.dv * 4;
     bool bad = overlaps(workspace, need, a.q, bq) || overlaps(workspace, need, a.k, bq);
     if (with_outputs)
         bad = bad || overlaps(workspace, need, a.v, bv) || overlaps(workspace, need, a.out, bo) ||
@@ -189,8 +207,8 @@ static ret_status check_workspace(const RetArgs& a, const char* who, const void*
 // may be the same buffer.  Sets a->initial_state.
 static ret_status check_initial_state(RetArgs* a, const char* who, const float* initial_state) {
     if (!initial_state) return RET_OK;
-    const size_t ntok = (size_t)a->B * a->N * a->H, bs = (size_t)a->B * a->H * a->dk * a->dv * 4;
-    const size_t bq = ntok * a->dk * 2, bv = ntok * a->dv * 2, bo = ntok * a->dv * (a->out_dt == RET_F32 ? 4 : 2);
+    const size_t ntok = (size_t)a->B * a->N * a->H, bs = (size_t)a->B * a->H * dk_of(*a) * a->dv * 4;
+    const size_t bq = ntok * dk_of(*a) * 2, bv = ntok * a->dv * 2, bo = ntok * a->dv * (a->out_dt == RET_F32 ? 4 : 2);
     if (!aligned(initial_state, 16)) return fail(RET_ERR_INVALID_ARG, "%s: initial_state must be 16-byte aligned", who);
     if (overlaps(initial_state, bs, a->out, bo) || overlaps(initial_state, bs, a->q, bq) ||
         overlaps(initial_state, bs, a->k, bq) || overlaps(initial_state, bs, a->v, bv) ||
@@ -224,6 +242,7 @@ ret_status ret_chunkwise_prepare(const void* q, const void* k, const double* gam
     a.in_dt = in_dt; a.out_dt = RET_BF16;
     a.xpos = xpos ? 1 : 0; a.pos_offset = pos_offset; a.theta_base = xpos ? theta_base : 10000.0;
     make_head_consts(gammas, H, &a.hc);
+    pad_small_dk(&a);
     if (!chunkwise_ws_supported(a))
         return fail(RET_ERR_UNSUPPORTED, "%s: shape outside the workspace path (ret_chunkwise_workspace_bytes is 0)",
                     who);
@@ -243,6 +262,7 @@ ret_status ret_forward_chunkwise_prepared(const void* q, const void* k, const vo
     ret_status st = make_args(&a, who, q, k, v, gammas, B, N, H, dk, dv, chunk, out, final_state, in_dt, out_dt,
                               xpos, pos_offset, theta_base);
     if (st != RET_OK) return st;
+    pad_small_dk(&a);
     if (!chunkwise_ws_supported(a))
         return fail(RET_ERR_UNSUPPORTED, "%s: shape outside the workspace path (ret_chunkwise_workspace_bytes is 0)",
                     who);
@@ -388,6 +408,7 @@ ret_status ret_forward_chunkwise_noalloc(const void* q, const void* k, const voi
     ret_status st = make_args(&a, "ret_forward_chunkwise_noalloc", q, k, v, gammas, B, N, H, dk, dv, chunk, out,
                               final_state, in_dt, out_dt, xpos, pos_offset, theta_base);
     if (st != RET_OK) return st;
+    pad_small_dk(&a);
     if (!chunkwise_ws_supported(a))
         return fail(RET_ERR_UNSUPPORTED,
                     "ret_forward_chunkwise_noalloc: needs bf16 inputs, chunk 128, dk 128 or 256, dv a multiple of "

@@ -195,3 +195,49 @@ def test_ws_scaled_gamma_schedule():
     ref, S = oracle.retention_recurrent(qr, kr, v.f64, g)
     assert err_out(host64(out), ref) < TOL_BF16
     assert err_state(host64(fs), S) < TOL_BF16
+
+
+@pytest.mark.parametrize("B,N,H,dv,chunk,xpos,off", [
+    (4, 2048, 8, 64, 64, True, 0),       # the pages' cost-analysis shape (d_model 512, 8 heads of 64)
+    (1, 300, 2, 128, 64, False, 0),      # ragged, no rotation
+    (2, 513, 3, 64, 128, True, 77),      # chunk 128, a position offset
+])
+def test_ws_d64_padded(B, N, H, dv, chunk, xpos, off):
+    """d_k = 64 on the tensor-core path, zero-padded to 128 (rotation at the
+    caller's d_k; states with 64 rows)."""
+    dk = 64
+    q, k, v = qkv(84 + N, B, N, H, dk, dv, dk ** -0.5)
+    g = gamma_schedule(H)
+    assert R.ret_chunkwise_workspace_bytes(B, N, H, dk, dv, chunk, torch.bfloat16, xpos) > 0
+    out, fs = run_ws(q, k, v, g, chunk, out_dtype=torch.float32, xpos=xpos, pos_offset=off, want_final_state=True)
+    R.ret_check_device_error()
+    assert fs.shape == (B, H, dk, dv)
+    qr, kr = rotated(q, k, xpos, off)
+    ref, S = oracle.retention_recurrent(qr, kr, v.f64, g)
+    assert err_out(host64(out), ref) < TOL_BF16
+    assert err_state(host64(fs), S) < TOL_BF16
+
+
+def test_ws_d64_continuation():
+    """Two calls of the prepared path at d_k = 64 handing the 64-row state on."""
+    B, N, H, dk, dv, split = 1, 400, 2, 64, 128, 200
+    q, k, v = qkv(85, B, N, H, dk, dv, dk ** -0.5)
+    g = gamma_schedule(H)
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    S = torch.empty((B, H, dk, dv), dtype=torch.float32, device="cuda")
+    outs = []
+    for lo, hi, init in ((0, split, None), (split, N, S)):
+        n = hi - lo
+        nb = R.ret_chunkwise_workspace_bytes(B, n, H, dk, dv, 64, torch.bfloat16, True)
+        ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+        qs, ks, vs = (t[:, lo:hi].contiguous() for t in (qd, kd, vd))
+        R.ret_chunkwise_prepare(qs, ks, g, 64, ws, dv, xpos=True, pos_offset=lo)
+        o, _ = R.ret_forward_chunkwise_prepared(qs, ks, vs, g, 64, ws, out_dtype=torch.float32, xpos=True,
+                                                pos_offset=lo, initial_state=init, final_state=S)
+        outs.append(host64(o))
+    torch.cuda.synchronize()
+    R.ret_check_device_error()
+    qr, kr = rotated(q, k, True)
+    ref, Sref = oracle.retention_recurrent(qr, kr, v.f64, g)
+    assert err_out(np.concatenate(outs, axis=1), ref) < TOL_BF16
+    assert err_state(host64(S), Sref) < TOL_BF16
