@@ -427,6 +427,16 @@ ret_status ret_linear_bf16(const void* X, const void* W, void* Y, int M, int N, 
                            cudaStream_t stream);
 
 /*
+ * Diagnostics: one device thread waits on a barrier that nothing arrives on,
+ * with the same bounded wait as the tensor-core kernels, for `polls` polls
+ * (1 .. 2^24), gives up and sets the device error word.  The following
+ * ret_check_device_error on the stream returns RET_ERR_TIMEOUT (and clears
+ * the word); the context stays usable.  It exercises the timeout path
+ * without hanging or faulting the GPU.
+ */
+ret_status ret_selftest_bounded_wait(uint32_t polls, cudaStream_t stream);
+
+/*
  * Synchronises `stream`, then reports (and clears) the device-side error word
  * that kernels set when a bounded wait gives up.  RET_OK if none was set.
  */

@@ -23,7 +23,7 @@ __all__ = [
     "ret_forward_chunkwise_noalloc", "ret_chunkwise_noalloc_max_bytes",
     "ret_decode_step", "ret_msr_forward", "ret_msr_workspace_bytes",
     "ret_forward_chunkwise_normalized", "ret_normalized_workspace_bytes", "ret_decode_step_normalized",
-    "ret_decode_step_positions",
+    "ret_decode_step_positions", "ret_selftest_bounded_wait",
     "NORM_DECAY", "NORM_SCORE",
     "ret_linear_bf16", "ret_retnet_block_forward", "ret_retnet_block_workspace_bytes",
     "ret_forward_parallel", "ret_forward_recurrent", "ret_check_device_error", "ret_last_error_string",
@@ -76,6 +76,7 @@ def _load_library():
     L.ret_forward_chunkwise_normalized.argtypes = [vp, vp, vp, dp, i, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, i,
                                                    i, i, i64, d, vp, ctypes.c_size_t]
     L.ret_decode_step_normalized.argtypes = [vp, vp, vp, dp, vp, vp, vp, i64, i, vp, i, i, i, i, i, i]
+    L.ret_selftest_bounded_wait.argtypes = [ctypes.c_uint32, vp]
     L.ret_decode_step_positions.argtypes = [vp, vp, vp, dp, vp, vp, vp, vp, i, d, i, vp, i, i, i, i, i, i]
     L.ret_forward_parallel.argtypes = [vp, vp, vp, dp, i, i, i, i, i, vp, vp, i, i, i, i64, d]
     L.ret_forward_recurrent.argtypes = [vp, vp, vp, dp, i, i, i, i, i, vp, vp, vp, i, i, i, i64, d]
@@ -419,6 +420,12 @@ def ret_decode_step_positions(q, k, v, gammas, state, positions, z=None, xpos: b
                                          int(norm_flags), _stream(stream), B, H, dk, dv, _dt(q.dtype),
                                          _dt(out.dtype)))
     return out
+
+
+def ret_selftest_bounded_wait(polls: int = 1 << 12, stream=None):
+    """Run the bounded-wait self-test: the next ret_check_device_error raises
+    with RET_ERR_TIMEOUT."""
+    _check(lib.ret_selftest_bounded_wait(int(polls), _stream(stream)))
 
 
 def ret_check_device_error(stream=None):

@@ -757,6 +757,21 @@ ret_status launch_main(const WsParams& p, cudaStream_t s) {
 
 }  // namespace
 
+// Self-test of the bounded wait: one thread waits on an mbarrier that
+// nothing arrives on, with the wait the kernels use, gives up after `polls`
+// polls and records the timeout in the device error word as they do.
+__global__ void k_wait_selftest(uint32_t polls) {
+    __shared__ uint64_t bar;
+    tc::mbar_init(&bar, 1);
+    tc::fence_barrier_init();
+    if (!tc::mbar_wait(&bar, 0, polls)) atomicExch(&g_err_chunk_ws, kErrTimeout);
+}
+
+ret_status launch_wait_selftest(uint32_t polls, cudaStream_t s) {
+    k_wait_selftest<<<1, 1, 0, s>>>(polls);
+    return check_launch("bounded-wait self-test");
+}
+
 // The workspace holds a copy of q (q_rot) when the queries are rotated or
 // padded to the kernel's d_k.
 static bool q_copied(const RetArgs& a) { return a.xpos || (a.dk_real && a.dk_real != a.dk); }

@@ -87,6 +87,10 @@ ret_status launch_decode_ex(const void* q, const void* k, const void* v, const H
                             void* out, int B, int H, int dk, int dv, ret_dtype in_dt, ret_dtype out_dt,
                             const DecodeOpts& o, cudaStream_t s);
 
+// One thread waits on a barrier nothing arrives on (bounded), then sets the
+// device error word: the timeout path without a hang or a fault.
+ret_status launch_wait_selftest(uint32_t polls, cudaStream_t s);
+
 // The tensor-core kernel alone, on prepared q_rot (or q) and k' (zeta-scaled keys).
 // q_rot: [B, N, H, dk] rows q_pitch elements apart.
 ret_status launch_chunkwise_main(const RetArgs& a, const void* q_rot, int q_pitch, const void* k_prime,

@@ -675,6 +675,13 @@ ret_status ret_linear_bf16(const void* X, const void* W, void* Y, int M, int N, 
     return launch_linear(X, W, Y, M, N, K, out_dt, stream);
 }
 
+ret_status ret_selftest_bounded_wait(uint32_t polls, cudaStream_t stream) {
+    t_err[0] = 0;
+    if (polls < 1 || polls > (1u << 24))
+        return fail(RET_ERR_INVALID_ARG, "ret_selftest_bounded_wait: polls must be in [1, 2^24]");
+    return launch_wait_selftest(polls, stream);
+}
+
 ret_status ret_check_device_error(cudaStream_t stream) {
     t_err[0] = 0;
     cudaError_t e = cudaStreamSynchronize(stream);
