@@ -39,6 +39,9 @@ struct GemmEpilogue {
     int xpos;               // rotations: 0 leaves the pairs unrotated
     long long pos_offset;
     double log2base;        // log2(theta_base)
+    // Rotations: (cos, sin) of every (token, pair) at position pos_offset +
+    // token, [seq][head_dim / 2] fp32, or null (computed in the epilogue).
+    const float2* rot_cs;
     double log2g[kMaxHeads];
 };
 

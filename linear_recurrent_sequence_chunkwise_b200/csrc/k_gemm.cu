@@ -42,7 +42,10 @@ constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kThreads = 320;          // TMA warp, MMA warp, two epilogue warpgroups
 constexpr int kSmemBytes = kStages * kStageBytes + 1024;
 
+constexpr int kMaxRotPairs = 256;  // rotated head width up to 512
+
 struct GemmParams {
+    int rot_pairs;  // pairs of a rotated head (head_dim / 2), 0 without rotation
     CUtensorMap ta;
     CUtensorMap tb[4];
     int M, K;
@@ -73,8 +76,10 @@ __device__ __forceinline__ float swish(float x) { return x / (1.f + expf(-x)); }
 __device__ __forceinline__ float gelu(float x) { return 0.5f * x * (1.f + erff(x * 0.70710678118654752f)); }
 
 // Store 32 consecutive fp32 values of row m, starting at segment column c0.
+// theta: the rotation frequencies theta_p of the rotated segments' heads,
+// one per pair (shared memory, filled once per CTA).
 __device__ __forceinline__ void epi_store(const GemmEpilogue& e, int seg, int m, int c0, const float (&v)[32],
-                                          int ncols_valid) {
+                                          int ncols_valid, const double* theta) {
     const GemmSegOut& o = e.seg[seg];
     if (m >= e.M) return;
     if (o.kind == kEpiRotate || o.kind == kEpiRotateScaleZeta) {
@@ -89,7 +94,8 @@ __device__ __forceinline__ void epi_store(const GemmEpilogue& e, int seg, int m,
         if (o.kind == kEpiRotateScaleZeta) {
             const int r = n % e.chunk;
             const int L = min(e.chunk, e.seq - (n - r));
-            mult = o.scale * (float)exp2((double)(L - 1 - r) * e.log2g[hh]);
+            // zeta = gamma^(L-1-r): the exponent in fp64, exp2 in fp32 (relative error ~1e-7)
+            mult = o.scale * exp2f((float)((double)(L - 1 - r) * e.log2g[hh]));
         } else {
             mult = o.scale;
         }
@@ -98,8 +104,13 @@ __device__ __forceinline__ void epi_store(const GemmEpilogue& e, int seg, int m,
             const int pidx = (d0 >> 1) + i;
             float sn = 0.f, cs = 1.f;
             if (e.xpos) {
-                const double theta = exp2(-2.0 * pidx / o.head_dim * e.log2base);
-                sincosf(rot_angle(e.pos_offset + n, theta), &sn, &cs);
+                if (e.rot_cs) {
+                    const float2 t = e.rot_cs[(size_t)n * (o.head_dim >> 1) + pidx];
+                    cs = t.x;
+                    sn = t.y;
+                } else {
+                    sincosf(rot_angle(e.pos_offset + n, theta[pidx]), &sn, &cs);
+                }
             }
             cs *= mult;
             sn *= mult;
@@ -181,6 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
     __shared__ GBars bars;
     __shared__ uint32_t s_tmem;
     __shared__ int s_fail;
+    __shared__ double s_theta[kMaxRotPairs];  // theta_p = base^(-2p/head_dim) of the rotated segments
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tiles_m = (p.M + BM - 1) / BM;
     const int ntiles = tiles_m * p.tiles_n;
@@ -201,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
         for (int s = 0; s < p.nseg; s++) tc::prefetch_tmap(&p.tb[s]);
     }
     if (warp == 1) tc::tmem_alloc(&s_tmem, 512);
+    for (int i = tid; i < p.rot_pairs; i += kThreads) s_theta[i] = exp2(-2.0 * i / (2 * p.rot_pairs) * p.epi.log2base);
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
@@ -274,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
 #pragma unroll
                 for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
                 const int c0 = (tn - p.seg_tile0[seg]) * BN + col;  // column within the segment
-                if (c0 < seg_cols) epi_store(p.epi, seg, m, c0, v, seg_cols - c0);
+                if (c0 < seg_cols) epi_store(p.epi, seg, m, c0, v, seg_cols - c0, s_theta);
             }
             tc::tc_fence_before();
             __syncwarp();
@@ -318,6 +331,15 @@ ret_status launch_gemm(const void* A, int M, int K, const GemmSegment* segs, int
     p.tiles_n = t0;
     p.epi = epi;
     p.epi.M = M;
+    p.rot_pairs = 0;
+    for (int i = 0; i < nseg; i++) {
+        const GemmSegOut& o = epi.seg[i];
+        if (epi.xpos && (o.kind == kEpiRotate || o.kind == kEpiRotateScaleZeta)) {
+            if (o.head_dim < 2 || o.head_dim / 2 > kMaxRotPairs || (p.rot_pairs && p.rot_pairs != o.head_dim / 2))
+                return fail(RET_ERR_UNSUPPORTED, "gemm: rotated heads of different widths or wider than 512");
+            p.rot_pairs = o.head_dim / 2;
+        }
+    }
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -5,6 +5,7 @@
 //     Y = Retention(Q, K, V)  per head with decay gamma_h
 //     Z = swish(G) (.) GroupNorm_h(Y),   out = Z W_O
 // as four launches on one stream:
+//   0. (xPos) the (cos, sin) of every (token, pair), once per call;
 //   1. tcgen05 GEMM X [W_Q | W_K | W_V | W_G] whose epilogue writes the
 //      rotated queries, the rotated keys already scaled by k_scale and by the
 //      zeta decay of their place in the chunk (the chunkwise kernel's k'),
@@ -19,6 +20,17 @@
 namespace ret {
 
 namespace {
+
+// (cos, sin) of angle (pos0 + n) theta_p, theta_p = base^(-2p/head_dim), for
+// n < seq, p < head_dim / 2; fp64 angle reduced to [-pi, pi], fp32 sincos.
+__global__ void k_rot_table(float2* __restrict__ cs, int seq, int pairs, long long pos0, double log2base) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)seq * pairs) return;
+    const int n = (int)(i / pairs), p = (int)(i % pairs);
+    float s, c;
+    sincosf(rot_angle(pos0 + n, exp2(-2.0 * p / (2 * pairs) * log2base)), &s, &c);
+    cs[i] = make_float2(c, s);
+}
 
 // One warp per (token, head): d_v values, lanes own d_v / 32 consecutive
 // elements each (d_v a multiple of 128, at most 1024).
@@ -68,8 +80,9 @@ __global__ void __launch_bounds__(256) k_gn_gate(const float* __restrict__ Y, __
 size_t msr_workspace_bytes(int B, int N, int dmodel, int H, int dk, int dv) {
     (void)dmodel;
     const size_t M = (size_t)B * N;
-    // q_rot, k' (bf16), v (bf16), swish(G) then Z (bf16), retention output (fp32)
-    return M * H * ((size_t)dk * 2 * 2 + (size_t)dv * 2 * 2 + (size_t)dv * 4) + 4 * 256;
+    // q_rot, k' (bf16), v (bf16), swish(G) then Z (bf16), retention output
+    // (fp32), the rotation's (cos, sin) table [N][dk/2]
+    return M * H * ((size_t)dk * 2 * 2 + (size_t)dv * 2 * 2 + (size_t)dv * 4) + (size_t)N * (dk / 2) * 8 + 6 * 256;
 }
 
 ret_status launch_msr(const MsrArgs& m, cudaStream_t s) {
@@ -86,6 +99,13 @@ ret_status launch_msr(const MsrArgs& m, cudaStream_t s) {
     __nv_bfloat16* v = reinterpret_cast<__nv_bfloat16*>(carve(M * HV * 2));
     __nv_bfloat16* g = reinterpret_cast<__nv_bfloat16*>(carve(M * HV * 2));
     float* y = reinterpret_cast<float*>(carve(M * HV * 4));
+    float2* rot = reinterpret_cast<float2*>(carve((size_t)m.N * (m.dk / 2) * 8));
+    if (m.xpos) {
+        const long long n_cs = (long long)m.N * (m.dk / 2);
+        k_rot_table<<<(int)((n_cs + 255) / 256), 256, 0, s>>>(rot, m.N, m.dk / 2, m.pos_offset, log2(m.theta_base));
+        ret_status st0 = check_launch("ret_msr_forward: rotation table");
+        if (st0 != RET_OK) return st0;
+    }
 
     // 1. projections with the fused epilogue
     GemmSegment segs[4] = {{m.Wq, HK}, {m.Wk, HK}, {m.Wv, HV}, {m.Wg, HV}};
@@ -100,6 +120,7 @@ ret_status launch_msr(const MsrArgs& m, cudaStream_t s) {
     epi.xpos = m.xpos;
     epi.pos_offset = m.pos_offset;
     epi.log2base = log2(m.theta_base);
+    epi.rot_cs = m.xpos ? rot : nullptr;
     memcpy(epi.log2g, m.hc.log2g, sizeof(epi.log2g));
     ret_status st = launch_gemm(m.X, (int)M, m.dmodel, segs, 4, epi, s);
     if (st != RET_OK) return st;
