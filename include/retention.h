@@ -373,9 +373,10 @@ ret_status ret_forward_recurrent(const void* q, const void* k, const void* v,
  * xpos/pos_offset/theta_base as in ret_forward_chunkwise.  Requires chunk
  * 128, dk 128 or 256, dv in {128, 256, 512, 1024}, d_model a multiple of 8
  * and every gamma_h^128 >= 2^-60 (else RET_ERR_UNSUPPORTED).
- * Four launches on `stream`: the projections (tcgen05 GEMM with the rotation,
- * k_scale, the chunkwise key decay and swish fused in its epilogue), the
- * chunkwise retention, GroupNorm with the gate, and the output projection.
+ * Five launches on `stream`: the (cos, sin) table of the rotation (xpos), the
+ * projections (tcgen05 GEMM with the rotation, k_scale, the chunkwise key
+ * decay and swish fused in its epilogue), the chunkwise retention, GroupNorm
+ * with the gate, and the output projection.
  */
 size_t ret_msr_workspace_bytes(int B, int N, int dmodel, int H, int dk, int dv);
 
@@ -401,7 +402,7 @@ ret_status ret_msr_forward(const void* X, const void* Wq, const void* Wk, const 
  * outputs and the FFN hidden layer are held in bf16 in the workspace
  * (device, 256-byte aligned, at least ret_retnet_block_workspace_bytes(...)
  * bytes, overlapping nothing).  d_model and d_ff multiples of 8.
- * Seven launches: LayerNorm, the MSR's four (the residual added in the output
+ * Eight launches: LayerNorm, the MSR's five (the residual added in the output
  * projection's epilogue), LayerNorm, and the two FFN GEMMs (gelu and the
  * residual in their epilogues).
  */
