@@ -4,7 +4,7 @@
 //     Q = rot(X W_Q), K = rot(k_scale X W_K), V = X W_V, G = X W_G
 //     Y = Retention(Q, K, V)  per head with decay gamma_h
 //     Z = swish(G) (.) GroupNorm_h(Y),   out = Z W_O
-// as four launches on one stream:
+// as launches on one stream:
 //   0. (xPos) the (cos, sin) of every (token, pair), once per call;
 //   1. tcgen05 GEMM X [W_Q | W_K | W_V | W_G] whose epilogue writes the
 //      rotated queries, the rotated keys already scaled by k_scale and by the

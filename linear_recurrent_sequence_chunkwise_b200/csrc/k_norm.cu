@@ -78,32 +78,36 @@ __global__ void __launch_bounds__(256) k_keysum(const __nv_bfloat16* __restrict_
 }
 
 // The decayed key sum before each chunk (zstart) and after the last one
-// (z1).  Block (batch, head, half of d_k), thread (segment t, component d):
-// the chunks are cut into kSeg segments; each thread carries its segment
-// from zero, the segments' end values are combined in order through shared
-// memory, and each thread carries its segment again from its true start.
-constexpr int kSeg = 8, kCarryD = 128;
+// (z1).  Block (batch, head, 32 key components), thread (segment t,
+// component): the chunks are cut into kSeg segments; each thread carries
+// its segment from zero, the segments' end values are combined in order
+// through shared memory (every segment before the last non-empty one spans
+// `per` full chunks, so one decay factor serves them all), and each thread
+// carries its segment again from its true start.
+constexpr int kSeg = 8, kCarryD = 32;
 __global__ void __launch_bounds__(kSeg * kCarryD) k_keycarry(const float* __restrict__ subsum, const float* z0,
                                                              float* zstart, float* z1, HeadConsts hc, int H, int DK,
                                                              int N, int nsub, int nch) {
     __shared__ float s_end[kSeg][kCarryD];
-    const int halves = DK / kCarryD;
-    const int bh = blockIdx.x / halves, h = bh % H;
-    const int d = (blockIdx.x % halves) * kCarryD + threadIdx.x % kCarryD, t = threadIdx.x / kCarryD;
+    const int slices = DK / kCarryD;
+    const int bh = blockIdx.x / slices, h = bh % H;
+    const int c = threadIdx.x % kCarryD, t = threadIdx.x / kCarryD;
+    const int d = (blockIdx.x % slices) * kCarryD + c;
     const double lg = hc.log2g[h];
     const float g_full = (float)exp2(kChunk * lg);
     const float g_last = (float)exp2((N - (nch - 1) * kChunk) * lg);
     const int per = (nch + kSeg - 1) / kSeg, j0 = t * per, j1 = min(nch, j0 + per);
+    const float g_seg = (float)exp2((double)per * kChunk * lg);  // decay over a full segment
     const float* ss = subsum + (size_t)bh * nsub * DK + d;
     constexpr int kPer = kChunk / kSub;
     auto chunk_sum = [&](int j) {
-        float c = 0.f;
+        float cs = 0.f;
 #pragma unroll
         for (int i = 0; i < kPer; i++) {
             const int sb = j * kPer + i;
-            if (sb < nsub) c += ss[(size_t)sb * DK];
+            if (sb < nsub) cs += ss[(size_t)sb * DK];
         }
-        return c;
+        return cs;
     };
     // read before anything is written: z1 may be the same buffer as z0
     float Z = z0 ? z0[(size_t)bh * DK + d] : 0.f;
@@ -116,24 +120,20 @@ __global__ void __launch_bounds__(kSeg * kCarryD) k_keycarry(const float* __rest
     for (int u = 0; u < kHeld; u++) cs[u] = (held && j0 + u < j1) ? chunk_sum(j0 + u) : 0.f;
     auto sum_at = [&](int j) {
         if (held) {
-            float c = 0.f;
+            float v = 0.f;
 #pragma unroll
-            for (int u = 0; u < kHeld; u++) c = (j - j0 == u) ? cs[u] : c;
-            return c;
+            for (int u = 0; u < kHeld; u++) v = (j - j0 == u) ? cs[u] : v;
+            return v;
         }
         return chunk_sum(j);
     };
     // pass 1: this segment from zero
     float E = 0.f;
     for (int j = j0; j < j1; j++) E = fmaf(j == nch - 1 ? g_last : g_full, E, sum_at(j));
-    s_end[t][threadIdx.x % kCarryD] = E;
+    s_end[t][c] = E;
     __syncthreads();
-    // the value entering this segment: earlier segments in order (all but the
-    // last chunk of the sequence span full chunks)
-    for (int u = 0; u < t; u++) {
-        const int len = min(nch, (u + 1) * per) - u * per;
-        Z = fmaf((float)exp2((double)len * kChunk * lg), Z, s_end[u][threadIdx.x % kCarryD]);
-    }
+    // the value entering this segment: the earlier (full) segments in order
+    for (int u = 0; u < t; u++) Z = fmaf(g_seg, Z, s_end[u][c]);
     // pass 2: this segment from its true start
     for (int j = j0; j < j1; j++) {
         zstart[((size_t)bh * nch + j) * DK + d] = Z;
@@ -144,14 +144,20 @@ __global__ void __launch_bounds__(kSeg * kCarryD) k_keycarry(const float* __rest
 }
 
 // One warp per (batch, head, 32-row block): the row sums s_n of its rows and
-// the factors f_n.
+// the factors f_n.  For row r of chunk j,
+//   s = gamma^(r+1-L) q . P_r + gamma^(r+1) q . z_{j-1},  P_r = sum_{c<=r} k'_c,
+// so each lane accumulates the two dot products over its 8 components, the
+// lanes' partials are summed per row through shared memory, and the decay
+// factors are applied once per row.
 constexpr int kRsWarps = 4;  // warps per block of k_rowscale
 template <int DK>
-__global__ void __launch_bounds__(kRsWarps * 32, 4) k_rowscale(const __nv_bfloat16* __restrict__ qe,
-                                                  const __nv_bfloat16* __restrict__ kp,
-                                                  const float* __restrict__ subsum, const float* __restrict__ zstart,
-                                                  float* __restrict__ rowscale, HeadConsts hc, int B, int N, int H,
-                                                  int nsub, int nch, long long pos0, int flags) {
+__global__ void __launch_bounds__(kRsWarps * 32, 6) k_rowscale(const __nv_bfloat16* __restrict__ qe,
+                                                               const __nv_bfloat16* __restrict__ kp,
+                                                               const float* __restrict__ subsum,
+                                                               const float* __restrict__ zstart,
+                                                               float* __restrict__ rowscale, HeadConsts hc, int B,
+                                                               int N, int H, int nsub, int nch, long long pos0,
+                                                               int flags) {
     static_assert(DK / 8 <= 32, "one 8-element group per lane");
     const int lane = threadIdx.x & 31;
     const long long w = (long long)blockIdx.x * kRsWarps + (threadIdx.x >> 5);
@@ -164,59 +170,68 @@ __global__ void __launch_bounds__(kRsWarps * 32, 4) k_rowscale(const __nv_bfloat
     const bool act = (flags & kNormScore) && lane < DK / 8;  // without it only c_n is needed
     const double lg = hc.log2g[h];
 
-    float Z[8], P[8];
+    __shared__ float part[2][kRsWarps][kSub][33];  // (q . P, q . z) per row and lane
+    float (*pp)[33] = part[0][threadIdx.x >> 5];
+    float (*pz)[33] = part[1][threadIdx.x >> 5];
+    if (flags & kNormScore) {
+        float Z[8], P[8];
 #pragma unroll
-    for (int e = 0; e < 8; e++) Z[e] = P[e] = 0.f;
-    if (act) {
-        const float* zs = zstart + ((size_t)bh * nch + j) * DK + 8 * lane;
-#pragma unroll
-        for (int e = 0; e < 8; e++) Z[e] = zs[e];
-        for (int s2 = j * (kChunk / kSub); s2 < s; s2++) {
-            const float* ps = subsum + ((size_t)bh * nsub + s2) * DK + 8 * lane;
-#pragma unroll
-            for (int e = 0; e < 8; e++) P[e] += ps[e];
-        }
-    }
-    // lane partials of each row, summed per row through shared memory (padded
-    // rows: lane l reading row l touches 32 different banks)
-    __shared__ float part[kRsWarps][kSub][33];
-    float (*pw)[33] = part[threadIdx.x >> 5];
-#pragma unroll
-    for (int rb = 0; rb < kSub; rb += 8) {
-        uint4 kx[8], qx[8];
-#pragma unroll
-        for (int u = 0; u < 8; u++) {
-            if (act && rb + u < nrows) {
-                const size_t row = ((size_t)b * N + n0c + r0 + rb + u) * H + h;
-                kx[u] = __ldg(reinterpret_cast<const uint4*>(kp + row * DK + 8 * lane));
-                qx[u] = __ldg(reinterpret_cast<const uint4*>(qe + row * DK + 8 * lane));
+        for (int e = 0; e < 8; e++) Z[e] = P[e] = 0.f;
+        if (act) {
+            const float4* zs = reinterpret_cast<const float4*>(zstart + ((size_t)bh * nch + j) * DK + 8 * lane);
+            const float4 z0 = zs[0], z1 = zs[1];
+            Z[0] = z0.x; Z[1] = z0.y; Z[2] = z0.z; Z[3] = z0.w; Z[4] = z1.x; Z[5] = z1.y; Z[6] = z1.z; Z[7] = z1.w;
+            for (int s2 = j * (kChunk / kSub); s2 < s; s2++) {
+                const float4* ps = reinterpret_cast<const float4*>(subsum + ((size_t)bh * nsub + s2) * DK + 8 * lane);
+                const float4 a0 = ps[0], a1 = ps[1];
+                P[0] += a0.x; P[1] += a0.y; P[2] += a0.z; P[3] += a0.w;
+                P[4] += a1.x; P[5] += a1.y; P[6] += a1.z; P[7] += a1.w;
             }
         }
 #pragma unroll
-        for (int u = 0; u < 8; u++) {
-            float val = 0.f;
-            if (act && rb + u < nrows) {
-                const int r = r0 + rb + u;
-                const float a = exp2f((float)((r + 1 - L) * lg));  // gamma^(r+1-L)
-                const float c = exp2f((float)((r + 1) * lg));      // gamma^(r+1)
-                float kf[8], qf[8];
-                unpack_bf16x8(kx[u], kf);
-                unpack_bf16x8(qx[u], qf);
+        for (int rb = 0; rb < kSub; rb += 4) {
+            uint4 kx[4], qx[4];
 #pragma unroll
-                for (int e = 0; e < 8; e++) {
-                    P[e] += kf[e];
-                    val = fmaf(qf[e], fmaf(a, P[e], c * Z[e]), val);
+            for (int u = 0; u < 4; u++) {
+                if (act && rb + u < nrows) {
+                    const size_t row = ((size_t)b * N + n0c + r0 + rb + u) * H + h;
+                    kx[u] = __ldg(reinterpret_cast<const uint4*>(kp + row * DK + 8 * lane));
+                    qx[u] = __ldg(reinterpret_cast<const uint4*>(qe + row * DK + 8 * lane));
                 }
             }
-            pw[rb + u][lane] = val;
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                float dP = 0.f, dZ = 0.f;
+                if (act && rb + u < nrows) {
+                    float kf[8], qf[8];
+                    unpack_bf16x8(kx[u], kf);
+                    unpack_bf16x8(qx[u], qf);
+#pragma unroll
+                    for (int e = 0; e < 8; e++) {
+                        P[e] += kf[e];
+                        dP = fmaf(qf[e], P[e], dP);
+                        dZ = fmaf(qf[e], Z[e], dZ);
+                    }
+                }
+                pp[rb + u][lane] = dP;
+                pz[rb + u][lane] = dZ;
+            }
         }
+        __syncwarp();
     }
-    __syncwarp();
-    float sn = 0.f;  // row r0 + lane
-#pragma unroll 8
-    for (int i = 0; i < 32; i++) sn += pw[lane][i];
     if (lane < nrows) {
-        const long long n = n0c + r0 + lane;
+        const int r = r0 + lane;
+        float sn = 0.f;
+        if (flags & kNormScore) {
+            float sP = 0.f, sZ = 0.f;
+#pragma unroll 8
+            for (int i = 0; i < 32; i++) {
+                sP += pp[lane][i];
+                sZ += pz[lane][i];
+            }
+            sn = exp2f((float)((r + 1 - L) * lg)) * sP + exp2f((float)((r + 1) * lg)) * sZ;
+        }
+        const long long n = n0c + r;
         double f = 1.0;
         if (flags & kNormDecay) {
             // sum_{i<=n} gamma^(n-i) over the whole sequence, position pos0 + n
@@ -272,16 +287,16 @@ ret_status launch_chunkwise_normalized(const RetArgs& a0, int flags, const float
     if (a0.dk == 256) {
         if (keys) {
             k_keysum<256><<<blocks, 256, 0, s>>>(kp, subsum, a0.B, a0.N, a0.H, L.nsub);
-            k_keycarry<<<a0.B * a0.H * 2, kSeg * kCarryD, 0, s>>>(subsum, z0, zstart, z1, a0.hc, a0.H, 256, a0.N,
-                                                                  L.nsub, L.nch);
+            k_keycarry<<<a0.B * a0.H * (256 / kCarryD), kSeg * kCarryD, 0, s>>>(subsum, z0, zstart, z1, a0.hc,
+                                                                                a0.H, 256, a0.N, L.nsub, L.nch);
         }
         k_rowscale<256><<<rs_blocks, kRsWarps * 32, 0, s>>>(qe, kp, subsum, zstart, rowscale, a0.hc, a0.B, a0.N, a0.H, L.nsub,
                                                L.nch, a0.pos_offset, flags);
     } else {
         if (keys) {
             k_keysum<128><<<blocks, 256, 0, s>>>(kp, subsum, a0.B, a0.N, a0.H, L.nsub);
-            k_keycarry<<<a0.B * a0.H, kSeg * kCarryD, 0, s>>>(subsum, z0, zstart, z1, a0.hc, a0.H, 128, a0.N, L.nsub,
-                                                              L.nch);
+            k_keycarry<<<a0.B * a0.H * (128 / kCarryD), kSeg * kCarryD, 0, s>>>(subsum, z0, zstart, z1, a0.hc,
+                                                                                a0.H, 128, a0.N, L.nsub, L.nch);
         }
         k_rowscale<128><<<rs_blocks, kRsWarps * 32, 0, s>>>(qe, kp, subsum, zstart, rowscale, a0.hc, a0.B, a0.N, a0.H, L.nsub,
                                                L.nch, a0.pos_offset, flags);
