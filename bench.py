@@ -611,8 +611,28 @@ def bench_fp32_small(R, torch, dev, stream, args, world, dist):
 
     ms = _timed(torch, stream, fn, 50, 5, world, dist, dev)
     R.ret_check_device_error()
+    # The same call replayed from a CUDA graph of 100 calls: the launch cost
+    # a serving loop pays when it captures its steps.
+    reps = 100
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        for _ in range(reps):
+            R.ret_forward_chunkwise(q, k, v, g, 16, out=out)
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    graph.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    R.ret_check_device_error()
+    us_graph = max_over_ranks(a.elapsed_time(b), world, dist, dev) * 1e3 / reps
+    del graph
     return {"workload": "retention_f32_1x64x8x16", "us_per_call": round(ms * 1e3, 2),
-            "bound": "latency", "kernel": "k_chunkwise_simt"}
+            "us_per_call_graph_replay": round(us_graph, 2), "bound": "latency", "kernel": "k_chunkwise_simt"}
 
 
 # ---------------------------------------------------------- the oracle ---
