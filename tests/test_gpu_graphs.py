@@ -68,3 +68,36 @@ def test_chunkwise_forward_replayed_from_a_graph():
     ref, Sref = oracle.retention_recurrent(oracle.xpos_rotate(q.f64), oracle.xpos_rotate(k.f64), v.f64, g)
     assert err_out(host64(out), ref) < TOL_BF16
     assert err_state(host64(fs), Sref) < TOL_BF16
+
+
+def test_backward_replayed_from_a_graph():
+    """The backward forks its dk passes onto a second stream and joins back
+    with events: under capture that is a fork/join in the graph."""
+    import linear_recurrent_sequence_chunkwise_b200 as R
+    B, N, H, dk, dv = 1, 300, 2, 128, 256
+    q = make_tensor(503, 1, (B, N, H, dk), "bf16", dk ** -0.5)
+    k = make_tensor(503, 2, (B, N, H, dk), "bf16", dk ** -0.5)
+    v = make_tensor(503, 3, (B, N, H, dv), "bf16")
+    do = make_tensor(503, 4, (B, N, H, dv), "bf16")
+    g = gamma_schedule(H)
+    qd, kd, vd, dod = dev(q), dev(k), dev(v), dev(do)
+    nb = R.ret_backward_workspace_bytes(B, N, H, dk, dv, 128, torch.bfloat16, True)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    dq = torch.empty((B, N, H, dk), dtype=torch.float32, device="cuda")
+    dkk = torch.empty_like(dq)
+    dvv = torch.empty((B, N, H, dv), dtype=torch.float32, device="cuda")
+    R.ret_backward_chunkwise(qd, kd, vd, dod, g, 128, workspace=ws, dq=dq, dk=dkk, dv=dvv, xpos=True)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        R.ret_backward_chunkwise(qd, kd, vd, dod, g, 128, workspace=ws, dq=dq, dk=dkk, dv=dvv, xpos=True)
+    for t in (dq, dkk, dvv):
+        t.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    R.ret_check_device_error()
+    ref = oracle.retention_backward(q.f64, k.f64, v.f64, do.f64, g, xpos=True)
+    for name, a, r in zip(("dq", "dk", "dv"), (dq, dkk, dvv), ref):
+        assert err_out(host64(a), r) < TOL_BF16, name
