@@ -91,11 +91,12 @@ struct SimtChunkLayout {
     size_t bytes;
 };
 
-static SimtChunkLayout simt_chunk_layout(int C, int dk, int W) {
+// R: rows of q, k, v held at once (the chunk, or the whole sequence).
+static SimtChunkLayout simt_chunk_layout(int C, int dk, int W, int R) {
     SimtChunkLayout l;
     l.W = W;
     l.ldk = dk + 1;
-    size_t floats = (size_t)2 * C * l.ldk + (size_t)C * W + (size_t)C * (C + 1) + (size_t)dk * W + (C + 2);
+    size_t floats = (size_t)2 * R * l.ldk + (size_t)R * W + (size_t)C * (C + 1) + (size_t)dk * W + (C + 2);
     floats = (floats + 1) & ~(size_t)1;  // 8-byte alignment for the theta table
     l.bytes = floats * sizeof(float) + (size_t)(dk / 2 + 1) * sizeof(double);
     return l;
@@ -106,18 +107,21 @@ __global__ void __launch_bounds__(256) k_chunkwise_simt(const Tin* __restrict__ 
                                                         const Tin* __restrict__ v, HeadConsts hc, int N, int H,
                                                         int dk, int dv, int C, int W, Tout* __restrict__ out,
                                                         float* __restrict__ fstate, int xpos, long long pos0,
-                                                        double log2base) {
+                                                        double log2base, int whole) {
+    // whole: the sequence is short enough that all its rows of q, k, v are
+    // loaded into shared memory once, before the chunk loop
     const int h = blockIdx.y, b = blockIdx.z, j0 = blockIdx.x * W;
     const int wt = min(W, dv - j0);
     const int ldk = dk + 1;
+    const int RR = whole ? N : C;  // rows the buffers hold
     extern __shared__ float sm[];
-    float* Qs = sm;
-    float* Ks = Qs + (size_t)C * ldk;
-    float* Vs = Ks + (size_t)C * ldk;
-    float* As = Vs + (size_t)C * W;
+    float* Qb = sm;
+    float* Kb = Qb + (size_t)RR * ldk;
+    float* Vb = Kb + (size_t)RR * ldk;
+    float* As = Vb + (size_t)RR * W;
     float* Ss = As + (size_t)C * (C + 1);
     float* pw = Ss + (size_t)dk * W;
-    size_t off = (size_t)2 * C * ldk + (size_t)C * W + (size_t)C * (C + 1) + (size_t)dk * W + (C + 2);
+    size_t off = (size_t)2 * RR * ldk + (size_t)RR * W + (size_t)C * (C + 1) + (size_t)dk * W + (C + 2);
     off = (off + 1) & ~(size_t)1;
     double* theta = reinterpret_cast<double*>(sm + off);
 
@@ -127,14 +131,21 @@ __global__ void __launch_bounds__(256) k_chunkwise_simt(const Tin* __restrict__ 
     for (int e = threadIdx.x; e < dk * W; e += blockDim.x) Ss[e] = 0.f;
     __syncthreads();
 
+    auto load = [&](int n0, int rows, float* Qd, float* Kd, float* Vd) {
+        load_rows_rotated(q, b, n0, rows, N, H, h, dk, Qd, ldk, xpos != 0, pos0, theta);
+        load_rows_rotated(k, b, n0, rows, N, H, h, dk, Kd, ldk, xpos != 0, pos0, theta);
+        for (int idx = threadIdx.x; idx < rows * wt; idx += blockDim.x) {
+            const int r = idx / wt, j = idx % wt;
+            Vd[r * W + j] = ld_as_float(v, (((size_t)b * N + n0 + r) * H + h) * dv + j0 + j);
+        }
+    };
+    if (whole) load(0, N, Qb, Kb, Vb);
     for (int c0 = 0; c0 < N; c0 += C) {
         const int L = min(C, N - c0);
-        load_rows_rotated(q, b, c0, L, N, H, h, dk, Qs, ldk, xpos != 0, pos0, theta);
-        load_rows_rotated(k, b, c0, L, N, H, h, dk, Ks, ldk, xpos != 0, pos0, theta);
-        for (int idx = threadIdx.x; idx < L * wt; idx += blockDim.x) {
-            const int r = idx / wt, j = idx % wt;
-            Vs[r * W + j] = ld_as_float(v, (((size_t)b * N + c0 + r) * H + h) * dv + j0 + j);
-        }
+        float* Qs = whole ? Qb + (size_t)c0 * ldk : Qb;
+        float* Ks = whole ? Kb + (size_t)c0 * ldk : Kb;
+        float* Vs = whole ? Vb + (size_t)c0 * W : Vb;
+        if (!whole) load(c0, L, Qs, Ks, Vs);
         __syncthreads();
         for (int idx = threadIdx.x; idx < L * L; idx += blockDim.x) {
             const int r = idx / L, c = idx % L;
@@ -179,8 +190,18 @@ ret_status launch_chunkwise_simt(const RetArgs& a, cudaStream_t s) {
     int W = 0;
     for (int w : {64, 32, 16, 8}) {
         if (w > a.dv && w != 8) continue;
-        lay = simt_chunk_layout(C, a.dk, w);
+        lay = simt_chunk_layout(C, a.dk, w, C);
         if (lay.bytes <= 200 * 1024) { W = w; break; }
+    }
+    // a short sequence is loaded once (one round of global-load latency
+    // instead of one per chunk)
+    int whole = 0;
+    if (W != 0 && a.N > C) {
+        const SimtChunkLayout lw = simt_chunk_layout(C, a.dk, W, a.N);
+        if (lw.bytes <= 64 * 1024) {
+            lay = lw;
+            whole = 1;
+        }
     }
     if (W == 0)
         return fail(RET_ERR_UNSUPPORTED, "chunkwise (CUDA-core path): chunk=%d dk=%d does not fit shared memory",
@@ -195,7 +216,7 @@ ret_status launch_chunkwise_simt(const RetArgs& a, cudaStream_t s) {
             return check_launch("chunkwise (CUDA-core path): smem attribute");                               \
         kern<<<grid, 256, lay.bytes, s>>>((const TI*)a.q, (const TI*)a.k, (const TI*)a.v, a.hc, a.N, a.H,    \
                                           a.dk, a.dv, C, W, (TO*)a.out, a.final_state, a.xpos, a.pos_offset, \
-                                          lb);                                                                \
+                                          lb, whole);                                                         \
     } while (0)
     if (a.in_dt == RET_F32 && a.out_dt == RET_F32) RET_LAUNCH_SIMT(float, float);
     else if (a.in_dt == RET_F32) RET_LAUNCH_SIMT(float, __nv_bfloat16);
