@@ -241,3 +241,19 @@ def test_ws_d64_continuation():
     ref, Sref = oracle.retention_recurrent(qr, kr, v.f64, g)
     assert err_out(np.concatenate(outs, axis=1), ref) < TOL_BF16
     assert err_state(host64(S), Sref) < TOL_BF16
+
+
+def test_ws_long_sequence_32k():
+    """32768 tokens (256 chunks in sequence per CTA) with the fastest and the
+    slowest decay of the schedule: the fp32 state and its bf16 read-out copy
+    carried across the whole sequence, every output and the final state
+    against the oracle."""
+    B, N, H, dk, dv = 1, 32768, 2, 256, 256
+    q, k, v = qkv(86, B, N, H, dk, dv, dk ** -0.5)
+    g = np.array([1 - 2.0 ** -5, 1 - 2.0 ** -12])
+    out, fs = run_ws(q, k, v, g, 128, out_dtype=torch.float32, xpos=True, want_final_state=True)
+    R.ret_check_device_error()
+    qr, kr = rotated(q, k, True)
+    ref, S = oracle.retention_recurrent(qr, kr, v.f64, g)
+    assert err_out(host64(out), ref) < TOL_BF16
+    assert err_state(host64(fs), S) < TOL_BF16
