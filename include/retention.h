@@ -192,8 +192,13 @@ ret_status ret_forward_chunkwise_prepared(const void* q, const void* k, const vo
  * dq, dk: device fp32 [B, N, H, dk]; dv: device fp32 [B, N, H, dv]; written,
  * 16-byte aligned, overlapping nothing else.
  * workspace: device, 256-byte aligned, at least
- * ret_backward_workspace_bytes(...) bytes (about 2x(q, k, v, dout) in bf16
- * plus k and v gradients in fp32), scratch, overlapping nothing else.
+ * ret_backward_workspace_bytes(...) bytes (the rotated keys in both time
+ * orders, the rotated queries, v and dout time-reversed, all bf16, and the
+ * scratch of two concurrent passes), overlapping nothing else.
+ * Half of the passes run on a second CUDA stream that the library creates
+ * per device on first use and keeps for the life of the process; the call
+ * joins it back into `stream` with events before returning (also under
+ * CUDA-graph capture).
  */
 size_t ret_backward_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk, ret_dtype in_dt,
                                     int xpos);
