@@ -436,8 +436,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                                               id_qt, k > 0);
                 }
                 tc::mma_commit_elect(&bars.qtm);  // Q in TMEM and T in smem are read
-                // ---- O += P V  (P from TMEM)
+                // ---- O += P V  (P from TMEM; V of this chunk must have landed:
+                // nothing else this warp waits on implies it, since the
+                // producer loads V after the chunk's K' parts)
                 ok = wait(&bars.pready, jc & 1);
+                if (ok) ok = wait(&bars.vfull[jc & 1], (jc >> 1) & 1);
                 if (!ok) break;
                 tc::tc_fence_after();
 #pragma unroll
