@@ -131,6 +131,30 @@ def _ptr(t: Optional[torch.Tensor], name: str):
     return ctypes.c_void_p(t.data_ptr())
 
 
+F32 = (torch.float32,)
+FLOATS = (torch.float32, torch.bfloat16)
+
+
+def _buf(t: Optional[torch.Tensor], name: str, shape, dtypes, like: torch.Tensor):
+    """A caller-provided buffer must have the shape and dtype the call reads or
+    writes and sit on the inputs' device: the C ABI takes plain pointers and
+    cannot check either."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {list(shape)} (got {list(t.shape)})")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} must be {' or '.join(str(d) for d in dtypes)} (got {t.dtype})")
+    if t.device != like.device:
+        raise ValueError(f"{name} is on {t.device}, the inputs on {like.device}")
+
+
+def _same_device(like: torch.Tensor, **tensors):
+    for name, t in tensors.items():
+        if t is not None and t.device != like.device:
+            raise ValueError(f"{name} is on {t.device}, the inputs on {like.device}")
+
+
 def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -159,8 +183,15 @@ def _seq_shapes(q, k, v):
         raise ValueError("expected q, k [B, N, H, dk] and v [B, N, H, dv]")
     if not (q.dtype == k.dtype == v.dtype):
         raise TypeError("q, k and v must share a dtype")
+    _same_device(q, k=k, v=v)
     B, N, H, dk = q.shape
     return B, N, H, dk, v.shape[3]
+
+
+def _seq_outputs(q, out, final_state, B, N, H, dk, dv, initial_state=None):
+    _buf(out, "out", (B, N, H, dv), FLOATS, q)
+    _buf(final_state, "final_state", (B, H, dk, dv), F32, q)
+    _buf(initial_state, "initial_state", (B, H, dk, dv), F32, q)
 
 
 def ret_forward_chunkwise(q, k, v, gammas, chunk: int, out=None, final_state=None, out_dtype=None,
@@ -174,8 +205,7 @@ def ret_forward_chunkwise(q, k, v, gammas, chunk: int, out=None, final_state=Non
         out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and want_final_state:
         final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
-    if final_state is not None and final_state.dtype != torch.float32:
-        raise TypeError("final_state must be float32")
+    _seq_outputs(q, out, final_state, B, N, H, dk, dv)
     _check(lib.ret_forward_chunkwise(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N, H, dk,
                                      dv, int(chunk), _ptr(out, "out"), _ptr(final_state, "final_state"),
                                      _stream(stream), _dt(q.dtype), _dt(out.dtype), int(bool(xpos)),
@@ -199,6 +229,8 @@ def ret_forward_chunkwise_ws(q, k, v, gammas, chunk: int, workspace, out=None, f
         out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and want_final_state:
         final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _seq_outputs(q, out, final_state, B, N, H, dk, dv)
+    _same_device(q, workspace=workspace)
     nbytes = workspace.numel() * workspace.element_size()
     _check(lib.ret_forward_chunkwise_ws(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N, H, dk,
                                         dv, int(chunk), _ptr(out, "out"), _ptr(final_state, "final_state"),
@@ -214,6 +246,7 @@ def ret_chunkwise_prepare(q, k, gammas, chunk: int, workspace, dv: int, xpos: bo
     if q.shape != k.shape or q.dim() != 4:
         raise ValueError("q and k must both be [B, N, H, dk]")
     B, N, H, dk = q.shape
+    _same_device(q, k=k, workspace=workspace)
     nbytes = workspace.numel() * workspace.element_size()
     _check(lib.ret_chunkwise_prepare(_ptr(q, "q"), _ptr(k, "k"), _gammas(gammas, H), B, N, H, dk, int(dv),
                                      int(chunk), _stream(stream), _dt(q.dtype), int(bool(xpos)), int(pos_offset),
@@ -231,9 +264,8 @@ def ret_forward_chunkwise_prepared(q, k, v, gammas, chunk: int, workspace, out=N
         out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and want_final_state:
         final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
-    if initial_state is not None and (initial_state.dtype != torch.float32 or
-                                      tuple(initial_state.shape) != (B, H, dk, dv)):
-        raise ValueError("initial_state must be fp32 [B, H, dk, dv]")
+    _seq_outputs(q, out, final_state, B, N, H, dk, dv, initial_state)
+    _same_device(q, workspace=workspace)
     nbytes = workspace.numel() * workspace.element_size()
     _check(lib.ret_forward_chunkwise_prepared(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N,
                                               H, dk, dv, int(chunk), _ptr(out, "out"),
@@ -254,14 +286,17 @@ def ret_backward_chunkwise(q, k, v, dout, gammas, chunk: int, workspace=None, dq
     """Gradients (dq, dk, dv) in fp32 of sum(out * dout) for the chunkwise
     forward of the same arguments."""
     B, N, H, dk_, dv_ = _seq_shapes(q, k, v)
-    if tuple(dout.shape) != (B, N, H, dv_):
-        raise ValueError("dout must be [B, N, H, dv]")
+    _buf(dout, "dout", (B, N, H, dv_), (q.dtype,), q)
     dq = torch.empty((B, N, H, dk_), dtype=torch.float32, device=q.device) if dq is None else dq
     dk = torch.empty((B, N, H, dk_), dtype=torch.float32, device=q.device) if dk is None else dk
     dv = torch.empty((B, N, H, dv_), dtype=torch.float32, device=q.device) if dv is None else dv
     if workspace is None:
         nb = ret_backward_workspace_bytes(B, N, H, dk_, dv_, chunk, q.dtype, xpos)
         workspace = torch.empty(max(nb, 1), dtype=torch.uint8, device=q.device)
+    _buf(dq, "dq", (B, N, H, dk_), F32, q)
+    _buf(dk, "dk", (B, N, H, dk_), F32, q)
+    _buf(dv, "dv", (B, N, H, dv_), F32, q)
+    _same_device(q, workspace=workspace)
     nbytes = workspace.numel() * workspace.element_size()
     _check(lib.ret_backward_chunkwise(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _ptr(dout, "dout"),
                                       _gammas(gammas, H), B, N, H, dk_, dv_, int(chunk), _ptr(dq, "dq"),
@@ -289,6 +324,7 @@ def ret_forward_chunkwise_noalloc(q, k, v, gammas, chunk: int, out=None, final_s
         out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and want_final_state:
         final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _seq_outputs(q, out, final_state, B, N, H, dk, dv)
     _check(lib.ret_forward_chunkwise_noalloc(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N,
                                              H, dk, dv, int(chunk), _ptr(out, "out"),
                                              _ptr(final_state, "final_state"), _stream(stream), _dt(q.dtype),
@@ -302,6 +338,7 @@ def ret_forward_parallel(q, k, v, gammas, out=None, out_dtype=None, xpos: bool =
     B, N, H, dk, dv = _seq_shapes(q, k, v)
     if out is None:
         out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
+    _seq_outputs(q, out, None, B, N, H, dk, dv)
     _check(lib.ret_forward_parallel(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N, H, dk,
                                     dv, _ptr(out, "out"), _stream(stream), _dt(q.dtype), _dt(out.dtype),
                                     int(bool(xpos)), int(pos_offset), float(theta_base)))
@@ -317,6 +354,7 @@ def ret_forward_recurrent(q, k, v, gammas, out=None, final_state=None, out_dtype
         out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
     if final_state is None and want_final_state:
         final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _seq_outputs(q, out, final_state, B, N, H, dk, dv)
     _check(lib.ret_forward_recurrent(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N, H, dk,
                                      dv, _ptr(out, "out"), _ptr(final_state, "final_state"), _stream(stream),
                                      _dt(q.dtype), _dt(out.dtype), int(bool(xpos)), int(pos_offset),
@@ -324,17 +362,27 @@ def ret_forward_recurrent(q, k, v, gammas, out=None, final_state=None, out_dtype
     return (out, final_state) if final_state is not None else out
 
 
+def _step_shapes(q, k, v, state):
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
+        raise ValueError("expected q, k [B, H, dk] and v [B, H, dv]")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k and v must share a dtype")
+    _same_device(q, k=k, v=v)
+    B, H, dk = q.shape
+    dv = v.shape[2]
+    if state is None:
+        raise ValueError("state must be float32 [B, H, dk, dv]")
+    _buf(state, "state", (B, H, dk, dv), F32, q)
+    return B, H, dk, dv
+
+
 def ret_decode_step(q, k, v, gammas, state, out=None, out_dtype=None, stream=None):
     """One decode step: state [B, H, dk, dv] fp32 updated in place; returns
     out [B, H, dv]."""
-    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
-        raise ValueError("expected q, k [B, H, dk] and v [B, H, dv]")
-    B, H, dk = q.shape
-    dv = v.shape[2]
-    if state.shape != (B, H, dk, dv) or state.dtype != torch.float32:
-        raise ValueError("state must be float32 [B, H, dk, dv]")
+    B, H, dk, dv = _step_shapes(q, k, v, state)
     if out is None:
         out = torch.empty((B, H, dv), dtype=out_dtype or torch.float32, device=q.device)
+    _buf(out, "out", (B, H, dv), FLOATS, q)
     _check(lib.ret_decode_step(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H),
                                _ptr(state, "state"), _ptr(out, "out"), _stream(stream), B, H, dk, dv,
                                _dt(q.dtype), _dt(out.dtype)))
@@ -359,13 +407,13 @@ def ret_forward_chunkwise_normalized(q, k, v, gammas, chunk: int, norm_flags: in
     B, N, H, dk, dv = _seq_shapes(q, k, v)
     if out is None:
         out = torch.empty((B, N, H, dv), dtype=out_dtype or q.dtype, device=q.device)
-    for name, t, shape in (("initial_state", initial_state, (B, H, dk, dv)), ("final_state", final_state, (B, H, dk, dv)),
-                           ("initial_z", initial_z, (B, H, dk)), ("final_z", final_z, (B, H, dk))):
-        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != shape):
-            raise ValueError(f"{name} must be fp32 {list(shape)}")
+    _seq_outputs(q, out, final_state, B, N, H, dk, dv, initial_state)
+    _buf(initial_z, "initial_z", (B, H, dk), F32, q)
+    _buf(final_z, "final_z", (B, H, dk), F32, q)
     if workspace is None:
         nb = ret_normalized_workspace_bytes(B, N, H, dk, dv, chunk, q.dtype, xpos)
         workspace = torch.empty(max(nb, 1), dtype=torch.uint8, device=q.device)
+    _same_device(q, workspace=workspace)
     nbytes = workspace.numel() * workspace.element_size()
     _check(lib.ret_forward_chunkwise_normalized(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H), B, N,
                                                 H, dk, dv, int(chunk), int(norm_flags), _ptr(out, "out"),
@@ -381,16 +429,11 @@ def ret_decode_step_normalized(q, k, v, gammas, state, z, position: int, norm_fl
                                out=None, out_dtype=None, stream=None):
     """One decode step with the score normalizations at 0-based ``position``:
     state [B, H, dk, dv] and z [B, H, dk] (fp32) updated in place."""
-    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
-        raise ValueError("expected q, k [B, H, dk] and v [B, H, dv]")
-    B, H, dk = q.shape
-    dv = v.shape[2]
-    if state.shape != (B, H, dk, dv) or state.dtype != torch.float32:
-        raise ValueError("state must be float32 [B, H, dk, dv]")
-    if z is not None and (z.shape != (B, H, dk) or z.dtype != torch.float32):
-        raise ValueError("z must be float32 [B, H, dk]")
+    B, H, dk, dv = _step_shapes(q, k, v, state)
+    _buf(z, "z", (B, H, dk), F32, q)
     if out is None:
         out = torch.empty((B, H, dv), dtype=out_dtype or torch.float32, device=q.device)
+    _buf(out, "out", (B, H, dv), FLOATS, q)
     _check(lib.ret_decode_step_normalized(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H),
                                           _ptr(state, "state"), _ptr(z, "z"), _ptr(out, "out"), int(position),
                                           int(norm_flags), _stream(stream), B, H, dk, dv, _dt(q.dtype),
@@ -404,16 +447,12 @@ def ret_decode_step_positions(q, k, v, gammas, state, positions, z=None, xpos: b
     """One decode step with each sequence at its own position: positions int64
     [B] on the device; xPos rotation of q, k inside the step; optional score
     normalizations with z [B, H, dk] fp32 (in place)."""
-    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[:2] != q.shape[:2]:
-        raise ValueError("expected q, k [B, H, dk] and v [B, H, dv]")
-    B, H, dk = q.shape
-    dv = v.shape[2]
-    if state.shape != (B, H, dk, dv) or state.dtype != torch.float32:
-        raise ValueError("state must be float32 [B, H, dk, dv]")
-    if positions.dtype != torch.int64 or tuple(positions.shape) != (B,):
-        raise ValueError("positions must be int64 [B]")
+    B, H, dk, dv = _step_shapes(q, k, v, state)
+    _buf(positions, "positions", (B,), (torch.int64,), q)
+    _buf(z, "z", (B, H, dk), F32, q)
     if out is None:
         out = torch.empty((B, H, dv), dtype=out_dtype or torch.float32, device=q.device)
+    _buf(out, "out", (B, H, dv), FLOATS, q)
     _check(lib.ret_decode_step_positions(_ptr(q, "q"), _ptr(k, "k"), _ptr(v, "v"), _gammas(gammas, H),
                                          _ptr(state, "state"), _ptr(z, "z"), _ptr(out, "out"),
                                          _ptr(positions, "positions"), int(bool(xpos)), float(theta_base),
@@ -433,6 +472,27 @@ def ret_check_device_error(stream=None):
     _check(lib.ret_check_device_error(_stream(stream)))
 
 
+BF16 = (torch.bfloat16,)
+
+
+def _msr_shapes(x, wq, wk, wv, wg, wo, H: int):
+    """B, N, d_model, dk, dv of an MSR layer from x [B, N, d_model] and the
+    (input, output) weights W_Q, W_K [d_model, H dk], W_V, W_G [d_model, H dv],
+    W_O [H dv, d_model], all bf16 on x's device."""
+    if x.dim() != 3 or x.dtype != torch.bfloat16:
+        raise ValueError("x must be bfloat16 [B, N, d_model]")
+    B, N, dm = x.shape
+    if H < 1 or wq.dim() != 2 or wv.dim() != 2 or wq.shape[1] % H or wv.shape[1] % H:
+        raise ValueError("W_Q and W_V must be [d_model, H * d] with H dividing their widths")
+    dk, dv = wq.shape[1] // H, wv.shape[1] // H
+    _buf(wq, "wq", (dm, H * dk), BF16, x)
+    _buf(wk, "wk", (dm, H * dk), BF16, x)
+    _buf(wv, "wv", (dm, H * dv), BF16, x)
+    _buf(wg, "wg", (dm, H * dv), BF16, x)
+    _buf(wo, "wo", (H * dv, dm), BF16, x)
+    return B, N, dm, dk, dv
+
+
 def ret_retnet_block_workspace_bytes(B, N, dmodel, H, dk, dv, dff) -> int:
     return int(lib.ret_retnet_block_workspace_bytes(B, N, dmodel, H, dk, dv, dff))
 
@@ -445,15 +505,19 @@ def ret_retnet_block_forward(x, wq, wk, wv, wg, wo, w1, w2, gammas, H: int, ln1_
     """One pre-LayerNorm RetNet block: Y = MSR(LN1(x)) + x, out = gelu(LN2(Y) W1) W2 + Y.
     x [B, N, d_model] bf16; weights bf16 [in, out]; LayerNorm gains/biases bf16
     [d_model] or None (1 / 0)."""
-    B, N, dm = x.shape
-    dk = wq.shape[1] // H
-    dv = wv.shape[1] // H
+    B, N, dm, dk, dv = _msr_shapes(x, wq, wk, wv, wg, wo, H)
     dff = w1.shape[1]
+    _buf(w1, "w1", (dm, dff), BF16, x)
+    _buf(w2, "w2", (dff, dm), BF16, x)
+    for name, t in (("ln1_gain", ln1_gain), ("ln1_bias", ln1_bias), ("ln2_gain", ln2_gain), ("ln2_bias", ln2_bias)):
+        _buf(t, name, (dm,), BF16, x)
     if out is None:
         out = torch.empty((B, N, dm), dtype=out_dtype, device=x.device)
+    _buf(out, "out", (B, N, dm), FLOATS, x)
     if workspace is None:
         workspace = torch.empty(ret_retnet_block_workspace_bytes(B, N, dm, H, dk, dv, dff), dtype=torch.uint8,
                                 device=x.device)
+    _same_device(x, workspace=workspace)
     nbytes = workspace.numel() * workspace.element_size()
     _check(lib.ret_retnet_block_forward(_ptr(x, "x"), _ptr(ln1_gain, "ln1_gain"), _ptr(ln1_bias, "ln1_bias"),
                                         _ptr(wq, "wq"), _ptr(wk, "wk"), _ptr(wv, "wv"), _ptr(wg, "wg"),
@@ -474,8 +538,10 @@ def ret_linear_bf16(x, w, out=None, out_dtype=torch.bfloat16, stream=None):
         raise ValueError("w must be [K, N]")
     N = w.shape[1]
     M = x.numel() // K
+    _same_device(x, w=w)
     if out is None:
         out = torch.empty((*x.shape[:-1], N), dtype=out_dtype, device=x.device)
+    _buf(out, "out", (*x.shape[:-1], N), FLOATS, x)
     _check(lib.ret_linear_bf16(_ptr(x, "x"), _ptr(w, "w"), _ptr(out, "out"), M, N, K, _dt(out.dtype),
                                _stream(stream)))
     return out
@@ -490,14 +556,14 @@ def ret_msr_forward(x, wq, wk, wv, wg, wo, gammas, H: int, chunk: int = 128, k_s
                     out=None, out_dtype=torch.bfloat16, workspace=None, stream=None):
     """MultiScaleRetention layer forward.  x [B, N, d_model] bf16; weights
     bf16 [in, out]; returns out [B, N, d_model]."""
-    B, N, dm = x.shape
-    dk = wq.shape[1] // H
-    dv = wv.shape[1] // H
+    B, N, dm, dk, dv = _msr_shapes(x, wq, wk, wv, wg, wo, H)
     if out is None:
         out = torch.empty((B, N, dm), dtype=out_dtype, device=x.device)
+    _buf(out, "out", (B, N, dm), FLOATS, x)
     need = ret_msr_workspace_bytes(B, N, dm, H, dk, dv)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _same_device(x, workspace=workspace)
     nbytes = workspace.numel() * workspace.element_size()
     _check(lib.ret_msr_forward(_ptr(x, "x"), _ptr(wq, "wq"), _ptr(wk, "wk"), _ptr(wv, "wv"), _ptr(wg, "wg"),
                                _ptr(wo, "wo"), _gammas(gammas, H), B, N, dm, H, dk, dv, int(chunk), float(k_scale),

@@ -262,3 +262,78 @@ def decode_positions_call(pos=ctypes.c_void_p(0xD0000000), z=ctypes.c_void_p(0xB
 def test_decode_positions_rejects_bad_arguments(kw, status):
     assert decode_positions_call(**kw) == status, (kw, R.ret_last_error_string())
     assert R.ret_last_error_string()
+
+
+# The binding checks every caller-provided buffer (shape, dtype, device)
+# before it marshals a pointer: the C ABI cannot see how large a buffer is.
+# These run on host tensors, so the checks fire before the CUDA-tensor one.
+def _seq(B=1, N=8, H=2, dk=16, dv=8, dt=torch.bfloat16):
+    return (torch.zeros(B, N, H, dk, dtype=dt), torch.zeros(B, N, H, dk, dtype=dt), torch.zeros(B, N, H, dv, dtype=dt))
+
+
+@pytest.mark.parametrize("kw,exc,msg", [
+    (dict(out=torch.zeros(1, 8, 2, 4, dtype=torch.bfloat16)), ValueError, "out must have shape"),
+    (dict(out=torch.zeros(1, 8, 2, 8, dtype=torch.float16)), TypeError, "out must be"),
+    (dict(final_state=torch.zeros(1, 2, 16, 4)), ValueError, "final_state must have shape"),
+    (dict(final_state=torch.zeros(1, 2, 16, 8, dtype=torch.bfloat16)), TypeError, "final_state must be"),
+])
+def test_binding_checks_output_buffers(kw, exc, msg):
+    q, k, v = _seq()
+    for fn in (lambda: R.ret_forward_chunkwise(q, k, v, [0.9, 0.8], 4, **kw),
+               lambda: R.ret_forward_chunkwise_ws(q, k, v, [0.9, 0.8], 4, torch.zeros(16, dtype=torch.uint8), **kw),
+               lambda: R.ret_forward_chunkwise_noalloc(q, k, v, [0.9, 0.8], 4, **kw),
+               lambda: R.ret_forward_recurrent(q, k, v, [0.9, 0.8], **kw)):
+        with pytest.raises(exc, match=msg):
+            fn()
+
+
+def test_binding_checks_initial_state_and_gradients():
+    q, k, v = _seq()
+    ws = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="initial_state must have shape"):
+        R.ret_forward_chunkwise_prepared(q, k, v, [0.9, 0.8], 128, ws, initial_state=torch.zeros(1, 2, 8, 16))
+    with pytest.raises(ValueError, match="dout must have shape"):
+        R.ret_backward_chunkwise(q, k, v, torch.zeros(1, 8, 2, 16, dtype=torch.bfloat16), [0.9, 0.8], 128)
+    with pytest.raises(TypeError, match="dout must be"):
+        R.ret_backward_chunkwise(q, k, v, torch.zeros(1, 8, 2, 8), [0.9, 0.8], 128)
+    with pytest.raises(ValueError, match="dq must have shape"):
+        R.ret_backward_chunkwise(q, k, v, torch.zeros(1, 8, 2, 8, dtype=torch.bfloat16), [0.9, 0.8], 128,
+                                 workspace=ws, dq=torch.zeros(1, 8, 2, 8))
+    with pytest.raises(ValueError, match="final_z must have shape"):
+        R.ret_forward_chunkwise_normalized(q, k, v, [0.9, 0.8], 128, workspace=ws, final_z=torch.zeros(1, 2, 8))
+
+
+def test_binding_checks_decode_buffers():
+    q, k, v = torch.zeros(3, 2, 16), torch.zeros(3, 2, 16), torch.zeros(3, 2, 8)
+    S = torch.zeros(3, 2, 16, 8)
+    with pytest.raises(ValueError, match="state must have shape"):
+        R.ret_decode_step(q, k, v, [0.9, 0.8], torch.zeros(3, 2, 8, 16))
+    with pytest.raises(TypeError, match="state must be"):
+        R.ret_decode_step(q, k, v, [0.9, 0.8], S.double())
+    with pytest.raises(ValueError, match="out must have shape"):
+        R.ret_decode_step(q, k, v, [0.9, 0.8], S, out=torch.zeros(3, 2, 16))
+    with pytest.raises(ValueError, match="z must have shape"):
+        R.ret_decode_step_normalized(q, k, v, [0.9, 0.8], S, torch.zeros(3, 16), 5)
+    with pytest.raises(TypeError, match="positions must be"):
+        R.ret_decode_step_positions(q, k, v, [0.9, 0.8], S, torch.zeros(3, dtype=torch.int32))
+    with pytest.raises(ValueError, match="positions must have shape"):
+        R.ret_decode_step_positions(q, k, v, [0.9, 0.8], S, torch.zeros(2, dtype=torch.int64))
+    with pytest.raises(TypeError, match="share a dtype"):
+        R.ret_decode_step(q, k.bfloat16(), v, [0.9, 0.8], S)
+
+
+def test_binding_checks_layer_weights():
+    B, N, dm, H, dk, dv = 1, 8, 32, 2, 16, 8
+    x = torch.zeros(B, N, dm, dtype=torch.bfloat16)
+    w = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    good = dict(wq=w(dm, H * dk), wk=w(dm, H * dk), wv=w(dm, H * dv), wg=w(dm, H * dv), wo=w(H * dv, dm))
+    for name, bad in (("wk", w(dm, H * dk + 2)), ("wg", w(dm, H * dk)), ("wo", w(dm, H * dv))):
+        ws = dict(good, **{name: bad})
+        with pytest.raises(ValueError, match=f"{name} must have shape"):
+            R.ret_msr_forward(x, ws["wq"], ws["wk"], ws["wv"], ws["wg"], ws["wo"], [0.9, 0.8], H)
+    with pytest.raises(ValueError, match="w2 must have shape"):
+        R.ret_retnet_block_forward(x, *good.values(), w(dm, 64), w(64, dm + 8), [0.9, 0.8], H)
+    with pytest.raises(ValueError, match="ln1_gain must have shape"):
+        R.ret_retnet_block_forward(x, *good.values(), w(dm, 64), w(64, dm), [0.9, 0.8], H, ln1_gain=w(dm + 1))
+    with pytest.raises(ValueError, match="x must be bfloat16"):
+        R.ret_msr_forward(x.float(), *good.values(), [0.9, 0.8], H)
