@@ -64,6 +64,12 @@ def flops_per_token_head(chunk, dk, dv):
     return 2 * chunk * dk + 2 * chunk * dv + 4 * dk * dv
 
 
+def flops_per_token_head_causal(chunk, dk, dv):
+    """The same count with only the causal half of each chunk's score block:
+    C replaced by (C + 1) / 2 in the two intra-chunk terms."""
+    return (chunk + 1) * dk + (chunk + 1) * dv + 4 * dk * dv
+
+
 def algo_bytes(w, out_bytes=2):
     """Read q, k, v once, write out once, write the final fp32 state once."""
     tok = w["B"] * w["N"] * w["H"]
@@ -261,6 +267,9 @@ def run_ours(args):
     roof["algo_flops"] = flops
     roof["algo_bytes"] = nbytes
     roof["tensor_tflops"] = round(tflops, 1)
+    flops_causal = flops_per_token_head_causal(C, dk, dv) * B * N * H
+    roof["algo_flops_causal"] = flops_causal
+    roof["tensor_tflops_causal"] = round(flops_causal / t_main / 1e12, 1)
     roof["tensor_frac"] = round(tflops / peaks["bf16_tflops"], 4)
     roof["hbm_gbs"] = round(gbs, 1)
     roof["hbm_frac"] = round(gbs / peaks["hbm_gbs"], 4)
@@ -273,7 +282,8 @@ def run_ours(args):
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "ms_per_step_median": round(statistics.median(times), 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1); q, k scaled by d_k^-0.5)",
         "config": {"workload": w["workload"], "B": B, "N": N, "H": H, "dk": dk, "dv": dv, "chunk": C, "xpos": True,
                    "out_dtype": "bf16", "final_state": True, "global_batch": B * world, "seq_len": N,
@@ -637,7 +647,7 @@ def bench_fp32_small(R, torch, dev, stream, args, world, dist):
 
 # ---------------------------------------------------------- the oracle ---
 
-def oracle_sample(w, heads, n_tok):
+def oracle_sample(w, heads, n_tok, nthreads=0):
     """One bounded oracle run: ``heads`` heads of the workload over the first
     ``n_tok`` tokens (rotation + recurrent definition, fp64, all host cores).
     Returns (seconds, tokens of the full workload this sample stands for)."""
@@ -651,7 +661,7 @@ def oracle_sample(w, heads, n_tok):
     v = rng.standard_normal((B, n_tok, heads, dv))
     g = np.array(gammas(w["H"])[:heads])
     t0 = time.perf_counter()
-    oracle.retention_recurrent(oracle.xpos_rotate(q), oracle.xpos_rotate(k), v, g)
+    oracle.retention_recurrent(oracle.xpos_rotate(q), oracle.xpos_rotate(k), v, g, nthreads=nthreads)
     dt = time.perf_counter() - t0
     return dt, B * n_tok * heads / w["H"]
 
@@ -663,9 +673,15 @@ def cpu_baseline(w, budget_s=20.0):
     dt, tok = oracle_sample(w, heads, 256)           # calibrate
     n = int(min(w["N"], max(256, 256 * budget_s / max(dt, 1e-3))))
     dt, tok = oracle_sample(w, heads, n)
+    # one host core: one head, a few seconds of work
+    d1, t1 = oracle_sample(w, 1, 256, nthreads=1)
+    n1 = int(min(w["N"], max(256, 256 * (budget_s / 5) / max(d1, 1e-3))))
+    d1, t1 = oracle_sample(w, 1, n1, nthreads=1)
     return {"value": round(tok / dt, 2), "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{heads} of {w['H']} heads x first {n} of {w['N']} tokens, fp64 recurrent definition "
-                      f"with xPos, {dt:.1f} s; value scaled to tokens of the full workload"}
+                      f"with xPos, {dt:.1f} s; value scaled to tokens of the full workload",
+            "single_core": {"value": round(t1 / d1, 2), "unit": UNIT, "cores": 1,
+                            "sample": f"1 head x first {n1} tokens, {d1:.1f} s; scaled to the full workload"}}
 
 
 def run_reference(args):
