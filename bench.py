@@ -31,7 +31,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 WORKLOAD = dict(workload="retention_bf16_1x8192x16x256x512", B=1, N=8192, H=16, dk=256, dv=512, chunk=128)
-DECODE = dict(workload="decode_bf16_64x16x256x512", B=64, H=16, dk=256, dv=512, prefill=1024, chunk=128)
+DECODE = dict(workload="decode_bf16_64x16x256x512", B=64, H=16, dk=256, dv=512, prefill=1024, chunk=128, steps=512)
 METRIC = "chunkwise retention fwd tokens/s"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
@@ -411,12 +411,45 @@ def bench_decode(R, torch, dev, stream, args, peaks, world, barrier, dist, rank)
         evs[i][1].record(stream)
     torch.cuda.synchronize()
     R.ret_check_device_error()
-    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    per_step = [a.elapsed_time(b) for a, b in evs]
+    ms = statistics.mean(per_step)
     ms = max_over_ranks(ms, world, dist, dev)
+    # The workload's whole generation loop: 512 steps back to back after the
+    # prefill, timed as one region, eagerly and replayed from a CUDA graph.
+    loop = d["steps"]
+
+    def run_loop(st):
+        for i in range(loop):
+            R.ret_decode_step(sq[i % pool], sk[i % pool], sv[i % pool], g, state, out=so, stream=st)
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run_loop(stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    loop_ms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        run_loop(None)  # the capturing stream
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    R.ret_check_device_error()
+    graph_ms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
+    del graph
     nbytes = 2 * B * H * dk * dv * 4 + B * H * (2 * dk * 2 + dv * 2 + dv * 4)
     gbs = nbytes / (ms / 1e3) / 1e9
     return {"workload": d["workload"], "metric": "decode-step state HBM GB/s", "value": round(gbs * world, 1),
-            "unit": "GB/s", "ms_per_step": round(ms, 4), "steps": steps, "bytes_per_step": nbytes,
+            "unit": "GB/s", "ms_per_step": round(ms, 4), "ms_per_step_median": round(statistics.median(per_step), 4),
+            "steps": steps, "bytes_per_step": nbytes,
+            "loop": {"steps": loop, "ms_total": round(loop_ms, 3), "ms_total_graph": round(graph_ms, 3),
+                     "ms_per_step": round(loop_ms / loop, 4), "ms_per_step_graph": round(graph_ms / loop, 4)},
             "tokens_per_s": round(world * B / (ms / 1e3), 1),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "kernel": "k_decode_step",
