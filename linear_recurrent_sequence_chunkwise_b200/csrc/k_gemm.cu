@@ -99,21 +99,31 @@ __device__ __forceinline__ void epi_store(const GemmEpilogue& e, int seg, int m,
         } else {
             mult = o.scale;
         }
+        // (cos, sin) of the 16 pairs: from the per-call table, two pairs per
+        // 16-byte load (the row's 16 pairs are 128 contiguous bytes, 128-byte
+        // aligned since d0 is a multiple of 32), else evaluated here
+        float csv[16], snv[16];
+        if (e.xpos && e.rot_cs) {
+            const float4* t4 = reinterpret_cast<const float4*>(e.rot_cs + (size_t)n * (o.head_dim >> 1) + (d0 >> 1));
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const float4 t = __ldg(t4 + i);
+                csv[2 * i] = t.x;
+                snv[2 * i] = t.y;
+                csv[2 * i + 1] = t.z;
+                snv[2 * i + 1] = t.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                csv[i] = 1.f;
+                snv[i] = 0.f;
+                if (e.xpos) sincosf(rot_angle(e.pos_offset + n, theta[(d0 >> 1) + i]), &snv[i], &csv[i]);
+            }
+        }
 #pragma unroll
         for (int i = 0; i < 16; i++) {
-            const int pidx = (d0 >> 1) + i;
-            float sn = 0.f, cs = 1.f;
-            if (e.xpos) {
-                if (e.rot_cs) {
-                    const float2 t = e.rot_cs[(size_t)n * (o.head_dim >> 1) + pidx];
-                    cs = t.x;
-                    sn = t.y;
-                } else {
-                    sincosf(rot_angle(e.pos_offset + n, theta[pidx]), &sn, &cs);
-                }
-            }
-            cs *= mult;
-            sn *= mult;
+            const float cs = csv[i] * mult, sn = snv[i] * mult;
             const float x0 = v[2 * i], x1 = v[2 * i + 1];
             w[2 * i] = x0 * cs - x1 * sn;
             w[2 * i + 1] = x0 * sn + x1 * cs;
