@@ -40,14 +40,15 @@ constexpr int kABytes = BM * BK * 2;   // 16 KB
 constexpr int kBBytes = BK * BN * 2;   // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kThreads = 320;          // TMA warp, MMA warp, two epilogue warpgroups
-constexpr int kSmemBytes = kStages * kStageBytes + 1024;
-
-constexpr int kMaxRotPairs = 256;  // rotated head width up to 512
+// Output staging: per epilogue warpgroup one 128-row box of 128-byte rows
+// (64 bf16 or 32 fp32 columns) in the TMA's 128-byte swizzle.
+constexpr int kOutBoxBytes = BM * 128;   // 16 KB
+constexpr int kSmemBytes = kStages * kStageBytes + 2 * kOutBoxBytes + 1024;
 
 struct GemmParams {
-    int rot_pairs;  // pairs of a rotated head (head_dim / 2), 0 without rotation
     CUtensorMap ta;
     CUtensorMap tb[4];
+    CUtensorMap to[4];   // each segment's output [M, N_seg], box 128 rows x 128 bytes
     int M, K;
     int nseg;
     int seg_n0[5];       // global column where segment s starts; seg_n0[nseg] = total N
@@ -75,20 +76,25 @@ __device__ __forceinline__ float swish(float x) { return x / (1.f + expf(-x)); }
 // gelu(x) = x Phi(x) with the exact normal CDF, Phi(x) = (1 + erf(x / sqrt 2)) / 2.
 __device__ __forceinline__ float gelu(float x) { return 0.5f * x * (1.f + erff(x * 0.70710678118654752f)); }
 
-// Store 32 consecutive fp32 values of row m, starting at segment column c0.
-// theta: the rotation frequencies theta_p of the rotated segments' heads,
-// one per pair (shared memory, filled once per CTA).
-__device__ __forceinline__ void epi_store(const GemmEpilogue& e, int seg, int m, int c0, const float (&v)[32],
-                                          int ncols_valid, const double* theta) {
+// The 32 epilogue values of row m at segment column c0 (ncols_valid of them
+// inside the segment; the rest, and rows past M, are zero).  Rotations use
+// the per-call (cos, sin) table, two pairs per 16-byte load (a row's 16
+// pairs are 128 contiguous bytes, 128-byte aligned since c0 is a multiple of
+// 32 within its head).
+__device__ __forceinline__ void epi_values(const GemmEpilogue& e, int seg, int m, int c0, const float (&v)[32],
+                                           int ncols_valid, float (&w)[32]) {
     const GemmSegOut& o = e.seg[seg];
-    if (m >= e.M) return;
+    if (m >= e.M) {
+#pragma unroll
+        for (int i = 0; i < 32; i++) w[i] = 0.f;
+        return;
+    }
     if (o.kind == kEpiRotate || o.kind == kEpiRotateScaleZeta) {
         // xPos rotation of consecutive pairs within a head of width o.head_dim
         // at position pos_offset + (m % seq), then (keys) the scale and zeta
         // of the row's place in its chunk.
         const int n = m % e.seq;
-        float w[32];
-        float mult = 1.f;
+        float mult = o.scale;
         const int d0 = c0 % o.head_dim;
         const int hh = c0 / o.head_dim;
         if (o.kind == kEpiRotateScaleZeta) {
@@ -96,14 +102,9 @@ __device__ __forceinline__ void epi_store(const GemmEpilogue& e, int seg, int m,
             const int L = min(e.chunk, e.seq - (n - r));
             // zeta = gamma^(L-1-r): the exponent in fp64, exp2 in fp32 (relative error ~1e-7)
             mult = o.scale * exp2f((float)((double)(L - 1 - r) * e.log2g[hh]));
-        } else {
-            mult = o.scale;
         }
-        // (cos, sin) of the 16 pairs: from the per-call table, two pairs per
-        // 16-byte load (the row's 16 pairs are 128 contiguous bytes, 128-byte
-        // aligned since d0 is a multiple of 32), else evaluated here
         float csv[16], snv[16];
-        if (e.xpos && e.rot_cs) {
+        if (e.xpos) {
             const float4* t4 = reinterpret_cast<const float4*>(e.rot_cs + (size_t)n * (o.head_dim >> 1) + (d0 >> 1));
 #pragma unroll
             for (int i = 0; i < 8; i++) {
@@ -118,7 +119,6 @@ __device__ __forceinline__ void epi_store(const GemmEpilogue& e, int seg, int m,
             for (int i = 0; i < 16; i++) {
                 csv[i] = 1.f;
                 snv[i] = 0.f;
-                if (e.xpos) sincosf(rot_angle(e.pos_offset + n, theta[(d0 >> 1) + i]), &snv[i], &csv[i]);
             }
         }
 #pragma unroll
@@ -128,20 +128,7 @@ __device__ __forceinline__ void epi_store(const GemmEpilogue& e, int seg, int m,
             w[2 * i] = x0 * cs - x1 * sn;
             w[2 * i + 1] = x0 * sn + x1 * cs;
         }
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(o.ptr) + (size_t)m * o.ld + c0;
-#pragma unroll
-        for (int c = 0; c < 4; c++) {
-            uint4 u;
-            u.x = tc::pack_bf16x2(w[8 * c + 0], w[8 * c + 1]);
-            u.y = tc::pack_bf16x2(w[8 * c + 2], w[8 * c + 3]);
-            u.z = tc::pack_bf16x2(w[8 * c + 4], w[8 * c + 5]);
-            u.w = tc::pack_bf16x2(w[8 * c + 6], w[8 * c + 7]);
-            reinterpret_cast<uint4*>(dst)[c] = u;
-        }
-        return;
-    }
-    float w[32];
-    if (o.kind == kEpiSwish) {
+    } else if (o.kind == kEpiSwish) {
 #pragma unroll
         for (int i = 0; i < 32; i++) w[i] = swish(v[i]);
     } else if (o.kind == kEpiGelu) {
@@ -159,41 +146,36 @@ __device__ __forceinline__ void epi_store(const GemmEpilogue& e, int seg, int m,
                 const uint4 u = reinterpret_cast<const uint4*>(r)[c];
                 const __nv_bfloat162* hp = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-                for (int e = 0; e < 4; e++) {
-                    const float2 f = __bfloat1622float2(hp[e]);
-                    w[8 * c + 2 * e] += f.x;
-                    w[8 * c + 2 * e + 1] += f.y;
+                for (int e2 = 0; e2 < 4; e2++) {
+                    const float2 f = __bfloat1622float2(hp[e2]);
+                    w[8 * c + 2 * e2] += f.x;
+                    w[8 * c + 2 * e2 + 1] += f.y;
                 }
             }
         } else {
             for (int i = 0; i < ncols_valid; i++) w[i] += __bfloat162float(r[i]);
         }
     }
-    if (o.dtype == RET_F32) {
-        float* dst = reinterpret_cast<float*>(o.ptr) + (size_t)m * o.ld + c0;
-        if (ncols_valid >= 32) {
+    if (ncols_valid < 32)
 #pragma unroll
-            for (int c = 0; c < 8; c++)
-                reinterpret_cast<float4*>(dst)[c] = make_float4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-        } else {
-            for (int i = 0; i < ncols_valid; i++) dst[i] = w[i];
-        }
-    } else {
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(o.ptr) + (size_t)m * o.ld + c0;
-        if (ncols_valid >= 32) {
-#pragma unroll
-            for (int c = 0; c < 4; c++) {
-                uint4 u;
-                u.x = tc::pack_bf16x2(w[8 * c + 0], w[8 * c + 1]);
-                u.y = tc::pack_bf16x2(w[8 * c + 2], w[8 * c + 3]);
-                u.z = tc::pack_bf16x2(w[8 * c + 4], w[8 * c + 5]);
-                u.w = tc::pack_bf16x2(w[8 * c + 6], w[8 * c + 7]);
-                reinterpret_cast<uint4*>(dst)[c] = u;
-            }
-        } else {
-            for (int i = 0; i < ncols_valid; i++) dst[i] = __float2bfloat16_rn(w[i]);
-        }
-    }
+        for (int i = 0; i < 32; i++)
+            if (i >= ncols_valid) w[i] = 0.f;
+}
+
+// Named barrier of one epilogue warpgroup (ids 1 and 2; 0 is __syncthreads),
+// and the same barrier returning whether x holds in all 128 threads.
+__device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory"); }
+__device__ __forceinline__ bool wg_all(int wg, bool x) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, %2, 128, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)x), "r"(1 + wg)
+        : "memory");
+    return r != 0;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ GemmParams p) {
@@ -202,7 +184,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
     __shared__ GBars bars;
     __shared__ uint32_t s_tmem;
     __shared__ int s_fail;
-    __shared__ double s_theta[kMaxRotPairs];  // theta_p = base^(-2p/head_dim) of the rotated segments
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tiles_m = (p.M + BM - 1) / BM;
     const int ntiles = tiles_m * p.tiles_n;
@@ -223,7 +204,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
         for (int s = 0; s < p.nseg; s++) tc::prefetch_tmap(&p.tb[s]);
     }
     if (warp == 1) tc::tmem_alloc(&s_tmem, 512);
-    for (int i = tid; i < p.rot_pairs; i += kThreads) s_theta[i] = exp2(-2.0 * i / (2 * p.rot_pairs) * p.epi.log2base);
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
@@ -276,33 +256,84 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm(const __grid_constant__ Ge
             }
         }
     } else {
+        // Epilogue warpgroups: warps 2-5 and 6-9, each on TMEM lanes 0..127
+        // (a warp reaches the lane quarter warp % 4), one 128-column half of
+        // the accumulator each.  Every 32 columns: TMEM -> registers, the
+        // segment's epilogue, then the values into the warpgroup's staging
+        // box (128 rows of 128 bytes: 64 bf16 or 32 fp32 columns, 128-byte
+        // swizzle); a full box goes out in one TMA store (rows past M and
+        // columns past the segment are clipped by the TMA).  The warpgroup
+        // agrees on every wait's outcome before any of its barriers, so a
+        // timed-out wait cannot leave part of it at a barrier.
         const int quarter = warp & 3, wg = (warp - 2) >> 2;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const bool leader = warp == 2 + 4 * wg && lane == 0;  // issues the warpgroup's stores
+        uint8_t* box = sm + kStages * kStageBytes + wg * kOutBoxBytes;
+        const uint32_t r = (uint32_t)(quarter * 32 + lane);   // row in the tile
         int tl = 0;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, tl++) {
             int tm, tn, seg;
             tile_coords(p, t, tm, tn, seg);
             const int ab = tl & 1;
-            ok = tc::mbar_wait(&bars.accfull[ab], (tl >> 1) & 1);
+            ok = wg_all(wg, tc::mbar_wait(&bars.accfull[ab], (tl >> 1) & 1));
             if (!ok) break;
             tc::tc_fence_after();
-            const int m = tm * BM + quarter * 32 + lane;
+            const int m = tm * BM + (int)r;
             const int seg_cols = p.seg_n0[seg + 1] - p.seg_n0[seg];
+            const bool f32 = p.epi.seg[seg].dtype == RET_F32;
             for (int c = 0; c < 4; c++) {
                 const int col = 128 * wg + 32 * c;
-                uint32_t r[32];
-                tc::tmem_ld32(tbase + lane_off + 256 * ab + col, r);
+                uint32_t rr[32];
+                tc::tmem_ld32(tbase + lane_off + 256 * ab + col, rr);
                 tc::tmem_ld_wait();
-                float v[32];
+                float v[32], w[32];
 #pragma unroll
-                for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
+                for (int i = 0; i < 32; i++) v[i] = __uint_as_float(rr[i]);
                 const int c0 = (tn - p.seg_tile0[seg]) * BN + col;  // column within the segment
-                if (c0 < seg_cols) epi_store(p.epi, seg, m, c0, v, seg_cols - c0, s_theta);
+                if (c0 < seg_cols) {
+                    epi_values(p.epi, seg, m, c0, v, seg_cols - c0, w);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; i++) w[i] = 0.f;
+                }
+                // a box starts at every chunk (fp32) or every even chunk (bf16)
+                const bool first = f32 || (c & 1) == 0, last = f32 || (c & 1) == 1;
+                if (first) {
+                    if (leader) tc::bulk_wait_group_read<0>();  // the previous box has been read
+                    wg_sync(wg);
+                }
+                if (f32) {
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; c4++)
+                        *reinterpret_cast<float4*>(box + tc::sw128_off(r, (uint32_t)c4)) =
+                            make_float4(w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]);
+                } else {
+                    const uint32_t h = (uint32_t)(c & 1);  // half of the 128-byte row
+#pragma unroll
+                    for (int c16 = 0; c16 < 4; c16++) {
+                        uint4 u;
+                        u.x = tc::pack_bf16x2(w[8 * c16 + 0], w[8 * c16 + 1]);
+                        u.y = tc::pack_bf16x2(w[8 * c16 + 2], w[8 * c16 + 3]);
+                        u.z = tc::pack_bf16x2(w[8 * c16 + 4], w[8 * c16 + 5]);
+                        u.w = tc::pack_bf16x2(w[8 * c16 + 6], w[8 * c16 + 7]);
+                        *reinterpret_cast<uint4*>(box + tc::sw128_off(r, 4 * h + (uint32_t)c16)) = u;
+                    }
+                }
+                if (last) {
+                    tc::fence_proxy_async_smem();
+                    wg_sync(wg);
+                    const int x0 = f32 ? c0 : c0 - 32;  // the box's first column
+                    if (leader && x0 < seg_cols) {
+                        tc::tma_store_2d(&p.to[seg], box, x0, tm * BM);
+                        tc::bulk_commit_group();
+                    }
+                }
             }
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bars.accempty[ab]);
         }
+        if (leader) tc::bulk_wait_group<0>();  // every box is in global memory
     }
     if (!ok) atomicExch(&s_fail, 1);
     tc::tc_fence_before();
@@ -341,14 +372,18 @@ ret_status launch_gemm(const void* A, int M, int K, const GemmSegment* segs, int
     p.tiles_n = t0;
     p.epi = epi;
     p.epi.M = M;
-    p.rot_pairs = 0;
     for (int i = 0; i < nseg; i++) {
         const GemmSegOut& o = epi.seg[i];
-        if (epi.xpos && (o.kind == kEpiRotate || o.kind == kEpiRotateScaleZeta)) {
-            if (o.head_dim < 2 || o.head_dim / 2 > kMaxRotPairs || (p.rot_pairs && p.rot_pairs != o.head_dim / 2))
-                return fail(RET_ERR_UNSUPPORTED, "gemm: rotated heads of different widths or wider than 512");
-            p.rot_pairs = o.head_dim / 2;
-        }
+        if (epi.xpos && (o.kind == kEpiRotate || o.kind == kEpiRotateScaleZeta) &&
+            (!epi.rot_cs || o.head_dim < 32 || o.head_dim % 32))
+            return fail(RET_ERR_UNSUPPORTED, "gemm: rotated heads need the (cos, sin) table and a width multiple of 32");
+        // output map: [M, N_seg] with row pitch ld, box 128 rows x 128 bytes
+        const bool f32 = o.dtype == RET_F32;
+        const uint64_t dout[2] = {(uint64_t)segs[i].N, (uint64_t)M};
+        const uint64_t sout[1] = {(uint64_t)o.ld * (f32 ? 4 : 2)};
+        const uint32_t bout[2] = {f32 ? 32u : 64u, (uint32_t)BM};
+        if (!(f32 ? make_tmap_f32 : make_tmap_bf16)(&p.to[i], o.ptr, 2, dout, sout, bout, CU_TENSOR_MAP_SWIZZLE_128B))
+            return RET_ERR_CUDA;
     }
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);

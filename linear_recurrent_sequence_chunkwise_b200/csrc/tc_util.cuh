@@ -271,6 +271,13 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void*
                  : "memory");
 }
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(smem_src)), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
 // Shared memory -> global tensor reduction: the tile is added element-wise
 // into global memory (fp32 adds), in the issuing thread's bulk group.
 __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* smem_src, int c0, int c1, int c2,
