@@ -24,7 +24,7 @@ struct GemmSegOut {
     void* ptr;          // [M, ld] row-major destination of this segment
     int ld;             // leading dimension (elements)
     int kind;           // kEpi*
-    ret_dtype dtype;    // kEpiStore / kEpiSwish: RET_F32 or RET_BF16; rotations write bf16
+    ret_dtype dtype;    // RET_F32 or RET_BF16 (rotations: bf16); ld * element size a multiple of 16 bytes
     float scale;
     int head_dim;       // rotations: width of a head (pairs rotate within it)
     const __nv_bfloat16* res;  // kEpiResidual: [M, res_ld] bf16 added to the result
@@ -40,7 +40,8 @@ struct GemmEpilogue {
     long long pos_offset;
     double log2base;        // log2(theta_base)
     // Rotations: (cos, sin) of every (token, pair) at position pos_offset +
-    // token, [seq][head_dim / 2] fp32, or null (computed in the epilogue).
+    // token, [seq][head_dim / 2] fp32, 16-byte aligned; required when xpos
+    // rotates a segment (head_dim a multiple of 32).
     const float2* rot_cs;
     double log2g[kMaxHeads];
 };

@@ -8,8 +8,9 @@
 // weight as stored, an MN-major operand).  Tiles 128 x 256 x 64, a 4-stage
 // TMA ring (48 KB per stage), one tcgen05.mma issuer, two 256-column fp32
 // accumulators in TMEM so that the epilogue of one tile overlaps the MMAs of
-// the next, and two epilogue warpgroups (128 columns each).  The grid is
-// persistent (one CTA per SM) and walks the tiles M-fastest.
+// the next, and two epilogue warpgroups (128 columns each) that stage each
+// 128-row output box in shared memory and store it with one TMA store.  The
+// grid is persistent (one CTA per SM) and walks the tiles M-fastest.
 //
 // The B operand may be split into up to four column segments, each with its
 // own tensor map and its own epilogue destination: that is how one launch
