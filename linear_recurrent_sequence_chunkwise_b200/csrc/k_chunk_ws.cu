@@ -23,7 +23,8 @@
 //      warp 1  tensor pipe, first issuer (one elected lane), per chunk j
 //                A  = Q K'^T          (Q from TMEM, K' from smem), part by part,
 //                O  = Q T             (read-out of the state before chunk j),
-//                O += P V             (P from TMEM);
+//                O += P V             (P from TMEM; each operand behind its
+//                                      own barrier, V's TMA barrier included);
 //      warp 3  tensor pipe, second issuer: the state update dS = K'^T V of
 //              each K' part, beside warp 1's stream (each K' slot is free
 //              once both issuers have read it);
