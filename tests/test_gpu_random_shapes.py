@@ -144,3 +144,33 @@ def test_random_decode(i):
     tol = TOL_F32 if dt == "f32" else TOL_BF16
     assert err_out(got, ref) < tol, c
     assert err_state(host64(S), Sref) < tol, c
+
+
+@pytest.mark.parametrize("n0,dt", [(77, "bf16"), (128, "bf16"), (300, "bf16"), (41, "f32")])
+def test_no_causal_leakage(n0, dt):
+    """Outputs before token n0 do not depend on tokens n0 and later: new
+    values from n0 on leave them bit for bit the same (the masked scores are
+    exact zeros, so the later keys and values add exact zeros), on the
+    tensor-core workspace path (bf16) and on the fp32 CUDA-core path."""
+    B, N, H = 2, 400, 2
+    dk, dv = (256, 128) if dt == "bf16" else (16, 16)
+    mk = lambda seed, st, d: make_tensor(seed, st, (B, N, H, d), dt, dk ** -0.5 if st < 3 else 1.0)
+    q, k, v = mk(800, 1, dk), mk(800, 2, dk), mk(800, 3, dv)
+    q2, k2, v2 = mk(801, 1, dk), mk(801, 2, dk), mk(801, 3, dv)
+    g = gamma_schedule(H)
+    outs = []
+    for tens in ((q, k, v), (q2, k2, v2)):
+        qd, kd, vd = (dev(t) for t in (q, k, v))
+        if tens[0] is q2:   # tokens from n0 on replaced by other values
+            for a, b in zip((qd, kd, vd), (dev(q2), dev(k2), dev(v2))):
+                a[:, n0:] = b[:, n0:]
+        if dt == "bf16":
+            nb = R.ret_chunkwise_workspace_bytes(B, N, H, dk, dv, 128, torch.bfloat16, True)
+            ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+            outs.append(R.ret_forward_chunkwise_ws(qd, kd, vd, g, 128, ws, out_dtype=torch.float32, xpos=True))
+        else:
+            outs.append(R.ret_forward_chunkwise(qd, kd, vd, g, 16, out_dtype=torch.float32))
+    torch.cuda.synchronize()
+    R.ret_check_device_error()
+    assert torch.equal(outs[0][:, :n0], outs[1][:, :n0])
+    assert not torch.equal(outs[0][:, n0:], outs[1][:, n0:])
