@@ -132,7 +132,37 @@ def _block_residual_of_the_normed_input(x, wq, wk, wv, wg, wo, w1, w2, gammas, H
     return (out, y) if return_y else out
 
 
+def _msr_without_rotation(x, wq, wk, wv, wg, wo, gammas, H, k_scale, eps, theta_base=10000.0, heads=None,
+                          return_parts=False):
+    """msr_forward with the xPos rotation of Q and K left out."""
+    x = np.asarray(x, np.float64)
+    B, N, _ = x.shape
+    dk, dv = wq.shape[1] // H, wv.shape[1] // H
+    q = omsr.project(x, wq).reshape(B, N, H, dk)
+    k = omsr.project(x, wk).reshape(B, N, H, dk) * k_scale
+    v = omsr.project(x, wv).reshape(B, N, H, dv)
+    ret, _ = oracle.retention_recurrent(q, k, v, np.asarray(gammas, np.float64))
+    z = omsr.swish(omsr.project(x, wg).reshape(B, N, H, dv)) * omsr.group_norm_heads(ret, eps)
+    return omsr.project(z.reshape(B, N, H * dv), wo)
+
+
+def _msr_gate_before_group_norm(x, wq, wk, wv, wg, wo, gammas, H, k_scale, eps, theta_base=10000.0, heads=None,
+                                return_parts=False):
+    """msr_forward with the swish gate applied before the GroupNorm."""
+    x = np.asarray(x, np.float64)
+    B, N, _ = x.shape
+    dk, dv = wq.shape[1] // H, wv.shape[1] // H
+    q = oracle.xpos_rotate(omsr.project(x, wq).reshape(B, N, H, dk), 0, theta_base)
+    k = oracle.xpos_rotate(omsr.project(x, wk).reshape(B, N, H, dk) * k_scale, 0, theta_base)
+    v = omsr.project(x, wv).reshape(B, N, H, dv)
+    ret, _ = oracle.retention_recurrent(q, k, v, np.asarray(gammas, np.float64))
+    z = omsr.group_norm_heads(omsr.swish(omsr.project(x, wg).reshape(B, N, H, dv)) * ret, eps)
+    return omsr.project(z.reshape(B, N, H * dv), wo)
+
+
 PY_MUTANTS = {
+    "msr_rotation_dropped": ("msr_forward", _msr_without_rotation),
+    "msr_gate_before_group_norm": ("msr_forward", _msr_gate_before_group_norm),
     "layer_norm_unbiased_variance": ("layer_norm", _ln_unbiased),
     "gelu_tanh_approximation": ("gelu", _gelu_tanh),
     "block_post_norm": ("retnet_block", _block_post_norm),

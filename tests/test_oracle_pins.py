@@ -317,6 +317,58 @@ def test_msr_layer_invariants():
     np.testing.assert_allclose(out, z.reshape(1, 10, H * dv) @ W["wo"], atol=1e-12)
 
 
+def test_msr_layer_brute_force_tiny():
+    """The MSR layer written out step by step with loops on a tiny case,
+    without calling msr_forward (P1 section 9.1, section 8.4 and the summary's
+    "Gated Multi-Scale Retention"): projections as explicit sums, the xPos
+    rotation of each consecutive pair by n theta_p with its own cos / sin
+    (P1 sections 6.6-6.8), retention through the pinned recurrent definition,
+    GroupNorm per (token, head) over d_v, then swish(G) times it, then W_O."""
+    rng = np.random.default_rng(17)
+    B, N, dm, H, dk, dv = 1, 7, 6, 2, 4, 3
+    x = rng.standard_normal((B, N, dm))
+    W = dict(wq=rng.standard_normal((dm, H * dk)), wk=rng.standard_normal((dm, H * dk)),
+             wv=rng.standard_normal((dm, H * dv)), wg=rng.standard_normal((dm, H * dv)),
+             wo=rng.standard_normal((H * dv, dm)))
+    g = np.array([0.8, 0.95])
+    k_scale, eps, base = 0.5, 1e-5, 10000.0
+
+    def proj(w, n, j):
+        return sum(x[0, n, i] * w[i, j] for i in range(dm))
+
+    def rotated(vec, n):
+        out = list(vec)
+        for p in range(dk // 2):
+            ang = n * base ** (-2.0 * p / dk)
+            c, s = math.cos(ang), math.sin(ang)
+            x0, x1 = vec[2 * p], vec[2 * p + 1]
+            out[2 * p], out[2 * p + 1] = x0 * c - x1 * s, x0 * s + x1 * c
+        return out
+
+    q = np.zeros((1, N, H, dk)); k = np.zeros((1, N, H, dk))
+    v = np.zeros((1, N, H, dv)); gate = np.zeros((N, H, dv))
+    for n in range(N):
+        for h in range(H):
+            q[0, n, h] = rotated([proj(W["wq"], n, h * dk + i) for i in range(dk)], n)
+            k[0, n, h] = rotated([k_scale * proj(W["wk"], n, h * dk + i) for i in range(dk)], n)
+            for j in range(dv):
+                v[0, n, h, j] = proj(W["wv"], n, h * dv + j)
+                gj = proj(W["wg"], n, h * dv + j)
+                gate[n, h, j] = gj / (1.0 + math.exp(-gj))
+    ret, _ = oracle.retention_recurrent(q, k, v, g)
+    z = np.zeros((N, H * dv))
+    for n in range(N):
+        for h in range(H):
+            row = ret[0, n, h]
+            mu = sum(row) / dv
+            var = sum((r - mu) ** 2 for r in row) / dv
+            for j in range(dv):
+                z[n, h * dv + j] = gate[n, h, j] * (row[j] - mu) / math.sqrt(var + eps)
+    want = np.array([[sum(z[n, c] * W["wo"][c, o] for c in range(H * dv)) for o in range(dm)] for n in range(N)])
+    got = omsr.msr_forward(x, **W, gammas=g, H=H, k_scale=k_scale, eps=eps, theta_base=base)
+    np.testing.assert_allclose(got[0], want, rtol=1e-10, atol=1e-10)
+
+
 # ---- gradients of the definition (oracle.retention_backward)
 
 def _loss(q, k, v, dout, g, xpos, off):
