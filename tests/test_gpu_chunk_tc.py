@@ -59,9 +59,9 @@ def test_chunkwise_tc_small(B, N, H, dk, dv, xpos, off, out_dtype):
     R.ret_check_device_error()
     qr, kr = rotated(q, k, xpos, off)
     ref, S = oracle.retention_recurrent(qr, kr, v.f64, g)
-    # small shapes: element-wise rounding bound; >= 1024 tokens also the relative L2 bar
+    # every shape: element-wise rounding bound; from 256 tokens on also the relative L2 bar
     bf16_bound_check(host64(out), host64(fs), qr, kr, v.f64, g, ref, S, out_dtype == torch.bfloat16)
-    if N >= 1024:
+    if N >= 256:
         assert err_out(host64(out), ref) < TOL_BF16
         assert err_state(host64(fs), S) < TOL_BF16
 
