@@ -159,6 +159,13 @@ ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
  * to rounding.  final_state may be the same buffer as initial_state (updated
  * in place); any other overlap is RET_ERR_INVALID_ARG.
  */
+/* Workspace bytes of ret_chunkwise_prepare / ret_forward_chunkwise_prepared
+ * (0 when the shape is outside the path): the rotated queries (xpos, or a
+ * dk of 64 padded to 128) and the rotated, zeta-scaled keys, [B, N, H, dk]
+ * bf16 each at the kernel's dk. */
+size_t ret_chunkwise_prepare_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk,
+                                             ret_dtype in_dt, int xpos);
+
 ret_status ret_chunkwise_prepare(const void* q, const void* k, const double* gammas, int B, int N,
                                  int H, int dk, int dv, int chunk, cudaStream_t stream,
                                  ret_dtype in_dt, int xpos, int64_t pos_offset, double theta_base,
@@ -305,12 +312,16 @@ ret_status ret_decode_step_positions(const void* q, const void* k, const void* v
  * is a fixed device array inside the library, of
  * ret_chunkwise_noalloc_max_bytes() bytes (64 MiB) on every GPU that loads
  * the library, held until the process exits.  Problems needing more scratch
- * than that (B*N*H*dk*4 bytes with xpos, B*N*H*dk*2 without) return
- * RET_ERR_INVALID_ARG, shapes outside the workspace path RET_ERR_UNSUPPORTED;
- * nothing is allocated in either case.
+ * than that return RET_ERR_INVALID_ARG, shapes outside the workspace path
+ * RET_ERR_UNSUPPORTED; nothing is allocated in either case.  The scratch is
+ * B*N*H*dk*4 bytes with xpos and B*N*H*dk*2 without, for dk 128 or 256;
+ * for dk = 64 (padded to 128 inside, the queries always copied) it is
+ * B*N*H*128*4 bytes with or without xpos.
  * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture.  All calls share the one array and leave their scratch in it;
+ * device and CUDA context, with that device current); make that first call
+ * before any stream capture.  After a cudaDeviceReset the next call looks
+ * the address up again in the new context.  All calls share the one array
+ * and leave their scratch in it;
  * nothing in it needs to start at zero.  Calls whose kernels overlap on the
  * GPU (other streams, other host threads) race on the array: serialise them.
  */

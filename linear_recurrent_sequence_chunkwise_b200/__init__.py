@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "RetentionError", "lib", "ret_xpos_rotate", "ret_forward_chunkwise", "ret_forward_chunkwise_ws",
-    "ret_chunkwise_workspace_bytes", "ret_chunkwise_prepare", "ret_forward_chunkwise_prepared",
+    "ret_chunkwise_workspace_bytes", "ret_chunkwise_prepare_workspace_bytes", "ret_chunkwise_prepare",
+    "ret_forward_chunkwise_prepared",
     "ret_backward_chunkwise", "ret_backward_workspace_bytes",
     "ret_forward_chunkwise_noalloc", "ret_chunkwise_noalloc_max_bytes",
     "ret_decode_step", "ret_msr_forward", "ret_msr_workspace_bytes",
@@ -50,7 +51,7 @@ def _load_library():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing: build it with "
-            "`python -m linear_recurrent_sequence_chunkwise_b200.build` (nvcc, sm_100a)")
+            "`python linear_recurrent_sequence_chunkwise_b200/build.py` (nvcc, sm_100a)")
     L = ctypes.CDLL(LIB_PATH)
     vp, i, d, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_int64
     dp = ctypes.POINTER(ctypes.c_double)
@@ -70,6 +71,8 @@ def _load_library():
     L.ret_chunkwise_noalloc_max_bytes.restype = ctypes.c_size_t
     L.ret_chunkwise_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
     L.ret_chunkwise_workspace_bytes.restype = ctypes.c_size_t
+    L.ret_chunkwise_prepare_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+    L.ret_chunkwise_prepare_workspace_bytes.restype = ctypes.c_size_t
     L.ret_decode_step.argtypes = [vp, vp, vp, dp, vp, vp, vp, i, i, i, i, i, i]
     L.ret_normalized_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
     L.ret_normalized_workspace_bytes.restype = ctypes.c_size_t
@@ -237,6 +240,11 @@ def ret_forward_chunkwise_ws(q, k, v, gammas, chunk: int, workspace, out=None, f
                                         _stream(stream), _dt(q.dtype), _dt(out.dtype), int(bool(xpos)),
                                         int(pos_offset), float(theta_base), _ptr(workspace, "workspace"), nbytes))
     return (out, final_state) if final_state is not None else out
+
+
+def ret_chunkwise_prepare_workspace_bytes(B, N, H, dk, dv, chunk, dtype=torch.bfloat16, xpos: bool = False) -> int:
+    """Workspace bytes of ret_chunkwise_prepare / ret_forward_chunkwise_prepared (0: shape not on that path)."""
+    return int(lib.ret_chunkwise_prepare_workspace_bytes(B, N, H, dk, dv, chunk, _dt(dtype), int(bool(xpos))))
 
 
 def ret_chunkwise_prepare(q, k, gammas, chunk: int, workspace, dv: int, xpos: bool = False, pos_offset: int = 0,

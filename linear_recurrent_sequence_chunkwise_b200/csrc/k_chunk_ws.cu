@@ -900,23 +900,48 @@ static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
 
 size_t chunkwise_static_ws_bytes() { return kStaticWsBytes; }
 
-// Device address of g_static_ws on the current device, looked up once per
-// device (the host-side symbol is only a stand-in for the device address).
+// Device address of g_static_ws in the current context, looked up once per
+// device and context (the host-side symbol is only a stand-in for the device
+// address).  The cache is keyed on the context as well as the device index:
+// after a cudaDeviceReset the runtime makes a new primary context with the
+// module loaded afresh, and the address is looked up again.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+static CUcontext current_context() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    CUcontext c = nullptr;
+    if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+    return c;
+}
+
 static ret_status static_ws_address(void** out) {
     constexpr int kMaxDev = 64;
     static void* addr[kMaxDev] = {};
+    static CUcontext ctx[kMaxDev] = {};
     static std::mutex mu;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(RET_ERR_CUDA, "static workspace: cudaGetDevice: %s", cudaGetErrorString(e));
     if (dev < 0 || dev >= kMaxDev) return fail(RET_ERR_UNSUPPORTED, "static workspace: device %d out of range", dev);
+    // (a thread that has made no runtime call yet has no current context:
+    // the lookup below binds the device's primary context)
+    const CUcontext c = current_context();
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    if (!addr[dev] || !c || ctx[dev] != c) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_static_ws);
         if (e != cudaSuccess || !p)
             return fail(RET_ERR_CUDA, "static workspace: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
         addr[dev] = p;
+        ctx[dev] = current_context();
     }
     *out = addr[dev];
     return RET_OK;
@@ -924,11 +949,15 @@ static ret_status static_ws_address(void** out) {
 
 ret_status launch_chunkwise_static(const RetArgs& a, cudaStream_t s) {
     const size_t need = chunkwise_ws_bytes(a);
-    if (need > kStaticWsBytes)
+    if (need > kStaticWsBytes) {
+        // a d_k below the kernel's is padded to it, with the queries always copied
+        const int dkc = a.dk_real ? a.dk_real : a.dk;
         return fail(RET_ERR_INVALID_ARG,
                     "ret_forward_chunkwise_noalloc: this problem needs %zu bytes of scratch, above the fixed %zu "
-                    "(B*N*H*dk*%d bytes must not exceed it)",
-                    need, kStaticWsBytes, a.xpos ? 4 : 2);
+                    "(B*N*H*%d*%d bytes for d_k = %d%s must not exceed it)",
+                    need, kStaticWsBytes, a.dk, q_copied(a) ? 4 : 2, dkc,
+                    a.dk_real && a.dk_real != a.dk ? ", padded to the kernel's d_k" : (a.xpos ? " with xpos" : ""));
+    }
     void* ws = nullptr;
     ret_status st = static_ws_address(&ws);
     if (st != RET_OK) return st;

@@ -155,6 +155,16 @@ size_t ret_chunkwise_workspace_bytes(int B, int N, int H, int dk, int dv, int ch
     return chunkwise_ws_supported(a) ? chunkwise_ws_bytes(a) : 0;
 }
 
+size_t ret_chunkwise_prepare_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk, ret_dtype in_dt,
+                                             int xpos) {
+    if (B < 1 || N < 1 || H < 1 || H > kMaxHeads || dk < 1 || dv < 1 || chunk < 1) return 0;
+    RetArgs a{};
+    a.B = B; a.N = N; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.in_dt = in_dt; a.xpos = xpos ? 1 : 0;
+    for (int h = 0; h < kMaxHeads; h++) a.hc.log2g[h] = 0.0;  // shape check only
+    pad_small_dk(&a);
+    return chunkwise_ws_supported(a) ? chunkwise_ws_bytes(a) : 0;
+}
+
 ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v, const double* gammas, int B, int N,
                                     int H, int dk, int dv, int chunk, void* out, float* final_state,
                                     cudaStream_t stream, ret_dtype in_dt, ret_dtype out_dt, int xpos,

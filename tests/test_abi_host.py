@@ -337,3 +337,18 @@ def test_binding_checks_layer_weights():
         R.ret_retnet_block_forward(x, *good.values(), w(dm, 64), w(64, dm), [0.9, 0.8], H, ln1_gain=w(dm + 1))
     with pytest.raises(ValueError, match="x must be bfloat16"):
         R.ret_msr_forward(x.float(), *good.values(), [0.9, 0.8], H)
+
+
+@needs_no_gpu
+@pytest.mark.parametrize("B,N,H,dk,xpos,refused", [
+    (4, 4097, 8, 64, 0, True),     # d_k 64 padded to 128 with the queries copied: 4*4097*8*128*4 > 64 MiB
+    (4, 4097, 8, 64, 1, True),
+    (1, 8193, 16, 256, 0, True),   # keys only: 8193*16*256*2 > 64 MiB
+])
+def test_noalloc_refuses_above_its_array_on_the_host(B, N, H, dk, xpos, refused):
+    g = (ctypes.c_double * H)(*([0.99] * H))
+    st = R.lib.ret_forward_chunkwise_noalloc(P, P2, P3, g, B, N, H, dk, 64, 128 if dk > 64 else 64, P4, None, S0,
+                                             1, 1, xpos, 0, 10000.0)
+    assert st == R.RET_ERR_INVALID_ARG
+    msg = R.ret_last_error_string()
+    assert "scratch" in msg and f"d_k = {dk}" in msg

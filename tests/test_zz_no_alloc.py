@@ -2,50 +2,88 @@
 
 Some callers cannot allocate device memory when they call the library (a
 plug-in inside a framework that owns all device memory, a service that fixes
-its footprint at start-up).  This entry point runs the workspace path on a
+its footprint at start-up).  This entry point runs the two kernels of the
+workspace path (the rotation / zeta pass, then the tensor-core kernel) on a
 fixed device array inside the library instead of a caller-provided buffer.
-The test compares it, through the C ABI, with the workspace entry point on
-two calls in a row with different inputs (the array keeps the first call's
-contents), and checks that a problem too large for the array is refused.
-The file name sorts last so that a run stopping at the first failure has
-already run every other test; it also passes alone in a fresh process."""
+
+The test calls it through the C ABI on two calls in a row with different
+inputs (the array keeps the first call's contents) and requires the same bits
+as the same two kernels run through ret_chunkwise_prepare +
+ret_forward_chunkwise_prepared on a caller workspace, for each layout of the
+scratch: rotated queries and keys (xpos), keys only (no xpos), and the d_k = 64
+shape padded to 128 with the queries always copied.  It also checks the
+result against the fp64 oracle, and that problems too large for the array are
+refused.  The file name sorts last so that a run stopping at the first
+failure has already run every other test; it also passes alone in a fresh
+process."""
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from retention_inputs import gamma_schedule, make_tensor
 from tests.helpers import TOL_BF16, dev, err_out, err_state, host64
 
 pytestmark = pytest.mark.gpu
 
 
-def test_noalloc_matches_workspace_entry_point_on_two_calls():
+def _scratch_bytes(B, N, H, dk, xpos):
+    """What the array must hold: k' (and the copied queries) at the kernel's d_k."""
+    dkk = 128 if dk == 64 else dk
+    copied = xpos or dk == 64
+    return B * N * H * dkk * 2 * (2 if copied else 1)
+
+
+@pytest.mark.parametrize("B,N,H,dk,dv,chunk,xpos", [
+    (1, 2000, 8, 256, 256, 128, True),
+    (2, 1500, 4, 256, 128, 128, False),
+    (4, 1000, 8, 64, 64, 64, True),
+])
+def test_noalloc_matches_the_workspace_kernels_on_two_calls(B, N, H, dk, dv, chunk, xpos):
     import linear_recurrent_sequence_chunkwise_b200 as R
-    B, N, H, dk, dv = 1, 2000, 8, 256, 256
     g = gamma_schedule(H)
-    assert B * N * H * dk * 4 <= R.ret_chunkwise_noalloc_max_bytes()
+    assert _scratch_bytes(B, N, H, dk, xpos) <= R.ret_chunkwise_noalloc_max_bytes()
     for call, seed in enumerate((301, 302)):
-        q = dev(make_tensor(seed, 1, (B, N, H, dk), "bf16", dk ** -0.5))
-        k = dev(make_tensor(seed, 2, (B, N, H, dk), "bf16", dk ** -0.5))
-        v = dev(make_tensor(seed, 3, (B, N, H, dv), "bf16"))
+        qt = make_tensor(seed, 1, (B, N, H, dk), "bf16", dk ** -0.5)
+        kt = make_tensor(seed, 2, (B, N, H, dk), "bf16", dk ** -0.5)
+        vt = make_tensor(seed, 3, (B, N, H, dv), "bf16")
+        q, k, v = dev(qt), dev(kt), dev(vt)
         out = torch.empty((B, N, H, dv), dtype=torch.float32, device="cuda")
         fs = torch.empty((B, H, dk, dv), dtype=torch.float32, device="cuda")
-        R.ret_forward_chunkwise_noalloc(q, k, v, g, 128, out=out, final_state=fs, xpos=True, pos_offset=call)
+        R.ret_forward_chunkwise_noalloc(q, k, v, g, chunk, out=out, final_state=fs, xpos=xpos, pos_offset=call)
         R.ret_check_device_error()
-        nb = R.ret_chunkwise_workspace_bytes(B, N, H, dk, dv, 128, torch.bfloat16, True)
+        nb = R.ret_chunkwise_prepare_workspace_bytes(B, N, H, dk, dv, chunk, torch.bfloat16, xpos)
         ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
-        ref, fref = R.ret_forward_chunkwise_ws(q, k, v, g, 128, ws, out_dtype=torch.float32, xpos=True,
-                                               pos_offset=call, want_final_state=True)
+        R.ret_chunkwise_prepare(q, k, g, chunk, ws, dv, xpos=xpos, pos_offset=call)
+        ref, fref = R.ret_forward_chunkwise_prepared(q, k, v, g, chunk, ws, out_dtype=torch.float32, xpos=xpos,
+                                                     pos_offset=call, want_final_state=True)
         R.ret_check_device_error()
-        assert err_out(host64(out), host64(ref)) < TOL_BF16
-        assert err_state(host64(fs), host64(fref)) < TOL_BF16
+        assert torch.equal(out, ref)
+        assert torch.equal(fs, fref)
+        qf, kf = qt.f64, kt.f64
+        if xpos:
+            qf, kf = oracle.xpos_rotate(qf, call), oracle.xpos_rotate(kf, call)
+        o_ref, s_ref = oracle.retention_recurrent(qf, kf, vt.f64, g)
+        assert err_out(host64(out), o_ref) < TOL_BF16
+        assert err_state(host64(fs), s_ref) < TOL_BF16
 
 
-def test_noalloc_refuses_problems_above_its_array():
+@pytest.mark.parametrize("B,N,H,dk,dv,xpos", [
+    (1, 16384, 16, 256, 64, True),    # 256 MiB of rotated queries and keys
+    (1, 4096, 16, 256, 64, False),    # exactly 32 MiB of keys: accepted
+    (4, 4097, 8, 64, 64, False),      # d_k 64 padded to 128, queries copied: just above 64 MiB
+])
+def test_noalloc_limit(B, N, H, dk, dv, xpos):
     import linear_recurrent_sequence_chunkwise_b200 as R
-    B, N, H, dk, dv = 1, 16384, 16, 256, 64     # 256 MiB of scratch with xpos
     q = torch.zeros((B, N, H, dk), dtype=torch.bfloat16, device="cuda")
     v = torch.zeros((B, N, H, dv), dtype=torch.bfloat16, device="cuda")
+    fits = _scratch_bytes(B, N, H, dk, xpos) <= R.ret_chunkwise_noalloc_max_bytes()
+    if fits:
+        out = R.ret_forward_chunkwise_noalloc(q, q.clone(), v, gamma_schedule(H), 128, xpos=xpos)
+        R.ret_check_device_error()
+        assert torch.count_nonzero(out) == 0
+        return
     with pytest.raises(R.RetentionError) as e:
-        R.ret_forward_chunkwise_noalloc(q, q.clone(), v, gamma_schedule(H), 128, xpos=True)
+        R.ret_forward_chunkwise_noalloc(q, q.clone(), v, gamma_schedule(H), 128, xpos=xpos)
     assert e.value.status == R.RET_ERR_INVALID_ARG
+    assert "scratch" in str(e.value)
