@@ -1,6 +1,7 @@
 """Build step of the CUDA library: compiles every ``csrc/*.cu`` for sm_100a
 into ``libretention.so`` next to this file (in-tree, so it travels with the
-source tree).  Run as ``python -m linear_recurrent_sequence_chunkwise_b200.build``."""
+source tree).  Run as ``python linear_recurrent_sequence_chunkwise_b200/build.py`` (by path:
+importing the package loads the library this script builds)."""
 from __future__ import annotations
 
 import glob
