@@ -1,10 +1,10 @@
 #!/usr/bin/env python
 """Throughput of the chunkwise retention forward on B200 (one JSON line).
 
-Step: one chunkwise retention forward (xPos rotation fused, fp32 inter-chunk
-state, final state written) over the long-sequence workload
-B=1, N=8192, H=16, d_k=256, d_v=512, chunk 128, bf16 in / bf16 out, through
-the C ABI (ret_forward_chunkwise).  value = tokens/s of the whole job
+Step: one chunkwise retention forward (xPos rotation fused into the
+tensor-core kernel, fp32 inter-chunk state, final state written) over the
+long-sequence workload B=1, N=8192, H=16, d_k=256, d_v=512, chunk 128,
+bf16 in / bf16 out, through the C ABI call ret_forward_chunkwise.  value = tokens/s of the whole job
 (B*N per step per rank, summed over ranks; weak scaling, one replica per
 GPU, no collective on the data path).  The decode step (64 sequences x 16
 heads of 256x512 fp32 state) is timed in the same run and reported under
@@ -202,21 +202,16 @@ def run_ours(args):
     fs = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    ws_bytes = R.ret_chunkwise_workspace_bytes(B, N, H, dk, dv, C, torch.bfloat16, True)
-    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
 
-    # One step = the two passes of the workspace path (ret_forward_chunkwise_ws
-    # split at its seam so that each kernel is timed on its own): the
-    # rotation + zeta pass, then the tensor-core kernel.
+    # One step = one call of the spec entry point ret_forward_chunkwise:
+    # the rotation, the zeta scaling and the chunkwise forward in one fused
+    # tensor-core launch (after a 512-byte reset of its exchange counters).
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        R.ret_chunkwise_prepare(q, k, g, C, ws, dv, xpos=True, stream=stream)
+        R.ret_forward_chunkwise(q, k, v, g, C, out=out, final_state=fs, xpos=True, stream=stream)
         if ev:
             ev[1].record(stream)
-        R.ret_forward_chunkwise_prepared(q, k, v, g, C, ws, out=out, final_state=fs, xpos=True, stream=stream)
-        if ev:
-            ev[2].record(stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -224,7 +219,7 @@ def run_ours(args):
     R.ret_check_device_error()
     torch.cuda.synchronize()
 
-    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(2)) for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
@@ -234,26 +229,26 @@ def run_ours(args):
         torch.cuda.synchronize()
         barrier()
     R.ret_check_device_error()
-    times = [a.elapsed_time(c) for a, b, c in evs]  # ms per step
-    t_prep = statistics.mean(a.elapsed_time(b) for a, b, c in evs) / 1e3
-    t_main = statistics.mean(b.elapsed_time(c) for a, b, c in evs) / 1e3
+    times = [a.elapsed_time(b) for a, b in evs]  # ms per step
+    t_main = statistics.mean(times) / 1e3
     total_ms = sum(times)
     total_ms = max_over_ranks(total_ms, world, dist, dev)
     ms_per_step = total_ms / args.steps
     value = job_throughput(B * N, world, ms_per_step)
 
     peaks = load_peaks()
-    # Dominant kernel: k_chunkwise_ws, timed alone (CUDA events around its
-    # launch on the launching stream, mean over the timed steps).  Its
-    # algorithmic work is the whole chunkwise forward: FLOPs of the method,
-    # bytes = read q_rot, k', v once, write out and the final state once.
+    # Dominant kernel: the fused k_chunkwise_ws, timed with CUDA events around
+    # the call on the launching stream (the call is the counter reset and this
+    # one launch), mean over the timed steps.  Its algorithmic work is the
+    # whole chunkwise forward: FLOPs of the method, bytes = read q, k, v once,
+    # write out and the final state once.
     flops = flops_per_token_head(C, dk, dv) * B * N * H
     nbytes = algo_bytes(w, out_bytes=2)
     tflops = flops / t_main / 1e12
     gbs = nbytes / t_main / 1e9
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
-    traffic = load_traffic("k_chunkwise_ws")
+    traffic = load_traffic("k_chunkwise_ws_fused")
     if t_hbm >= t_tc:
         roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(gbs / peaks["hbm_gbs"], 4)}
@@ -262,7 +257,7 @@ def run_ours(args):
                 "frac": round(tflops / peaks["bf16_tflops"], 4)}
     roof["traffic"] = traffic["bytes_per_launch"] if traffic else None
     roof["peak_source"] = peaks["source"] + " (burst; the kernel is timed alone)"
-    roof["kernel"] = "k_chunkwise_ws"
+    roof["kernel"] = "k_chunkwise_ws<256, bf16, fused>"
     roof["kernel_ms"] = round(t_main * 1e3, 4)
     roof["algo_flops"] = flops
     roof["algo_bytes"] = nbytes
@@ -273,13 +268,6 @@ def run_ours(args):
     roof["tensor_frac"] = round(tflops / peaks["bf16_tflops"], 4)
     roof["hbm_gbs"] = round(gbs, 1)
     roof["hbm_frac"] = round(gbs / peaks["hbm_gbs"], 4)
-    # The rotation + zeta pass: reads q, k and writes q_rot, k' (bf16).
-    prep_bytes = 4 * B * N * H * dk * 2
-    prep = {"kernel": "k_prep_qk", "bound": "hbm", "ms": round(t_prep * 1e3, 4),
-            "achieved": round(prep_bytes / t_prep / 1e9, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(prep_bytes / t_prep / 1e9 / peaks["hbm_gbs"], 4), "algo_bytes": prep_bytes,
-            "traffic": (load_traffic("k_prep_qk") or {}).get("bytes_per_launch")}
-
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -288,10 +276,23 @@ def run_ours(args):
         "config": {"workload": w["workload"], "B": B, "N": N, "H": H, "dk": dk, "dv": dv, "chunk": C, "xpos": True,
                    "out_dtype": "bf16", "final_state": True, "global_batch": B * world, "seq_len": N,
                    "parallelism": f"replicas x{world}", "l2": "flushed before every timed step (256 MiB write)"},
-        "roofline": roof, "prep_pass": prep, "clocks": clk.summary(), "gpu_launches": 2 * args.steps,
-        "path": "ret_chunkwise_prepare (rotation + zeta pass) then ret_forward_chunkwise_prepared "
-                "(warp-specialized tcgen05 kernel), i.e. ret_forward_chunkwise_ws in two calls",
+        "roofline": roof, "clocks": clk.summary(), "gpu_launches": args.steps,
+        "path": "ret_forward_chunkwise: one cooperative launch of the warp-specialized tcgen05 kernel with the "
+                "xPos rotation and zeta scaling fused (each head's 8 CTAs share the rotated rows through an "
+                "L2-resident exchange ring), after a 512-byte counter reset",
     }
+    # the same forward as two calls (rotation + zeta pass, then the tensor-core
+    # kernel on the prepared rows), timed the same way, for comparison
+    ws2 = torch.empty(R.ret_chunkwise_prepare_workspace_bytes(B, N, H, dk, dv, C, torch.bfloat16, True),
+                      dtype=torch.uint8, device=dev)
+
+    def two_pass():
+        R.ret_chunkwise_prepare(q, k, g, C, ws2, dv, xpos=True, stream=stream)
+        R.ret_forward_chunkwise_prepared(q, k, v, g, C, ws2, out=out, final_state=fs, xpos=True, stream=stream)
+
+    result["two_pass_ms"] = round(_timed_flushed(torch, stream, two_pass, min(args.steps, 10), 3, world, dist, dev,
+                                                 flush), 4)
+    del ws2
     if not args.no_e2e:
         result["e2e"] = e2e_ours(R, torch, dev, stream, w, g, args, world, barrier, dist)
     if not args.no_decode:
@@ -328,8 +329,6 @@ def e2e_ours(R, torch, dev, stream, w, g, args, world, barrier, dist):
     ho = [torch.empty((B, N, H, dv), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
     dbuf = [tuple(torch.empty_like(x, device=dev) for x in (hq, hk, hv)) for _ in range(2)]
     do = [torch.empty((B, N, H, dv), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-    ws = torch.empty(max(R.ret_chunkwise_workspace_bytes(B, N, H, dk, dv, C, torch.bfloat16, True), 1),
-                     dtype=torch.uint8, device=dev)
     steps = max(3, min(args.steps, 10))
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     ev = lambda: torch.cuda.Event()
@@ -351,7 +350,7 @@ def e2e_ours(R, torch, dev, stream, w, g, args, world, barrier, dist):
         stream.wait_event(in_ready[b])
         if used[b]:
             stream.wait_event(out_free[b])           # step i-2's output has left this buffer
-        R.ret_forward_chunkwise_ws(dq, dk_, dv_, g, C, ws, out=do[b], xpos=True, stream=stream)
+        R.ret_forward_chunkwise(dq, dk_, dv_, g, C, out=do[b], xpos=True, stream=stream)
         comp_done[b].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(comp_done[b])
@@ -609,10 +608,31 @@ def bench_block(R, torch, dev, stream, args, peaks, world, dist):
                                     "k_gemm (W2, residual)"}}
 
 
+def _timed_flushed(torch, stream, fn, steps, warmup, world, dist, dev, flush):
+    """Mean CUDA-event time (ms) of fn() over `steps` calls after `warmup`,
+    with the L2 flushed (a 256 MiB write) before every call, outside the
+    events; max over ranks."""
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world, dist, dev)
+
+
 def bench_c2(R, torch, dev, stream, args, peaks, world, dist):
     """The pages' cost-analysis shape [4, 2048, 8 heads of 64], bf16, xPos,
-    chunk 64: the workspace path (d_k padded to 128 on the tensor cores)
-    beside the single-call path (CUDA cores, fp32 arithmetic)."""
+    chunk 64, L2 flushed before every call: the spec call
+    ret_forward_chunkwise (fused rotation, d_k padded to 128 on the tensor
+    cores, 128-token blocks) beside the two-pass form (rotation pass, then
+    the tensor-core kernel).  HBM-bound: algorithmic bytes = read q, k, v
+    once, write out once (bf16)."""
     B, N, H, dk, dv, C = 4, 2048, 8, 64, 64, 64
     gen = torch.Generator(device=dev)
     gen.manual_seed(0x5EED0009)
@@ -621,22 +641,30 @@ def bench_c2(R, torch, dev, stream, args, peaks, world, dist):
     v = torch.randn((B, N, H, dv), generator=gen, device=dev).to(torch.bfloat16)
     out = torch.empty((B, N, H, dv), dtype=torch.bfloat16, device=dev)
     g = gammas(H)
-    ws = torch.empty(R.ret_chunkwise_workspace_bytes(B, N, H, dk, dv, C, torch.bfloat16, True), dtype=torch.uint8,
-                     device=dev)
+    ws = torch.empty(R.ret_chunkwise_prepare_workspace_bytes(B, N, H, dk, dv, C, torch.bfloat16, True),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def tc():
-        R.ret_forward_chunkwise_ws(q, k, v, g, C, ws, out=out, xpos=True, stream=stream)
-
-    def cc():
+    def fused():
         R.ret_forward_chunkwise(q, k, v, g, C, out=out, xpos=True, stream=stream)
 
+    def two_pass():
+        R.ret_chunkwise_prepare(q, k, g, C, ws, dv, xpos=True, stream=stream)
+        R.ret_forward_chunkwise_prepared(q, k, v, g, C, ws, out=out, xpos=True, stream=stream)
+
     steps = max(5, min(args.steps, 20))
-    ms_tc = _timed(torch, stream, tc, steps, 3, world, dist, dev)
-    ms_cc = _timed(torch, stream, cc, steps, 3, world, dist, dev)
+    ms = _timed_flushed(torch, stream, fused, steps, 3, world, dist, dev, flush)
+    ms_two = _timed_flushed(torch, stream, two_pass, steps, 3, world, dist, dev, flush)
     R.ret_check_device_error()
-    return {"workload": "retention_bf16_4x2048x8x64", "tokens_per_s": round(world * B * N / (ms_tc / 1e3), 1),
-            "ms_per_step": round(ms_tc, 4), "single_call_cuda_cores_ms": round(ms_cc, 4),
-            "path": "ret_forward_chunkwise_ws: k_prep_qk + k_chunkwise_ws<128>, d_k padded to 128, 128-token blocks"}
+    nbytes = B * N * H * (2 * dk * 2 + dv * 2 + dv * 2)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": "retention_bf16_4x2048x8x64", "tokens_per_s": round(world * B * N / (ms / 1e3), 1),
+            "ms_per_step": round(ms, 4), "two_pass_ms": round(ms_two, 4),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "algo_bytes": nbytes,
+                         "peak_source": peaks["source"]},
+            "l2": "flushed before every timed call (256 MiB write)",
+            "path": "ret_forward_chunkwise: fused k_chunkwise_ws<128>, d_k padded to 128, 128-token blocks"}
 
 
 def bench_fp32_small(R, torch, dev, stream, args, world, dist):

@@ -20,7 +20,19 @@ ret_status check_launch(const char* what);
 constexpr int kMaxHeads = 128;
 struct HeadConsts {
     double log2g[kMaxHeads];  // log2(gamma_h); -inf for gamma_h = 0
+    // Row a of a 128-row chunk the tensor-core kernels scale the decay about
+    // (keys by gamma^(a-c), output rows by gamma^(r-a)): 127 when
+    // gamma^128 >= 2^-60, 63 when gamma^64 >= 2^-100 (every factor then stays
+    // within 2^+-100), -1 for a head the tensor-core kernels do not take.
+    int anchor[kMaxHeads];
 };
+constexpr int kChunkAnchorFull = 127, kChunkAnchorMid = 63;
+// The anchor rule above, for one head.
+inline int decay_anchor(double log2g) {
+    if (log2g * 128.0 >= -60.0) return kChunkAnchorFull;
+    if (log2g * 64.0 >= -100.0) return kChunkAnchorMid;
+    return -1;
+}
 // Fill `hc` from the host array; returns false if H is out of range.
 bool make_head_consts(const double* gammas, int H, HeadConsts* hc);
 
@@ -30,7 +42,6 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 // mbarriers keeps its own word (no relocatable device code) and exposes a
 // host reader that returns and clears it (cudaSuccess or the CUDA error).
 constexpr int kErrTimeout = 1;
-cudaError_t read_clear_error_chunk_tc(int* flag);
 cudaError_t read_clear_error_chunk_ws(int* flag);
 
 // ---------------------------------------------------------------- device side

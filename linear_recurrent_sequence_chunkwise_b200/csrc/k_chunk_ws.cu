@@ -1,19 +1,34 @@
-// k_chunk_ws.cu -- chunkwise retention forward with a caller-provided
-// workspace: a bandwidth-bound prep kernel plus a warp-specialized
-// tcgen05 / TMEM / TMA kernel.
+// k_chunk_ws.cu -- chunkwise retention forward on the tensor cores: a
+// warp-specialized tcgen05 / TMEM / TMA kernel, fed either by a
+// bandwidth-bound rotation pass (two-pass form) or by its own CTAs (fused
+// form).
 //
-// Same mathematics as k_chunk_tc.cu ("Hybrid Architectures: RetNet and the
-// Three Computation Paradigms", section 7.2; RetNet paper summary, Eq. 7),
-// with the decay folded into a scaled key k'_c = gamma^(L-1-c) k_c (c the row
-// in its chunk of L rows), a pre-scaled state T = gamma^L R and a row scale:
-//     out_r = gamma^(r+1-L) [ sum_{c<=r} (q_r . k'_c) v_c + q_r^T T ],
-//     R     = T + K'^T V.
+// Mathematics ("Hybrid Architectures: RetNet and the Three Computation
+// Paradigms", section 7.2; RetNet paper summary, Eq. 7).  For a chunk of L
+// rows and 0-based rows r, c:
+//     out_r = sum_{c<=r} gamma^(r-c) (q_r . k_c) v_c + gamma^(r+1) q_r^T R_prev
+//     R     = gamma^L R_prev + sum_c gamma^(L-1-c) k_c v_c^T
+// The kernel folds every decay factor into one scaled key and one row scale
+// about an anchor row a (a = min(anchor_h, L-1), anchor_h 127 or 63):
+//     k'_c  = gamma^(a-c) k_c
+//     T     = gamma^(a+1) R_prev                      (read-out copy, bf16)
+//     out_r = gamma^(r-a) [ sum_{c<=r} (q_r . k'_c) v_c + q_r^T T ]
+//     R     = gamma^L R_prev + gamma^(L-1-a) K'^T V
+// since gamma^(r-c) = gamma^(r-a) gamma^(a-c) and gamma^(r+1) = gamma^(r-a)
+// gamma^(a+1).  So the decay mask D becomes a plain causal mask on Q K'^T,
+// generated in registers, and the intra-chunk scores, the cross read-out and
+// the state update each feed one fp32 TMEM accumulator.  With a = L-1 (heads
+// with gamma^128 >= 2^-60) the factors are those of the pages' zeta and xi;
+// faster-decaying heads take a = 63, which keeps every factor within
+// 2^+-100 for gamma^64 >= 2^-100; heads below that are left to the recurrent
+// kernel (their CTAs return at once).
 //
-// 1. k_prep_qk (HBM-bound, one pass): rotates q and k once per head (xPos,
-//    consecutive pairs, angle (pos_offset + n) theta_p with the sine and
-//    cosine of each (position, pair) evaluated once for all heads), scales
-//    each rotated key row by its zeta, and writes q_rot and k' (bf16) into the
-//    workspace.  Without rotation only k' is written and q is read in place.
+// 1. k_prep_qk (HBM-bound, one pass, two-pass form): rotates q and k once per
+//    head (xPos, consecutive pairs, angle (pos_offset + n) theta_p with the
+//    sine and cosine of each (position, pair) evaluated once for all heads),
+//    scales each rotated key row by gamma^(a-c), and writes q_rot and k'
+//    (bf16) into the workspace.  Without rotation only k' is written and q is
+//    read in place.
 // 2. k_chunkwise_ws: one CTA per (batch, head, 64 value columns), 16 warps
 //    in five roles (registers rebalanced with setmaxnreg):
 //      warp 0  TMA producer: L2 prefetch two chunks ahead (the CTAs of a
@@ -34,15 +49,19 @@
 //                soon as it lands, -> TMEM once the read-out of chunk j is
 //                done; a plain smem read keeps the load traffic on the TMA
 //                path (per-row global loads from these threads measurably
-//                slow the tensor pipe down);
+//                slow the tensor pipe down).  In the fused form these warps
+//                also rotate this CTA's share of each chunk into the head's
+//                exchange ring (see q_role_fused);
 //      warps 8-15 (two warpgroups on TMEM lanes 0..127, one column half each):
 //                mask:     P = tril(A) -> packed bf16 in TMEM,
-//                state:    R = gamma^L R + dS in registers (fp32), then the
-//                          bf16 T = gamma^L' R into smem for the next read-out,
-//                epilogue: out = gamma^(r+1-L) O staged in the chunk's V slot.
+//                state:    R = gamma^L R + gamma^(L-1-a) dS in registers
+//                          (fp32), then the bf16 T = gamma^(a'+1) R into smem
+//                          for the next read-out,
+//                epilogue: out = gamma^(r-a) O staged in the chunk's V slot.
 //    TMEM columns: A [0,128), P [128,192), O [192,256), Q [256,384),
 //    dS [384,512).  Every hand-off between the roles has at least one block
 //    of MMAs in between, so no role waits on another in the steady state.
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -128,8 +147,10 @@ __global__ void __launch_bounds__(256) k_prep_qk(const __nv_bfloat16* __restrict
             for (int hh = 0; hh < kHB; hh++) {
                 if (h0 + hh >= H) continue;
                 const size_t e = ((size_t)t * H + h0 + hh) * DK + 8 * g;
-                // zeta = gamma^(L-1-r): the exponent in fp64, exp2 in fp32 (relative error ~1e-7)
-                const float zeta = exp2f((float)((double)(L - 1 - r) * hc.log2g[h0 + hh]));
+                // k' scale gamma^(a-r), a = min(anchor, L-1): the exponent in fp64,
+                // exp2 in fp32 (relative error ~1e-7)
+                const int a = min(hc.anchor[h0 + hh], L - 1);
+                const float zeta = exp2f((float)((double)(a - r) * hc.log2g[h0 + hh]));
                 uint32_t* kwv = reinterpret_cast<uint32_t*>(&kw[hh]);
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
@@ -168,7 +189,69 @@ struct WsParams {
     const float* rowscale;  // [B, N, H] factor of each output row, or null
     int nmain;            // CTAs: B * H * (dv / 64), one per (b, h, 64 value columns)
     HeadConsts hc;
+    // Fused rotation (FUSED instances).  A launch takes the (b, h) pairs
+    // bh0 .. bh0 + gridDim.x / nt - 1 (nt = dv / 64 CTAs per head; bh0 = 0
+    // otherwise).  Each of a head's nt CTAs turns its 1/nt share of the rows
+    // of every chunk (xPos) from the raw q and k, scales the keys by zeta,
+    // and writes them into the head's exchange ring (kRing chunk slots in
+    // global memory, small enough to stay in L2); the tensor maps tq / tk
+    // then point at the ring.  Per (head g, slot) two counts: ready[g][slot]
+    // the shares written into the slot, consumed[g][slot] the CTAs whose
+    // loads of the slot's chunk have landed (which frees it).  Chunk i lives
+    // in slot i % kRing as its generation u = i / kRing, so it is complete
+    // when ready reaches nt (u + 1), and the slot may take chunk i + kRing
+    // once consumed reaches nt (u + 1).  (The CTAs of a head drift apart by
+    // up to kLead chunks, so one count per head would not say which chunk.)
+    int bh0;
+    const __nv_bfloat16* q_raw;
+    const __nv_bfloat16* k_raw;
+    int q_ld, k_ld;       // elements between consecutive (token, head) rows of q_raw / k_raw
+    __nv_bfloat16* ring_q;
+    __nv_bfloat16* ring_k;
+    unsigned int* ready;
+    unsigned int* consumed;
+    int xpos;
+    long long pos0;
+    double log2base;
 };
+
+// Exchange ring of the fused rotation: chunk slots per head, and how many
+// chunks ahead of the one being computed the shares are written.
+constexpr int kRing = 6, kLead = 3;
+
+// Wait (bounded) until *ctr >= target, with acquire semantics at GPU scope,
+// then order the caller's later async-proxy (TMA) accesses after what it saw.
+__device__ __forceinline__ bool wait_count(const unsigned int* ctr, unsigned int target) {
+    for (uint32_t i = 0; i < (1u << 22); i++) {
+        unsigned int v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        if (v >= target) {
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            return true;
+        }
+        __nanosleep(32);
+    }
+    return false;
+}
+
+__device__ __forceinline__ void count_release(unsigned int* ctr) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+}
+
+// Named barrier 1 over the Q warpgroup (warps 4-7): returns whether x holds
+// in all 128 threads; also orders their memory accesses around it.
+__device__ __forceinline__ bool qwg_all(bool x) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, 1, 128, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)x)
+        : "memory");
+    return r != 0;
+}
 
 constexpr int kKSlots = 3;                         // K' ring depth (parts of 128 d_k rows)
 constexpr int kKPartBytes = kPartDk * kC * 2;      // 32 KB
@@ -212,7 +295,245 @@ __device__ __forceinline__ void regs_inc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-template <int DK, typename Tout>
+// An angle (fp64) reduced to [-pi, pi] and rounded to fp32, for the fast
+// fp32 sine and cosine (absolute error a few 1e-7 there).
+__device__ __forceinline__ float angle_mod_2pi(double a) {
+    const double two_pi = 6.283185307179586476925286766559, inv_two_pi = 0.15915494309189533576888376337251;
+    return (float)fma(-two_pi, rint(a * inv_two_pi), a);
+}
+
+// One 16-byte group (4 consecutive pairs) of a row, turned by the angles
+// whose cosines and sines are c[], s[] (k rows: already scaled by zeta).
+__device__ __forceinline__ uint4 turn_group(uint4 x, const float (&c)[4], const float (&s)[4]) {
+    uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const float x0 = tc::bf16lo(w[i]), x1 = tc::bf16hi(w[i]);
+        w[i] = tc::pack_bf16x2(x0 * c[i] - x1 * s[i], x0 * s[i] + x1 * c[i]);
+    }
+    return x;
+}
+
+// The Q warpgroup of the fused instances.  Per chunk jq:
+//   * once the read-out of chunk jq - 1 has consumed the previous Q, the
+//     staged Q goes from shared memory into TMEM one 64-column slab at a time
+//     (few registers held), and the tensor pipe is told (qready);
+//   * the count of the chunk written in the previous iteration is released
+//     (its bulk stores have long completed, so this is cheap);
+//   * this CTA's share of chunk jq + kLead is written into the exchange ring,
+//     once the slot is free (every CTA of the head has loaded the chunk that
+//     last used it: consumed[g][slot] = nt * generation; the count is read one
+//     iteration early).  The share is the rows [r0, r0 + R) of the chunk,
+//     R = ceil(128 / nt); each thread turns one 16-byte group (pairs
+//     4g .. 4g+3) of every kStep-th row, writes it into the Q staging buffer
+//     (free until the staging buffer is handed back), and one thread copies
+//     the rows into the ring with bulk stores (pieces of up to 64 rows);
+//   * the staging buffer goes back to the TMA producer (qempty), and the raw
+//     rows of chunk jq + kLead + 1 are loaded into registers for the next
+//     iteration (their latency is hidden).
+// The rotation of a thread's first row is evaluated from the position (fp64
+// angle, reduced, then fp32 sine and cosine), the next ones by turning it
+// through kStep * theta_p; keys are also scaled by gamma^(a-r); rows past the
+// end of the sequence and groups past the caller's d_k are written as zeros.
+// The rows of the prologue (chunks 0 .. kLead - 1) are written before the
+// loop, and the staging buffer is handed to the producer once (qempty phase
+// 0) before it loads the first Q.  The warpgroup agrees on every wait's
+// outcome (named barrier 1), so a timed-out wait cannot strand part of it at
+// a barrier.  Returns false on a timeout.
+template <int DK>
+__device__ __forceinline__ bool q_role_fused(const WsParams& p, uint8_t* sQ, uint32_t tb, uint32_t lane_off, int r,
+                                             int quarter, int lane, int nt, int jt, int gl, int b, int h,
+                                             int nchunks, double lg, int anc, Bars& bars) {
+    constexpr int kGpr = DK / 8;             // 16-byte groups in a row
+    constexpr int kRpw = 32 / kGpr;          // rows one warp covers at a time
+    constexpr int kStep = 4 * kRpw;          // rows between one thread's rows
+    constexpr int kBatch = 4;                // rows whose loads are in flight together
+    constexpr int kPiece = (DK * kC * 2) / (4 * DK);   // rows of q and k the staging buffer holds (64)
+    const int N = p.N, H = p.H;
+    const int grp = lane % kGpr;
+    const int rsub = quarter * kRpw + lane / kGpr;     // row offset within a step
+    const bool real = 8 * grp < p.dks;       // inside the caller's d_k
+    const bool turn = p.xpos && real;
+    const int wtid = quarter * 32 + lane;
+    const int R = (kC + nt - 1) / nt;
+    const int r0 = min(R * jt, kC), r1 = min(r0 + R, kC);
+    // theta_p = base^(-2p/d_k) of the thread's four pairs (fp64), and the
+    // turn through kStep positions
+    double theta[4];
+    float cstep[4], sstep[4];
+    {
+        const double inv_dk = 1.0 / p.dks;
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            theta[k] = turn ? exp2(-2.0 * (4 * grp + k) * inv_dk * p.log2base) : 0.0;
+            cstep[k] = 1.f;
+            sstep[k] = 0.f;
+            if (turn) __sincosf(angle_mod_2pi((double)kStep * theta[k]), &sstep[k], &cstep[k]);
+        }
+    }
+    auto raw_row = [&](int i, int rr) { return ((size_t)b * N + (size_t)i * kC + rr) * H + h; };
+    // the raw rows rb, rb + kStep, ... (kBatch of them) of chunk i
+    auto load_rows = [&](int i, int rb, uint4 (&qw)[kBatch], uint4 (&kw)[kBatch]) {
+        const int L = i < nchunks ? min(kC, N - i * kC) : 0;
+#pragma unroll
+        for (int u = 0; u < kBatch; u++) {
+            const int rr = rb + u * kStep;
+            qw[u] = kw[u] = make_uint4(0, 0, 0, 0);
+            if (real && rr < L && rr < r1) {
+                const size_t row = raw_row(i, rr);
+                qw[u] = __ldg(reinterpret_cast<const uint4*>(p.q_raw + row * p.q_ld + 8 * grp));
+                kw[u] = __ldg(reinterpret_cast<const uint4*>(p.k_raw + row * p.k_ld + 8 * grp));
+            }
+        }
+    };
+    // thread 0: the consumed count of the slot the next write takes
+    unsigned seen = 0;
+    auto peek = [&](int i) {
+        if (wtid == 0 && i >= kRing && i < nchunks)
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];"
+                         : "=r"(seen)
+                         : "l"(p.consumed + gl * kRing + i % kRing)
+                         : "memory");
+    };
+    uint4 aq[kBatch], ak[kBatch];   // raw rows of the next chunk to write, loaded ahead
+
+    // This CTA's share of chunk i into the ring (the first kBatch rows of the
+    // thread from aq / ak); the bulk stores are left in flight.
+    auto write_share = [&](int i) -> bool {
+        bool okp = true;
+        if (i >= kRing && wtid == 0) {
+            const unsigned need = (unsigned)(nt * (i / kRing));
+            if (seen < need) okp = wait_count(p.consumed + gl * kRing + i % kRing, need);
+        }
+        if (!qwg_all(okp)) return false;
+        const int n0 = i * kC, L = min(kC, N - n0);
+        const size_t slot0 = ((size_t)gl * kRing + (size_t)(i % kRing)) * kC;   // ring row of the slot's row 0
+        float cs[4], sn[4];
+        const double pos = (double)(p.pos0 + n0 + r0 + rsub);
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            cs[k] = 1.f;
+            sn[k] = 0.f;
+            if (turn) __sincosf(angle_mod_2pi(pos * theta[k]), &sn[k], &cs[k]);
+        }
+        for (int p0 = r0; p0 < r1; p0 += kPiece) {
+            const int p1 = min(p0 + kPiece, r1);
+            uint8_t* stq = sQ;
+            uint8_t* stk = sQ + (size_t)kPiece * DK * 2;
+            // rows rb, rb + kStep, ... (kBatch of them) from qw / kw into the staging buffer
+            auto put = [&](int rb, uint4 (&qw)[kBatch], uint4 (&kw)[kBatch]) {
+#pragma unroll
+                for (int u = 0; u < kBatch; u++) {
+                    const int rr = rb + u * kStep;
+                    if (rr >= p1) break;
+                    uint4 qo = qw[u], ko = kw[u];
+                    if (real && rr < L) {
+                        // k' scale gamma^(a-r), a = min(anchor, L-1): exponent in fp64, exp2 in fp32
+                        const float zeta = exp2f((float)((double)(min(anc, L - 1) - rr) * lg));
+                        float ck[4], sk[4];
+#pragma unroll
+                        for (int k = 0; k < 4; k++) {
+                            ck[k] = cs[k] * zeta;
+                            sk[k] = sn[k] * zeta;
+                        }
+                        qo = turn_group(qo, cs, sn);
+                        ko = turn_group(ko, ck, sk);
+                    }
+                    const size_t o = ((size_t)(rr - p0) * DK + 8 * grp) * 2;
+                    *reinterpret_cast<uint4*>(stq + o) = qo;
+                    *reinterpret_cast<uint4*>(stk + o) = ko;
+                    if (turn) {
+#pragma unroll
+                        for (int k = 0; k < 4; k++) {
+                            const float c2 = cs[k] * cstep[k] - sn[k] * sstep[k];
+                            sn[k] = sn[k] * cstep[k] + cs[k] * sstep[k];
+                            cs[k] = c2;
+                        }
+                    }
+                }
+            };
+            for (int rb = p0 + rsub; rb < p1; rb += kBatch * kStep) {
+                if (rb == r0 + rsub) {
+                    put(rb, aq, ak);
+                } else {
+                    uint4 qw[kBatch], kw[kBatch];
+                    load_rows(i, rb, qw, kw);
+                    put(rb, qw, kw);
+                }
+            }
+            // the staged rows go to the ring by one thread's bulk stores; the
+            // staging buffer is reused once they have been read
+            tc::fence_proxy_async_smem();
+            qwg_all(true);
+            if (wtid == 0) {
+                const uint32_t bytes = (uint32_t)(p1 - p0) * DK * 2;
+                tc::bulk_store(p.ring_q + (slot0 + p0) * DK, stq, bytes);
+                tc::bulk_store(p.ring_k + (slot0 + p0) * DK, stk, bytes);
+                tc::bulk_commit_group();
+                tc::bulk_wait_group_read<0>();
+            }
+            qwg_all(true);
+        }
+        return true;
+    };
+    // thread 0: once the bulk stores of chunk i have completed, its count
+    auto release = [&](int i) {
+        if (wtid == 0) {
+            tc::bulk_wait_group<0>();
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            count_release(p.ready + gl * kRing + i % kRing);
+        }
+    };
+
+    for (int i = 0; i < kLead && i < nchunks; i++) {
+        load_rows(i, r0 + rsub, aq, ak);
+        if (!write_share(i)) return false;
+        release(i);
+    }
+    // the staging buffer is the producer's from here on (qempty phase 0)
+    elect_arrive(&bars.qempty, lane);
+    load_rows(kLead, r0 + rsub, aq, ak);
+    for (int jq = 0; jq < nchunks; jq++) {
+        peek(jq + kLead);
+        if (jq > 0 && !qwg_all(tc::mbar_wait(&bars.qtm, (jq - 1) & 1))) return false;
+        if (!qwg_all(tc::mbar_wait(&bars.qfull, jq & 1))) return false;
+        tc::tc_fence_after();
+        // one slab at a time (32 registers of Q in flight)
+#pragma unroll 1
+        for (int g = 0; g < DK / 64; g++) {
+            uint32_t w[32];
+#pragma unroll
+            for (int c16 = 0; c16 < 8; c16++) {
+                const uint4 x = *reinterpret_cast<const uint4*>(sQ + g * (kC * 128) +
+                                                                tc::sw128_off((uint32_t)r, (uint32_t)c16));
+                w[4 * c16 + 0] = x.x;
+                w[4 * c16 + 1] = x.y;
+                w[4 * c16 + 2] = x.z;
+                w[4 * c16 + 3] = x.w;
+            }
+            tc::tmem_st32(tb + lane_off + kTQ + 32 * g, w);
+        }
+        tc::tmem_st_wait();
+        tc::tc_fence_before();
+        elect_arrive(&bars.qready, lane);
+        const int i = jq + kLead;
+        if (jq > 0 && i - 1 < nchunks) release(i - 1);
+        if (i < nchunks) {
+            // (the staging buffer's reads above are done: the TMEM stores
+            // consumed their registers, and every thread has passed them)
+            qwg_all(true);
+            if (!write_share(i)) return false;
+        }
+        // the staging buffer goes back to the producer: the generic reads and
+        // writes above are ordered before its next async-proxy write
+        tc::fence_proxy_async_smem();
+        elect_arrive(&bars.qempty, lane);
+        if (i < nchunks) load_rows(i + 1, r0 + rsub, aq, ak);
+    }
+    return true;
+}
+
+template <int DK, typename Tout, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_constant__ WsParams p) {
     constexpr int kParts = DK / kPartDk;
     constexpr int kQSlabs = DK / 64;
@@ -224,11 +545,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nt = p.dv / kW, jt = (int)blockIdx.x % nt;     // this CTA's 64 value columns
-    const int h = ((int)blockIdx.x / nt) % p.H, b = (int)blockIdx.x / (nt * p.H);
+    const int gl = (int)blockIdx.x / nt;                      // this launch's head index
+    const int h = (p.bh0 + gl) % p.H, b = (p.bh0 + gl) / p.H;
     const int j0 = jt * kW;
     const int N = p.N;
     const int nchunks = (N + kC - 1) / kC;
     const double lg = p.hc.log2g[h];
+    // a head whose decay is too fast for the folded factors is computed by
+    // the recurrent kernel; its CTAs (all of them, so none waits on another)
+    // leave before touching anything
+    if (p.hc.anchor[h] < 0) return;
     const int has_init = p.istate != nullptr;
     constexpr int kXfWarps = 8;  // transform warps arriving on the warpgroup barriers
 
@@ -278,23 +604,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             // -------------------------------------------- TMA producer
             // L2 prefetch of chunk jp: the CTAs of one head split the Q and K'
             // boxes between them; each prefetches its own V tile.
+            // (the fused ring is written into L2 by the CTAs themselves)
             auto prefetch = [&](int jp) {
                 if (jp >= nchunks) return;
                 const int n0p = jp * kC;
-                for (int i = jt; i < 2 * kQSlabs; i += nt)
-                    tc::tma_prefetch_l2_4d(i < kQSlabs ? &p.tq : &p.tk, 64 * (i % kQSlabs), h, n0p, b);
+                if constexpr (!FUSED)
+                    for (int i = jt; i < 2 * kQSlabs; i += nt)
+                        tc::tma_prefetch_l2_4d(i < kQSlabs ? &p.tq : &p.tk, 64 * (i % kQSlabs), h, n0p, b);
                 tc::tma_prefetch_l2_4d(&p.tv, j0, h, n0p, b);
             };
             prefetch(0);
             prefetch(1);
             for (int jc = 0; jc < nchunks && ok; jc++) {
                 const int n0 = jc * kC;
+                // coordinates of the chunk's rows in the q / k' tensor maps:
+                // (head, token, batch), or (ring row, head of the launch, 0)
+                const int c1 = FUSED ? (jc % kRing) * kC : h, c2 = FUSED ? gl : n0, c3 = FUSED ? 0 : b;
                 prefetch(jc + 2);
-                if (jc > 0) ok = tc::mbar_wait(&bars.qempty, (jc - 1) & 1);
+                // (fused: the Q warpgroup hands the staging buffer over once after
+                // writing its first ring rows, so chunk jc waits for phase jc)
+                if (FUSED) ok = tc::mbar_wait(&bars.qempty, jc & 1);
+                else if (jc > 0) ok = tc::mbar_wait(&bars.qempty, (jc - 1) & 1);
+                // fused: every CTA of the head has written its share of the chunk
+                if (FUSED && ok)
+                    ok = wait_count(p.ready + gl * kRing + jc % kRing, (unsigned)(nt * (jc / kRing + 1)));
                 if (!ok) break;
                 tc::mbar_arrive_expect_tx(&bars.qfull, DK * kC * 2);
                 for (int s = 0; s < kQSlabs; s++)
-                    tc::tma_load_4d(sm + WsSmem<DK>::kQ + s * (kC * 128), &p.tq, &bars.qfull, 64 * s, h, n0, b);
+                    tc::tma_load_4d(sm + WsSmem<DK>::kQ + s * (kC * 128), &p.tq, &bars.qfull, 64 * s, c1, c2, c3);
                 for (int part = 0; part < kParts && ok; part++) {
                     const int g = jc * kParts + part, slot = g % kKSlots, u = g / kKSlots;
                     if (u > 0) ok = tc::mbar_wait(&bars.kempty[slot], (u - 1) & 1);
@@ -302,8 +639,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                     uint8_t* dst = sm + WsSmem<DK>::kK + slot * kKPartBytes;
                     tc::mbar_arrive_expect_tx(&bars.kfull[slot], kKPartBytes);
                     for (int s = 0; s < 2; s++)
-                        tc::tma_load_4d(dst + s * (kC * 128), &p.tk, &bars.kfull[slot], part * kPartDk + 64 * s, h,
-                                        n0, b);
+                        tc::tma_load_4d(dst + s * (kC * 128), &p.tk, &bars.kfull[slot], part * kPartDk + 64 * s, c1,
+                                        c2, c3);
                 }
                 const int vs = jc & 1;
                 if (ok && jc >= 2) ok = tc::mbar_wait(&bars.vempty[vs], ((jc >> 1) & 1) ^ 1);
@@ -467,6 +804,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const uint8_t* sQ = sm + WsSmem<DK>::kQ;
         uint4 qv[DK / 8];
+        if constexpr (FUSED) {
+            ok = q_role_fused<DK>(p, const_cast<uint8_t*>(sQ), tb, lane_off, r, quarter, lane, nt, jt, gl, b, h,
+                                  nchunks, lg, p.hc.anchor[h], bars);
+        } else
         for (int jq = 0; jq < nchunks && ok; jq++) {
             ok = tc::mbar_wait(&bars.qfull, jq & 1);
             if (!ok) break;
@@ -521,16 +862,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         uint8_t* sT = sm + WsSmem<DK>::kT;
         float R[kParts][32];
-        // decay powers of a full chunk and of the (possibly shorter) last one
+        // decay powers of a full chunk and of the (possibly shorter) last one:
+        // state decay gamma^L, row scale gamma^(r-a), read-out copy gamma^(a+1),
+        // and gamma^(L-1-a) on dS (exactly 1 when a = L-1)
+        // (the last chunk's are evaluated where they are used, once)
         const int L_last = N - (nchunks - 1) * kC;
-        const float g_full = (float)exp2((double)kC * lg);
-        const float sc_full = (float)exp2((double)(r + 1 - kC) * lg);
-        const float g_last = (float)exp2((double)L_last * lg);
-        const float sc_last = (float)exp2((double)(r + 1 - L_last) * lg);
+        const int a_full = p.hc.anchor[h], a_last = min(a_full, L_last - 1);
+        auto pw = [&](int e) { return (float)exp2((double)e * lg); };
+        const float g_full = pw(kC), sc_full = pw(r - a_full), t_full = pw(a_full + 1), f_full = pw(kC - 1 - a_full);
         if (has_init) {
             // Continue from the given state: R = S_init, and the first read-out
-            // uses T = gamma^L0 S_init (L0 the first chunk's length).
-            const float g0 = nchunks == 1 ? g_last : g_full;
+            // uses T = gamma^(a0+1) S_init (a0 the first chunk's anchor).
+            const float g0 = nchunks == 1 ? pw(a_last + 1) : t_full;
 #pragma unroll
             for (int part = 0; part < kParts; part++) {
                 const int dr = part * kPartDk + r;
@@ -573,6 +916,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             // ---- mask: P = tril(A) as packed bf16 into TMEM, 32 A columns at a time
             ok = tc::mbar_wait(&bars.afull, jc & 1);
             if (!ok) break;
+            // fused: every load of this chunk from the ring has landed (A read
+            // all of Q and K'), so the slot may be rewritten as far as this CTA goes
+            if constexpr (FUSED)
+                if (warp == 8 && lane == 0) count_release(p.consumed + gl * kRing + jc % kRing);
             tc::tc_fence_after();
             {
 #pragma unroll
@@ -600,19 +947,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             if (!ok) break;
             tc::tc_fence_after();
             {
-                const float gL = last ? g_last : g_full;
+                const float gL = last ? pw(L_last) : g_full, fD = last ? pw(L_last - 1 - a_last) : f_full;
 #pragma unroll
                 for (int part = 0; part < kParts; part++) {
                     uint32_t d[32];
                     tc::tmem_ld32(tb + lane_off + kTD + part * kW + 32 * wg, d);
                     tc::tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; i++) R[part][i] = fmaf(gL, R[part][i], __uint_as_float(d[i]));
+                    for (int i = 0; i < 32; i++) R[part][i] = fmaf(gL, R[part][i], fD * __uint_as_float(d[i]));
                 }
                 tc::tc_fence_before();
                 elect_arrive(&bars.dsfree, lane);
                 if (!last) {
-                    const float gN = (jc + 1 == nchunks - 1) ? g_last : g_full;
+                    const float gN = (jc + 1 == nchunks - 1) ? pw(a_last + 1) : t_full;
                     // T is overwritten only once this chunk's read-out has consumed it
                     ok = tc::mbar_wait(&bars.qtm, jc & 1);
                     if (!ok) break;
@@ -662,7 +1009,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                         // P V completed) in the TMA's 128-byte swizzle, then one
                         // thread stores it: rows past N are clipped by the TMA.
                         uint8_t* sO = sm + WsSmem<DK>::kV + (jc & 1) * kVBytes;
-                        const float sc = (last ? sc_last : sc_full) * rs;
+                        const float sc = (last ? pw(r - a_last) : sc_full) * rs;
 #pragma unroll
                         for (int c16 = 0; c16 < 4; c16++) {
                             const int base = c16 * 8;
@@ -687,7 +1034,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                         const bool direct = p.out_rev && last && L < kC;
                         if (!direct) {
                             uint8_t* sO = sm + WsSmem<DK>::kV + (jc & 1) * kVBytes;
-                            const float sc = (last ? sc_last : sc_full) * rs;
+                            const float sc = (last ? pw(r - a_last) : sc_full) * rs;
                             const uint32_t srow = p.out_rev ? (uint32_t)(kC - 1 - r) : (uint32_t)r;
                             if (wg == 1) {
                                 ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars.ohalf[jc & 1], (jc >> 1) & 1));
@@ -708,7 +1055,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                     }
                 }
                 if (r < L) {
-                    const float sc = (last ? sc_last : sc_full) * rs;
+                    const float sc = (last ? pw(r - a_last) : sc_full) * rs;
                     const int n = p.out_rev ? N - 1 - (n0 + r) : n0 + r;
                     Tout* dst = reinterpret_cast<Tout*>(p.out) + (((size_t)b * N + n) * p.H + h) * p.dv + j0 + 32 * wg;
                     if constexpr (sizeof(Tout) == 2) {
@@ -751,7 +1098,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
 
 template <int DK, typename Tout>
 ret_status launch_main(const WsParams& p, cudaStream_t s) {
-    auto kern = k_chunkwise_ws<DK, Tout>;
+    auto kern = k_chunkwise_ws<DK, Tout, false>;
     const int smem = (int)WsSmem<DK>::kBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return check_launch("chunkwise (workspace path): smem attribute");
@@ -786,14 +1133,22 @@ size_t chunkwise_ws_bytes(const RetArgs& a) {
     return q_copied(a) ? 2 * qk : qk;
 }
 
-bool chunkwise_ws_supported(const RetArgs& a) {
+bool chunkwise_ws_shape_ok(const RetArgs& a) {
     if (a.in_dt != RET_BF16) return false;
     if (a.chunk != kC || !(a.dk == 128 || a.dk == 256) || a.dv % kW != 0) return false;
     if (a.N > (1 << 30)) return false;
     if ((long long)a.B * a.H * (a.dv / kW) > (1ll << 30)) return false;
-    for (int h = 0; h < a.H; h++)
-        if (!(a.hc.log2g[h] * kC >= -60.0)) return false;
     return true;
+}
+
+int chunkwise_heads_below(const RetArgs& a, int min_anchor) {
+    int n = 0;
+    for (int h = 0; h < a.H; h++) n += a.hc.anchor[h] < min_anchor;
+    return n;
+}
+
+bool chunkwise_ws_supported(const RetArgs& a) {
+    return chunkwise_ws_shape_ok(a) && chunkwise_heads_below(a, 0) == 0;
 }
 
 // Tensor maps and per-launch fields shared by both kernel variants.
@@ -834,6 +1189,161 @@ static ret_status fill_params(WsParams* p, const RetArgs& a, const void* q_src, 
         }
         p->tma_out = 1;
     }
+    return RET_OK;
+}
+
+// ------------------------------------------------------ fused rotation
+//
+// The CTAs of one head wait on one another's ring writes, so a launch holds
+// no more heads than can be resident at once; it is launched cooperatively,
+// which makes the runtime refuse (rather than run) a grid that could not be
+// co-resident.  Larger problems run as several launches, one per group of
+// heads, on the same scratch.
+
+constexpr int kFusedCtaCap = 148;   // CTAs the scratch of one launch is sized for (one per SM of a B200)
+
+static int fused_group_cap(const RetArgs& a) {
+    const int nt = a.dv / kW;
+    const long long bh = (long long)a.B * a.H;
+    return (int)std::min<long long>(bh, std::max(1, kFusedCtaCap / nt));
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Scratch: ready[G][kRing], consumed[G][kRing] (u32), then the q and k'
+// rings, [G, kRing, 128, dk] bf16 each.
+static size_t fused_counter_bytes(size_t G) { return align256(2 * G * kRing * sizeof(unsigned)); }
+
+size_t chunkwise_fused_bytes(const RetArgs& a) {
+    const size_t G = (size_t)fused_group_cap(a);
+    return fused_counter_bytes(G) + 2 * G * kRing * kC * (size_t)a.dk * 2;
+}
+
+template <int DK, typename Tout>
+ret_status launch_fused(const WsParams& p, int grid, cudaStream_t s) {
+    auto kern = k_chunkwise_ws<DK, Tout, true>;
+    const int smem = (int)WsSmem<DK>::kBytes;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return check_launch("chunkwise (fused): smem attribute");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "chunkwise (fused): launch: %s", cudaGetErrorString(e));
+    return check_launch("chunkwise (fused)");
+}
+
+// CTAs of the fused kernel that fit on the current device at once.
+template <int DK, typename Tout>
+static int fused_resident(int* out) {
+    auto kern = k_chunkwise_ws<DK, Tout, true>;
+    const int smem = (int)WsSmem<DK>::kBytes;
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) != cudaSuccess)
+        return 0;
+    *out = per_sm * sms;
+    return 1;
+}
+
+ret_status launch_chunkwise_fused(const RetArgs& a, void* scratch, cudaStream_t s) {
+    const int nt = a.dv / kW;
+    const bool f32 = a.out_dt == RET_F32;
+    int resident = 0;
+    const int okr = a.dk == 256 ? (f32 ? fused_resident<256, float>(&resident) : fused_resident<256, __nv_bfloat16>(&resident))
+                                : (f32 ? fused_resident<128, float>(&resident) : fused_resident<128, __nv_bfloat16>(&resident));
+    if (!okr) return fail(RET_ERR_CUDA, "chunkwise (fused): occupancy query failed");
+    const int cap = fused_group_cap(a);
+    const int G = std::min(cap, resident / nt);
+    if (G < 1) return fail(RET_ERR_UNSUPPORTED, "chunkwise (fused): no room for the %d CTAs of one head", nt);
+    unsigned* ctr = reinterpret_cast<unsigned*>(scratch);
+    __nv_bfloat16* ring_q =
+        reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(scratch) + fused_counter_bytes((size_t)cap));
+    __nv_bfloat16* ring_k = ring_q + (size_t)cap * kRing * kC * a.dk;
+    // the tensor maps of q and k' read the rings: {dk, ring rows, head of the launch, 1}
+    WsParams p;
+    ret_status st = fill_params(&p, a, a.q, a.dk, a.k);
+    if (st != RET_OK) return st;
+    {
+        const uint64_t dk = a.dk, rows = (uint64_t)kRing * kC;
+        const uint64_t dr[4] = {dk, rows, (uint64_t)cap, 1};
+        const uint64_t sr[3] = {dk * 2, rows * dk * 2, (uint64_t)cap * rows * dk * 2};
+        const uint32_t box[4] = {64, (uint32_t)kC, 1, 1};
+        if (!make_tmap_bf16(&p.tq, ring_q, 4, dr, sr, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tmap_bf16(&p.tk, ring_k, 4, dr, sr, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return RET_ERR_CUDA;
+    }
+    const int dkr = a.dk_real ? a.dk_real : a.dk;
+    p.q_raw = reinterpret_cast<const __nv_bfloat16*>(a.q);
+    p.k_raw = reinterpret_cast<const __nv_bfloat16*>(a.k);
+    p.q_ld = a.q_ld ? a.q_ld : dkr;
+    p.k_ld = a.k_ld ? a.k_ld : dkr;
+    p.ring_q = ring_q;
+    p.ring_k = ring_k;
+    p.ready = ctr;
+    p.consumed = ctr + (size_t)cap * kRing;
+    p.xpos = a.xpos;
+    p.pos0 = a.pos_offset;
+    p.log2base = log2(a.theta_base);
+    const int BH = a.B * a.H;
+    for (int bh0 = 0; bh0 < BH; bh0 += G) {
+        const int g = std::min(G, BH - bh0);
+        p.bh0 = bh0;
+        p.nmain = g * nt;
+        cudaError_t e = cudaMemsetAsync(ctr, 0, 2 * (size_t)cap * kRing * sizeof(unsigned), s);
+        if (e != cudaSuccess) return fail(RET_ERR_CUDA, "chunkwise (fused): counter reset: %s", cudaGetErrorString(e));
+        if (a.dk == 256) st = f32 ? launch_fused<256, float>(p, g * nt, s) : launch_fused<256, __nv_bfloat16>(p, g * nt, s);
+        else st = f32 ? launch_fused<128, float>(p, g * nt, s) : launch_fused<128, __nv_bfloat16>(p, g * nt, s);
+        if (st != RET_OK) return st;
+    }
+    return RET_OK;
+}
+
+// The fused path on scratch from a stream-ordered pool the library keeps per
+// device (created on the first call, never trimmed): allocated and freed in
+// stream order around the launches, so concurrent calls on other streams get
+// their own scratch.
+ret_status launch_chunkwise_fused_pooled(const RetArgs& a, cudaStream_t s) {
+    constexpr int kMaxDev = 64;
+    static cudaMemPool_t pools[kMaxDev] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "chunkwise: cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDev) return fail(RET_ERR_UNSUPPORTED, "chunkwise: device %d out of range", dev);
+    cudaMemPool_t pool;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!pools[dev]) {
+            cudaMemPoolProps props = {};
+            props.allocType = cudaMemAllocationTypePinned;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            e = cudaMemPoolCreate(&pools[dev], &props);
+            if (e != cudaSuccess) {
+                pools[dev] = nullptr;
+                return fail(RET_ERR_CUDA, "chunkwise: scratch pool: %s", cudaGetErrorString(e));
+            }
+            uint64_t keep = ~0ull;
+            cudaMemPoolSetAttribute(pools[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+        }
+        pool = pools[dev];
+    }
+    void* scratch = nullptr;
+    e = cudaMallocFromPoolAsync(&scratch, chunkwise_fused_bytes(a), pool, s);
+    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "chunkwise: scratch: %s", cudaGetErrorString(e));
+    const ret_status st = launch_chunkwise_fused(a, scratch, s);
+    e = cudaFreeAsync(scratch, s);
+    if (st != RET_OK) return st;
+    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "chunkwise: scratch release: %s", cudaGetErrorString(e));
     return RET_OK;
 }
 

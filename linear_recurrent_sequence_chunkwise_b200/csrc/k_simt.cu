@@ -330,8 +330,10 @@ __global__ void __launch_bounds__(256) k_recurrent_simt(const Tin* __restrict__ 
                                                         const Tin* __restrict__ v, HeadConsts hc, int N, int H,
                                                         int dk, int dv, Tout* __restrict__ out,
                                                         float* __restrict__ fstate, int xpos, long long pos0,
-                                                        double log2base) {
+                                                        double log2base, int untaken_only) {
     const int h = blockIdx.y, b = blockIdx.z;
+    // beside the tensor-core kernel: only the heads it leaves out
+    if (untaken_only && hc.anchor[h] >= 0) return;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int j = blockIdx.x * 32 + lane;
     extern __shared__ double smd[];
@@ -379,7 +381,7 @@ __global__ void __launch_bounds__(256) k_recurrent_simt(const Tin* __restrict__ 
     }
 }
 
-ret_status launch_recurrent_simt(const RetArgs& a, cudaStream_t s) {
+ret_status launch_recurrent_simt(const RetArgs& a, cudaStream_t s, bool untaken_only) {
     if (a.dk > 8 * kRecMaxRows) return fail(RET_ERR_UNSUPPORTED, "ret_forward_recurrent: dk > 256");
     const size_t bytes = (size_t)(a.dk / 2 + 1) * sizeof(double) + ((size_t)4 * a.dk + 256) * sizeof(float);
     dim3 grid((a.dv + 31) / 32, a.H, a.B);
@@ -387,7 +389,7 @@ ret_status launch_recurrent_simt(const RetArgs& a, cudaStream_t s) {
 #define RET_LAUNCH_REC(TI, TO)                                                                                \
     k_recurrent_simt<TI, TO><<<grid, 256, bytes, s>>>((const TI*)a.q, (const TI*)a.k, (const TI*)a.v, a.hc,  \
                                                       a.N, a.H, a.dk, a.dv, (TO*)a.out, a.final_state,       \
-                                                      a.xpos, a.pos_offset, lb)
+                                                      a.xpos, a.pos_offset, lb, untaken_only ? 1 : 0)
     if (a.in_dt == RET_F32 && a.out_dt == RET_F32) RET_LAUNCH_REC(float, float);
     else if (a.in_dt == RET_F32) RET_LAUNCH_REC(float, __nv_bfloat16);
     else if (a.out_dt == RET_F32) RET_LAUNCH_REC(__nv_bfloat16, float);

@@ -41,18 +41,21 @@ struct RetArgs {
 ret_status launch_xpos_rotate(void* x, ret_dtype dt, int B, int N, int H, int d, long long pos_offset,
                               double theta_base, cudaStream_t s, bool inverse = false);
 ret_status launch_chunkwise_simt(const RetArgs& a, cudaStream_t s);
-ret_status launch_chunkwise_tc(const RetArgs& a, cudaStream_t s);
 ret_status launch_parallel_simt(const RetArgs& a, cudaStream_t s);
-ret_status launch_recurrent_simt(const RetArgs& a, cudaStream_t s);
+// untaken_only: only the heads the tensor-core kernels leave out (anchor -1).
+ret_status launch_recurrent_simt(const RetArgs& a, cudaStream_t s, bool untaken_only = false);
 ret_status launch_decode(const void* q, const void* k, const void* v, const HeadConsts& hc, float* state,
                          void* out, int B, int H, int dk, int dv, ret_dtype in_dt, ret_dtype out_dt,
                          cudaStream_t s);
 
-// Does the tensor-core chunkwise kernel take this problem?
-bool chunkwise_tc_supported(const RetArgs& a);
 
 // Workspace path: prep kernel (rotation + zeta scaling into the workspace)
-// and the warp-specialized tensor-core kernel.
+// and the warp-specialized tensor-core kernel.  The shape check alone; the
+// number of heads whose anchor (HeadConsts) is below min_anchor (0: heads the
+// kernel does not take; kChunkAnchorFull: heads not on the plain factors);
+// and both together (shape on the path, every head taken).
+bool chunkwise_ws_shape_ok(const RetArgs& a);
+int chunkwise_heads_below(const RetArgs& a, int min_anchor);
 bool chunkwise_ws_supported(const RetArgs& a);
 size_t chunkwise_ws_bytes(const RetArgs& a);
 ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s);
@@ -60,6 +63,13 @@ ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s);
 // workspace the prep pass has filled (a.initial_state honoured).
 ret_status launch_chunkwise_prep(const RetArgs& a, void* ws, cudaStream_t s);
 ret_status launch_chunkwise_prepared(const RetArgs& a, void* ws, cudaStream_t s);
+// The fused path: the rotation and zeta scaling inside the tensor-core
+// kernel, the rotated rows shared by the CTAs of a head through an exchange
+// ring in `scratch` (chunkwise_fused_bytes of it, 256-byte aligned).  The
+// pooled form takes the scratch from a stream-ordered pool of the library.
+size_t chunkwise_fused_bytes(const RetArgs& a);
+ret_status launch_chunkwise_fused(const RetArgs& a, void* scratch, cudaStream_t s);
+ret_status launch_chunkwise_fused_pooled(const RetArgs& a, cudaStream_t s);
 // The workspace path on the library's fixed device array (no allocation).
 size_t chunkwise_static_ws_bytes();
 ret_status launch_chunkwise_static(const RetArgs& a, cudaStream_t s);

@@ -1,5 +1,6 @@
 // ret_api.cu -- the C ABI: argument validation, per-head constants and
-// dispatch to the kernels.  Nothing here allocates device memory.
+// dispatch to the kernels.  Nothing here allocates device memory, apart from
+// ret_forward_chunkwise's small stream-ordered scratch (see k_chunk_ws.cu).
 #include <cstring>
 #include <math.h>
 #include <stdarg.h>
@@ -30,6 +31,7 @@ bool make_head_consts(const double* gammas, int H, HeadConsts* hc) {
     if (H < 1 || H > kMaxHeads) return false;
     for (int h = 0; h < H; h++) hc->log2g[h] = log2(gammas[h]);  // -inf for gamma = 0
     for (int h = H; h < kMaxHeads; h++) hc->log2g[h] = 0.0;
+    for (int h = 0; h < kMaxHeads; h++) hc->anchor[h] = decay_anchor(hc->log2g[h]);
     return true;
 }
 
@@ -96,6 +98,19 @@ static ret_status make_args(RetArgs* a, const char* who, const void* q, const vo
 
 using namespace ret;
 
+// The workspace path's kernel takes d_k = 128 or 256.  A d_k of 64 runs on it
+// zero-padded to 128: the padded components add nothing to q . k and leave
+// the padded state rows at zero.  Its kernel blocks the sequence by 128
+// tokens, so a chunk of 64 is computed in blocks of 128 (the chunkwise form
+// gives the recurrence's result for any block length).
+static void pad_small_dk(RetArgs* a) {
+    if (a->in_dt == RET_BF16 && a->dk == 64 && (a->chunk == 64 || a->chunk == 128)) {
+        a->dk_real = 64;
+        a->dk = 128;
+        a->chunk = 128;
+    }
+}
+
 extern "C" {
 
 const char* ret_last_error_string(void) { return t_err; }
@@ -122,25 +137,23 @@ ret_status ret_forward_chunkwise(const void* q, const void* k, const void* v, co
     ret_status st = make_args(&a, "ret_forward_chunkwise", q, k, v, gammas, B, N, H, dk, dv, chunk, out,
                               final_state, in_dt, out_dt, xpos, pos_offset, theta_base);
     if (st != RET_OK) return st;
-    if (in_dt == RET_BF16 && chunkwise_tc_supported(a)) return launch_chunkwise_tc(a, stream);
+    {
+        // the tensor-core path with the rotation fused (d_k = 64 padded to 128);
+        // heads too fast for it (gamma^64 < 2^-100), if any, token by token
+        RetArgs f = a;
+        pad_small_dk(&f);
+        const int left = chunkwise_heads_below(f, 0);
+        if (chunkwise_ws_shape_ok(f) && left < H) {
+            st = launch_chunkwise_fused_pooled(f, stream);
+            if (st != RET_OK || left == 0) return st;
+            return launch_recurrent_simt(a, stream, true);
+        }
+    }
     st = launch_chunkwise_simt(a, stream);
     if (st != RET_ERR_UNSUPPORTED) return st;
     // Same function, token by token: the shape fits neither chunkwise kernel.
     t_err[0] = 0;
     return launch_recurrent_simt(a, stream);
-}
-
-// The workspace path's kernel takes d_k = 128 or 256.  A d_k of 64 runs on it
-// zero-padded to 128: the padded components add nothing to q . k and leave
-// the padded state rows at zero.  Its kernel blocks the sequence by 128
-// tokens, so a chunk of 64 is computed in blocks of 128 (the chunkwise form
-// gives the recurrence's result for any block length).
-static void pad_small_dk(RetArgs* a) {
-    if (a->in_dt == RET_BF16 && a->dk == 64 && (a->chunk == 64 || a->chunk == 128)) {
-        a->dk_real = 64;
-        a->dk = 128;
-        a->chunk = 128;
-    }
 }
 
 // The caller's d_k (before padding).
@@ -150,9 +163,9 @@ size_t ret_chunkwise_workspace_bytes(int B, int N, int H, int dk, int dv, int ch
     if (B < 1 || N < 1 || H < 1 || H > kMaxHeads || dk < 1 || dv < 1 || chunk < 1) return 0;
     RetArgs a{};
     a.B = B; a.N = N; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.in_dt = in_dt; a.xpos = xpos ? 1 : 0;
-    for (int h = 0; h < kMaxHeads; h++) a.hc.log2g[h] = 0.0;  // shape check only
+    for (int h = 0; h < kMaxHeads; h++) a.hc.log2g[h] = 0.0, a.hc.anchor[h] = kChunkAnchorFull;  // shape check only
     pad_small_dk(&a);
-    return chunkwise_ws_supported(a) ? chunkwise_ws_bytes(a) : 0;
+    return chunkwise_ws_supported(a) ? chunkwise_fused_bytes(a) : 0;
 }
 
 size_t ret_chunkwise_prepare_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk, ret_dtype in_dt,
@@ -160,7 +173,7 @@ size_t ret_chunkwise_prepare_workspace_bytes(int B, int N, int H, int dk, int dv
     if (B < 1 || N < 1 || H < 1 || H > kMaxHeads || dk < 1 || dv < 1 || chunk < 1) return 0;
     RetArgs a{};
     a.B = B; a.N = N; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.in_dt = in_dt; a.xpos = xpos ? 1 : 0;
-    for (int h = 0; h < kMaxHeads; h++) a.hc.log2g[h] = 0.0;  // shape check only
+    for (int h = 0; h < kMaxHeads; h++) a.hc.log2g[h] = 0.0, a.hc.anchor[h] = kChunkAnchorFull;  // shape check only
     pad_small_dk(&a);
     return chunkwise_ws_supported(a) ? chunkwise_ws_bytes(a) : 0;
 }
@@ -174,11 +187,13 @@ ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
     ret_status st = make_args(&a, "ret_forward_chunkwise_ws", q, k, v, gammas, B, N, H, dk, dv, chunk, out,
                               final_state, in_dt, out_dt, xpos, pos_offset, theta_base);
     if (st != RET_OK) return st;
+    const RetArgs caller = a;
     pad_small_dk(&a);
-    if (!chunkwise_ws_supported(a)) return ret_forward_chunkwise(q, k, v, gammas, B, N, H, dk, dv, chunk, out,
-                                                                 final_state, stream, in_dt, out_dt, xpos,
-                                                                 pos_offset, theta_base);
-    const size_t need = chunkwise_ws_bytes(a);
+    const int left = chunkwise_heads_below(a, 0);
+    if (!chunkwise_ws_shape_ok(a) || left == H)
+        return ret_forward_chunkwise(q, k, v, gammas, B, N, H, dk, dv, chunk, out, final_state, stream, in_dt,
+                                     out_dt, xpos, pos_offset, theta_base);
+    const size_t need = chunkwise_fused_bytes(a);
     if (!workspace || workspace_bytes < need)
         return fail(RET_ERR_INVALID_ARG, "ret_forward_chunkwise_ws: workspace of %zu bytes needed (got %zu)", need,
                     workspace ? workspace_bytes : (size_t)0);
@@ -190,7 +205,10 @@ ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
         overlaps(workspace, need, out, bo) ||
         (final_state && overlaps(workspace, need, final_state, (size_t)B * H * dk * dv * 4)))
         return fail(RET_ERR_INVALID_ARG, "ret_forward_chunkwise_ws: workspace overlaps another buffer");
-    return launch_chunkwise_ws(a, workspace, stream);
+    st = launch_chunkwise_fused(a, workspace, stream);
+    if (st != RET_OK || left == 0) return st;
+    // heads too fast for the tensor-core kernel, token by token
+    return launch_recurrent_simt(caller, stream, true);
 }
 
 // Workspace checks shared by the workspace-path entry points.
@@ -287,7 +305,7 @@ size_t ret_normalized_workspace_bytes(int B, int N, int H, int dk, int dv, int c
     if (B < 1 || N < 1 || H < 1 || H > kMaxHeads || dk < 1 || dv < 1 || chunk < 1) return 0;
     RetArgs a{};
     a.B = B; a.N = N; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.in_dt = in_dt; a.xpos = xpos ? 1 : 0;
-    for (int h = 0; h < kMaxHeads; h++) a.hc.log2g[h] = 0.0;  // shape check only
+    for (int h = 0; h < kMaxHeads; h++) a.hc.log2g[h] = 0.0, a.hc.anchor[h] = kChunkAnchorFull;  // shape check only
     return chunkwise_ws_supported(a) ? normalized_ws_bytes(a) : 0;
 }
 
@@ -306,7 +324,7 @@ ret_status ret_forward_chunkwise_normalized(const void* q, const void* k, const 
     if (norm_flags & ~(RET_NORM_DECAY | RET_NORM_SCORE))
         return fail(RET_ERR_INVALID_ARG, "%s: norm_flags must combine RET_NORM_DECAY and RET_NORM_SCORE", who);
     if (pos_offset < 0) return fail(RET_ERR_INVALID_ARG, "%s: pos_offset must be >= 0", who);
-    if (!chunkwise_ws_supported(a))
+    if (!chunkwise_ws_supported(a) || chunkwise_heads_below(a, kChunkAnchorFull) > 0)
         return fail(RET_ERR_UNSUPPORTED,
                     "%s: needs bf16 inputs, chunk 128, dk 128 or 256, dv a multiple of 64 and every "
                     "gamma_h^128 >= 2^-60",
@@ -422,7 +440,7 @@ ret_status ret_forward_chunkwise_noalloc(const void* q, const void* k, const voi
     if (!chunkwise_ws_supported(a))
         return fail(RET_ERR_UNSUPPORTED,
                     "ret_forward_chunkwise_noalloc: needs bf16 inputs, chunk 128, dk 128 or 256, dv a multiple of "
-                    "64 and every gamma_h^128 >= 2^-60");
+                    "64 and every gamma_h^64 >= 2^-100");
     return launch_chunkwise_static(a, stream);
 }
 
@@ -601,7 +619,8 @@ ret_status ret_msr_forward(const void* X, const void* Wq, const void* Wk, const 
     // the retention step runs on the tensor-core kernel only
     RetArgs a{};
     a.B = B; a.in_dt = RET_BF16; a.chunk = chunk; a.dk = dk; a.dv = dv; a.N = N; a.H = H; a.hc = m.hc;
-    if (!chunkwise_ws_supported(a))
+    // (the projection epilogue scales the keys by the plain zeta)
+    if (!chunkwise_ws_supported(a) || chunkwise_heads_below(a, kChunkAnchorFull) > 0)
         return fail(RET_ERR_UNSUPPORTED, "%s: needs chunk 128, d_k 128 or 256, d_v a multiple of 64 and "
                     "gamma_h^128 >= 2^-60", who);
     if (!(dv == 128 || dv == 256 || dv == 512 || dv == 1024))
@@ -650,7 +669,7 @@ ret_status ret_retnet_block_forward(const void* X, const void* ln1_gain, const v
     RetArgs a{};
     a.B = B; a.in_dt = RET_BF16; a.chunk = chunk; a.dk = dk; a.dv = dv; a.N = N; a.H = H;
     make_head_consts(gammas, H, &a.hc);
-    if (!chunkwise_ws_supported(a))
+    if (!chunkwise_ws_supported(a) || chunkwise_heads_below(a, kChunkAnchorFull) > 0)
         return fail(RET_ERR_UNSUPPORTED, "%s: needs chunk 128, d_k 128 or 256, d_v a multiple of 64 and "
                     "gamma_h^128 >= 2^-60", who);
     if (!(dv == 128 || dv == 256 || dv == 512 || dv == 1024))
@@ -696,12 +715,11 @@ ret_status ret_check_device_error(cudaStream_t stream) {
     t_err[0] = 0;
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return fail(RET_ERR_CUDA, "ret_check_device_error: %s", cudaGetErrorString(e));
-    int flag = 0, flag2 = 0, flag3 = 0;
-    e = read_clear_error_chunk_tc(&flag);
-    if (e == cudaSuccess) e = read_clear_error_chunk_ws(&flag2);
-    if (e == cudaSuccess) e = read_clear_error_gemm(&flag3);
+    int flag = 0, flag2 = 0;
+    e = read_clear_error_chunk_ws(&flag);
+    if (e == cudaSuccess) e = read_clear_error_gemm(&flag2);
     if (e != cudaSuccess) return fail(RET_ERR_CUDA, "ret_check_device_error: %s", cudaGetErrorString(e));
-    flag |= flag2 | flag3;
+    flag |= flag2;
     if (flag) return fail(RET_ERR_TIMEOUT, "a kernel gave up a bounded wait (device error word %d)", flag);
     return RET_OK;
 }

@@ -137,9 +137,31 @@ def prepared_call(ws=WS, nbytes=WS_BYTES, init=None, fs=None, dk=128, out=P4):
 
 
 def test_workspace_size_matches_the_two_pass_shape():
-    assert R.ret_chunkwise_workspace_bytes(1, 128, 2, 128, 64, 128, torch.bfloat16, False) == WS_BYTES
-    assert R.ret_chunkwise_workspace_bytes(1, 128, 2, 128, 64, 128, torch.bfloat16, True) == 2 * QK_BYTES
-    assert R.ret_chunkwise_workspace_bytes(3, 1000, 2, 128, 64, 128, torch.bfloat16, True) == 2 * 3 * 1000 * 2 * 128 * 2
+    ws = R.ret_chunkwise_prepare_workspace_bytes
+    assert ws(1, 128, 2, 128, 64, 128, torch.bfloat16, False) == WS_BYTES
+    assert ws(1, 128, 2, 128, 64, 128, torch.bfloat16, True) == 2 * QK_BYTES
+    assert ws(3, 1000, 2, 128, 64, 128, torch.bfloat16, True) == 2 * 3 * 1000 * 2 * 128 * 2
+    assert ws(1, 128, 2, 16, 64, 128, torch.bfloat16, False) == 0
+
+
+def _fused_bytes(B, H, dk, dv):
+    """Scratch of the fused forward: per head of one launch (at most 148 CTAs,
+    dv / 64 per head) two u32 counts per ring slot, then the q and k' rings of
+    6 chunk slots of 128 rows each."""
+    G = min(B * H, 148 // (dv // 64))
+    ctr = (2 * G * 6 * 4 + 255) // 256 * 256
+    return ctr + 2 * G * 6 * 128 * dk * 2
+
+
+@pytest.mark.parametrize("B,N,H,dk,dv,xpos", [
+    (1, 128, 2, 128, 64, False), (1, 8192, 16, 256, 512, True), (64, 1024, 16, 256, 512, False),
+    (4, 2048, 8, 64, 64, True),
+])
+def test_fused_workspace_size_is_a_ring_not_the_sequence(B, N, H, dk, dv, xpos):
+    dkk = 128 if dk == 64 else dk
+    got = R.ret_chunkwise_workspace_bytes(B, N, H, dk, dv, 64 if dk == 64 else 128, torch.bfloat16, xpos)
+    assert got == _fused_bytes(B, H, dkk, dv)
+    assert got <= 160 << 20      # independent of N; at most 148 heads of rings
     assert R.ret_chunkwise_workspace_bytes(1, 128, 2, 16, 64, 128, torch.bfloat16, False) == 0
 
 
@@ -201,7 +223,7 @@ def test_backward_rejects_bad_arguments(kw, status):
 
 def test_normalized_workspace_size():
     nb = R.ret_normalized_workspace_bytes(1, 200, 2, 128, 64, 128, torch.bfloat16, True)
-    ws = R.ret_chunkwise_workspace_bytes(1, 200, 2, 128, 64, 128, torch.bfloat16, True)
+    ws = R.ret_chunkwise_prepare_workspace_bytes(1, 200, 2, 128, 64, 128, torch.bfloat16, True)
     # the prepared q, k, then row factors [B, N, H], key sums per 32 rows and per chunk start
     al = lambda x: (x + 255) // 256 * 256
     assert nb == al(ws) + al(200 * 2 * 4) + al(2 * 7 * 128 * 4) + al(2 * 2 * 128 * 4)

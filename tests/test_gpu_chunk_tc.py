@@ -68,8 +68,10 @@ def test_chunkwise_tc_small(B, N, H, dk, dv, xpos, off, out_dtype):
 
 @pytest.mark.parametrize("gam", [1.0, 0.75, 0.6, 0.0])
 def test_chunkwise_degenerate_decays(gam):
-    """gamma 1 and 0.75 (0.75^128 = 2^-53) run on the tensor cores; 0.6 and 0
-    (gamma^128 below 2^-60) take the recurrent GPU kernel; all must match the
+    """gamma 1 and 0.75 (0.75^128 = 2^-53) run on the tensor cores with the
+    decay anchored at the chunk's last row; 0.6 (0.6^128 below 2^-60, 0.6^64
+    above 2^-100) with the anchor at row 63; gamma 0 is left to the recurrent
+    kernel while the other head stays on the tensor cores; all must match the
     oracle."""
     q, k, v = qkv(50, 1, 260, 2, 256, 64, 1 / 16)
     g = np.array([gam, 0.99])
@@ -154,3 +156,64 @@ def test_msr_core_shape():
     o = out.cpu().numpy()
     got = np.stack([o[b, :, h] for b, h in picks], axis=1)[None].astype(np.float64)
     assert err_out(got, ref) < TOL_BF16
+
+
+def _kernels_launched(fn):
+    """Names of the CUDA kernels fn() launches, from torch's profiler (CUPTI);
+    None when the profiler records no device activity here."""
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    names = {e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA}
+    return names or None
+
+
+@pytest.mark.parametrize("slow", [0.5, 0.36])
+def test_mixed_decays_stay_on_the_tensor_cores(slow):
+    """One fast-decaying head (gamma 0.5 or 0.36: gamma^128 far below 2^-60)
+    among heads on the pages' schedule: every head runs on the fused
+    tensor-core kernel (the fast one with its decay anchored at row 63), no
+    CUDA-core kernel is launched, and the result matches the oracle at the
+    workload's bar (RetNet paper summary, multi-scale decay; the pages'
+    schedule has no such head, a caller may)."""
+    B, N, H, dk, dv = 1, 1000, 4, 256, 128
+    q, k, v = qkv(61, B, N, H, dk, dv, dk ** -0.5)
+    g = np.array(list(gamma_schedule(H - 1)) + [slow])
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    res = {}
+
+    def run():
+        res["o"], res["s"] = R.ret_forward_chunkwise(qd, kd, vd, g, 128, out_dtype=torch.float32, xpos=True,
+                                                     want_final_state=True)
+    names = _kernels_launched(run)
+    R.ret_check_device_error()
+    if names is not None:
+        assert any("k_chunkwise_ws" in n for n in names), names
+        assert not any("simt" in n for n in names), names
+    ref, S = ref_of(q, k, v, g, True)
+    assert err_out(host64(res["o"]), ref) < TOL_BF16
+    assert err_state(host64(res["s"]), S) < TOL_BF16
+
+
+def test_very_fast_head_goes_to_the_recurrent_kernel_alone():
+    """gamma 0.2 (0.2^64 below 2^-100) is computed token by token while the
+    other heads stay on the tensor cores; both kernels run, and every head
+    matches the oracle."""
+    B, N, H, dk, dv = 2, 300, 3, 128, 64
+    q, k, v = qkv(62, B, N, H, dk, dv, dk ** -0.5)
+    g = np.array([0.96875, 0.2, 0.99])
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    res = {}
+
+    def run():
+        res["o"], res["s"] = R.ret_forward_chunkwise(qd, kd, vd, g, 128, out_dtype=torch.float32, xpos=True,
+                                                     want_final_state=True)
+    names = _kernels_launched(run)
+    R.ret_check_device_error()
+    if names is not None:
+        assert any("k_chunkwise_ws" in n for n in names), names
+        assert any("k_recurrent_simt" in n for n in names), names
+    ref, S = ref_of(q, k, v, g, True)
+    assert err_out(host64(res["o"]), ref) < TOL_BF16
+    assert err_state(host64(res["s"]), S) < TOL_BF16

@@ -98,8 +98,8 @@ def test_random_forward_in_two_calls(i):
     outs = []
     for lo, hi, init in ((0, split, None), (split, c["N"], S)):
         part = [t[:, lo:hi].contiguous() for t in (qd, kd, vd)]
-        nb = R.ret_chunkwise_workspace_bytes(c["B"], hi - lo, c["H"], c["dk"], c["dv"], 128, torch.bfloat16,
-                                             c["xpos"])
+        nb = R.ret_chunkwise_prepare_workspace_bytes(c["B"], hi - lo, c["H"], c["dk"], c["dv"], 128,
+                                                     torch.bfloat16, c["xpos"])
         ws = torch.full((nb,), 0x5A, dtype=torch.uint8, device="cuda")
         R.ret_chunkwise_prepare(part[0], part[1], g, 128, ws, c["dv"], xpos=c["xpos"], pos_offset=c["off"] + lo)
         outs.append(R.ret_forward_chunkwise_prepared(*part, g, 128, ws, final_state=S, initial_state=init,
