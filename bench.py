@@ -1,10 +1,11 @@
 #!/usr/bin/env python
 """Throughput of the chunkwise retention forward on B200 (one JSON line).
 
-Step: one chunkwise retention forward (xPos rotation fused into the
-tensor-core kernel, fp32 inter-chunk state, final state written) over the
-long-sequence workload B=1, N=8192, H=16, d_k=256, d_v=512, chunk 128,
-bf16 in / bf16 out, through the C ABI call ret_forward_chunkwise.  value = tokens/s of the whole job
+Step: one chunkwise retention forward (xPos rotation, fp32 inter-chunk
+state, final state written) over the long-sequence workload B=1, N=8192,
+H=16, d_k=256, d_v=512, chunk 128, bf16 in / bf16 out, through the C ABI
+call ret_forward_chunkwise (a tensor-core scores pass, then the
+warp-specialized tensor-core kernel).  value = tokens/s of the whole job
 (B*N per step per rank, summed over ranks; weak scaling, one replica per
 GPU, no collective on the data path).  The decode step (64 sequences x 16
 heads of 256x512 fp32 state) is timed in the same run and reported under
@@ -204,8 +205,9 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     # One step = one call of the spec entry point ret_forward_chunkwise:
-    # the rotation, the zeta scaling and the chunkwise forward in one fused
-    # tensor-core launch (after a 512-byte reset of its exchange counters).
+    # the scores pass (rotation, key scaling, masked intra-chunk scores on the
+    # tensor cores) and the warp-specialized tensor-core kernel, on scratch
+    # from the library's stream-ordered pool.
     def step(ev=None):
         if ev:
             ev[0].record(stream)
@@ -230,25 +232,46 @@ def run_ours(args):
         barrier()
     R.ret_check_device_error()
     times = [a.elapsed_time(b) for a, b in evs]  # ms per step
-    t_main = statistics.mean(times) / 1e3
+
+    # The same forward through the two-call form (same kernels, same work),
+    # with CUDA events between the two launches, to time each kernel alone.
+    ws2 = torch.empty(R.ret_chunkwise_prepare_workspace_bytes(B, N, H, dk, dv, C, torch.bfloat16, True),
+                      dtype=torch.uint8, device=dev)
+    split = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        e = split[i - args.warmup] if i >= args.warmup else None
+        if e:
+            e[0].record(stream)
+        R.ret_chunkwise_prepare(q, k, g, C, ws2, dv, xpos=True, stream=stream)
+        if e:
+            e[1].record(stream)
+        R.ret_forward_chunkwise_prepared(q, k, v, g, C, ws2, out=out, final_state=fs, xpos=True, stream=stream)
+        if e:
+            e[2].record(stream)
+    torch.cuda.synchronize()
+    R.ret_check_device_error()
+    del ws2
+    t_prep = statistics.mean(a.elapsed_time(b) for a, b, c in split) / 1e3
+    t_main = statistics.mean(b.elapsed_time(c) for a, b, c in split) / 1e3
     total_ms = sum(times)
     total_ms = max_over_ranks(total_ms, world, dist, dev)
     ms_per_step = total_ms / args.steps
     value = job_throughput(B * N, world, ms_per_step)
 
     peaks = load_peaks()
-    # Dominant kernel: the fused k_chunkwise_ws, timed with CUDA events around
-    # the call on the launching stream (the call is the counter reset and this
-    # one launch), mean over the timed steps.  Its algorithmic work is the
-    # whole chunkwise forward: FLOPs of the method, bytes = read q, k, v once,
-    # write out and the final state once.
+    # Dominant kernel: k_chunkwise_ws (the read-out, P V and the state
+    # update on the scores pass's output), timed with CUDA events around its
+    # launch on the launching stream, mean over the timed steps.  Its
+    # algorithmic work is taken as the whole chunkwise forward: FLOPs of the
+    # method, bytes = read q, k, v once, write out and the final state once.
     flops = flops_per_token_head(C, dk, dv) * B * N * H
     nbytes = algo_bytes(w, out_bytes=2)
     tflops = flops / t_main / 1e12
     gbs = nbytes / t_main / 1e9
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
-    traffic = load_traffic("k_chunkwise_ws_fused")
+    traffic = load_traffic("k_chunkwise_ws")
     if t_hbm >= t_tc:
         roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(gbs / peaks["hbm_gbs"], 4)}
@@ -257,7 +280,7 @@ def run_ours(args):
                 "frac": round(tflops / peaks["bf16_tflops"], 4)}
     roof["traffic"] = traffic["bytes_per_launch"] if traffic else None
     roof["peak_source"] = peaks["source"] + " (burst; the kernel is timed alone)"
-    roof["kernel"] = "k_chunkwise_ws<256, bf16, fused>"
+    roof["kernel"] = "k_chunkwise_ws<256, bf16, scores given>"
     roof["kernel_ms"] = round(t_main * 1e3, 4)
     roof["algo_flops"] = flops
     roof["algo_bytes"] = nbytes
@@ -268,6 +291,14 @@ def run_ours(args):
     roof["tensor_frac"] = round(tflops / peaks["bf16_tflops"], 4)
     roof["hbm_gbs"] = round(gbs, 1)
     roof["hbm_frac"] = round(gbs / peaks["hbm_gbs"], 4)
+    # The scores pass: reads q, k; writes q_rot, k' and P (bf16); 2 C dk
+    # FLOPs per (token, head) for the scores.
+    nchunks = (N + C - 1) // C
+    sc_bytes = 4 * B * N * H * dk * 2 + B * H * nchunks * C * C * 2
+    scores = {"kernel": "k_prep_scores<256>", "bound": "hbm", "ms": round(t_prep * 1e3, 4),
+              "achieved": round(sc_bytes / t_prep / 1e9, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+              "frac": round(sc_bytes / t_prep / 1e9 / peaks["hbm_gbs"], 4), "algo_bytes": sc_bytes,
+              "traffic": (load_traffic("k_prep_scores") or {}).get("bytes_per_launch")}
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -276,23 +307,10 @@ def run_ours(args):
         "config": {"workload": w["workload"], "B": B, "N": N, "H": H, "dk": dk, "dv": dv, "chunk": C, "xpos": True,
                    "out_dtype": "bf16", "final_state": True, "global_batch": B * world, "seq_len": N,
                    "parallelism": f"replicas x{world}", "l2": "flushed before every timed step (256 MiB write)"},
-        "roofline": roof, "clocks": clk.summary(), "gpu_launches": args.steps,
-        "path": "ret_forward_chunkwise: one cooperative launch of the warp-specialized tcgen05 kernel with the "
-                "xPos rotation and zeta scaling fused (each head's 8 CTAs share the rotated rows through an "
-                "L2-resident exchange ring), after a 512-byte counter reset",
+        "roofline": roof, "scores_pass": scores, "clocks": clk.summary(), "gpu_launches": 2 * args.steps,
+        "path": "ret_forward_chunkwise: k_prep_scores (rotation, key scaling and the masked intra-chunk scores "
+                "on tcgen05, once per head) then k_chunkwise_ws (read-out, P V, state update on tcgen05)",
     }
-    # the same forward as two calls (rotation + zeta pass, then the tensor-core
-    # kernel on the prepared rows), timed the same way, for comparison
-    ws2 = torch.empty(R.ret_chunkwise_prepare_workspace_bytes(B, N, H, dk, dv, C, torch.bfloat16, True),
-                      dtype=torch.uint8, device=dev)
-
-    def two_pass():
-        R.ret_chunkwise_prepare(q, k, g, C, ws2, dv, xpos=True, stream=stream)
-        R.ret_forward_chunkwise_prepared(q, k, v, g, C, ws2, out=out, final_state=fs, xpos=True, stream=stream)
-
-    result["two_pass_ms"] = round(_timed_flushed(torch, stream, two_pass, min(args.steps, 10), 3, world, dist, dev,
-                                                 flush), 4)
-    del ws2
     if not args.no_e2e:
         result["e2e"] = e2e_ours(R, torch, dev, stream, w, g, args, world, barrier, dist)
     if not args.no_decode:
@@ -528,7 +546,7 @@ def bench_normalized(R, torch, dev, stream, w, g, args, peaks, world, dist):
                                            out=out, final_state=fs, final_z=fz, xpos=True, stream=stream)
 
     def plain():
-        R.ret_forward_chunkwise_ws(q, k, v, g, C, ws, out=out, final_state=fs, xpos=True, stream=stream)
+        R.ret_forward_chunkwise(q, k, v, g, C, out=out, final_state=fs, xpos=True, stream=stream)
 
     steps = max(5, min(args.steps, 20))
     ms = _timed(torch, stream, norm, steps, 3, world, dist, dev)
@@ -537,7 +555,8 @@ def bench_normalized(R, torch, dev, stream, w, g, args, peaks, world, dist):
     return {"workload": w["workload"], "flags": "decay + score", "ms_per_step": round(ms, 4),
             "tokens_per_s": round(world * B * N / (ms / 1e3), 1), "plain_ms_per_step": round(ms_plain, 4),
             "overhead": round(ms / ms_plain - 1.0, 4),
-            "kernels": "k_prep_qk, k_keysum, k_keycarry, k_rowscale, k_chunkwise_ws (row factors in the epilogue)"}
+            "kernels": "k_prep_qk, k_keysum, k_keycarry, k_rowscale, k_chunkwise_ws (row factors in the epilogue)",
+            "plain": "ret_forward_chunkwise (k_prep_scores + k_chunkwise_ws)"}
 
 
 def bench_msr(R, torch, dev, stream, args, peaks, world, dist):
@@ -629,10 +648,9 @@ def _timed_flushed(torch, stream, fn, steps, warmup, world, dist, dev, flush):
 def bench_c2(R, torch, dev, stream, args, peaks, world, dist):
     """The pages' cost-analysis shape [4, 2048, 8 heads of 64], bf16, xPos,
     chunk 64, L2 flushed before every call: the spec call
-    ret_forward_chunkwise (fused rotation, d_k padded to 128 on the tensor
-    cores, 128-token blocks) beside the two-pass form (rotation pass, then
-    the tensor-core kernel).  HBM-bound: algorithmic bytes = read q, k, v
-    once, write out once (bf16)."""
+    ret_forward_chunkwise (d_k padded to 128 on the tensor cores, 128-token
+    blocks).  HBM-bound: algorithmic bytes = read q, k, v once, write out
+    once (bf16)."""
     B, N, H, dk, dv, C = 4, 2048, 8, 64, 64, 64
     gen = torch.Generator(device=dev)
     gen.manual_seed(0x5EED0009)
@@ -641,30 +659,24 @@ def bench_c2(R, torch, dev, stream, args, peaks, world, dist):
     v = torch.randn((B, N, H, dv), generator=gen, device=dev).to(torch.bfloat16)
     out = torch.empty((B, N, H, dv), dtype=torch.bfloat16, device=dev)
     g = gammas(H)
-    ws = torch.empty(R.ret_chunkwise_prepare_workspace_bytes(B, N, H, dk, dv, C, torch.bfloat16, True),
-                     dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def fused():
         R.ret_forward_chunkwise(q, k, v, g, C, out=out, xpos=True, stream=stream)
 
-    def two_pass():
-        R.ret_chunkwise_prepare(q, k, g, C, ws, dv, xpos=True, stream=stream)
-        R.ret_forward_chunkwise_prepared(q, k, v, g, C, ws, out=out, xpos=True, stream=stream)
-
     steps = max(5, min(args.steps, 20))
     ms = _timed_flushed(torch, stream, fused, steps, 3, world, dist, dev, flush)
-    ms_two = _timed_flushed(torch, stream, two_pass, steps, 3, world, dist, dev, flush)
     R.ret_check_device_error()
     nbytes = B * N * H * (2 * dk * 2 + dv * 2 + dv * 2)
     gbs = nbytes / (ms / 1e3) / 1e9
     return {"workload": "retention_bf16_4x2048x8x64", "tokens_per_s": round(world * B * N / (ms / 1e3), 1),
-            "ms_per_step": round(ms, 4), "two_pass_ms": round(ms_two, 4),
+            "ms_per_step": round(ms, 4),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gbs / peaks["hbm_gbs"], 4), "algo_bytes": nbytes,
                          "peak_source": peaks["source"]},
             "l2": "flushed before every timed call (256 MiB write)",
-            "path": "ret_forward_chunkwise: fused k_chunkwise_ws<128>, d_k padded to 128, 128-token blocks"}
+            "path": "ret_forward_chunkwise: k_prep_scores<128> + k_chunkwise_ws<128>, d_k padded to 128, "
+                    "128-token blocks"}
 
 
 def bench_fp32_small(R, torch, dev, stream, args, world, dist):

@@ -1,7 +1,7 @@
 // k_chunk_ws.cu -- chunkwise retention forward on the tensor cores: a
-// warp-specialized tcgen05 / TMEM / TMA kernel, fed either by a
-// bandwidth-bound rotation pass (two-pass form) or by its own CTAs (fused
-// form).
+// warp-specialized tcgen05 / TMEM / TMA kernel fed by a pass that rotates q
+// and k and scales the keys (and, in the scores form, also computes the
+// masked intra-chunk scores P on the tensor cores).
 //
 // Mathematics ("Hybrid Architectures: RetNet and the Three Computation
 // Paradigms", section 7.2; RetNet paper summary, Eq. 7).  For a chunk of L
@@ -49,9 +49,7 @@
 //                soon as it lands, -> TMEM once the read-out of chunk j is
 //                done; a plain smem read keeps the load traffic on the TMA
 //                path (per-row global loads from these threads measurably
-//                slow the tensor pipe down).  In the fused form these warps
-//                also rotate this CTA's share of each chunk into the head's
-//                exchange ring (see q_role_fused);
+//                slow the tensor pipe down);
 //      warps 8-15 (two warpgroups on TMEM lanes 0..127, one column half each):
 //                mask:     P = tril(A) -> packed bf16 in TMEM,
 //                state:    R = gamma^L R + gamma^(L-1-a) dS in registers
@@ -189,78 +187,27 @@ struct WsParams {
     const float* rowscale;  // [B, N, H] factor of each output row, or null
     int nmain;            // CTAs: B * H * (dv / 64), one per (b, h, 64 value columns)
     HeadConsts hc;
-    // Fused rotation (FUSED instances).  A launch takes the (b, h) pairs
-    // bh0 .. bh0 + gridDim.x / nt - 1 (nt = dv / 64 CTAs per head; bh0 = 0
-    // otherwise).  Each of a head's nt CTAs turns its 1/nt share of the rows
-    // of every chunk (xPos) from the raw q and k, scales the keys by zeta,
-    // and writes them into the head's exchange ring (kRing chunk slots in
-    // global memory, small enough to stay in L2); the tensor maps tq / tk
-    // then point at the ring.  Per (head g, slot) two counts: ready[g][slot]
-    // the shares written into the slot, consumed[g][slot] the CTAs whose
-    // loads of the slot's chunk have landed (which frees it).  Chunk i lives
-    // in slot i % kRing as its generation u = i / kRing, so it is complete
-    // when ready reaches nt (u + 1), and the slot may take chunk i + kRing
-    // once consumed reaches nt (u + 1).  (The CTAs of a head drift apart by
-    // up to kLead chunks, so one count per head would not say which chunk.)
-    int bh0;
-    const __nv_bfloat16* q_raw;
-    const __nv_bfloat16* k_raw;
-    int q_ld, k_ld;       // elements between consecutive (token, head) rows of q_raw / k_raw
-    __nv_bfloat16* ring_q;
-    __nv_bfloat16* ring_k;
-    unsigned int* ready;
-    unsigned int* consumed;
-    int xpos;
-    long long pos0;
-    double log2base;
+    // PREP instances: the masked scores P of every (b, h, chunk), bf16
+    // [B, H, nchunks, 128 query rows, 128 key columns]: tile rows
+    // ((b H + h) nchunks + j) 128 of a 2-D map {128, rows}.
+    CUtensorMap tp;
 };
-
-// Exchange ring of the fused rotation: chunk slots per head, and how many
-// chunks ahead of the one being computed the shares are written.
-constexpr int kRing = 6, kLead = 3;
-
-// Wait (bounded) until *ctr >= target, with acquire semantics at GPU scope,
-// then order the caller's later async-proxy (TMA) accesses after what it saw.
-__device__ __forceinline__ bool wait_count(const unsigned int* ctr, unsigned int target) {
-    for (uint32_t i = 0; i < (1u << 22); i++) {
-        unsigned int v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-        if (v >= target) {
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            return true;
-        }
-        __nanosleep(32);
-    }
-    return false;
-}
-
-__device__ __forceinline__ void count_release(unsigned int* ctr) {
-    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
-}
-
-// Named barrier 1 over the Q warpgroup (warps 4-7): returns whether x holds
-// in all 128 threads; also orders their memory accesses around it.
-__device__ __forceinline__ bool qwg_all(bool x) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred pi, po;\n\t"
-        "setp.ne.u32 pi, %1, 0;\n\t"
-        "bar.red.and.pred po, 1, 128, pi;\n\t"
-        "selp.u32 %0, 1, 0, po;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)x)
-        : "memory");
-    return r != 0;
-}
 
 constexpr int kKSlots = 3;                         // K' ring depth (parts of 128 d_k rows)
 constexpr int kKPartBytes = kPartDk * kC * 2;      // 32 KB
 
-template <int DK>
+constexpr int kPBytes = kC * kC * 2;              // 32 KB: the masked scores P of one chunk (bf16)
+
+// With precomputed scores (PREP) the K' parts are read by the state-update
+// issuer alone, so their ring takes two slots and the third one's space
+// holds the chunk's P tile.
+template <int DK, bool PREP>
 struct WsSmem {
+    static constexpr int kSlots = PREP ? 2 : kKSlots;
     static constexpr uint32_t kQ = 0;                              // Q staging, DK x 128 rows
     static constexpr uint32_t kK = kQ + DK * kC * 2;               // K' ring
-    static constexpr uint32_t kV = kK + kKSlots * kKPartBytes;     // 2 x 16 KB
+    static constexpr uint32_t kP = kK + kSlots * kKPartBytes;      // P tile (PREP)
+    static constexpr uint32_t kV = kP + (PREP ? kPBytes : 0);      // 2 x 16 KB
     static constexpr uint32_t kT = kV + 2 * kVBytes;               // DK x 128 B
     static constexpr uint32_t kEnd = kT + DK * 128;
     static constexpr uint32_t kBytes = kEnd + 1024;
@@ -279,6 +226,7 @@ static_assert(128 * (kRegsCtl + kRegsQ) + 256 * kRegsXf <= 512 * 128, "register 
 struct Bars {
     uint64_t qfull, qempty, kfull[kKSlots], kempty[kKSlots], vfull[2], vempty[2];
     uint64_t qready, qtm, afull, aread, pready, dsdone, dsfree, tready, ofull, ofree, ostaged[2], ostaged2[2], ohalf[2];
+    uint64_t pfull, pempty;   // the P tile's slot (precomputed scores)
 };
 
 __device__ __forceinline__ void elect_arrive(uint64_t* bar, int lane) {
@@ -314,227 +262,10 @@ __device__ __forceinline__ uint4 turn_group(uint4 x, const float (&c)[4], const 
     return x;
 }
 
-// The Q warpgroup of the fused instances.  Per chunk jq:
-//   * once the read-out of chunk jq - 1 has consumed the previous Q, the
-//     staged Q goes from shared memory into TMEM one 64-column slab at a time
-//     (few registers held), and the tensor pipe is told (qready);
-//   * the count of the chunk written in the previous iteration is released
-//     (its bulk stores have long completed, so this is cheap);
-//   * this CTA's share of chunk jq + kLead is written into the exchange ring,
-//     once the slot is free (every CTA of the head has loaded the chunk that
-//     last used it: consumed[g][slot] = nt * generation; the count is read one
-//     iteration early).  The share is the rows [r0, r0 + R) of the chunk,
-//     R = ceil(128 / nt); each thread turns one 16-byte group (pairs
-//     4g .. 4g+3) of every kStep-th row, writes it into the Q staging buffer
-//     (free until the staging buffer is handed back), and one thread copies
-//     the rows into the ring with bulk stores (pieces of up to 64 rows);
-//   * the staging buffer goes back to the TMA producer (qempty), and the raw
-//     rows of chunk jq + kLead + 1 are loaded into registers for the next
-//     iteration (their latency is hidden).
-// The rotation of a thread's first row is evaluated from the position (fp64
-// angle, reduced, then fp32 sine and cosine), the next ones by turning it
-// through kStep * theta_p; keys are also scaled by gamma^(a-r); rows past the
-// end of the sequence and groups past the caller's d_k are written as zeros.
-// The rows of the prologue (chunks 0 .. kLead - 1) are written before the
-// loop, and the staging buffer is handed to the producer once (qempty phase
-// 0) before it loads the first Q.  The warpgroup agrees on every wait's
-// outcome (named barrier 1), so a timed-out wait cannot strand part of it at
-// a barrier.  Returns false on a timeout.
-template <int DK>
-__device__ __forceinline__ bool q_role_fused(const WsParams& p, uint8_t* sQ, uint32_t tb, uint32_t lane_off, int r,
-                                             int quarter, int lane, int nt, int jt, int gl, int b, int h,
-                                             int nchunks, double lg, int anc, Bars& bars) {
-    constexpr int kGpr = DK / 8;             // 16-byte groups in a row
-    constexpr int kRpw = 32 / kGpr;          // rows one warp covers at a time
-    constexpr int kStep = 4 * kRpw;          // rows between one thread's rows
-    constexpr int kBatch = 4;                // rows whose loads are in flight together
-    constexpr int kPiece = (DK * kC * 2) / (4 * DK);   // rows of q and k the staging buffer holds (64)
-    const int N = p.N, H = p.H;
-    const int grp = lane % kGpr;
-    const int rsub = quarter * kRpw + lane / kGpr;     // row offset within a step
-    const bool real = 8 * grp < p.dks;       // inside the caller's d_k
-    const bool turn = p.xpos && real;
-    const int wtid = quarter * 32 + lane;
-    const int R = (kC + nt - 1) / nt;
-    const int r0 = min(R * jt, kC), r1 = min(r0 + R, kC);
-    // theta_p = base^(-2p/d_k) of the thread's four pairs (fp64), and the
-    // turn through kStep positions
-    double theta[4];
-    float cstep[4], sstep[4];
-    {
-        const double inv_dk = 1.0 / p.dks;
-#pragma unroll
-        for (int k = 0; k < 4; k++) {
-            theta[k] = turn ? exp2(-2.0 * (4 * grp + k) * inv_dk * p.log2base) : 0.0;
-            cstep[k] = 1.f;
-            sstep[k] = 0.f;
-            if (turn) __sincosf(angle_mod_2pi((double)kStep * theta[k]), &sstep[k], &cstep[k]);
-        }
-    }
-    auto raw_row = [&](int i, int rr) { return ((size_t)b * N + (size_t)i * kC + rr) * H + h; };
-    // the raw rows rb, rb + kStep, ... (kBatch of them) of chunk i
-    auto load_rows = [&](int i, int rb, uint4 (&qw)[kBatch], uint4 (&kw)[kBatch]) {
-        const int L = i < nchunks ? min(kC, N - i * kC) : 0;
-#pragma unroll
-        for (int u = 0; u < kBatch; u++) {
-            const int rr = rb + u * kStep;
-            qw[u] = kw[u] = make_uint4(0, 0, 0, 0);
-            if (real && rr < L && rr < r1) {
-                const size_t row = raw_row(i, rr);
-                qw[u] = __ldg(reinterpret_cast<const uint4*>(p.q_raw + row * p.q_ld + 8 * grp));
-                kw[u] = __ldg(reinterpret_cast<const uint4*>(p.k_raw + row * p.k_ld + 8 * grp));
-            }
-        }
-    };
-    // thread 0: the consumed count of the slot the next write takes
-    unsigned seen = 0;
-    auto peek = [&](int i) {
-        if (wtid == 0 && i >= kRing && i < nchunks)
-            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];"
-                         : "=r"(seen)
-                         : "l"(p.consumed + gl * kRing + i % kRing)
-                         : "memory");
-    };
-    uint4 aq[kBatch], ak[kBatch];   // raw rows of the next chunk to write, loaded ahead
-
-    // This CTA's share of chunk i into the ring (the first kBatch rows of the
-    // thread from aq / ak); the bulk stores are left in flight.
-    auto write_share = [&](int i) -> bool {
-        bool okp = true;
-        if (i >= kRing && wtid == 0) {
-            const unsigned need = (unsigned)(nt * (i / kRing));
-            if (seen < need) okp = wait_count(p.consumed + gl * kRing + i % kRing, need);
-        }
-        if (!qwg_all(okp)) return false;
-        const int n0 = i * kC, L = min(kC, N - n0);
-        const size_t slot0 = ((size_t)gl * kRing + (size_t)(i % kRing)) * kC;   // ring row of the slot's row 0
-        float cs[4], sn[4];
-        const double pos = (double)(p.pos0 + n0 + r0 + rsub);
-#pragma unroll
-        for (int k = 0; k < 4; k++) {
-            cs[k] = 1.f;
-            sn[k] = 0.f;
-            if (turn) __sincosf(angle_mod_2pi(pos * theta[k]), &sn[k], &cs[k]);
-        }
-        for (int p0 = r0; p0 < r1; p0 += kPiece) {
-            const int p1 = min(p0 + kPiece, r1);
-            uint8_t* stq = sQ;
-            uint8_t* stk = sQ + (size_t)kPiece * DK * 2;
-            // rows rb, rb + kStep, ... (kBatch of them) from qw / kw into the staging buffer
-            auto put = [&](int rb, uint4 (&qw)[kBatch], uint4 (&kw)[kBatch]) {
-#pragma unroll
-                for (int u = 0; u < kBatch; u++) {
-                    const int rr = rb + u * kStep;
-                    if (rr >= p1) break;
-                    uint4 qo = qw[u], ko = kw[u];
-                    if (real && rr < L) {
-                        // k' scale gamma^(a-r), a = min(anchor, L-1): exponent in fp64, exp2 in fp32
-                        const float zeta = exp2f((float)((double)(min(anc, L - 1) - rr) * lg));
-                        float ck[4], sk[4];
-#pragma unroll
-                        for (int k = 0; k < 4; k++) {
-                            ck[k] = cs[k] * zeta;
-                            sk[k] = sn[k] * zeta;
-                        }
-                        qo = turn_group(qo, cs, sn);
-                        ko = turn_group(ko, ck, sk);
-                    }
-                    const size_t o = ((size_t)(rr - p0) * DK + 8 * grp) * 2;
-                    *reinterpret_cast<uint4*>(stq + o) = qo;
-                    *reinterpret_cast<uint4*>(stk + o) = ko;
-                    if (turn) {
-#pragma unroll
-                        for (int k = 0; k < 4; k++) {
-                            const float c2 = cs[k] * cstep[k] - sn[k] * sstep[k];
-                            sn[k] = sn[k] * cstep[k] + cs[k] * sstep[k];
-                            cs[k] = c2;
-                        }
-                    }
-                }
-            };
-            for (int rb = p0 + rsub; rb < p1; rb += kBatch * kStep) {
-                if (rb == r0 + rsub) {
-                    put(rb, aq, ak);
-                } else {
-                    uint4 qw[kBatch], kw[kBatch];
-                    load_rows(i, rb, qw, kw);
-                    put(rb, qw, kw);
-                }
-            }
-            // the staged rows go to the ring by one thread's bulk stores; the
-            // staging buffer is reused once they have been read
-            tc::fence_proxy_async_smem();
-            qwg_all(true);
-            if (wtid == 0) {
-                const uint32_t bytes = (uint32_t)(p1 - p0) * DK * 2;
-                tc::bulk_store(p.ring_q + (slot0 + p0) * DK, stq, bytes);
-                tc::bulk_store(p.ring_k + (slot0 + p0) * DK, stk, bytes);
-                tc::bulk_commit_group();
-                tc::bulk_wait_group_read<0>();
-            }
-            qwg_all(true);
-        }
-        return true;
-    };
-    // thread 0: once the bulk stores of chunk i have completed, its count
-    auto release = [&](int i) {
-        if (wtid == 0) {
-            tc::bulk_wait_group<0>();
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            count_release(p.ready + gl * kRing + i % kRing);
-        }
-    };
-
-    for (int i = 0; i < kLead && i < nchunks; i++) {
-        load_rows(i, r0 + rsub, aq, ak);
-        if (!write_share(i)) return false;
-        release(i);
-    }
-    // the staging buffer is the producer's from here on (qempty phase 0)
-    elect_arrive(&bars.qempty, lane);
-    load_rows(kLead, r0 + rsub, aq, ak);
-    for (int jq = 0; jq < nchunks; jq++) {
-        peek(jq + kLead);
-        if (jq > 0 && !qwg_all(tc::mbar_wait(&bars.qtm, (jq - 1) & 1))) return false;
-        if (!qwg_all(tc::mbar_wait(&bars.qfull, jq & 1))) return false;
-        tc::tc_fence_after();
-        // one slab at a time (32 registers of Q in flight)
-#pragma unroll 1
-        for (int g = 0; g < DK / 64; g++) {
-            uint32_t w[32];
-#pragma unroll
-            for (int c16 = 0; c16 < 8; c16++) {
-                const uint4 x = *reinterpret_cast<const uint4*>(sQ + g * (kC * 128) +
-                                                                tc::sw128_off((uint32_t)r, (uint32_t)c16));
-                w[4 * c16 + 0] = x.x;
-                w[4 * c16 + 1] = x.y;
-                w[4 * c16 + 2] = x.z;
-                w[4 * c16 + 3] = x.w;
-            }
-            tc::tmem_st32(tb + lane_off + kTQ + 32 * g, w);
-        }
-        tc::tmem_st_wait();
-        tc::tc_fence_before();
-        elect_arrive(&bars.qready, lane);
-        const int i = jq + kLead;
-        if (jq > 0 && i - 1 < nchunks) release(i - 1);
-        if (i < nchunks) {
-            // (the staging buffer's reads above are done: the TMEM stores
-            // consumed their registers, and every thread has passed them)
-            qwg_all(true);
-            if (!write_share(i)) return false;
-        }
-        // the staging buffer goes back to the producer: the generic reads and
-        // writes above are ordered before its next async-proxy write
-        tc::fence_proxy_async_smem();
-        elect_arrive(&bars.qempty, lane);
-        if (i < nchunks) load_rows(i + 1, r0 + rsub, aq, ak);
-    }
-    return true;
-}
-
-template <int DK, typename Tout, bool FUSED>
+template <int DK, typename Tout, bool PREP>
 __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_constant__ WsParams p) {
+    using Sm = WsSmem<DK, PREP>;
+    constexpr int kSl = Sm::kSlots;   // K' ring slots
     constexpr int kParts = DK / kPartDk;
     constexpr int kQSlabs = DK / 64;
     extern __shared__ uint8_t smem_raw[];
@@ -545,8 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nt = p.dv / kW, jt = (int)blockIdx.x % nt;     // this CTA's 64 value columns
-    const int gl = (int)blockIdx.x / nt;                      // this launch's head index
-    const int h = (p.bh0 + gl) % p.H, b = (p.bh0 + gl) / p.H;
+    const int h = ((int)blockIdx.x / nt) % p.H, b = (int)blockIdx.x / (nt * p.H);
     const int j0 = jt * kW;
     const int N = p.N;
     const int nchunks = (N + kC - 1) / kC;
@@ -561,10 +291,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
     if (tid == 0) {
         tc::mbar_init(&bars.qfull, 1);
         tc::mbar_init(&bars.qempty, 4);
-        for (int i = 0; i < kKSlots; i++) {
+        for (int i = 0; i < kSl; i++) {
             tc::mbar_init(&bars.kfull[i], 1);
-            tc::mbar_init(&bars.kempty[i], 2);  // read by both issuers
+            tc::mbar_init(&bars.kempty[i], PREP ? 1 : 2);  // read by both issuers (one with P given)
         }
+        tc::mbar_init(&bars.pfull, 1);
+        tc::mbar_init(&bars.pempty, 1);
         for (int i = 0; i < 2; i++) {
             tc::mbar_init(&bars.vfull[i], 1);
             tc::mbar_init(&bars.vempty[i], p.tma_out ? 1 : 2);
@@ -590,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         tc::prefetch_tmap(&p.tq);
         tc::prefetch_tmap(&p.tk);
         tc::prefetch_tmap(&p.tv);
+        if (PREP) tc::prefetch_tmap(&p.tp);
     }
     if (warp == 1) tc::tmem_alloc(&s_tmem, 512);
     tc::tc_fence_before();
@@ -604,49 +337,48 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             // -------------------------------------------- TMA producer
             // L2 prefetch of chunk jp: the CTAs of one head split the Q and K'
             // boxes between them; each prefetches its own V tile.
-            // (the fused ring is written into L2 by the CTAs themselves)
+            // (the CTAs of a head split the Q and K' boxes between them)
             auto prefetch = [&](int jp) {
                 if (jp >= nchunks) return;
                 const int n0p = jp * kC;
-                if constexpr (!FUSED)
-                    for (int i = jt; i < 2 * kQSlabs; i += nt)
-                        tc::tma_prefetch_l2_4d(i < kQSlabs ? &p.tq : &p.tk, 64 * (i % kQSlabs), h, n0p, b);
+                for (int i = jt; i < 2 * kQSlabs; i += nt)
+                    tc::tma_prefetch_l2_4d(i < kQSlabs ? &p.tq : &p.tk, 64 * (i % kQSlabs), h, n0p, b);
                 tc::tma_prefetch_l2_4d(&p.tv, j0, h, n0p, b);
             };
             prefetch(0);
             prefetch(1);
             for (int jc = 0; jc < nchunks && ok; jc++) {
                 const int n0 = jc * kC;
-                // coordinates of the chunk's rows in the q / k' tensor maps:
-                // (head, token, batch), or (ring row, head of the launch, 0)
-                const int c1 = FUSED ? (jc % kRing) * kC : h, c2 = FUSED ? gl : n0, c3 = FUSED ? 0 : b;
                 prefetch(jc + 2);
-                // (fused: the Q warpgroup hands the staging buffer over once after
-                // writing its first ring rows, so chunk jc waits for phase jc)
-                if (FUSED) ok = tc::mbar_wait(&bars.qempty, jc & 1);
-                else if (jc > 0) ok = tc::mbar_wait(&bars.qempty, (jc - 1) & 1);
-                // fused: every CTA of the head has written its share of the chunk
-                if (FUSED && ok)
-                    ok = wait_count(p.ready + gl * kRing + jc % kRing, (unsigned)(nt * (jc / kRing + 1)));
+                if (jc > 0) ok = tc::mbar_wait(&bars.qempty, (jc - 1) & 1);
                 if (!ok) break;
                 tc::mbar_arrive_expect_tx(&bars.qfull, DK * kC * 2);
                 for (int s = 0; s < kQSlabs; s++)
-                    tc::tma_load_4d(sm + WsSmem<DK>::kQ + s * (kC * 128), &p.tq, &bars.qfull, 64 * s, c1, c2, c3);
+                    tc::tma_load_4d(sm + Sm::kQ + s * (kC * 128), &p.tq, &bars.qfull, 64 * s, h, n0, b);
                 for (int part = 0; part < kParts && ok; part++) {
-                    const int g = jc * kParts + part, slot = g % kKSlots, u = g / kKSlots;
+                    const int g = jc * kParts + part, slot = g % kSl, u = g / kSl;
                     if (u > 0) ok = tc::mbar_wait(&bars.kempty[slot], (u - 1) & 1);
                     if (!ok) break;
-                    uint8_t* dst = sm + WsSmem<DK>::kK + slot * kKPartBytes;
+                    uint8_t* dst = sm + Sm::kK + slot * kKPartBytes;
                     tc::mbar_arrive_expect_tx(&bars.kfull[slot], kKPartBytes);
                     for (int s = 0; s < 2; s++)
-                        tc::tma_load_4d(dst + s * (kC * 128), &p.tk, &bars.kfull[slot], part * kPartDk + 64 * s, c1,
-                                        c2, c3);
+                        tc::tma_load_4d(dst + s * (kC * 128), &p.tk, &bars.kfull[slot], part * kPartDk + 64 * s, h,
+                                        n0, b);
                 }
                 const int vs = jc & 1;
                 if (ok && jc >= 2) ok = tc::mbar_wait(&bars.vempty[vs], ((jc >> 1) & 1) ^ 1);
                 if (!ok) break;
                 tc::mbar_arrive_expect_tx(&bars.vfull[vs], kVBytes);
-                tc::tma_load_4d(sm + WsSmem<DK>::kV + vs * kVBytes, &p.tv, &bars.vfull[vs], j0, h, n0, b);
+                tc::tma_load_4d(sm + Sm::kV + vs * kVBytes, &p.tv, &bars.vfull[vs], j0, h, n0, b);
+                if constexpr (PREP) {
+                    // the chunk's masked scores, once the P V of the previous chunk is done
+                    if (jc > 0) ok = tc::mbar_wait(&bars.pempty, (jc - 1) & 1);
+                    if (!ok) break;
+                    const int prow = ((b * p.H + h) * nchunks + jc) * kC;
+                    tc::mbar_arrive_expect_tx(&bars.pfull, kPBytes);
+                    for (int s = 0; s < 2; s++)
+                        tc::tma_load_2d(sm + Sm::kP + s * (kC * 128), &p.tp, &bars.pfull, 64 * s, prow);
+                }
             }
         } else if (warp == 2) {
             // ------------------------------------------ output store (bf16)
@@ -672,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                     // a reversed partial last chunk would start before row 0: the
                     // transform warps store it directly
                     const bool direct = p.out_rev && jc == nchunks - 1 && N - jc * kC < kC;
-                    uint8_t* slot = sm + WsSmem<DK>::kV + vs * kVBytes;
+                    uint8_t* slot = sm + Sm::kV + vs * kVBytes;
                     ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars.ostaged[vs], par));
                     if (!ok) break;
                     if (lane == 0) {
@@ -696,8 +428,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         } else if (warp == 3) {
             // ------------------------------------ state-update issuer
             const uint32_t id_st = tc::idesc_bf16_f32(128, kW, 1, 1);
-            const uint64_t dk_mn = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kK), kC * 128, 1024);
-            const uint64_t dv_mn = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kV), kC * 128, 1024);
+            const uint64_t dk_mn = tc::sdesc_sw128(tc::smem_u32(sm + Sm::kK), kC * 128, 1024);
+            const uint64_t dv_mn = tc::sdesc_sw128(tc::smem_u32(sm + Sm::kV), kC * 128, 1024);
             auto wait = [&](uint64_t* bar, uint32_t parity) {
                 return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity));
             };
@@ -708,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 if (!ok) break;
                 tc::tc_fence_after();
                 for (int part = 0; part < kParts && ok; part++) {
-                    const int g = jc * kParts + part, slot = g % kKSlots, u = g / kKSlots;
+                    const int g = jc * kParts + part, slot = g % kSl, u = g / kSl;
                     ok = wait(&bars.kfull[slot], u & 1);
                     if (!ok) break;
                     tc::tc_fence_after();
@@ -731,9 +463,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             const uint32_t id_qt = tc::idesc_bf16_f32(128, kW, 0, 1);
             const uint32_t id_pv = tc::idesc_bf16_f32(128, kW, 0, 1);
             // descriptor bases; offsets are added in 16-byte units
-            const uint64_t dk_k = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kK), 16, 1024);         // K' as B, K-major
-            const uint64_t dv_mn = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kV), kC * 128, 1024);  // V as B, MN-major
-            const uint64_t dt_mn = tc::sdesc_sw128(tc::smem_u32(sm + WsSmem<DK>::kT), DK * 128, 1024);  // T as B, MN-major
+            const uint64_t dk_k = tc::sdesc_sw128(tc::smem_u32(sm + Sm::kK), 16, 1024);         // K' as B, K-major
+            const uint64_t dv_mn = tc::sdesc_sw128(tc::smem_u32(sm + Sm::kV), kC * 128, 1024);  // V as B, MN-major
+            const uint64_t dt_mn = tc::sdesc_sw128(tc::smem_u32(sm + Sm::kT), DK * 128, 1024);  // T as B, MN-major
             // a timed-out wait must leave the warp converged for elect.sync
             auto wait = [&](uint64_t* bar, uint32_t parity) {
                 return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity));
@@ -741,13 +473,44 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             // Per chunk: A = Q K'^T part by part with dS = K'^T V of every part
             // but the last right behind it (so each K' part is released early),
             // then the read-out O = Q T, the last dS part, and O += P V.
-            for (int jc = 0; jc < nchunks && ok; jc++) {
+            // With precomputed scores: the read-out, then O += P V with P as the
+            // shared-memory A operand (K-major, 128-byte swizzle).
+            const uint64_t dp_k = tc::sdesc_sw128(tc::smem_u32(sm + Sm::kP), 16, 1024);
+            for (int jc = 0; PREP && jc < nchunks && ok; jc++) {
+                const uint32_t vo = (uint32_t)((jc & 1) * kVBytes) >> 4;
+                ok = wait(&bars.qready, jc & 1);
+                if (!ok) break;
+                if (jc > 0 || has_init) {
+                    ok = wait(&bars.tready, (jc - 1 + has_init) & 1);
+                    if (ok && jc > 0) ok = wait(&bars.ofree, (jc - 1) & 1);
+                    if (!ok) break;
+                    tc::tc_fence_after();
+#pragma unroll 4
+                    for (int k = 0; k < DK / 16; k++)
+                        tc::mma_bf16_ts_elect(tb + kTO, tb + kTQ + 8 * k, dt_mn + (uint32_t)((16 * k * 128) >> 4),
+                                              id_qt, k > 0);
+                }
+                tc::mma_commit_elect(&bars.qtm);  // Q in TMEM and T in smem are read
+                ok = wait(&bars.pfull, jc & 1);
+                if (ok) ok = wait(&bars.vfull[jc & 1], (jc >> 1) & 1);
+                if (!ok) break;
+                tc::tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < kC / 16; k++)
+                    tc::mma_bf16_ss_elect(tb + kTO, dp_k + (uint32_t)(((k / 4) * (kC * 128) + (k % 4) * 32) >> 4),
+                                          dv_mn + vo + (uint32_t)((k * 2048) >> 4), id_pv,
+                                          (jc > 0) || has_init || (k > 0));
+                tc::mma_commit_elect(&bars.ofull);
+                tc::mma_commit_elect(&bars.pempty);
+                if (!p.tma_out) tc::mma_commit_elect(&bars.vempty[jc & 1]);
+            }
+            for (int jc = 0; !PREP && jc < nchunks && ok; jc++) {
                 const uint32_t vo = (uint32_t)((jc & 1) * kVBytes) >> 4;
                 ok = wait(&bars.qready, jc & 1);
                 if (ok && jc > 0) ok = wait(&bars.aread, (jc - 1) & 1);
                 if (!ok) break;
                 for (int part = 0; part < kParts && ok; part++) {
-                    const int g = jc * kParts + part, slot = g % kKSlots, u = g / kKSlots;
+                    const int g = jc * kParts + part, slot = g % kSl, u = g / kSl;
                     ok = wait(&bars.kfull[slot], u & 1);
                     if (!ok) break;
                     tc::tc_fence_after();
@@ -802,12 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const uint8_t* sQ = sm + WsSmem<DK>::kQ;
+        const uint8_t* sQ = sm + Sm::kQ;
         uint4 qv[DK / 8];
-        if constexpr (FUSED) {
-            ok = q_role_fused<DK>(p, const_cast<uint8_t*>(sQ), tb, lane_off, r, quarter, lane, nt, jt, gl, b, h,
-                                  nchunks, lg, p.hc.anchor[h], bars);
-        } else
         for (int jq = 0; jq < nchunks && ok; jq++) {
             ok = tc::mbar_wait(&bars.qfull, jq & 1);
             if (!ok) break;
@@ -860,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
         const int wg = (warp - 8) >> 2;               // column half
         const int r = quarter * 32 + lane;            // chunk row / state row in a block
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        uint8_t* sT = sm + WsSmem<DK>::kT;
+        uint8_t* sT = sm + Sm::kT;
         float R[kParts][32];
         // decay powers of a full chunk and of the (possibly shorter) last one:
         // state decay gamma^L, row scale gamma^(r-a), read-out copy gamma^(a+1),
@@ -914,14 +673,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
             // the row's normalization factor, loaded now and used by the epilogue
             const float rs = (p.rowscale && r < L) ? __ldg(p.rowscale + ((size_t)b * N + n0 + r) * p.H + h) : 1.f;
             // ---- mask: P = tril(A) as packed bf16 into TMEM, 32 A columns at a time
-            ok = tc::mbar_wait(&bars.afull, jc & 1);
+            // (with precomputed scores there is no mask step)
+            if (!PREP) ok = tc::mbar_wait(&bars.afull, jc & 1);
             if (!ok) break;
-            // fused: every load of this chunk from the ring has landed (A read
-            // all of Q and K'), so the slot may be rewritten as far as this CTA goes
-            if constexpr (FUSED)
-                if (warp == 8 && lane == 0) count_release(p.consumed + gl * kRing + jc % kRing);
             tc::tc_fence_after();
-            {
+            if (!PREP) {
 #pragma unroll
                 for (int hh = 0; hh < 2; hh++) {
                     uint32_t a[32], w[16];
@@ -939,9 +695,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                 tc::tc_fence_before();
                 elect_arrive(&bars.aread, lane);
                 tc::tmem_st_wait();
+                tc::tc_fence_before();
+                elect_arrive(&bars.pready, lane);
             }
-            tc::tc_fence_before();
-            elect_arrive(&bars.pready, lane);
             // ---- state: R = gamma^L R + dS; T = gamma^L_next R (bf16, read-out of the next chunk)
             ok = tc::mbar_wait(&bars.dsdone, jc & 1);
             if (!ok) break;
@@ -1008,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                         // Stage the bf16 tile in the V slot of this chunk (free since
                         // P V completed) in the TMA's 128-byte swizzle, then one
                         // thread stores it: rows past N are clipped by the TMA.
-                        uint8_t* sO = sm + WsSmem<DK>::kV + (jc & 1) * kVBytes;
+                        uint8_t* sO = sm + Sm::kV + (jc & 1) * kVBytes;
                         const float sc = (last ? pw(r - a_last) : sc_full) * rs;
 #pragma unroll
                         for (int c16 = 0; c16 < 4; c16++) {
@@ -1033,7 +789,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
                         // directly below, the store warp only told it is staged.
                         const bool direct = p.out_rev && last && L < kC;
                         if (!direct) {
-                            uint8_t* sO = sm + WsSmem<DK>::kV + (jc & 1) * kVBytes;
+                            uint8_t* sO = sm + Sm::kV + (jc & 1) * kVBytes;
                             const float sc = (last ? pw(r - a_last) : sc_full) * rs;
                             const uint32_t srow = p.out_rev ? (uint32_t)(kC - 1 - r) : (uint32_t)r;
                             if (wg == 1) {
@@ -1096,10 +852,206 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
     if (warp == 1) tc::tmem_dealloc(tb, 512);
 }
 
-template <int DK, typename Tout>
+// ------------------------------------------------------------ scores pass
+//
+// k_prep_scores: one CTA of 128 threads per (batch, head, chunk), taking
+// d_k in two halves through one shared-memory slot (so that three CTAs share
+// an SM and one's loads overlap another's arithmetic).  Per half:
+//   TMA     the half's columns of the chunk's raw q and k rows (128-byte
+//           swizzled slabs; a d_k below DK reads as zeros past its end, and
+//           so do rows past the sequence);
+//   CUDA    turn each consecutive pair in place (xPos, angle (pos_offset + n)
+//           theta_p: the first row of a thread from the position, fp64 angle
+//           reduced, fp32 sine and cosine; its next rows by turning through
+//           the row step) and scale each key row by gamma^(a-r);
+//   TMA     the half of q_rot (when copied) and of k' back to the workspace,
+//           for the main kernel's read-out and state update;
+//   tcgen05 A' += Q_half K'_half^T (M = N = 128, both operands from shared
+//           memory) into TMEM.
+// Then P = tril(A') -> bf16 in the 128-byte swizzle of the K-major A operand
+// the main kernel's P V reads, staged in the slot, and stored by TMA.  So the
+// intra-chunk scores, and the key scaling the main kernel's state update
+// needs, are computed once per head instead of once per value slice.
+struct ScoreParams {
+    CUtensorMap tq_in, tk_in;      // raw q, k: {dk, H, N, B}, row pitch q_ld / k_ld
+    CUtensorMap tq_out, tk_out;    // q_rot, k' in the workspace: {DK, H, N, B}
+    CUtensorMap tp;                // P tiles: {128, B H nchunks 128}
+    HeadConsts hc;
+    int N, H, nchunks, dks, xpos, qcopy;
+    long long pos0;
+    double log2base;
+};
+
+constexpr int kScThreads = 128;
+
+template <int DK>
+struct ScSmem {
+    static constexpr int kHalfSlabs = DK / 128;                     // 64-column slabs per half
+    static constexpr uint32_t kHalf = kHalfSlabs * kC * 128;        // one tensor's half: 32 KB (DK 256)
+    static constexpr uint32_t kQ = 0;
+    static constexpr uint32_t kK = kQ + kHalf;
+    static constexpr uint32_t kEnd = (2 * kHalf > (uint32_t)kPBytes ? 2 * kHalf : (uint32_t)kPBytes);
+    static constexpr uint32_t kBytes = kEnd + 1024;
+};
+
+template <int DK>
+__global__ void __launch_bounds__(kScThreads) k_prep_scores(const __grid_constant__ ScoreParams p) {
+    using Sm = ScSmem<DK>;
+    constexpr int kHS = Sm::kHalfSlabs;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t bar_ld, bar_mma;
+    __shared__ uint32_t s_tmem;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int jc = (int)(blockIdx.x % (unsigned)p.nchunks);
+    const int bh = (int)(blockIdx.x / (unsigned)p.nchunks);
+    const int h = bh % p.H, b = bh / p.H;
+    if (p.hc.anchor[h] < 0) return;   // left to the recurrent kernel
+    const int n0 = jc * kC, L = min(kC, p.N - n0);
+    const double lg = p.hc.log2g[h];
+    auto load_half = [&](int hf) {
+        tc::mbar_arrive_expect_tx(&bar_ld, 2 * Sm::kHalf);
+        for (int s = 0; s < kHS; s++) {
+            const int x = 64 * (kHS * hf + s);
+            tc::tma_load_4d(sm + Sm::kQ + s * (kC * 128), &p.tq_in, &bar_ld, x, h, n0, b);
+            tc::tma_load_4d(sm + Sm::kK + s * (kC * 128), &p.tk_in, &bar_ld, x, h, n0, b);
+        }
+    };
+    if (tid == 0) {
+        tc::mbar_init(&bar_ld, 1);
+        tc::mbar_init(&bar_mma, 1);
+        tc::fence_barrier_init();
+        load_half(0);
+    }
+    if (warp == 0) tc::tmem_alloc(&s_tmem, 128);
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tb = s_tmem;
+    bool ok = true;
+
+    constexpr int kGpr = DK / 16;               // 16-byte groups in a row's half
+    constexpr int kRows = kScThreads / kGpr;    // rows one pass of the block covers
+    const int cc = tid % kGpr, rfirst = tid / kGpr;
+    const int slab = cc / 8, c16 = cc % 8;
+    const int a = min(p.hc.anchor[h], L - 1);
+    const uint32_t id = tc::idesc_bf16_f32(128, 128, 0, 0);
+    for (int hf = 0; hf < 2; hf++) {
+        ok = ok && tc::mbar_wait(&bar_ld, hf & 1);
+        // ---- rotation and key scale of this half, in place
+        const int col = DK / 2 * hf + 8 * cc;   // first of the thread's 8 columns
+        const bool real = col < p.dks;
+        const bool turn = p.xpos && real;
+        if (real && ok) {
+            float cs[4], sn[4], cst[4], sst[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                cs[k] = cst[k] = 1.f;
+                sn[k] = sst[k] = 0.f;
+                if (turn) {
+                    const double th = exp2(-2.0 * (col / 2 + k) / p.dks * p.log2base);
+                    __sincosf(angle_mod_2pi((double)(p.pos0 + n0 + rfirst) * th), &sn[k], &cs[k]);
+                    __sincosf(angle_mod_2pi((double)kRows * th), &sst[k], &cst[k]);
+                }
+            }
+            for (int r = rfirst; r < L; r += kRows) {
+                const uint32_t off = (uint32_t)slab * (kC * 128) + tc::sw128_off((uint32_t)r, (uint32_t)c16);
+                uint4* qa = reinterpret_cast<uint4*>(sm + Sm::kQ + off);
+                uint4* ka = reinterpret_cast<uint4*>(sm + Sm::kK + off);
+                // k' scale gamma^(a-r): the exponent in fp64, exp2 in fp32
+                const float zeta = exp2f((float)((double)(a - r) * lg));
+                float ck[4], sk[4];
+#pragma unroll
+                for (int k = 0; k < 4; k++) {
+                    ck[k] = cs[k] * zeta;
+                    sk[k] = sn[k] * zeta;
+                }
+                if (turn) *qa = turn_group(*qa, cs, sn);
+                *ka = turn_group(*ka, ck, sk);
+                if (turn) {
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        const float c2 = cs[k] * cst[k] - sn[k] * sst[k];
+                        sn[k] = sn[k] * cst[k] + cs[k] * sst[k];
+                        cs[k] = c2;
+                    }
+                }
+            }
+        }
+        tc::fence_proxy_async_smem();
+        ok = __syncthreads_and(ok ? 1 : 0) != 0;
+        // ---- the half of q_rot and k' out; A' += Q_half K'_half^T
+        if (tid == 0 && ok) {
+            for (int s = 0; s < kHS; s++) {
+                const int x = 64 * (kHS * hf + s);
+                if (p.qcopy) tc::tma_store_4d(&p.tq_out, sm + Sm::kQ + s * (kC * 128), x, h, n0, b);
+                tc::tma_store_4d(&p.tk_out, sm + Sm::kK + s * (kC * 128), x, h, n0, b);
+            }
+            tc::bulk_commit_group();
+            tc::tc_fence_after();
+            const uint64_t dq = tc::sdesc_sw128(tc::smem_u32(sm + Sm::kQ), 16, 1024);
+            const uint64_t dk = tc::sdesc_sw128(tc::smem_u32(sm + Sm::kK), 16, 1024);
+#pragma unroll
+            for (int k = 0; k < DK / 32; k++) {
+                const uint32_t o = (uint32_t)(((k / 4) * (kC * 128) + (k % 4) * 32) >> 4);
+                tc::mma_bf16_ss(tb, dq + o, dk + o, id, (hf > 0) || (k > 0));
+            }
+            tc::mma_commit(&bar_mma);
+            // the slot is reused once the stores have read it and the MMAs are done
+            tc::bulk_wait_group_read<0>();
+            ok = tc::mbar_wait(&bar_mma, hf & 1);
+            if (ok && hf == 0) load_half(1);
+        }
+        ok = __syncthreads_and(ok ? 1 : 0) != 0;
+    }
+    tc::tc_fence_after();
+
+    // ---- P = tril(A') as bf16 into the slot: warp w reads TMEM lanes
+    // 32 w .. (its rows), all 128 key columns
+    if (ok) {
+        const int r = warp * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+#pragma unroll
+        for (int q32 = 0; q32 < 4; q32++) {
+            uint32_t av[32], w[16];
+            tc::tmem_ld32(tb + lane_off + 32 * q32, av);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const int c = 32 * q32 + 2 * i;
+                const float lo = (c <= r) ? __uint_as_float(av[2 * i]) : 0.f;
+                const float hi = (c + 1 <= r) ? __uint_as_float(av[2 * i + 1]) : 0.f;
+                w[i] = tc::pack_bf16x2(lo, hi);
+            }
+            // columns 32 q32 .. + 31: slab q32 / 2, 16-byte chunks 4 (q32 % 2) ..
+#pragma unroll
+            for (int q4 = 0; q4 < 4; q4++)
+                *reinterpret_cast<uint4*>(sm + (q32 / 2) * (kC * 128) +
+                                          tc::sw128_off((uint32_t)r, (uint32_t)(4 * (q32 % 2) + q4))) =
+                    make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+        }
+    }
+    tc::tc_fence_before();
+    tc::fence_proxy_async_smem();
+    ok = __syncthreads_and(ok ? 1 : 0) != 0;
+    if (tid == 0) {
+        if (ok) {
+            const int prow = (bh * p.nchunks + jc) * kC;
+            for (int s = 0; s < 2; s++) tc::tma_store_2d(&p.tp, sm + s * (kC * 128), 64 * s, prow);
+            tc::bulk_commit_group();
+        }
+        tc::bulk_wait_group<0>();   // every store has read its tile (and is done)
+        if (!ok) atomicExch(&g_err_chunk_ws, kErrTimeout);
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tb, 128);
+}
+
+template <int DK, typename Tout, bool PREP = false>
 ret_status launch_main(const WsParams& p, cudaStream_t s) {
-    auto kern = k_chunkwise_ws<DK, Tout, false>;
-    const int smem = (int)WsSmem<DK>::kBytes;
+    auto kern = k_chunkwise_ws<DK, Tout, PREP>;
+    const int smem = (int)WsSmem<DK, PREP>::kBytes;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return check_launch("chunkwise (workspace path): smem attribute");
     kern<<<p.nmain, kThreads, smem, s>>>(p);
@@ -1192,161 +1144,6 @@ static ret_status fill_params(WsParams* p, const RetArgs& a, const void* q_src, 
     return RET_OK;
 }
 
-// ------------------------------------------------------ fused rotation
-//
-// The CTAs of one head wait on one another's ring writes, so a launch holds
-// no more heads than can be resident at once; it is launched cooperatively,
-// which makes the runtime refuse (rather than run) a grid that could not be
-// co-resident.  Larger problems run as several launches, one per group of
-// heads, on the same scratch.
-
-constexpr int kFusedCtaCap = 148;   // CTAs the scratch of one launch is sized for (one per SM of a B200)
-
-static int fused_group_cap(const RetArgs& a) {
-    const int nt = a.dv / kW;
-    const long long bh = (long long)a.B * a.H;
-    return (int)std::min<long long>(bh, std::max(1, kFusedCtaCap / nt));
-}
-
-static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-
-// Scratch: ready[G][kRing], consumed[G][kRing] (u32), then the q and k'
-// rings, [G, kRing, 128, dk] bf16 each.
-static size_t fused_counter_bytes(size_t G) { return align256(2 * G * kRing * sizeof(unsigned)); }
-
-size_t chunkwise_fused_bytes(const RetArgs& a) {
-    const size_t G = (size_t)fused_group_cap(a);
-    return fused_counter_bytes(G) + 2 * G * kRing * kC * (size_t)a.dk * 2;
-}
-
-template <int DK, typename Tout>
-ret_status launch_fused(const WsParams& p, int grid, cudaStream_t s) {
-    auto kern = k_chunkwise_ws<DK, Tout, true>;
-    const int smem = (int)WsSmem<DK>::kBytes;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return check_launch("chunkwise (fused): smem attribute");
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
-    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "chunkwise (fused): launch: %s", cudaGetErrorString(e));
-    return check_launch("chunkwise (fused)");
-}
-
-// CTAs of the fused kernel that fit on the current device at once.
-template <int DK, typename Tout>
-static int fused_resident(int* out) {
-    auto kern = k_chunkwise_ws<DK, Tout, true>;
-    const int smem = (int)WsSmem<DK>::kBytes;
-    int dev = 0, sms = 0, per_sm = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) ||
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) != cudaSuccess)
-        return 0;
-    *out = per_sm * sms;
-    return 1;
-}
-
-ret_status launch_chunkwise_fused(const RetArgs& a, void* scratch, cudaStream_t s) {
-    const int nt = a.dv / kW;
-    const bool f32 = a.out_dt == RET_F32;
-    int resident = 0;
-    const int okr = a.dk == 256 ? (f32 ? fused_resident<256, float>(&resident) : fused_resident<256, __nv_bfloat16>(&resident))
-                                : (f32 ? fused_resident<128, float>(&resident) : fused_resident<128, __nv_bfloat16>(&resident));
-    if (!okr) return fail(RET_ERR_CUDA, "chunkwise (fused): occupancy query failed");
-    const int cap = fused_group_cap(a);
-    const int G = std::min(cap, resident / nt);
-    if (G < 1) return fail(RET_ERR_UNSUPPORTED, "chunkwise (fused): no room for the %d CTAs of one head", nt);
-    unsigned* ctr = reinterpret_cast<unsigned*>(scratch);
-    __nv_bfloat16* ring_q =
-        reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(scratch) + fused_counter_bytes((size_t)cap));
-    __nv_bfloat16* ring_k = ring_q + (size_t)cap * kRing * kC * a.dk;
-    // the tensor maps of q and k' read the rings: {dk, ring rows, head of the launch, 1}
-    WsParams p;
-    ret_status st = fill_params(&p, a, a.q, a.dk, a.k);
-    if (st != RET_OK) return st;
-    {
-        const uint64_t dk = a.dk, rows = (uint64_t)kRing * kC;
-        const uint64_t dr[4] = {dk, rows, (uint64_t)cap, 1};
-        const uint64_t sr[3] = {dk * 2, rows * dk * 2, (uint64_t)cap * rows * dk * 2};
-        const uint32_t box[4] = {64, (uint32_t)kC, 1, 1};
-        if (!make_tmap_bf16(&p.tq, ring_q, 4, dr, sr, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_tmap_bf16(&p.tk, ring_k, 4, dr, sr, box, CU_TENSOR_MAP_SWIZZLE_128B))
-            return RET_ERR_CUDA;
-    }
-    const int dkr = a.dk_real ? a.dk_real : a.dk;
-    p.q_raw = reinterpret_cast<const __nv_bfloat16*>(a.q);
-    p.k_raw = reinterpret_cast<const __nv_bfloat16*>(a.k);
-    p.q_ld = a.q_ld ? a.q_ld : dkr;
-    p.k_ld = a.k_ld ? a.k_ld : dkr;
-    p.ring_q = ring_q;
-    p.ring_k = ring_k;
-    p.ready = ctr;
-    p.consumed = ctr + (size_t)cap * kRing;
-    p.xpos = a.xpos;
-    p.pos0 = a.pos_offset;
-    p.log2base = log2(a.theta_base);
-    const int BH = a.B * a.H;
-    for (int bh0 = 0; bh0 < BH; bh0 += G) {
-        const int g = std::min(G, BH - bh0);
-        p.bh0 = bh0;
-        p.nmain = g * nt;
-        cudaError_t e = cudaMemsetAsync(ctr, 0, 2 * (size_t)cap * kRing * sizeof(unsigned), s);
-        if (e != cudaSuccess) return fail(RET_ERR_CUDA, "chunkwise (fused): counter reset: %s", cudaGetErrorString(e));
-        if (a.dk == 256) st = f32 ? launch_fused<256, float>(p, g * nt, s) : launch_fused<256, __nv_bfloat16>(p, g * nt, s);
-        else st = f32 ? launch_fused<128, float>(p, g * nt, s) : launch_fused<128, __nv_bfloat16>(p, g * nt, s);
-        if (st != RET_OK) return st;
-    }
-    return RET_OK;
-}
-
-// The fused path on scratch from a stream-ordered pool the library keeps per
-// device (created on the first call, never trimmed): allocated and freed in
-// stream order around the launches, so concurrent calls on other streams get
-// their own scratch.
-ret_status launch_chunkwise_fused_pooled(const RetArgs& a, cudaStream_t s) {
-    constexpr int kMaxDev = 64;
-    static cudaMemPool_t pools[kMaxDev] = {};
-    static std::mutex mu;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "chunkwise: cudaGetDevice: %s", cudaGetErrorString(e));
-    if (dev < 0 || dev >= kMaxDev) return fail(RET_ERR_UNSUPPORTED, "chunkwise: device %d out of range", dev);
-    cudaMemPool_t pool;
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        if (!pools[dev]) {
-            cudaMemPoolProps props = {};
-            props.allocType = cudaMemAllocationTypePinned;
-            props.location.type = cudaMemLocationTypeDevice;
-            props.location.id = dev;
-            e = cudaMemPoolCreate(&pools[dev], &props);
-            if (e != cudaSuccess) {
-                pools[dev] = nullptr;
-                return fail(RET_ERR_CUDA, "chunkwise: scratch pool: %s", cudaGetErrorString(e));
-            }
-            uint64_t keep = ~0ull;
-            cudaMemPoolSetAttribute(pools[dev], cudaMemPoolAttrReleaseThreshold, &keep);
-        }
-        pool = pools[dev];
-    }
-    void* scratch = nullptr;
-    e = cudaMallocFromPoolAsync(&scratch, chunkwise_fused_bytes(a), pool, s);
-    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "chunkwise: scratch: %s", cudaGetErrorString(e));
-    const ret_status st = launch_chunkwise_fused(a, scratch, s);
-    e = cudaFreeAsync(scratch, s);
-    if (st != RET_OK) return st;
-    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "chunkwise: scratch release: %s", cudaGetErrorString(e));
-    return RET_OK;
-}
-
 ret_status launch_chunkwise_main(const RetArgs& a, const void* q_src, int q_pitch, const void* k_prime,
                                  cudaStream_t s) {
     WsParams p;
@@ -1394,6 +1191,140 @@ ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s) {
     ret_status st = launch_chunkwise_prep(a, ws, s);
     if (st != RET_OK) return st;
     return launch_chunkwise_prepared(a, ws, s);
+}
+
+// ------------------------------------------------------- the scores form
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static int chunks_of(const RetArgs& a) { return (a.N + kC - 1) / kC; }
+
+// Workspace of the scores form: that of the two-pass form (k', then q_rot),
+// then the P tiles [B, H, nchunks, 128, 128] bf16.
+size_t chunkwise_scores_bytes(const RetArgs& a) {
+    return align256(chunkwise_ws_bytes(a)) + (size_t)a.B * a.H * chunks_of(a) * kPBytes;
+}
+
+// The P tiles' tensor map (both passes use the same one).
+static bool scores_map(const RetArgs& a, void* ws, CUtensorMap* tp) {
+    void* pbuf = reinterpret_cast<uint8_t*>(ws) + align256(chunkwise_ws_bytes(a));
+    const uint64_t prows = (uint64_t)a.B * a.H * chunks_of(a) * kC;
+    const uint64_t dpp[2] = {(uint64_t)kC, prows};
+    const uint64_t spp[1] = {(uint64_t)kC * 2};
+    const uint32_t bpp[2] = {64, (uint32_t)kC};
+    return make_tmap_bf16(tp, pbuf, 2, dpp, spp, bpp, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Pass 1: rotation, key scale and the masked scores into the workspace.
+ret_status launch_chunkwise_scores_pass1(const RetArgs& a, void* ws, cudaStream_t s) {
+    __nv_bfloat16 *k_out, *q_rot;
+    ws_parts(a, ws, &k_out, &q_rot);
+    const bool qc = q_copied(a);
+    const int nchunks = chunks_of(a);
+    {
+        ScoreParams sp;
+        memset(&sp, 0, sizeof(sp));
+        const int dkr = a.dk_real ? a.dk_real : a.dk;
+        const uint64_t B = a.B, N = a.N, H = a.H, dk = a.dk;
+        const uint64_t qld = a.q_ld ? a.q_ld : dkr, kld = a.k_ld ? a.k_ld : dkr;
+        const uint32_t box[4] = {64, 1, (uint32_t)kC, 1};
+        const uint64_t dr[4] = {(uint64_t)dkr, H, N, B};
+        const uint64_t sq[3] = {qld * 2, H * qld * 2, N * H * qld * 2};
+        const uint64_t sk[3] = {kld * 2, H * kld * 2, N * H * kld * 2};
+        const uint64_t dw[4] = {dk, H, N, B};
+        const uint64_t sw[3] = {dk * 2, H * dk * 2, N * H * dk * 2};
+        if (!make_tmap_bf16(&sp.tq_in, a.q, 4, dr, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tmap_bf16(&sp.tk_in, a.k, 4, dr, sk, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tmap_bf16(&sp.tk_out, k_out, 4, dw, sw, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            (qc && !make_tmap_bf16(&sp.tq_out, q_rot, 4, dw, sw, box, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+            !scores_map(a, ws, &sp.tp))
+            return RET_ERR_CUDA;
+        sp.hc = a.hc;
+        sp.N = a.N;
+        sp.H = a.H;
+        sp.nchunks = nchunks;
+        sp.dks = dkr;
+        sp.xpos = a.xpos;
+        sp.qcopy = qc ? 1 : 0;
+        sp.pos0 = a.pos_offset;
+        sp.log2base = log2(a.theta_base);
+        const long long grid = (long long)a.B * a.H * nchunks;
+        if (grid > (1ll << 31) - 1) return fail(RET_ERR_UNSUPPORTED, "chunkwise (scores): too many chunks");
+        if (a.dk == 256) {
+            auto kern = k_prep_scores<256>;
+            const int smem = (int)ScSmem<256>::kBytes;
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+                return check_launch("chunkwise (scores pass): smem attribute");
+            kern<<<(unsigned)grid, kScThreads, smem, s>>>(sp);
+        } else {
+            auto kern = k_prep_scores<128>;
+            const int smem = (int)ScSmem<128>::kBytes;
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+                return check_launch("chunkwise (scores pass): smem attribute");
+            kern<<<(unsigned)grid, kScThreads, smem, s>>>(sp);
+        }
+        return check_launch("chunkwise (scores pass)");
+    }
+}
+
+// Pass 2: read-out, P V and state update on the prepared rows and scores
+// (a.initial_state honoured).
+ret_status launch_chunkwise_scores_pass2(const RetArgs& a, void* ws, cudaStream_t s) {
+    __nv_bfloat16 *k_out, *q_rot;
+    ws_parts(a, ws, &k_out, &q_rot);
+    const bool qc = q_copied(a);
+    WsParams p;
+    ret_status st = fill_params(&p, a, qc ? (const void*)q_rot : a.q, qc || !a.q_ld ? a.dk : a.q_ld, k_out);
+    if (st != RET_OK) return st;
+    if (!scores_map(a, ws, &p.tp)) return RET_ERR_CUDA;
+    const bool f32 = a.out_dt == RET_F32;
+    if (a.dk == 256) return f32 ? launch_main<256, float, true>(p, s) : launch_main<256, __nv_bfloat16, true>(p, s);
+    return f32 ? launch_main<128, float, true>(p, s) : launch_main<128, __nv_bfloat16, true>(p, s);
+}
+
+ret_status launch_chunkwise_scores(const RetArgs& a, void* ws, cudaStream_t s) {
+    const ret_status st = launch_chunkwise_scores_pass1(a, ws, s);
+    return st != RET_OK ? st : launch_chunkwise_scores_pass2(a, ws, s);
+}
+
+// The scores form on scratch from a stream-ordered pool the library keeps per
+// device (created on the first call, never trimmed): allocated and freed in
+// stream order around the launches, so concurrent calls on other streams get
+// their own scratch.
+ret_status launch_chunkwise_scores_pooled(const RetArgs& a, cudaStream_t s) {
+    constexpr int kMaxDev = 64;
+    static cudaMemPool_t pools[kMaxDev] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "chunkwise: cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDev) return fail(RET_ERR_UNSUPPORTED, "chunkwise: device %d out of range", dev);
+    cudaMemPool_t pool;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!pools[dev]) {
+            cudaMemPoolProps props = {};
+            props.allocType = cudaMemAllocationTypePinned;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            e = cudaMemPoolCreate(&pools[dev], &props);
+            if (e != cudaSuccess) {
+                pools[dev] = nullptr;
+                return fail(RET_ERR_CUDA, "chunkwise: scratch pool: %s", cudaGetErrorString(e));
+            }
+            uint64_t keep = ~0ull;
+            cudaMemPoolSetAttribute(pools[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+        }
+        pool = pools[dev];
+    }
+    void* scratch = nullptr;
+    e = cudaMallocFromPoolAsync(&scratch, chunkwise_scores_bytes(a), pool, s);
+    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "chunkwise: scratch: %s", cudaGetErrorString(e));
+    const ret_status st = launch_chunkwise_scores(a, scratch, s);
+    e = cudaFreeAsync(scratch, s);
+    if (st != RET_OK) return st;
+    if (e != cudaSuccess) return fail(RET_ERR_CUDA, "chunkwise: scratch release: %s", cudaGetErrorString(e));
+    return RET_OK;
 }
 
 // ------------------------------------------------- allocation-free variant

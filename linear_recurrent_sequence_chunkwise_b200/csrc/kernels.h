@@ -63,13 +63,17 @@ ret_status launch_chunkwise_ws(const RetArgs& a, void* ws, cudaStream_t s);
 // workspace the prep pass has filled (a.initial_state honoured).
 ret_status launch_chunkwise_prep(const RetArgs& a, void* ws, cudaStream_t s);
 ret_status launch_chunkwise_prepared(const RetArgs& a, void* ws, cudaStream_t s);
-// The fused path: the rotation and zeta scaling inside the tensor-core
-// kernel, the rotated rows shared by the CTAs of a head through an exchange
-// ring in `scratch` (chunkwise_fused_bytes of it, 256-byte aligned).  The
-// pooled form takes the scratch from a stream-ordered pool of the library.
-size_t chunkwise_fused_bytes(const RetArgs& a);
-ret_status launch_chunkwise_fused(const RetArgs& a, void* scratch, cudaStream_t s);
-ret_status launch_chunkwise_fused_pooled(const RetArgs& a, cudaStream_t s);
+// The scores form: a tensor-core pass that rotates q and k, scales the keys
+// and computes the masked intra-chunk scores P of every (b, h, chunk), then
+// the warp-specialized kernel on those (read-out, P V, state update).  `ws`
+// holds chunkwise_scores_bytes (256-byte aligned).  The pooled form takes it
+// from a stream-ordered pool of the library.
+size_t chunkwise_scores_bytes(const RetArgs& a);
+ret_status launch_chunkwise_scores(const RetArgs& a, void* ws, cudaStream_t s);
+// Its two passes on their own (the second honours a.initial_state).
+ret_status launch_chunkwise_scores_pass1(const RetArgs& a, void* ws, cudaStream_t s);
+ret_status launch_chunkwise_scores_pass2(const RetArgs& a, void* ws, cudaStream_t s);
+ret_status launch_chunkwise_scores_pooled(const RetArgs& a, cudaStream_t s);
 // The workspace path on the library's fixed device array (no allocation).
 size_t chunkwise_static_ws_bytes();
 ret_status launch_chunkwise_static(const RetArgs& a, cudaStream_t s);

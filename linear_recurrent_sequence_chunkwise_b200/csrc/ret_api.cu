@@ -1,6 +1,7 @@
 // ret_api.cu -- the C ABI: argument validation, per-head constants and
 // dispatch to the kernels.  Nothing here allocates device memory, apart from
-// ret_forward_chunkwise's small stream-ordered scratch (see k_chunk_ws.cu).
+// ret_forward_chunkwise's stream-ordered scratch from the library's pool
+// (see k_chunk_ws.cu).
 #include <cstring>
 #include <math.h>
 #include <stdarg.h>
@@ -138,13 +139,13 @@ ret_status ret_forward_chunkwise(const void* q, const void* k, const void* v, co
                               final_state, in_dt, out_dt, xpos, pos_offset, theta_base);
     if (st != RET_OK) return st;
     {
-        // the tensor-core path with the rotation fused (d_k = 64 padded to 128);
+        // the tensor-core path, scores form (d_k = 64 padded to 128);
         // heads too fast for it (gamma^64 < 2^-100), if any, token by token
         RetArgs f = a;
         pad_small_dk(&f);
         const int left = chunkwise_heads_below(f, 0);
         if (chunkwise_ws_shape_ok(f) && left < H) {
-            st = launch_chunkwise_fused_pooled(f, stream);
+            st = launch_chunkwise_scores_pooled(f, stream);
             if (st != RET_OK || left == 0) return st;
             return launch_recurrent_simt(a, stream, true);
         }
@@ -165,7 +166,7 @@ size_t ret_chunkwise_workspace_bytes(int B, int N, int H, int dk, int dv, int ch
     a.B = B; a.N = N; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.in_dt = in_dt; a.xpos = xpos ? 1 : 0;
     for (int h = 0; h < kMaxHeads; h++) a.hc.log2g[h] = 0.0, a.hc.anchor[h] = kChunkAnchorFull;  // shape check only
     pad_small_dk(&a);
-    return chunkwise_ws_supported(a) ? chunkwise_fused_bytes(a) : 0;
+    return chunkwise_ws_supported(a) ? chunkwise_scores_bytes(a) : 0;
 }
 
 size_t ret_chunkwise_prepare_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk, ret_dtype in_dt,
@@ -175,7 +176,7 @@ size_t ret_chunkwise_prepare_workspace_bytes(int B, int N, int H, int dk, int dv
     a.B = B; a.N = N; a.H = H; a.dk = dk; a.dv = dv; a.chunk = chunk; a.in_dt = in_dt; a.xpos = xpos ? 1 : 0;
     for (int h = 0; h < kMaxHeads; h++) a.hc.log2g[h] = 0.0, a.hc.anchor[h] = kChunkAnchorFull;  // shape check only
     pad_small_dk(&a);
-    return chunkwise_ws_supported(a) ? chunkwise_ws_bytes(a) : 0;
+    return chunkwise_ws_supported(a) ? chunkwise_scores_bytes(a) : 0;
 }
 
 ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v, const double* gammas, int B, int N,
@@ -193,7 +194,7 @@ ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
     if (!chunkwise_ws_shape_ok(a) || left == H)
         return ret_forward_chunkwise(q, k, v, gammas, B, N, H, dk, dv, chunk, out, final_state, stream, in_dt,
                                      out_dt, xpos, pos_offset, theta_base);
-    const size_t need = chunkwise_fused_bytes(a);
+    const size_t need = chunkwise_scores_bytes(a);
     if (!workspace || workspace_bytes < need)
         return fail(RET_ERR_INVALID_ARG, "ret_forward_chunkwise_ws: workspace of %zu bytes needed (got %zu)", need,
                     workspace ? workspace_bytes : (size_t)0);
@@ -205,7 +206,7 @@ ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
         overlaps(workspace, need, out, bo) ||
         (final_state && overlaps(workspace, need, final_state, (size_t)B * H * dk * dv * 4)))
         return fail(RET_ERR_INVALID_ARG, "ret_forward_chunkwise_ws: workspace overlaps another buffer");
-    st = launch_chunkwise_fused(a, workspace, stream);
+    st = launch_chunkwise_scores(a, workspace, stream);
     if (st != RET_OK || left == 0) return st;
     // heads too fast for the tensor-core kernel, token by token
     return launch_recurrent_simt(caller, stream, true);
@@ -214,7 +215,7 @@ ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
 // Workspace checks shared by the workspace-path entry points.
 static ret_status check_workspace(const RetArgs& a, const char* who, const void* workspace, size_t workspace_bytes,
                                   bool with_outputs) {
-    const size_t need = chunkwise_ws_bytes(a);
+    const size_t need = chunkwise_scores_bytes(a);
     if (!workspace || workspace_bytes < need)
         return fail(RET_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed (got %zu)", who, need,
                     workspace ? workspace_bytes : (size_t)0);
@@ -276,7 +277,7 @@ ret_status ret_chunkwise_prepare(const void* q, const void* k, const double* gam
                     who);
     st = check_workspace(a, who, workspace, workspace_bytes, false);
     if (st != RET_OK) return st;
-    return launch_chunkwise_prep(a, workspace, stream);
+    return launch_chunkwise_scores_pass1(a, workspace, stream);
 }
 
 ret_status ret_forward_chunkwise_prepared(const void* q, const void* k, const void* v, const double* gammas, int B,
@@ -298,7 +299,7 @@ ret_status ret_forward_chunkwise_prepared(const void* q, const void* k, const vo
     if (st != RET_OK) return st;
     st = check_workspace(a, who, workspace, workspace_bytes, true);
     if (st != RET_OK) return st;
-    return launch_chunkwise_prepared(a, const_cast<void*>(workspace), stream);
+    return launch_chunkwise_scores_pass2(a, const_cast<void*>(workspace), stream);
 }
 
 size_t ret_normalized_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk, ret_dtype in_dt, int xpos) {

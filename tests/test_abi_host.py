@@ -124,7 +124,8 @@ def test_binding_requires_cuda_tensors():
 # chunk 128, dk 128, dv 64 (q, k 64 KB each at the fake addresses above).
 WS = ctypes.c_void_p(0xA0000000)
 QK_BYTES = 1 * 128 * 2 * 128 * 2          # one bf16 [B, N, H, dk] tensor
-WS_BYTES = QK_BYTES                       # k' alone (no rotation)
+P_BYTES = 1 * 2 * 1 * 128 * 128 * 2       # the masked scores of every (b, h, chunk), bf16
+WS_BYTES = QK_BYTES + P_BYTES             # k' alone (no rotation), then the scores
 
 
 def prepare_call(q=P, k=P2, g=G2, dk=128, dv=64, ws=WS, nbytes=WS_BYTES, xpos=0):
@@ -136,38 +137,35 @@ def prepared_call(ws=WS, nbytes=WS_BYTES, init=None, fs=None, dk=128, out=P4):
                                                 1e4, ws, nbytes)
 
 
+def _scores_bytes(B, N, H, dk, copied):
+    """Workspace of the scores form: k' (and the copied queries) [B, N, H, dk]
+    bf16, 256-byte aligned, then P [B, H, ceil(N / 128), 128, 128] bf16."""
+    qk = B * N * H * dk * 2 * (2 if copied else 1)
+    return (qk + 255) // 256 * 256 + B * H * ((N + 127) // 128) * 128 * 128 * 2
+
+
 def test_workspace_size_matches_the_two_pass_shape():
     ws = R.ret_chunkwise_prepare_workspace_bytes
     assert ws(1, 128, 2, 128, 64, 128, torch.bfloat16, False) == WS_BYTES
-    assert ws(1, 128, 2, 128, 64, 128, torch.bfloat16, True) == 2 * QK_BYTES
-    assert ws(3, 1000, 2, 128, 64, 128, torch.bfloat16, True) == 2 * 3 * 1000 * 2 * 128 * 2
+    assert ws(1, 128, 2, 128, 64, 128, torch.bfloat16, True) == 2 * QK_BYTES + P_BYTES
+    assert ws(3, 1000, 2, 128, 64, 128, torch.bfloat16, True) == _scores_bytes(3, 1000, 2, 128, True)
     assert ws(1, 128, 2, 16, 64, 128, torch.bfloat16, False) == 0
-
-
-def _fused_bytes(B, H, dk, dv):
-    """Scratch of the fused forward: per head of one launch (at most 148 CTAs,
-    dv / 64 per head) two u32 counts per ring slot, then the q and k' rings of
-    6 chunk slots of 128 rows each."""
-    G = min(B * H, 148 // (dv // 64))
-    ctr = (2 * G * 6 * 4 + 255) // 256 * 256
-    return ctr + 2 * G * 6 * 128 * dk * 2
 
 
 @pytest.mark.parametrize("B,N,H,dk,dv,xpos", [
     (1, 128, 2, 128, 64, False), (1, 8192, 16, 256, 512, True), (64, 1024, 16, 256, 512, False),
-    (4, 2048, 8, 64, 64, True),
+    (4, 2048, 8, 64, 64, True), (2, 300, 3, 128, 192, True),
 ])
-def test_fused_workspace_size_is_a_ring_not_the_sequence(B, N, H, dk, dv, xpos):
-    dkk = 128 if dk == 64 else dk
-    got = R.ret_chunkwise_workspace_bytes(B, N, H, dk, dv, 64 if dk == 64 else 128, torch.bfloat16, xpos)
-    assert got == _fused_bytes(B, H, dkk, dv)
-    assert got <= 160 << 20      # independent of N; at most 148 heads of rings
-    assert R.ret_chunkwise_workspace_bytes(1, 128, 2, 16, 64, 128, torch.bfloat16, False) == 0
+def test_single_call_workspace_is_the_scores_form(B, N, H, dk, dv, xpos):
+    dkk, chunk = (128, 64) if dk == 64 else (dk, 128)
+    want = _scores_bytes(B, N, H, dkk, xpos or dk == 64)
+    assert R.ret_chunkwise_workspace_bytes(B, N, H, dk, dv, chunk, torch.bfloat16, xpos) == want
+    assert R.ret_chunkwise_prepare_workspace_bytes(B, N, H, dk, dv, chunk, torch.bfloat16, xpos) == want
 
 
 @needs_no_gpu
 @pytest.mark.parametrize("kw,status", [
-    (dict(q=None), 1), (dict(ws=None), 1), (dict(nbytes=100), 1), (dict(nbytes=2 * QK_BYTES - 1, xpos=1), 1),
+    (dict(q=None), 1), (dict(ws=None), 1), (dict(nbytes=100), 1), (dict(nbytes=2 * QK_BYTES + P_BYTES - 1, xpos=1), 1),
     (dict(ws=ctypes.c_void_p(0xA0000010)), 1), (dict(ws=ctypes.c_void_p(0x10000)), 1),
     (dict(g=(ctypes.c_double * 2)(0.9, 1.5)), 1), (dict(dk=16), 2), (dict(dv=48), 2),
 ])
@@ -223,7 +221,7 @@ def test_backward_rejects_bad_arguments(kw, status):
 
 def test_normalized_workspace_size():
     nb = R.ret_normalized_workspace_bytes(1, 200, 2, 128, 64, 128, torch.bfloat16, True)
-    ws = R.ret_chunkwise_prepare_workspace_bytes(1, 200, 2, 128, 64, 128, torch.bfloat16, True)
+    ws = 2 * 200 * 2 * 128 * 2
     # the prepared q, k, then row factors [B, N, H], key sums per 32 rows and per chunk start
     al = lambda x: (x + 255) // 256 * 256
     assert nb == al(ws) + al(200 * 2 * 4) + al(2 * 7 * 128 * 4) + al(2 * 2 * 128 * 4)
