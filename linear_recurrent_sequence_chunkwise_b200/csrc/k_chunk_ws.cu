@@ -854,198 +854,320 @@ __global__ void __launch_bounds__(kThreads, 1) k_chunkwise_ws(const __grid_const
 
 // ------------------------------------------------------------ scores pass
 //
-// k_prep_scores: one CTA of 128 threads per (batch, head, chunk), taking
-// d_k in two halves through one shared-memory slot (so that three CTAs share
-// an SM and one's loads overlap another's arithmetic).  Per half:
-//   TMA     the half's columns of the chunk's raw q and k rows (128-byte
-//           swizzled slabs; a d_k below DK reads as zeros past its end, and
-//           so do rows past the sequence);
-//   CUDA    turn each consecutive pair in place (xPos, angle (pos_offset + n)
-//           theta_p: the first row of a thread from the position, fp64 angle
-//           reduced, fp32 sine and cosine; its next rows by turning through
-//           the row step) and scale each key row by gamma^(a-r);
-//   TMA     the half of q_rot (when copied) and of k' back to the workspace,
-//           for the main kernel's read-out and state update;
-//   tcgen05 A' += Q_half K'_half^T (M = N = 128, both operands from shared
-//           memory) into TMEM.
-// Then P = tril(A') -> bf16 in the 128-byte swizzle of the K-major A operand
-// the main kernel's P V reads, staged in the slot, and stored by TMA.  So the
-// intra-chunk scores, and the key scaling the main kernel's state update
-// needs, are computed once per head instead of once per value slice.
+// k_prep_scores: persistent and warp-specialized; each CTA walks the tiles
+// (batch, head, chunk) blockIdx.x, blockIdx.x + gridDim.x, ..., one 64-column
+// slab of d_k at a time through a ring of kScStages shared-memory stages:
+//   warp 0 (one lane)   TMA: the slab of the chunk's raw q and k rows into a
+//                       stage (128-byte swizzle; a d_k below DK reads as
+//                       zeros past its end, and so do rows past the sequence);
+//   warps 4-7           turn each consecutive pair in place (xPos, angle
+//                       (pos_offset + n) theta_p: a thread's first row from the
+//                       position, fp64 angle reduced, fp32 sine and cosine; its
+//                       next rows by turning through the row step), scale each
+//                       key row by gamma^(a-r), and store the slab of q_rot
+//                       (when copied) and of k' to the workspace by TMA;
+//   warp 1 (one lane)   tcgen05: A' += Q_slab K'_slab^T (M = N = 128, K = 64,
+//                       both operands from the stage) into one of two TMEM
+//                       accumulators;
+//   warps 8-11          P = tril(A') -> bf16 in the 128-byte swizzle of the
+//                       K-major A operand the main kernel's P V reads, staged
+//                       and stored by TMA.
+// A stage is free once its MMAs are done and its stores have read it; an
+// accumulator once the previous tile's P has been read out of it.  Every wait
+// is bounded; a warpgroup agrees on each wait's outcome (named barriers 1
+// and 2), and a timed-out wait ends the CTA's walk with the error word set.
 struct ScoreParams {
     CUtensorMap tq_in, tk_in;      // raw q, k: {dk, H, N, B}, row pitch q_ld / k_ld
     CUtensorMap tq_out, tk_out;    // q_rot, k' in the workspace: {DK, H, N, B}
     CUtensorMap tp;                // P tiles: {128, B H nchunks 128}
     HeadConsts hc;
-    int N, H, nchunks, dks, xpos, qcopy;
+    int N, H, nchunks, ntiles, dks, xpos, qcopy;
     long long pos0;
-    double log2base;
+    double theta[128];             // theta_p = base^(-2p/d_k) of every pair, fp64
 };
 
-constexpr int kScThreads = 128;
+constexpr int kScThreads = 384;
+constexpr int kScStages = 5;
+constexpr int kScLag = 2;                        // slabs whose stores may still be reading their stages
+constexpr uint32_t kScSlab = kC * 128;           // one 64-column slab of 128 rows: 16 KB
+constexpr uint32_t kScStage = 2 * kScSlab;       // q and k slabs
 
-template <int DK>
+// The rotation's tables (fp32 cosine, sine pairs): rows 0..15 the turn
+// through r theta_p, row 16 through 16 theta_p (a thread's row step), row 17
+// the current tile's base angle (pos_offset + n0) theta_p.
+constexpr int kScTabRows = 18;
+
 struct ScSmem {
-    static constexpr int kHalfSlabs = DK / 128;                     // 64-column slabs per half
-    static constexpr uint32_t kHalf = kHalfSlabs * kC * 128;        // one tensor's half: 32 KB (DK 256)
-    static constexpr uint32_t kQ = 0;
-    static constexpr uint32_t kK = kQ + kHalf;
-    static constexpr uint32_t kEnd = (2 * kHalf > (uint32_t)kPBytes ? 2 * kHalf : (uint32_t)kPBytes);
+    static constexpr uint32_t kRing = 0;
+    static constexpr uint32_t kP = kRing + kScStages * kScStage;
+    static constexpr uint32_t kTab = kP + kPBytes;
+    static constexpr uint32_t kEnd = kTab + kScTabRows * 128 * 8;
     static constexpr uint32_t kBytes = kEnd + 1024;
 };
 
+struct ScBars {
+    uint64_t full[kScStages], empty[kScStages], rotated[kScStages], accfull[2], accempty[2];
+};
+
+// Named barrier `id` over 128 threads, returning whether x holds in all of them.
+__device__ __forceinline__ bool wg_all_id(int id, bool x) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, %2, 128, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)x), "r"(id)
+        : "memory");
+    return r != 0;
+}
+
 template <int DK>
-__global__ void __launch_bounds__(kScThreads) k_prep_scores(const __grid_constant__ ScoreParams p) {
-    using Sm = ScSmem<DK>;
-    constexpr int kHS = Sm::kHalfSlabs;
+__global__ void __launch_bounds__(kScThreads, 1) k_prep_scores(const __grid_constant__ ScoreParams p) {
+    constexpr int kSlabs = DK / 64;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar_ld, bar_mma;
+    __shared__ ScBars bars;
     __shared__ uint32_t s_tmem;
+    __shared__ int s_fail;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int jc = (int)(blockIdx.x % (unsigned)p.nchunks);
-    const int bh = (int)(blockIdx.x / (unsigned)p.nchunks);
-    const int h = bh % p.H, b = bh / p.H;
-    if (p.hc.anchor[h] < 0) return;   // left to the recurrent kernel
-    const int n0 = jc * kC, L = min(kC, p.N - n0);
-    const double lg = p.hc.log2g[h];
-    auto load_half = [&](int hf) {
-        tc::mbar_arrive_expect_tx(&bar_ld, 2 * Sm::kHalf);
-        for (int s = 0; s < kHS; s++) {
-            const int x = 64 * (kHS * hf + s);
-            tc::tma_load_4d(sm + Sm::kQ + s * (kC * 128), &p.tq_in, &bar_ld, x, h, n0, b);
-            tc::tma_load_4d(sm + Sm::kK + s * (kC * 128), &p.tk_in, &bar_ld, x, h, n0, b);
-        }
+    // the tile of local index i: (bh, jc), the (batch, head) pairs of one chunk
+    // next to each other, so that the CTAs at work read whole token rows of q
+    // and k together; heads the tensor cores do not take are skipped
+    const int BH = p.ntiles / p.nchunks;
+    auto tile_of = [&](int i, int* bh, int* jc) {
+        const int t = (int)blockIdx.x + i * (int)gridDim.x;
+        *jc = t / BH;
+        *bh = t % BH;
     };
+    const int ntile = p.ntiles > (int)blockIdx.x ? (p.ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
     if (tid == 0) {
-        tc::mbar_init(&bar_ld, 1);
-        tc::mbar_init(&bar_mma, 1);
+        for (int i = 0; i < kScStages; i++) {
+            tc::mbar_init(&bars.full[i], 1);
+            tc::mbar_init(&bars.empty[i], 2);     // the MMAs and the stores have read it
+            tc::mbar_init(&bars.rotated[i], 1);
+        }
+        for (int i = 0; i < 2; i++) {
+            tc::mbar_init(&bars.accfull[i], 1);
+            tc::mbar_init(&bars.accempty[i], 4);  // the epilogue warps have read it
+        }
+        s_fail = 0;
         tc::fence_barrier_init();
-        load_half(0);
     }
-    if (warp == 0) tc::tmem_alloc(&s_tmem, 128);
+    if (warp == 1) tc::tmem_alloc(&s_tmem, 256);
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tb = s_tmem;
     bool ok = true;
 
-    constexpr int kGpr = DK / 16;               // 16-byte groups in a row's half
-    constexpr int kRows = kScThreads / kGpr;    // rows one pass of the block covers
-    const int cc = tid % kGpr, rfirst = tid / kGpr;
-    const int slab = cc / 8, c16 = cc % 8;
-    const int a = min(p.hc.anchor[h], L - 1);
-    const uint32_t id = tc::idesc_bf16_f32(128, 128, 0, 0);
-    for (int hf = 0; hf < 2; hf++) {
-        ok = ok && tc::mbar_wait(&bar_ld, hf & 1);
-        // ---- rotation and key scale of this half, in place
-        const int col = DK / 2 * hf + 8 * cc;   // first of the thread's 8 columns
-        const bool real = col < p.dks;
-        const bool turn = p.xpos && real;
-        if (real && ok) {
-            float cs[4], sn[4], cst[4], sst[4];
-#pragma unroll
-            for (int k = 0; k < 4; k++) {
-                cs[k] = cst[k] = 1.f;
-                sn[k] = sst[k] = 0.f;
-                if (turn) {
-                    const double th = exp2(-2.0 * (col / 2 + k) / p.dks * p.log2base);
-                    __sincosf(angle_mod_2pi((double)(p.pos0 + n0 + rfirst) * th), &sn[k], &cs[k]);
-                    __sincosf(angle_mod_2pi((double)kRows * th), &sst[k], &cst[k]);
+    if (warp == 0) {
+        // ---------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int done = 0;   // tiles loaded (the stages run over their slabs in order)
+            for (int i = 0; i < ntile && ok; i++) {
+                int bh, jc;
+                tile_of(i, &bh, &jc);
+                const int h = bh % p.H, b = bh / p.H;
+                if (p.hc.anchor[h] < 0) continue;
+                for (int s = 0; s < kSlabs && ok; s++) {
+                    const int g = done * kSlabs + s, st = g % kScStages, u = g / kScStages;
+                    if (u > 0) ok = tc::mbar_wait(&bars.empty[st], (u - 1) & 1);
+                    if (!ok) break;
+                    uint8_t* dst = sm + ScSmem::kRing + st * kScStage;
+                    tc::mbar_arrive_expect_tx(&bars.full[st], kScStage);
+                    tc::tma_load_4d(dst, &p.tq_in, &bars.full[st], 64 * s, h, jc * kC, b);
+                    tc::tma_load_4d(dst + kScSlab, &p.tk_in, &bars.full[st], 64 * s, h, jc * kC, b);
                 }
+                done++;
             }
-            for (int r = rfirst; r < L; r += kRows) {
-                const uint32_t off = (uint32_t)slab * (kC * 128) + tc::sw128_off((uint32_t)r, (uint32_t)c16);
-                uint4* qa = reinterpret_cast<uint4*>(sm + Sm::kQ + off);
-                uint4* ka = reinterpret_cast<uint4*>(sm + Sm::kK + off);
-                // k' scale gamma^(a-r): the exponent in fp64, exp2 in fp32
-                const float zeta = exp2f((float)((double)(a - r) * lg));
-                float ck[4], sk[4];
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------- MMA issuer
+        const uint32_t id = tc::idesc_bf16_f32(128, 128, 0, 0);
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity));
+        };
+        int done = 0;   // tiles issued (the accumulators alternate over them)
+        for (int i = 0; i < ntile && ok; i++) {
+            int bh, jc;
+            tile_of(i, &bh, &jc);
+            if (p.hc.anchor[bh % p.H] < 0) continue;
+            const int buf = done & 1;
+            if (done >= 2) ok = wait(&bars.accempty[buf], ((done >> 1) - 1) & 1);
+            if (!ok) break;
+            for (int s = 0; s < kSlabs && ok; s++) {
+                const int g = done * kSlabs + s, st = g % kScStages, u = g / kScStages;
+                ok = wait(&bars.rotated[st], u & 1);
+                if (!ok) break;
+                tc::tc_fence_after();
+                const uint32_t base = tc::smem_u32(sm + ScSmem::kRing + st * kScStage);
+                const uint64_t dq = tc::sdesc_sw128(base, 16, 1024);
+                const uint64_t dk = tc::sdesc_sw128(base + kScSlab, 16, 1024);
 #pragma unroll
-                for (int k = 0; k < 4; k++) {
-                    ck[k] = cs[k] * zeta;
-                    sk[k] = sn[k] * zeta;
+                for (int k = 0; k < 4; k++)
+                    tc::mma_bf16_ss_elect(tb + 128 * buf, dq + (uint32_t)(k * 2), dk + (uint32_t)(k * 2), id,
+                                          (s > 0) || (k > 0));
+                tc::mma_commit_elect(&bars.empty[st]);
+            }
+            if (!ok) break;
+            tc::mma_commit_elect(&bars.accfull[buf]);
+            done++;
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------- rotation warpgroup
+        const int wt = tid - 128;             // 0..127
+        const int c16 = wt % 8;               // the thread's 16-byte chunk of a slab row
+        const int rfirst = wt / 8;            // rows rfirst, rfirst + 16, ...
+        float2* tab = reinterpret_cast<float2*>(sm + ScSmem::kTab);   // [kScTabRows][128]
+        const int npairs = p.dks / 2;
+        if (p.xpos) {
+            // turns through r theta_p, r = 0..16 (small angles: fp32 sine and cosine)
+            for (int e = wt; e < 17 * 128; e += 128) {
+                const int r = e / 128, pp = e % 128;
+                float sv = 0.f, cv = 1.f;
+                if (pp < npairs) sincosf((float)(r * p.theta[pp]), &sv, &cv);
+                tab[e] = make_float2(cv, sv);
+            }
+        }
+        int done = 0;
+        for (int i = 0; i < ntile && ok; i++) {
+            int bh, jc;
+            tile_of(i, &bh, &jc);
+            const int h = bh % p.H, b = bh / p.H;
+            if (p.hc.anchor[h] < 0) continue;
+            const int n0 = jc * kC, L = min(kC, p.N - n0);
+            const float lgf = (float)p.hc.log2g[h];
+            const int a = min(p.hc.anchor[h], L - 1);
+            if (p.xpos) {
+                // the tile's base angle of every pair: fp64 product, reduced, then fp32
+                if (wt < npairs) {
+                    float sv, cv;
+                    __sincosf(angle_mod_2pi((double)(p.pos0 + n0) * p.theta[wt]), &sv, &cv);
+                    tab[17 * 128 + wt] = make_float2(cv, sv);
                 }
-                if (turn) *qa = turn_group(*qa, cs, sn);
-                *ka = turn_group(*ka, ck, sk);
-                if (turn) {
+                wg_all_id(1, true);
+            }
+            for (int s = 0; s < kSlabs && ok; s++) {
+                const int g = done * kSlabs + s, st = g % kScStages, u = g / kScStages;
+                ok = wg_all_id(1, tc::mbar_wait(&bars.full[st], u & 1));
+                if (!ok) break;
+                uint8_t* base = sm + ScSmem::kRing + st * kScStage;
+                const int col = 64 * s + 8 * c16;   // first of the thread's 8 columns
+                const bool real = col < p.dks;
+                const bool turn = p.xpos && real;
+                if (real) {
+                    float cs[4], sn[4], cst[4], sst[4];
 #pragma unroll
                     for (int k = 0; k < 4; k++) {
-                        const float c2 = cs[k] * cst[k] - sn[k] * sst[k];
-                        sn[k] = sn[k] * cst[k] + cs[k] * sst[k];
-                        cs[k] = c2;
+                        cs[k] = cst[k] = 1.f;
+                        sn[k] = sst[k] = 0.f;
+                        if (turn) {
+                            const int pp = col / 2 + k;
+                            const float2 t0 = tab[17 * 128 + pp], t1 = tab[rfirst * 128 + pp], t2 = tab[16 * 128 + pp];
+                            cs[k] = t0.x * t1.x - t0.y * t1.y;   // turn through (pos0 + n0 + rfirst) theta_p
+                            sn[k] = t0.y * t1.x + t0.x * t1.y;
+                            cst[k] = t2.x;
+                            sst[k] = t2.y;
+                        }
+                    }
+                    for (int r = rfirst; r < L; r += 16) {
+                        const uint32_t off = tc::sw128_off((uint32_t)r, (uint32_t)c16);
+                        uint4* qa = reinterpret_cast<uint4*>(base + off);
+                        uint4* ka = reinterpret_cast<uint4*>(base + kScSlab + off);
+                        // k' scale gamma^(a-r) (fp32: relative error a few 1e-7)
+                        const float zeta = exp2f((float)(a - r) * lgf);
+                        float ck[4], sk[4];
+#pragma unroll
+                        for (int k = 0; k < 4; k++) {
+                            ck[k] = cs[k] * zeta;
+                            sk[k] = sn[k] * zeta;
+                        }
+                        if (turn) *qa = turn_group(*qa, cs, sn);
+                        *ka = turn_group(*ka, ck, sk);
+                        if (turn) {
+#pragma unroll
+                            for (int k = 0; k < 4; k++) {
+                                const float c2 = cs[k] * cst[k] - sn[k] * sst[k];
+                                sn[k] = sn[k] * cst[k] + cs[k] * sst[k];
+                                cs[k] = c2;
+                            }
+                        }
                     }
                 }
+                tc::fence_proxy_async_smem();
+                wg_all_id(1, true);
+                if (wt == 0) {
+                    if (p.qcopy) tc::tma_store_4d(&p.tq_out, base, 64 * s, h, n0, b);
+                    tc::tma_store_4d(&p.tk_out, base + kScSlab, 64 * s, h, n0, b);
+                    tc::bulk_commit_group();
+                    tc::mbar_arrive(&bars.rotated[st]);
+                    // the stores of slab g - kScLag have read their stage by now
+                    // (one bulk group per slab): that stage goes back
+                    tc::bulk_wait_group_read<kScLag>();
+                    if (g >= kScLag) tc::mbar_arrive(&bars.empty[(g - kScLag) % kScStages]);
+                }
             }
+            done++;
         }
-        tc::fence_proxy_async_smem();
-        ok = __syncthreads_and(ok ? 1 : 0) != 0;
-        // ---- the half of q_rot and k' out; A' += Q_half K'_half^T
-        if (tid == 0 && ok) {
-            for (int s = 0; s < kHS; s++) {
-                const int x = 64 * (kHS * hf + s);
-                if (p.qcopy) tc::tma_store_4d(&p.tq_out, sm + Sm::kQ + s * (kC * 128), x, h, n0, b);
-                tc::tma_store_4d(&p.tk_out, sm + Sm::kK + s * (kC * 128), x, h, n0, b);
-            }
-            tc::bulk_commit_group();
+        if (wt == 0) tc::bulk_wait_group<0>();   // (no load waits for the last stages)
+    } else if (warp >= 8) {
+        // ------------------------------------------- epilogue warpgroup
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const int wt = tid - 256;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        int done = 0;
+        for (int i = 0; i < ntile && ok; i++) {
+            int bh, jc;
+            tile_of(i, &bh, &jc);
+            if (p.hc.anchor[bh % p.H] < 0) continue;
+            const int buf = done & 1;
+            ok = wg_all_id(2, tc::mbar_wait(&bars.accfull[buf], (done >> 1) & 1));
+            if (!ok) break;
             tc::tc_fence_after();
-            const uint64_t dq = tc::sdesc_sw128(tc::smem_u32(sm + Sm::kQ), 16, 1024);
-            const uint64_t dk = tc::sdesc_sw128(tc::smem_u32(sm + Sm::kK), 16, 1024);
+            // the staging tile is reused once the previous P store has read it
+            if (wt == 0) tc::bulk_wait_group_read<0>();
+            wg_all_id(2, true);
 #pragma unroll
-            for (int k = 0; k < DK / 32; k++) {
-                const uint32_t o = (uint32_t)(((k / 4) * (kC * 128) + (k % 4) * 32) >> 4);
-                tc::mma_bf16_ss(tb, dq + o, dk + o, id, (hf > 0) || (k > 0));
+            for (int q32 = 0; q32 < 4; q32++) {
+                uint32_t av[32], w[16];
+                tc::tmem_ld32(tb + lane_off + 128 * buf + 32 * q32, av);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int k = 0; k < 16; k++) {
+                    const int c = 32 * q32 + 2 * k;
+                    const float lo = (c <= r) ? __uint_as_float(av[2 * k]) : 0.f;
+                    const float hi = (c + 1 <= r) ? __uint_as_float(av[2 * k + 1]) : 0.f;
+                    w[k] = tc::pack_bf16x2(lo, hi);
+                }
+                // columns 32 q32 .. + 31: slab q32 / 2, 16-byte chunks 4 (q32 % 2) ..
+#pragma unroll
+                for (int q4 = 0; q4 < 4; q4++)
+                    *reinterpret_cast<uint4*>(sm + ScSmem::kP + (q32 / 2) * kScSlab +
+                                              tc::sw128_off((uint32_t)r, (uint32_t)(4 * (q32 % 2) + q4))) =
+                        make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
             }
-            tc::mma_commit(&bar_mma);
-            // the slot is reused once the stores have read it and the MMAs are done
-            tc::bulk_wait_group_read<0>();
-            ok = tc::mbar_wait(&bar_mma, hf & 1);
-            if (ok && hf == 0) load_half(1);
-        }
-        ok = __syncthreads_and(ok ? 1 : 0) != 0;
-    }
-    tc::tc_fence_after();
-
-    // ---- P = tril(A') as bf16 into the slot: warp w reads TMEM lanes
-    // 32 w .. (its rows), all 128 key columns
-    if (ok) {
-        const int r = warp * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-#pragma unroll
-        for (int q32 = 0; q32 < 4; q32++) {
-            uint32_t av[32], w[16];
-            tc::tmem_ld32(tb + lane_off + 32 * q32, av);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; i++) {
-                const int c = 32 * q32 + 2 * i;
-                const float lo = (c <= r) ? __uint_as_float(av[2 * i]) : 0.f;
-                const float hi = (c + 1 <= r) ? __uint_as_float(av[2 * i + 1]) : 0.f;
-                w[i] = tc::pack_bf16x2(lo, hi);
+            tc::tc_fence_before();
+            elect_arrive(&bars.accempty[buf], lane);
+            tc::fence_proxy_async_smem();
+            wg_all_id(2, true);
+            if (wt == 0) {
+                const int prow = (bh * p.nchunks + jc) * kC;
+                for (int s = 0; s < 2; s++) tc::tma_store_2d(&p.tp, sm + ScSmem::kP + s * kScSlab, 64 * s, prow);
+                tc::bulk_commit_group();
             }
-            // columns 32 q32 .. + 31: slab q32 / 2, 16-byte chunks 4 (q32 % 2) ..
-#pragma unroll
-            for (int q4 = 0; q4 < 4; q4++)
-                *reinterpret_cast<uint4*>(sm + (q32 / 2) * (kC * 128) +
-                                          tc::sw128_off((uint32_t)r, (uint32_t)(4 * (q32 % 2) + q4))) =
-                    make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+            done++;
         }
+        if (wt == 0) tc::bulk_wait_group<0>();
     }
-    tc::tc_fence_before();
-    tc::fence_proxy_async_smem();
-    ok = __syncthreads_and(ok ? 1 : 0) != 0;
-    if (tid == 0) {
-        if (ok) {
-            const int prow = (bh * p.nchunks + jc) * kC;
-            for (int s = 0; s < 2; s++) tc::tma_store_2d(&p.tp, sm + s * (kC * 128), 64 * s, prow);
-            tc::bulk_commit_group();
-        }
-        tc::bulk_wait_group<0>();   // every store has read its tile (and is done)
-        if (!ok) atomicExch(&g_err_chunk_ws, kErrTimeout);
-    }
+    if (!ok) atomicExch(&s_fail, 1);
     tc::tc_fence_before();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tb, 128);
+    if (s_fail && tid == 0) atomicExch(&g_err_chunk_ws, kErrTimeout);
+    if (warp == 1) tc::tmem_dealloc(tb, 256);
 }
 
 template <int DK, typename Tout, bool PREP = false>
@@ -1247,21 +1369,26 @@ ret_status launch_chunkwise_scores_pass1(const RetArgs& a, void* ws, cudaStream_
         sp.xpos = a.xpos;
         sp.qcopy = qc ? 1 : 0;
         sp.pos0 = a.pos_offset;
-        sp.log2base = log2(a.theta_base);
-        const long long grid = (long long)a.B * a.H * nchunks;
-        if (grid > (1ll << 31) - 1) return fail(RET_ERR_UNSUPPORTED, "chunkwise (scores): too many chunks");
+        for (int i = 0; i < 128; i++) sp.theta[i] = i < dkr / 2 ? pow(a.theta_base, -2.0 * i / dkr) : 0.0;
+        const long long ntiles = (long long)a.B * a.H * nchunks;
+        if (ntiles > (1ll << 30)) return fail(RET_ERR_UNSUPPORTED, "chunkwise (scores): too many chunks");
+        sp.ntiles = (int)ntiles;
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                      cudaSuccess)
+            return fail(RET_ERR_CUDA, "chunkwise (scores pass): device query failed");
+        const unsigned grid = (unsigned)std::min<long long>(ntiles, sms);
+        const int smem = (int)ScSmem::kBytes;
         if (a.dk == 256) {
             auto kern = k_prep_scores<256>;
-            const int smem = (int)ScSmem<256>::kBytes;
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
                 return check_launch("chunkwise (scores pass): smem attribute");
-            kern<<<(unsigned)grid, kScThreads, smem, s>>>(sp);
+            kern<<<grid, kScThreads, smem, s>>>(sp);
         } else {
             auto kern = k_prep_scores<128>;
-            const int smem = (int)ScSmem<128>::kBytes;
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
                 return check_launch("chunkwise (scores pass): smem attribute");
-            kern<<<(unsigned)grid, kScThreads, smem, s>>>(sp);
+            kern<<<grid, kScThreads, smem, s>>>(sp);
         }
         return check_launch("chunkwise (scores pass)");
     }
