@@ -271,7 +271,7 @@ def run_ours(args):
     gbs = nbytes / t_main / 1e9
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
-    traffic = load_traffic("k_chunkwise_ws")
+    traffic = load_traffic("k_chunkwise_ws_scores")
     if t_hbm >= t_tc:
         roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(gbs / peaks["hbm_gbs"], 4)}
