@@ -90,13 +90,23 @@ ret_status ret_xpos_rotate(void* x, ret_dtype dt, int B, int N, int H, int d,
  * xpos != 0 applies the rotation of ret_xpos_rotate (positions pos_offset + n,
  *      base theta_base) to q and k as they are loaded; the inputs are not
  *      modified.
- * Kernels: in_dt RET_BF16 with dk in {128, 256}, dv a multiple of 64,
- * chunk = 128 and every gamma_h^128 >= 2^-60 runs on the tensor cores
- * (tcgen05/TMEM/TMA).  Otherwise the fp32 CUDA-core chunkwise kernel runs
- * when its per-block working set (about 4 * chunk * (2 dk + chunk + 64)
- * + 256 dk bytes) fits in shared memory, and else the token-by-token
- * recurrent kernel (dk <= 256), which computes the same function.  Larger dk
- * on neither path: RET_ERR_UNSUPPORTED.
+ * Kernels: in_dt RET_BF16 with chunk 128, dk 128 or 256 and dv a multiple
+ * of 64 (and dk 64 with chunk 64 or 128, zero-padded to 128 and computed in
+ * 128-token blocks) runs on the tensor cores (tcgen05/TMEM/TMA) in two
+ * launches: a pass that rotates q and k, scales the keys by the folded decay
+ * and computes each head's masked intra-chunk scores once, then the kernel
+ * of the read-out, P V and the state update.  Their scratch comes from a
+ * stream-ordered memory pool the library keeps per device (allocated and
+ * freed in stream order on `stream`; the pool keeps its memory for later
+ * calls).  Heads whose decay is too fast for the folded factors
+ * (gamma_h^64 < 2^-100) are computed by the token-by-token recurrent kernel
+ * in the same call.  Other shapes: the fp32 CUDA-core chunkwise kernel when
+ * its per-block working set (about 4 * chunk * (2 dk + chunk + 64)
+ * + 256 dk bytes) fits in shared memory, else the recurrent kernel
+ * (dk <= 256), which computes the same function.  Larger dk on neither path:
+ * RET_ERR_UNSUPPORTED.  A failure to get scratch from the pool is
+ * RET_ERR_CUDA; ret_forward_chunkwise_ws and ret_forward_chunkwise_noalloc
+ * take none.
  */
 ret_status ret_forward_chunkwise(const void* q, const void* k, const void* v,
                                  const double* gammas, int B, int N, int H, int dk, int dv,
@@ -108,14 +118,17 @@ ret_status ret_forward_chunkwise(const void* q, const void* k, const void* v,
  * Chunkwise forward with a caller-provided device workspace: the same
  * computation and arguments as ret_forward_chunkwise, plus `workspace`
  * (device, 256-byte aligned, not overlapping any other buffer) of at least
- * ret_chunkwise_workspace_bytes(...) bytes.  The workspace receives, in one
- * bandwidth-bound pass, the rotated queries (when xpos != 0) and the rotated
- * keys scaled by zeta = gamma^(chunk-1-j) (the decay of section 7.2 folded
- * into the keys), so that the tensor-core kernel that follows runs TMA ->
- * tcgen05 with no per-element work on q and k.  Its contents are scratch and
- * undefined after the call.  When the problem does not take this path
- * (ret_chunkwise_workspace_bytes returns 0, or some gamma_h^chunk < 2^-60)
- * the call behaves as ret_forward_chunkwise and does not touch the workspace.
+ * ret_chunkwise_workspace_bytes(...) bytes.  The first launch writes into
+ * it the rotated queries (when xpos != 0, or dk padded), the rotated keys
+ * scaled by gamma^(a-j) (the decay of section 7.2 folded into the keys about
+ * an anchor row a of each chunk: a = 127, or 63 for heads with
+ * gamma^128 < 2^-60) and the masked scores P = tril(Q K'^T) of every
+ * (batch, head, chunk) in bf16; the tensor-core kernel that follows reads
+ * them by TMA.  Its contents are scratch and undefined after the call.  When
+ * the shape does not take this path (ret_chunkwise_workspace_bytes returns
+ * 0) or no head does (every gamma_h^64 < 2^-100), the call behaves as
+ * ret_forward_chunkwise and does not touch the workspace; heads with
+ * gamma_h^64 < 2^-100 among others are computed token by token beside it.
  * The path takes bf16 inputs with chunk 128, dk 128 or 256 and dv a multiple
  * of 64; dk = 64 with chunk 64 or 128 also runs on it, zero-padded to dk 128
  * in the workspace and blocked by 128 tokens (the result is the
@@ -132,16 +145,17 @@ ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
                                     size_t workspace_bytes);
 
 /*
- * The two passes of ret_forward_chunkwise_ws as separate calls, on the same
- * workspace, in stream order (prepare, then prepared).  Shapes outside the
- * workspace path (ret_chunkwise_workspace_bytes returns 0, or some
- * gamma_h^chunk < 2^-60) return RET_ERR_UNSUPPORTED from both; use
+ * The two launches of ret_forward_chunkwise_ws as separate calls, on the
+ * same workspace, in stream order (prepare, then prepared).  Shapes outside
+ * the workspace path (ret_chunkwise_workspace_bytes returns 0, or some head
+ * with gamma_h^64 < 2^-100) return RET_ERR_UNSUPPORTED from both; use
  * ret_forward_chunkwise for them.
  *
  * ret_chunkwise_prepare reads q and k (device [B, N, H, dk], bf16, 16-byte
- * aligned) and fills the workspace with the rotated queries (xpos != 0) and
- * the rotated, zeta-scaled keys.  Its arguments mean what they mean for
- * ret_forward_chunkwise_ws; dv only selects the path (a multiple of 64).
+ * aligned) and fills the workspace with the rotated queries (xpos != 0), the
+ * rotated, decay-scaled keys and the masked scores P of every chunk.  Its
+ * arguments mean what they mean for ret_forward_chunkwise_ws; dv only
+ * selects the path (a multiple of 64).
  *
  * ret_forward_chunkwise_prepared runs the tensor-core kernel on a workspace
  * that ret_chunkwise_prepare filled with the same q, k, gammas, B, N, H, dk,
@@ -161,8 +175,10 @@ ret_status ret_forward_chunkwise_ws(const void* q, const void* k, const void* v,
  */
 /* Workspace bytes of ret_chunkwise_prepare / ret_forward_chunkwise_prepared
  * (0 when the shape is outside the path): the rotated queries (xpos, or a
- * dk of 64 padded to 128) and the rotated, zeta-scaled keys, [B, N, H, dk]
- * bf16 each at the kernel's dk. */
+ * dk of 64 padded to 128) and the rotated, decay-scaled keys, [B, N, H, dk]
+ * bf16 each at the kernel's dk, then (256-byte aligned) the P tiles,
+ * [B, H, ceil(N / 128), 128, 128] bf16.  The same as
+ * ret_chunkwise_workspace_bytes. */
 size_t ret_chunkwise_prepare_workspace_bytes(int B, int N, int H, int dk, int dv, int chunk,
                                              ret_dtype in_dt, int xpos);
 
@@ -308,8 +324,10 @@ ret_status ret_decode_step_positions(const void* q, const void* k, const void* v
  * forbids allocation afterwards.  The pages have no counterpart; this is a
  * deployment convenience of this library.
  * Same arguments and results as ret_forward_chunkwise (the caller still
- * passes every input and output buffer); the scratch of the workspace path
- * is a fixed device array inside the library, of
+ * passes every input and output buffer).  It runs the two-pass form (the
+ * rotation / key-scaling pass, then the tensor-core kernel computing the
+ * masked scores itself, so no P tiles), whose scratch is a fixed device
+ * array inside the library, of
  * ret_chunkwise_noalloc_max_bytes() bytes (64 MiB) on every GPU that loads
  * the library, held until the process exits.  Problems needing more scratch
  * than that return RET_ERR_INVALID_ARG, shapes outside the workspace path
