@@ -886,7 +886,7 @@ struct ScoreParams {
     double theta[128];             // theta_p = base^(-2p/d_k) of every pair, fp64
 };
 
-constexpr int kScThreads = 384;
+constexpr int kScThreads = 512;
 constexpr int kScStages = 5;
 constexpr int kScLag = 2;                        // slabs whose stores may still be reading their stages
 constexpr uint32_t kScSlab = kC * 128;           // one 64-column slab of 128 rows: 16 KB
@@ -909,16 +909,17 @@ struct ScBars {
     uint64_t full[kScStages], empty[kScStages], rotated[kScStages], accfull[2], accempty[2];
 };
 
-// Named barrier `id` over 128 threads, returning whether x holds in all of them.
-__device__ __forceinline__ bool wg_all_id(int id, bool x) {
+// Named barrier `id` over n threads (128 unless given), returning whether x
+// holds in all of them.
+__device__ __forceinline__ bool wg_all_id(int id, bool x, int n = 128) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred pi, po;\n\t"
         "setp.ne.u32 pi, %1, 0;\n\t"
-        "bar.red.and.pred po, %2, 128, pi;\n\t"
+        "bar.red.and.pred po, %2, %3, pi;\n\t"
         "selp.u32 %0, 1, 0, po;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)x), "r"(id)
+        : "r"((uint32_t)x), "r"(id), "r"(n)
         : "memory");
     return r != 0;
 }
@@ -1016,16 +1017,17 @@ __global__ void __launch_bounds__(kScThreads, 1) k_prep_scores(const __grid_cons
             tc::mma_commit_elect(&bars.accfull[buf]);
             done++;
         }
-    } else if (warp >= 4 && warp < 8) {
-        // ------------------------------------------- rotation warpgroup
-        const int wt = tid - 128;             // 0..127
+    } else if ((warp >= 4 && warp < 8) || warp >= 12) {
+        // ------------------------------------------ rotation (two warpgroups)
+        constexpr int kRot = 256;             // rotation threads
+        const int wt = warp < 8 ? tid - 128 : tid - 256;   // 0..255
         const int c16 = wt % 8;               // the thread's 16-byte chunk of a slab row
-        const int rfirst = wt / 8;            // rows rfirst, rfirst + 16, ...
+        const int rfirst = wt / 8;            // rows rfirst, rfirst + 32, ...
         float2* tab = reinterpret_cast<float2*>(sm + ScSmem::kTab);   // [kScTabRows][128]
         const int npairs = p.dks / 2;
         if (p.xpos) {
             // turns through r theta_p, r = 0..16 (small angles: fp32 sine and cosine)
-            for (int e = wt; e < 17 * 128; e += 128) {
+            for (int e = wt; e < 17 * 128; e += kRot) {
                 const int r = e / 128, pp = e % 128;
                 float sv = 0.f, cv = 1.f;
                 if (pp < npairs) sincosf((float)(r * p.theta[pp]), &sv, &cv);
@@ -1048,11 +1050,11 @@ __global__ void __launch_bounds__(kScThreads, 1) k_prep_scores(const __grid_cons
                     __sincosf(angle_mod_2pi((double)(p.pos0 + n0) * p.theta[wt]), &sv, &cv);
                     tab[17 * 128 + wt] = make_float2(cv, sv);
                 }
-                wg_all_id(1, true);
+                wg_all_id(1, true, kRot);
             }
             for (int s = 0; s < kSlabs && ok; s++) {
                 const int g = done * kSlabs + s, st = g % kScStages, u = g / kScStages;
-                ok = wg_all_id(1, tc::mbar_wait(&bars.full[st], u & 1));
+                ok = wg_all_id(1, tc::mbar_wait(&bars.full[st], u & 1), kRot);
                 if (!ok) break;
                 uint8_t* base = sm + ScSmem::kRing + st * kScStage;
                 const int col = 64 * s + 8 * c16;   // first of the thread's 8 columns
@@ -1066,39 +1068,56 @@ __global__ void __launch_bounds__(kScThreads, 1) k_prep_scores(const __grid_cons
                         sn[k] = sst[k] = 0.f;
                         if (turn) {
                             const int pp = col / 2 + k;
-                            const float2 t0 = tab[17 * 128 + pp], t1 = tab[rfirst * 128 + pp], t2 = tab[16 * 128 + pp];
+                            const float2 t0 = tab[17 * 128 + pp], t2 = tab[16 * 128 + pp];
+                            float2 t1 = tab[(rfirst & 15) * 128 + pp];
+                            if (rfirst >= 16) t1 = make_float2(t1.x * t2.x - t1.y * t2.y, t1.y * t2.x + t1.x * t2.y);
                             cs[k] = t0.x * t1.x - t0.y * t1.y;   // turn through (pos0 + n0 + rfirst) theta_p
                             sn[k] = t0.y * t1.x + t0.x * t1.y;
-                            cst[k] = t2.x;
-                            sst[k] = t2.y;
+                            cst[k] = t2.x * t2.x - t2.y * t2.y;  // the row step: 32 theta_p
+                            sst[k] = 2.f * t2.x * t2.y;
                         }
                     }
-                    for (int r = rfirst; r < L; r += 16) {
-                        const uint32_t off = tc::sw128_off((uint32_t)r, (uint32_t)c16);
-                        uint4* qa = reinterpret_cast<uint4*>(base + off);
-                        uint4* ka = reinterpret_cast<uint4*>(base + kScSlab + off);
-                        // k' scale gamma^(a-r) (fp32: relative error a few 1e-7)
-                        const float zeta = exp2f((float)(a - r) * lgf);
-                        float ck[4], sk[4];
+                    // the thread's rows rfirst + 32 i, i < nr: every load first, then
+                    // the turns and stores (two warps per sub-partition here, so the
+                    // loads' latency is hidden mostly by the thread's own work)
+                    const int nr = (L - rfirst + 31) >> 5;
+                    uint4 qv[4], kv[4];
 #pragma unroll
-                        for (int k = 0; k < 4; k++) {
-                            ck[k] = cs[k] * zeta;
-                            sk[k] = sn[k] * zeta;
+                    for (int i = 0; i < 4; i++) {
+                        if (i < nr) {
+                            const uint32_t off = tc::sw128_off((uint32_t)(rfirst + 32 * i), (uint32_t)c16);
+                            if (turn) qv[i] = *reinterpret_cast<const uint4*>(base + off);
+                            kv[i] = *reinterpret_cast<const uint4*>(base + kScSlab + off);
                         }
-                        if (turn) *qa = turn_group(*qa, cs, sn);
-                        *ka = turn_group(*ka, ck, sk);
-                        if (turn) {
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; i++) {
+                        if (i < nr) {
+                            const int r = rfirst + 32 * i;
+                            const uint32_t off = tc::sw128_off((uint32_t)r, (uint32_t)c16);
+                            // k' scale gamma^(a-r) (fp32: relative error a few 1e-7)
+                            const float zeta = exp2f((float)(a - r) * lgf);
+                            float ck[4], sk[4];
 #pragma unroll
                             for (int k = 0; k < 4; k++) {
-                                const float c2 = cs[k] * cst[k] - sn[k] * sst[k];
-                                sn[k] = sn[k] * cst[k] + cs[k] * sst[k];
-                                cs[k] = c2;
+                                ck[k] = cs[k] * zeta;
+                                sk[k] = sn[k] * zeta;
+                            }
+                            if (turn) *reinterpret_cast<uint4*>(base + off) = turn_group(qv[i], cs, sn);
+                            *reinterpret_cast<uint4*>(base + kScSlab + off) = turn_group(kv[i], ck, sk);
+                            if (turn) {
+#pragma unroll
+                                for (int k = 0; k < 4; k++) {
+                                    const float c2 = cs[k] * cst[k] - sn[k] * sst[k];
+                                    sn[k] = sn[k] * cst[k] + cs[k] * sst[k];
+                                    cs[k] = c2;
+                                }
                             }
                         }
                     }
                 }
                 tc::fence_proxy_async_smem();
-                wg_all_id(1, true);
+                wg_all_id(1, true, kRot);
                 if (wt == 0) {
                     if (p.qcopy) tc::tma_store_4d(&p.tq_out, base, 64 * s, h, n0, b);
                     tc::tma_store_4d(&p.tk_out, base + kScSlab, 64 * s, h, n0, b);
@@ -1114,7 +1133,7 @@ __global__ void __launch_bounds__(kScThreads, 1) k_prep_scores(const __grid_cons
         }
         if (wt == 0) tc::bulk_wait_group<0>();   // (no load waits for the last stages)
     } else if (warp >= 8) {
-        // ------------------------------------------- epilogue warpgroup
+        // ------------------------------------------- epilogue warpgroup (warps 8-11)
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const int wt = tid - 256;
