@@ -288,14 +288,6 @@ __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const 
                  : "memory");
 }
 
-// Shared memory -> global memory bulk copy (untiled) in the issuing thread's
-// bulk async group: both addresses 16-byte aligned, size a multiple of 16.
-__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
-                 "r"(bytes)
-                 : "memory");
-}
-
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Wait until at most N of this thread's bulk groups still read shared memory.
