@@ -291,6 +291,11 @@ def run_ours(args):
     roof["tensor_frac"] = round(tflops / peaks["bf16_tflops"], 4)
     roof["hbm_gbs"] = round(gbs, 1)
     roof["hbm_frac"] = round(gbs / peaks["hbm_gbs"], 4)
+    # the same algorithmic work over the whole step (both kernels, mean step)
+    t_step = ms_per_step / 1e3
+    roof["step"] = {"ms": round(ms_per_step, 4), "hbm_frac": round(nbytes / t_step / 1e9 / peaks["hbm_gbs"], 4),
+                    "tensor_frac": round(flops / t_step / 1e12 / peaks["bf16_tflops"], 4),
+                    "roofline_ms": round(max(t_tc, t_hbm) * 1e3, 4)}
     # The scores pass: reads q, k; writes q_rot, k' and P (bf16); 2 C dk
     # FLOPs per (token, head) for the scores.
     nchunks = (N + C - 1) // C
