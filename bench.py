@@ -204,7 +204,7 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    # One step = one call of the spec entry point ret_forward_chunkwise:
+    # One step = one call of the library's chunkwise entry point ret_forward_chunkwise:
     # the scores pass (rotation, key scaling, masked intra-chunk scores on the
     # tensor cores) and the warp-specialized tensor-core kernel, on scratch
     # from the library's stream-ordered pool.
@@ -652,7 +652,7 @@ def _timed_flushed(torch, stream, fn, steps, warmup, world, dist, dev, flush):
 
 def bench_c2(R, torch, dev, stream, args, peaks, world, dist):
     """The pages' cost-analysis shape [4, 2048, 8 heads of 64], bf16, xPos,
-    chunk 64, L2 flushed before every call: the spec call
+    chunk 64, L2 flushed before every call: the single allocating call
     ret_forward_chunkwise (d_k padded to 128 on the tensor cores, 128-token
     blocks).  HBM-bound: algorithmic bytes = read q, k, v once, write out
     once (bf16)."""
