@@ -560,7 +560,7 @@ def bench_normalized(R, torch, dev, stream, w, g, args, peaks, world, dist):
     return {"workload": w["workload"], "flags": "decay + score", "ms_per_step": round(ms, 4),
             "tokens_per_s": round(world * B * N / (ms / 1e3), 1), "plain_ms_per_step": round(ms_plain, 4),
             "overhead": round(ms / ms_plain - 1.0, 4),
-            "kernels": "k_prep_qk, k_keysum, k_keycarry, k_rowscale, k_chunkwise_ws (row factors in the epilogue)",
+            "kernels": "k_prep_scores, k_keysum, k_keycarry, k_rowscale, k_chunkwise_ws (scores given, row factors in the epilogue)",
             "plain": "ret_forward_chunkwise (k_prep_scores + k_chunkwise_ws)"}
 
 

@@ -255,7 +255,7 @@ NormLayout norm_layout(const RetArgs& a) {
     NormLayout L;
     L.nsub = (a.N + kSub - 1) / kSub;
     L.nch = (a.N + kChunk - 1) / kChunk;
-    size_t o = al(chunkwise_ws_bytes(a));
+    size_t o = al(chunkwise_scores_bytes(a));   // the scores form's k', q_rot and P tiles
     L.rowscale = o; o += al((size_t)a.B * a.N * a.H * 4);
     L.subsum = o; o += al((size_t)a.B * a.H * L.nsub * a.dk * 4);
     L.zstart = o; o += al((size_t)a.B * a.H * L.nch * a.dk * 4);
@@ -274,9 +274,11 @@ ret_status launch_chunkwise_normalized(const RetArgs& a0, int flags, const float
     float* rowscale = reinterpret_cast<float*>(base + L.rowscale);
     float* subsum = reinterpret_cast<float*>(base + L.subsum);
     float* zstart = reinterpret_cast<float*>(base + L.zstart);
-    ret_status st = launch_chunkwise_prep(a0, ws, s);
+    // the scores pass: k' opens the workspace, the rotated q follows it (xpos)
+    // or is q itself, then the P tiles (the row factors scale whole output
+    // rows, so the scores need no change)
+    ret_status st = launch_chunkwise_scores_pass1(a0, ws, s);
     if (st != RET_OK) return st;
-    // the prepared k' opens the workspace; the rotated q follows it (xpos) or is q itself
     const size_t qk = (size_t)a0.B * a0.N * a0.H * a0.dk;
     const __nv_bfloat16* kp = reinterpret_cast<const __nv_bfloat16*>(ws);
     const __nv_bfloat16* qe = a0.xpos ? kp + qk : reinterpret_cast<const __nv_bfloat16*>(a0.q);
@@ -305,7 +307,7 @@ ret_status launch_chunkwise_normalized(const RetArgs& a0, int flags, const float
     if (st != RET_OK) return st;
     RetArgs a = a0;
     a.rowscale = rowscale;
-    return launch_chunkwise_prepared(a, ws, s);
+    return launch_chunkwise_scores_pass2(a, ws, s);
 }
 
 }  // namespace ret

@@ -222,9 +222,10 @@ def test_backward_rejects_bad_arguments(kw, status):
 def test_normalized_workspace_size():
     nb = R.ret_normalized_workspace_bytes(1, 200, 2, 128, 64, 128, torch.bfloat16, True)
     ws = 2 * 200 * 2 * 128 * 2
-    # the prepared q, k, then row factors [B, N, H], key sums per 32 rows and per chunk start
+    # the scores form's q_rot, k' and P tiles [B, H, 2 chunks, 128, 128], then row
+    # factors [B, N, H], key sums per 32 rows and per chunk start
     al = lambda x: (x + 255) // 256 * 256
-    assert nb == al(ws) + al(200 * 2 * 4) + al(2 * 7 * 128 * 4) + al(2 * 2 * 128 * 4)
+    assert nb == al(ws) + 2 * 2 * 128 * 128 * 2 + al(200 * 2 * 4) + al(2 * 7 * 128 * 4) + al(2 * 2 * 128 * 4)
     assert R.ret_normalized_workspace_bytes(1, 200, 2, 16, 64, 128, torch.bfloat16, True) == 0
     assert R.ret_normalized_workspace_bytes(1, 200, 2, 128, 64, 128, torch.float32, True) == 0
 
