@@ -23,6 +23,16 @@
 // 2^+-100 for gamma^64 >= 2^-100; heads below that are left to the recurrent
 // kernel (their CTAs return at once).
 //
+// Two forms share the main kernel.  The scores form (the allocating call,
+// the workspace call, prepare/prepared and the normalised forward) runs
+// k_prep_scores (below, after the main kernel) and then k_chunkwise_ws with
+// PREP = true: the scores P = tril(Q K'^T) of each (batch, head, chunk) come
+// from the workspace, warp 1 issues only the read-out and P V (P as the
+// shared-memory A operand, loaded by the producer), and the transform
+// warpgroups skip the mask.  The two-pass form (the backward's passes, the
+// MSR layer, the allocation-free call) runs k_prep_qk and then
+// k_chunkwise_ws with PREP = false, as laid out here:
+//
 // 1. k_prep_qk (HBM-bound, one pass, two-pass form): rotates q and k once per
 //    head (xPos, consecutive pairs, angle (pos_offset + n) theta_p with the
 //    sine and cosine of each (position, pair) evaluated once for all heads),
@@ -57,8 +67,11 @@
 //                          for the next read-out,
 //                epilogue: out = gamma^(r-a) O staged in the chunk's V slot.
 //    TMEM columns: A [0,128), P [128,192), O [192,256), Q [256,384),
-//    dS [384,512).  Every hand-off between the roles has at least one block
-//    of MMAs in between, so no role waits on another in the steady state.
+//    dS [384,512) (the scores form leaves A and P unused).  Every hand-off
+//    between the roles has at least one block of MMAs in between, so no role
+//    waits on another in the steady state.  On B200 the kernel is bound by
+//    its SM's shared-memory port (TMA fills, tensor-core operand reads and
+//    the warps' staging traffic, about 560 KB a chunk in the scores form).
 #include <algorithm>
 #include <cstring>
 #include <mutex>
