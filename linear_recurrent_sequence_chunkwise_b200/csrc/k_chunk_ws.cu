@@ -939,7 +939,9 @@ __device__ __forceinline__ bool wg_all_id(int id, bool x, int n = 128) {
 
 template <int DK>
 __global__ void __launch_bounds__(kScThreads, 1) k_prep_scores(const __grid_constant__ ScoreParams p) {
-    constexpr int kSlabs = DK / 64;
+    // the slabs of d_k a tile has: a d_k below DK (zero-padded) skips the
+    // slabs past it, which the main kernel reads as TMA zero-fill
+    const int nslabs = (p.dks + 63) / 64;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ ScBars bars;
@@ -986,8 +988,8 @@ __global__ void __launch_bounds__(kScThreads, 1) k_prep_scores(const __grid_cons
                 tile_of(i, &bh, &jc);
                 const int h = bh % p.H, b = bh / p.H;
                 if (p.hc.anchor[h] < 0) continue;
-                for (int s = 0; s < kSlabs && ok; s++) {
-                    const int g = done * kSlabs + s, st = g % kScStages, u = g / kScStages;
+                for (int s = 0; s < nslabs && ok; s++) {
+                    const int g = done * nslabs + s, st = g % kScStages, u = g / kScStages;
                     if (u > 0) ok = tc::mbar_wait(&bars.empty[st], (u - 1) & 1);
                     if (!ok) break;
                     uint8_t* dst = sm + ScSmem::kRing + st * kScStage;
@@ -1012,8 +1014,8 @@ __global__ void __launch_bounds__(kScThreads, 1) k_prep_scores(const __grid_cons
             const int buf = done & 1;
             if (done >= 2) ok = wait(&bars.accempty[buf], ((done >> 1) - 1) & 1);
             if (!ok) break;
-            for (int s = 0; s < kSlabs && ok; s++) {
-                const int g = done * kSlabs + s, st = g % kScStages, u = g / kScStages;
+            for (int s = 0; s < nslabs && ok; s++) {
+                const int g = done * nslabs + s, st = g % kScStages, u = g / kScStages;
                 ok = wait(&bars.rotated[st], u & 1);
                 if (!ok) break;
                 tc::tc_fence_after();
@@ -1065,8 +1067,8 @@ __global__ void __launch_bounds__(kScThreads, 1) k_prep_scores(const __grid_cons
                 }
                 wg_all_id(1, true, kRot);
             }
-            for (int s = 0; s < kSlabs && ok; s++) {
-                const int g = done * kSlabs + s, st = g % kScStages, u = g / kScStages;
+            for (int s = 0; s < nslabs && ok; s++) {
+                const int g = done * nslabs + s, st = g % kScStages, u = g / kScStages;
                 ok = wg_all_id(1, tc::mbar_wait(&bars.full[st], u & 1), kRot);
                 if (!ok) break;
                 uint8_t* base = sm + ScSmem::kRing + st * kScStage;
@@ -1261,7 +1263,9 @@ bool chunkwise_ws_supported(const RetArgs& a) {
 static ret_status fill_params(WsParams* p, const RetArgs& a, const void* q_src, int q_pitch, const void* k_prime) {
     memset(p, 0, sizeof(*p));
     const uint64_t B = a.B, N = a.N, H = a.H, dk = a.dk, dv = a.dv, qp = (uint64_t)q_pitch;
-    const uint64_t dq[4] = {dk, H, N, B};
+    // a d_k padded to the kernel's: the padded columns are read as TMA
+    // zero-fill, so the workspace need not hold them
+    const uint64_t dq[4] = {(uint64_t)(a.dk_real ? a.dk_real : a.dk), H, N, B};
     const uint64_t sq[3] = {dk * 2, H * dk * 2, N * H * dk * 2};
     const uint64_t sqq[3] = {qp * 2, H * qp * 2, N * H * qp * 2};
     const uint32_t box[4] = {64, 1, (uint32_t)kC, 1};
